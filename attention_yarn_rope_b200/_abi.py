@@ -1,0 +1,105 @@
+"""ctypes declarations of libgptoss_attn's C ABI (include/gptoss.h).
+
+Argument marshalling only.  The library must exist in-tree (built by
+``attention_yarn_rope_b200.build_lib``); a missing library raises, there is
+no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptoss_attn.so")
+
+GPTOSS_OK = 0
+GPTOSS_ERR_INVALID_ARG = 1
+GPTOSS_ERR_UNSUPPORTED = 2
+GPTOSS_ERR_CUDA = 3
+GPTOSS_ERR_TIMEOUT = 4
+
+STATUS_NAMES = {
+    0: "GPTOSS_OK",
+    1: "GPTOSS_ERR_INVALID_ARG",
+    2: "GPTOSS_ERR_UNSUPPORTED",
+    3: "GPTOSS_ERR_CUDA",
+    4: "GPTOSS_ERR_TIMEOUT",
+}
+
+# Every symbol include/gptoss.h declares.
+EXPORTED = (
+    "gptoss_status_string",
+    "gptoss_rope_qk",
+    "gptoss_attn_fwd",
+    "gptoss_attn_decode_workspace_size",
+    "gptoss_attn_decode",
+    "gptoss_read_device_status",
+    "gptoss_set_wait_limit",
+    "gptoss_selftest_wait_timeout",
+)
+
+
+class RopeParams(ctypes.Structure):
+    _fields_ = [
+        ("base", ctypes.c_double),
+        ("factor", ctypes.c_double),
+        ("initial_context", ctypes.c_int32),
+        ("rotary_dim", ctypes.c_int32),
+        ("ntk_alpha", ctypes.c_double),
+        ("ntk_beta", ctypes.c_double),
+    ]
+
+
+class Strides(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("tok", ctypes.c_int64), ("head", ctypes.c_int64)]
+
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_u32 = ctypes.c_uint32
+_f32 = ctypes.c_float
+_st = ctypes.c_int  # gptoss_status (enum)
+
+_SIGNATURES = {
+    "gptoss_status_string": (ctypes.c_char_p, [_st]),
+    "gptoss_rope_qk": (_st, [_vp, Strides, _vp, Strides, _vp, Strides, _vp, Strides, _vp, _vp, _i32, _i32, _i32,
+                             _i32, _i32, ctypes.POINTER(RopeParams), _vp]),
+    "gptoss_attn_fwd": (_st, [_vp, Strides, _vp, Strides, _vp, Strides, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                              _i32, _i32, _i32, _f32, ctypes.POINTER(RopeParams), _vp, Strides, _vp, _vp]),
+    "gptoss_attn_decode_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
+    "gptoss_attn_decode": (_st, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
+                                 ctypes.POINTER(RopeParams), _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "gptoss_read_device_status": (_st, [ctypes.POINTER(_i32), _i32, _vp]),
+    "gptoss_set_wait_limit": (_st, [_u32]),
+    "gptoss_selftest_wait_timeout": (_st, [_u32, _vp, _vp]),
+}
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree library once.  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libgptoss_attn.so not found at {LIB_PATH}; build it with "
+                "`python -m attention_yarn_rope_b200.build_lib` (there is no CPU fallback)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+class GptossError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+
+
+def check(fn: str, status: int) -> None:
+    if status != GPTOSS_OK:
+        raise GptossError(fn, status)

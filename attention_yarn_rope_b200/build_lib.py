@@ -1,0 +1,69 @@
+"""Builds libgptoss_attn.so in-tree with nvcc for sm_100a.
+
+Usage: ``python -m attention_yarn_rope_b200.build_lib [--verbose-ptxas]``.
+The library is one translation unit (``csrc/gptoss_lib.cu``) linked against
+the static CUDA runtime, so it needs no libcudart at load time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+SRC = os.path.join(PKG, "csrc", "gptoss_lib.cu")
+OUT = os.path.join(PKG, "libgptoss_attn.so")
+DEPS = [os.path.join(PKG, "csrc", f) for f in os.listdir(os.path.join(PKG, "csrc"))] + [
+    os.path.join(ROOT, "include", "gptoss.h")
+]
+
+
+def nvcc_path() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", shutil.which("nvcc")):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(OUT):
+        return False
+    t = os.path.getmtime(OUT)
+    return all(os.path.getmtime(d) <= t for d in DEPS if os.path.exists(d))
+
+
+def build(force: bool = False, ptxas_verbose: bool = False) -> str:
+    if not force and up_to_date():
+        return OUT
+    cmd = [
+        nvcc_path(),
+        "-gencode", "arch=compute_100a,code=sm_100a",
+        "-O3", "-lineinfo", "-std=c++17",
+        "--use_fast_math" if False else "-Xptxas=-O3",
+        "-Xcompiler", "-fPIC",
+        "-shared", "-cudart", "static",
+        "-I", os.path.join(ROOT, "include"),
+        "-o", OUT + ".tmp", SRC,
+    ]
+    if ptxas_verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    proc = subprocess.run(cmd, capture_output=True, text=True)
+    if proc.returncode != 0:
+        sys.stderr.write(proc.stdout + proc.stderr)
+        raise RuntimeError("nvcc failed building libgptoss_attn.so")
+    if ptxas_verbose:
+        sys.stderr.write(proc.stderr)
+    os.replace(OUT + ".tmp", OUT)
+    return OUT
+
+
+if __name__ == "__main__":
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose-ptxas", action="store_true")
+    a = ap.parse_args()
+    print(build(force=a.force, ptxas_verbose=a.verbose_ptxas))

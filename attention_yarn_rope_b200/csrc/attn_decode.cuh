@@ -1,0 +1,343 @@
+// attn_decode.cuh -- single-token decode over a bf16 KV cache (gptoss_attn_decode).
+//
+// Rule: the sink attention of GptOssAttention (NeMo AutoModel gpt_oss.layers
+// page: sinks, sliding_window, softmax_scale) for one new query per sequence
+// at position len-1 (RoPE rule of the gpt_oss.rope_utils page), keys already
+// rotated in the cache.
+//
+// Design: the op streams the cache once, so it is HBM-bound (8 FLOP per cache
+// byte at 8 q-heads per kv-head).  Split-KV: CTA (g, split, b) owns one kv
+// head and a contiguous chunk of keys and computes all G = Hq/Hkv query heads
+// of that group, so each cache byte is read exactly once.  A producer warp
+// streams 64-key K and V tiles with TMA (128-byte swizzled rows) through a
+// ring of stages; four consumer warps each take 16 keys of a stage and run
+// QK^T and PV on the tensor cores with warp-level mma.sync m16n8k16 (query
+// heads as the 16-row M side), an online softmax per head with quad shuffles,
+// and fp32 accumulators in registers.  The CTA writes an unnormalised partial
+// (m, l, O) per head; a second kernel merges the splits of each (b, g) and
+// folds exp(sink) into the denominator exactly once.
+#pragma once
+
+#include "host_util.cuh"
+#include "rope_qk.cuh"
+#include "sm100_ptx.cuh"
+
+namespace gptoss {
+
+constexpr int kDecTileKeys = 64;       // keys per pipeline stage
+constexpr int kDecStages = 6;
+constexpr int kDecConsumerWarps = 4;   // 16 keys of a stage each
+constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
+constexpr int kDecTileBytes = kDecTileKeys * kHeadDim * 2;  // 8 KB
+constexpr int kDecMaxGroup = 16;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct DecodeParams {
+  CUtensorMap tmap_k;  // dims (64, Hkv, Lmax, B), box (64, 1, 64, 1)
+  CUtensorMap tmap_v;
+  const __nv_bfloat16* q;  // [B, Hq, 64]
+  __nv_bfloat16* out;      // [B, Hq, 64]
+  float* lse;              // [B, Hq] nullable
+  const int32_t* seqlens;  // [B]
+  const float* sinks;      // [Hq]
+  float* ws_o;             // [B, Hkv, nsplit, G, 64]
+  float* ws_ml;            // [B, Hkv, nsplit, G, 2]
+  int B, Lmax, Hq, Hkv, G, window, chunk, nsplit;
+  float scale_log2;
+  uint64_t wait_ns;
+  RopeTable tab;
+};
+
+// Split count and chunk length for a decode launch.  They depend only on the
+// cache shape (not on the window), so the workspace sized for window 0 also
+// covers every window.
+__host__ __device__ inline int decode_chunk(int B, int Lmax, int Hkv) {
+  // aim at about 16 CTAs per SM over the whole launch, chunks of 256..4096 keys
+  const long long bh = static_cast<long long>(B) * Hkv;
+  long long c = (static_cast<long long>(Lmax) * bh + 2367) / 2368;
+  c = (c + kDecTileKeys - 1) / kDecTileKeys * kDecTileKeys;
+  if (c < 256) c = 256;
+  if (c > 4096) c = 4096;
+  return static_cast<int>(c);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Address of 16-byte chunk `c` of row `r` in a 128B-swizzled tile at `base`.
+__device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int r, int c) {
+  return base + r * 128 + ((c ^ (r & 7)) << 4);
+}
+
+struct __align__(1024) DecodeSmem {
+  uint8_t k[kDecStages][kDecTileBytes];
+  uint8_t v[kDecStages][kDecTileBytes];
+  __nv_bfloat16 q[kDecMaxGroup][kHeadDim + 8];  // rotated query rows, padded
+  float wm[kDecConsumerWarps][kDecMaxGroup];
+  float wl[kDecConsumerWarps][kDecMaxGroup];
+  uint64_t full[kDecStages];
+  uint64_t empty[kDecStages];
+};
+
+__global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int g = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = __ldg(p.seqlens + b);
+  const int lo = p.window > 0 ? max(0, n - p.window) : 0;
+  const int k_begin = lo + split * p.chunk;
+  const int k_end = min(n, k_begin + p.chunk);
+  if (k_begin >= k_end) return;  // this split is past the sequence: the merge skips it
+  const int ntile = (k_end - k_begin + kDecTileKeys - 1) / kDecTileKeys;
+  const int G = p.G;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kDecConsumerWarps);
+    }
+    fence_mbar_init();
+  }
+  // rotated query rows of this group (zero rows past G)
+  for (int idx = threadIdx.x; idx < kDecMaxGroup * kPairs; idx += kDecThreads) {
+    const int h = idx / kPairs, j = idx % kPairs;
+    float x = 0.f, y = 0.f;
+    if (h < G) {
+      const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(b) * p.Hq + g * G + h) * kHeadDim;
+      x = __bfloat162float(qr[j]);
+      y = __bfloat162float(qr[j + kPairs]);
+      if (p.tab.enabled) {
+        const float2 cs = rope_cs(n - 1, p.tab.inv_freq[j], p.tab.conc);
+        const float xr = x * cs.x - y * cs.y;
+        const float yr = y * cs.x + x * cs.y;
+        x = xr;
+        y = yr;
+      }
+    }
+    sm.q[h][j] = __float2bfloat16_rn(x);
+    sm.q[h][j + kPairs] = __float2bfloat16_rn(y);
+  }
+  __syncthreads();
+
+  if (warp == kDecConsumerWarps) {
+    // ---------------- producer warp ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tmap_k);
+      tma_prefetch_desc(&p.tmap_v);
+      for (int it = 0; it < ntile; ++it) {
+        const int s = it % kDecStages;
+        if (!mbar_wait(&sm.empty[s], ((it / kDecStages) & 1) ^ 1, p.wait_ns)) break;
+        mbar_arrive_expect_tx(&sm.full[s], 2 * kDecTileBytes);
+        const int key0 = k_begin + it * kDecTileKeys;
+        tma_load_4d(sm.k[s], &p.tmap_k, &sm.full[s], 0, g, key0, b);
+        tma_load_4d(sm.v[s], &p.tmap_v, &sm.full[s], 0, g, key0, b);
+      }
+      // drain: every issued stage must land before the CTA may exit
+      const int first = ntile > kDecStages ? ntile - kDecStages : 0;
+      for (int it = first; it < ntile; ++it)
+        mbar_wait(&sm.full[it % kDecStages], (it / kDecStages) & 1, p.wait_ns);
+    }
+    return;
+  }
+
+  // ---------------- consumer warps ----------------
+  const int gr = lane >> 2, tq = lane & 3;  // fragment row / column-pair index
+  // query A fragments: rows gr and gr+8, k-tiles of 16 features
+  uint32_t qa[4][4];
+#pragma unroll
+  for (int kt = 0; kt < 4; ++kt) {
+    const int c0 = kt * 16 + 2 * tq;
+    qa[kt][0] = *reinterpret_cast<const uint32_t*>(&sm.q[gr][c0]);
+    qa[kt][1] = *reinterpret_cast<const uint32_t*>(&sm.q[gr + 8][c0]);
+    qa[kt][2] = *reinterpret_cast<const uint32_t*>(&sm.q[gr][c0 + 8]);
+    qa[kt][3] = *reinterpret_cast<const uint32_t*>(&sm.q[gr + 8][c0 + 8]);
+  }
+  float o[8][4];
+#pragma unroll
+  for (int dt = 0; dt < 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of rows gr, gr+8
+  float l0 = 0.f, l1 = 0.f;              // this thread's share of the running sums
+
+  for (int it = 0; it < ntile; ++it) {
+    const int s = it % kDecStages;
+    if (!mbar_wait(&sm.full[s], (it / kDecStages) & 1, p.wait_ns)) break;
+    const uint32_t kb = smem_u32(sm.k[s]);
+    const uint32_t vb = smem_u32(sm.v[s]);
+    const int r0 = warp * 16;  // first key row of this warp in the tile
+    // S = Q K^T for two 8-key blocks
+    float sc[2][4];
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+      sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
+      const int row = r0 + nb * 8 + (lane & 7);
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sw128_addr(kb, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
+        mma_bf16_16816(sc[nb], qa[2 * kp], b0, b1);
+        mma_bf16_16816(sc[nb], qa[2 * kp + 1], b2, b3);
+      }
+    }
+    // mask keys past the chunk, scale into log2 units
+    const int key_base = k_begin + it * kDecTileKeys + r0;
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = key_base + nb * 8 + 2 * tq + (e & 1);
+        sc[nb][e] = key < k_end ? sc[nb][e] * p.scale_log2 : -INFINITY;
+      }
+    // online softmax, rows gr (e = 0, 1) and gr + 8 (e = 2, 3)
+    float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+    const float b0s = n0 == -INFINITY ? 0.f : n0;  // safe subtrahends
+    const float b1s = n1 == -INFINITY ? 0.f : n1;
+    const float a0 = ex2_approx(m0 - b0s), a1 = ex2_approx(m1 - b1s);
+    m0 = n0;
+    m1 = n1;
+    float pr[2][4];
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+      pr[nb][0] = ex2_approx(sc[nb][0] - b0s);
+      pr[nb][1] = ex2_approx(sc[nb][1] - b0s);
+      pr[nb][2] = ex2_approx(sc[nb][2] - b1s);
+      pr[nb][3] = ex2_approx(sc[nb][3] - b1s);
+    }
+    l0 = l0 * a0 + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
+    l1 = l1 * a1 + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
+#pragma unroll
+    for (int dt = 0; dt < 8; ++dt) {
+      o[dt][0] *= a0;
+      o[dt][1] *= a0;
+      o[dt][2] *= a1;
+      o[dt][3] *= a1;
+    }
+    // P as the A operand (16 heads x 16 keys)
+    uint32_t pa[4];
+    pa[0] = pack_bf16(pr[0][0], pr[0][1]);
+    pa[1] = pack_bf16(pr[0][2], pr[0][3]);
+    pa[2] = pack_bf16(pr[1][0], pr[1][1]);
+    pa[3] = pack_bf16(pr[1][2], pr[1][3]);
+    // O += P V over 8 feature blocks of 8
+#pragma unroll
+    for (int dp = 0; dp < 4; ++dp) {
+      uint32_t v0, v1, v2, v3;
+      const int row = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      ldsm_x4_t(sw128_addr(vb, row, 2 * dp + (lane >> 4)), v0, v1, v2, v3);
+      mma_bf16_16816(o[2 * dp], pa, v0, v1);
+      mma_bf16_16816(o[2 * dp + 1], pa, v2, v3);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.empty[s]);
+  }
+
+  // ---------------- merge the four warps ----------------
+  // The per-warp accumulators reuse the K stages once every warp is done.
+  named_barrier_sync(1, kDecConsumerWarps * 32);
+  float(*wo)[kDecMaxGroup][kHeadDim] = reinterpret_cast<float(*)[kDecMaxGroup][kHeadDim]>(&sm.k[0][0]);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  if (tq == 0) {
+    sm.wm[warp][gr] = m0;
+    sm.wm[warp][gr + 8] = m1;
+    sm.wl[warp][gr] = l0;
+    sm.wl[warp][gr + 8] = l1;
+  }
+#pragma unroll
+  for (int dt = 0; dt < 8; ++dt) {
+    wo[warp][gr][dt * 8 + 2 * tq] = o[dt][0];
+    wo[warp][gr][dt * 8 + 2 * tq + 1] = o[dt][1];
+    wo[warp][gr + 8][dt * 8 + 2 * tq] = o[dt][2];
+    wo[warp][gr + 8][dt * 8 + 2 * tq + 1] = o[dt][3];
+  }
+  named_barrier_sync(1, kDecConsumerWarps * 32);
+  const int tid = threadIdx.x;  // 128 consumer threads: (head, 4 features) x 2 passes
+  for (int idx = tid; idx < kDecMaxGroup * 16; idx += kDecConsumerWarps * 32) {
+    const int h = idx >> 4, d4 = (idx & 15) * 4;
+    if (h >= G) continue;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, sm.wm[w][h]);
+    const float Ms = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kDecConsumerWarps; ++w) {
+      const float sc = ex2_approx(sm.wm[w][h] - Ms);
+      L += sm.wl[w][h] * sc;
+      acc.x += wo[w][h][d4] * sc;
+      acc.y += wo[w][h][d4 + 1] * sc;
+      acc.z += wo[w][h][d4 + 2] * sc;
+      acc.w += wo[w][h][d4 + 3] * sc;
+    }
+    const int64_t slot = ((static_cast<int64_t>(b) * p.Hkv + g) * p.nsplit + split) * G + h;
+    *reinterpret_cast<float4*>(p.ws_o + slot * kHeadDim + d4) = acc;
+    if (d4 == 0) {
+      p.ws_ml[slot * 2] = M;
+      p.ws_ml[slot * 2 + 1] = L;
+    }
+  }
+}
+
+// Merge the splits of one (b, g): fold exp(sink) once, normalise, write bf16.
+__global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int n = __ldg(p.seqlens + b);
+  const int lo = p.window > 0 ? max(0, n - p.window) : 0;
+  const int nsp = min(p.nsplit, (n - lo + p.chunk - 1) / p.chunk);
+  const int G = p.G;
+  for (int idx = threadIdx.x; idx < G * 32; idx += 256) {
+    const int h = idx >> 5, d2 = (idx & 31) * 2;
+    const int head = g * G + h;
+    const float sink = __ldg(p.sinks + head) * kLog2e;
+    const int64_t base = (static_cast<int64_t>(b) * p.Hkv + g) * p.nsplit;
+    float M = sink;
+    for (int s = 0; s < nsp; ++s) M = fmaxf(M, p.ws_ml[((base + s) * G + h) * 2]);
+    const float Ms = M == -INFINITY ? 0.f : M;
+    float L = ex2_approx(sink - Ms);
+    float ox = 0.f, oy = 0.f;
+    for (int s = 0; s < nsp; ++s) {
+      const int64_t slot = (base + s) * G + h;
+      const float sc = ex2_approx(p.ws_ml[slot * 2] - Ms);
+      L += p.ws_ml[slot * 2 + 1] * sc;
+      const float2 ov = *reinterpret_cast<const float2*>(p.ws_o + slot * kHeadDim + d2);
+      ox += ov.x * sc;
+      oy += ov.y * sc;
+    }
+    const float inv = 1.f / L;
+    __nv_bfloat162 r;
+    r.x = __float2bfloat16_rn(ox * inv);
+    r.y = __float2bfloat16_rn(oy * inv);
+    *reinterpret_cast<__nv_bfloat162*>(p.out + (static_cast<int64_t>(b) * p.Hq + head) * kHeadDim + d2) = r;
+    if (p.lse != nullptr && d2 == 0) p.lse[static_cast<int64_t>(b) * p.Hq + head] = (M + log2f(L)) * kLn2;
+  }
+}
+
+}  // namespace gptoss

@@ -1,0 +1,251 @@
+// gptoss_lib.cu -- the C ABI of libgptoss_attn (declared in include/gptoss.h).
+// One translation unit: the kernels live in the headers included below.
+// Every entry point validates on the host, encodes its TMA descriptors and
+// launches asynchronously on the caller's stream; nothing is allocated.
+
+#include <cuda_runtime.h>
+
+#include "attn_decode.cuh"
+#include "attn_fwd.cuh"
+#include "gptoss.h"
+#include "host_util.cuh"
+#include "rope_qk.cuh"
+#include "sm100_ptx.cuh"
+
+using namespace gptoss;
+
+namespace {
+
+// One mbarrier that nothing ever arrives at: the kernel's bounded wait must
+// give up and record GPTOSS_ERR_TIMEOUT.  Exercises the device failure path.
+__global__ void wait_timeout_probe_kernel(uint64_t limit_ns, int* result) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(&bar, 0, limit_ns);
+  if (threadIdx.x == 0) *result = ok ? 1 : 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gptoss_status_string(gptoss_status s) {
+  switch (s) {
+    case GPTOSS_OK: return "GPTOSS_OK";
+    case GPTOSS_ERR_INVALID_ARG: return "GPTOSS_ERR_INVALID_ARG";
+    case GPTOSS_ERR_UNSUPPORTED: return "GPTOSS_ERR_UNSUPPORTED";
+    case GPTOSS_ERR_CUDA: return "GPTOSS_ERR_CUDA";
+    case GPTOSS_ERR_TIMEOUT: return "GPTOSS_ERR_TIMEOUT";
+  }
+  return "GPTOSS_ERR_UNKNOWN";
+}
+
+gptoss_status gptoss_set_wait_limit(uint32_t microseconds) {
+  wait_limit_ns() = microseconds == 0 ? 2000000000ull : static_cast<uint64_t>(microseconds) * 1000ull;
+  return GPTOSS_OK;
+}
+
+gptoss_status gptoss_read_device_status(int32_t* status_out, int32_t reset, struct CUstream_st* stream) {
+  if (status_out == nullptr) return GPTOSS_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return GPTOSS_ERR_CUDA;
+  if (reset) {
+    static const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return GPTOSS_ERR_CUDA;
+  }
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GPTOSS_ERR_CUDA;
+  *status_out = v;
+  return GPTOSS_OK;
+}
+
+gptoss_status gptoss_selftest_wait_timeout(uint32_t limit_us, int32_t* result_dev, struct CUstream_st* stream) {
+  if (result_dev == nullptr || limit_us == 0 || limit_us > 1000000) return GPTOSS_ERR_INVALID_ARG;
+  wait_timeout_probe_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<uint64_t>(limit_us) * 1000ull,
+                                                             reinterpret_cast<int*>(result_dev));
+  return check_launch();
+}
+
+gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk, void* q_out,
+                             gptoss_strides sq_out, void* k_out, gptoss_strides sk_out, const int32_t* positions,
+                             const int32_t* cu_seqlens, int32_t B, int32_t S_or_T, int32_t Hq, int32_t Hkv,
+                             int32_t D, const gptoss_rope_params* rope, struct CUstream_st* stream) {
+  if (rope == nullptr) return GPTOSS_ERR_INVALID_ARG;
+  if (B < 0 || S_or_T < 0 || Hq <= 0 || Hkv <= 0) return GPTOSS_ERR_INVALID_ARG;
+  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  gptoss_status st = check_rope(rope, D);
+  if (st != GPTOSS_OK) return st;
+  const bool thd = cu_seqlens != nullptr;
+  const int64_t ntok = thd ? S_or_T : static_cast<int64_t>(B) * S_or_T;
+  if (ntok == 0 || B == 0) return GPTOSS_OK;
+  if (ntok > INT32_MAX) return GPTOSS_ERR_INVALID_ARG;
+  if (!q || !k || !q_out || !k_out) return GPTOSS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out)) return GPTOSS_ERR_INVALID_ARG;
+  if (!strides_ok(sq, !thd) || !strides_ok(sk, !thd) || !strides_ok(sq_out, !thd) || !strides_ok(sk_out, !thd))
+    return GPTOSS_ERR_INVALID_ARG;
+  RopeQkParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.q_out = static_cast<__nv_bfloat16*>(q_out);
+  p.k_out = static_cast<__nv_bfloat16*>(k_out);
+  p.sq = sq;
+  p.sk = sk;
+  p.sqo = sq_out;
+  p.sko = sk_out;
+  p.tm.positions = positions;
+  p.tm.cu_seqlens = cu_seqlens;
+  p.tm.nseq = B;
+  p.tm.S = thd ? 0 : S_or_T;
+  p.tm.ntok = static_cast<int>(ntok);
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  yarn_table(*rope, &p.tab);
+  const int grid = static_cast<int>((ntok + kRopeTokensPerCta - 1) / kRopeTokensPerCta);
+  rope_qk_kernel<<<grid, kRopeThreads, 0, as_stream(stream)>>>(p);
+  return check_launch();
+}
+
+gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk, const void* v,
+                              gptoss_strides sv, const float* sinks, const int32_t* positions,
+                              const int32_t* cu_seqlens, int32_t B, int32_t S, int32_t total_tokens, int32_t Hq,
+                              int32_t Hkv, int32_t D, int32_t window, float softmax_scale,
+                              const gptoss_rope_params* rope, void* out, gptoss_strides so, float* lse,
+                              struct CUstream_st* stream) {
+  if (B < 0 || S < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0 || window < 0) return GPTOSS_ERR_INVALID_ARG;
+  if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
+  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
+  gptoss_status st = check_rope(rope, D);
+  if (st != GPTOSS_OK) return st;
+  const bool thd = cu_seqlens != nullptr;
+  if (!thd && static_cast<int64_t>(B) * S != total_tokens) return GPTOSS_ERR_INVALID_ARG;
+  if (total_tokens == 0 || B == 0 || S == 0) return GPTOSS_OK;
+  if (!q || !k || !v || !sinks || !out) return GPTOSS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GPTOSS_ERR_INVALID_ARG;
+  if (!strides_ok(sq, !thd) || !strides_ok(sk, !thd) || !strides_ok(sv, !thd) || !strides_ok(so, !thd))
+    return GPTOSS_ERR_INVALID_ARG;
+  const int n_qtiles = (S + kFwdTile - 1) / kFwdTile;
+  const int64_t grid = static_cast<int64_t>(n_qtiles) * Hq * B;
+  if (grid > INT32_MAX) return GPTOSS_ERR_UNSUPPORTED;
+
+  FwdParams p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t dimS = thd ? static_cast<uint64_t>(total_tokens) : static_cast<uint64_t>(S);
+  const uint64_t dimB = thd ? 1 : static_cast<uint64_t>(B);
+  const uint64_t kb_stride = thd ? dimS * sk.tok * 2 : static_cast<uint64_t>(sk.batch) * 2;
+  const uint64_t vb_stride = thd ? dimS * sv.tok * 2 : static_cast<uint64_t>(sv.batch) * 2;
+  st = make_tmap_bf16_4d(&p.tmap_k, k, kHeadDim, Hkv, dimS, dimB, sk.head * 2, sk.tok * 2,
+                         kb_stride == 0 ? 16 : kb_stride, kHeadDim, 1, kFwdTile, 1);
+  if (st != GPTOSS_OK) return st;
+  st = make_tmap_bf16_4d(&p.tmap_v, v, kHeadDim, Hkv, dimS, dimB, sv.head * 2, sv.tok * 2,
+                         vb_stride == 0 ? 16 : vb_stride, kHeadDim, 1, kFwdTile, 1);
+  if (st != GPTOSS_OK) return st;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.sq = sq;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.so = so;
+  p.lse = lse;
+  p.sinks = sinks;
+  p.positions = positions;
+  p.cu_seqlens = cu_seqlens;
+  p.B = B;
+  p.S = S;
+  p.T = total_tokens;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.window = window;
+  p.n_qtiles = n_qtiles;
+  p.scale_log2 = softmax_scale * kLog2e;
+  p.wait_ns = wait_limit_ns();
+  if (rope != nullptr) yarn_table(*rope, &p.tab);
+  else p.tab.enabled = 0;
+  const size_t smem = sizeof(FwdSmem) + 1024;
+  if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return GPTOSS_ERR_CUDA;
+  attn_fwd_kernel<<<static_cast<int>(grid), kFwdThreads, smem, as_stream(stream)>>>(p);
+  return check_launch();
+}
+
+size_t gptoss_attn_decode_workspace_size(int32_t B, int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D) {
+  if (B <= 0 || Lmax <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D != kHeadDim) return 0;
+  const int chunk = decode_chunk(B, Lmax, Hkv);
+  const int64_t nsplit = (Lmax + chunk - 1) / chunk;
+  const int64_t slots = static_cast<int64_t>(B) * Hkv * nsplit * (Hq / Hkv);
+  return static_cast<size_t>(slots * (kHeadDim + 2) * sizeof(float));
+}
+
+gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* cache_seqlens, const float* sinks, int32_t B, int32_t Lmax,
+                                 int32_t Hq, int32_t Hkv, int32_t D, int32_t window, float softmax_scale,
+                                 const gptoss_rope_params* rope, void* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, struct CUstream_st* stream) {
+  if (B < 0 || Lmax <= 0 || Hq <= 0 || Hkv <= 0 || window < 0) return GPTOSS_ERR_INVALID_ARG;
+  if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
+  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (Hq / Hkv > kDecMaxGroup) return GPTOSS_ERR_UNSUPPORTED;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
+  gptoss_status st = check_rope(rope, D);
+  if (st != GPTOSS_OK) return st;
+  if (B == 0) return GPTOSS_OK;
+  if (!q || !k_cache || !v_cache || !cache_seqlens || !sinks || !out || !workspace) return GPTOSS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace))
+    return GPTOSS_ERR_INVALID_ARG;
+  const size_t need = gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D);
+  if (need == 0 || workspace_bytes < need) return GPTOSS_ERR_INVALID_ARG;
+  const int64_t max_b = static_cast<int64_t>(B) * Lmax * Hkv * kHeadDim;
+  if (max_b > (int64_t(1) << 40)) return GPTOSS_ERR_UNSUPPORTED;
+
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
+  const uint64_t bat_b = tok_b * Lmax;
+  st = make_tmap_bf16_4d(&p.tmap_k, k_cache, kHeadDim, Hkv, Lmax, B, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
+                         kDecTileKeys, 1);
+  if (st != GPTOSS_OK) return st;
+  st = make_tmap_bf16_4d(&p.tmap_v, v_cache, kHeadDim, Hkv, Lmax, B, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
+                         kDecTileKeys, 1);
+  if (st != GPTOSS_OK) return st;
+  const int G = Hq / Hkv;
+  const int chunk = decode_chunk(B, Lmax, Hkv);
+  const int nsplit_max = (Lmax + chunk - 1) / chunk;
+  const int span = window > 0 ? (window < Lmax ? window : Lmax) : Lmax;
+  const int nsplit = (span + chunk - 1) / chunk;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.seqlens = cache_seqlens;
+  p.sinks = sinks;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = p.ws_o + static_cast<int64_t>(B) * Hkv * nsplit_max * G * kHeadDim;
+  p.B = B;
+  p.Lmax = Lmax;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.window = window;
+  p.chunk = chunk;
+  p.nsplit = nsplit_max;
+  p.scale_log2 = softmax_scale * kLog2e;
+  p.wait_ns = wait_limit_ns();
+  if (rope != nullptr) yarn_table(*rope, &p.tab);
+  else p.tab.enabled = 0;
+  const size_t smem = sizeof(DecodeSmem) + 1024;
+  if (cudaFuncSetAttribute(attn_decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return GPTOSS_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  attn_decode_split_kernel<<<dim3(Hkv, nsplit, B), kDecThreads, smem, s>>>(p);
+  if (check_launch() != GPTOSS_OK) return GPTOSS_ERR_CUDA;
+  attn_decode_merge_kernel<<<dim3(Hkv, B), 256, 0, s>>>(p);
+  return check_launch();
+}
+
+}  // extern "C"

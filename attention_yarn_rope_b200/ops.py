@@ -1,0 +1,170 @@
+"""Python binding of libgptoss_attn: the three entry points under the same
+names, taking torch tensors.
+
+PyTorch supplies device memory and the current CUDA stream; every step of the
+computation runs in the library's CUDA kernels.  Functions raise
+:class:`~attention_yarn_rope_b200._abi.GptossError` on any non-OK status, and
+:func:`~attention_yarn_rope_b200._abi.load` raises when the library is
+missing.  There is no CPU path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _abi
+
+
+@dataclass(frozen=True)
+class RopeConfig:
+    """YaRN parameters (RotaryEmbedding on the NeMo AutoModel gpt_oss.rope_utils page)."""
+
+    base: float = 150000.0
+    factor: float = 32.0
+    initial_context: int = 4096
+    ntk_alpha: float = 1.0
+    ntk_beta: float = 32.0
+    rotary_dim: int = 64
+
+    def to_c(self) -> _abi.RopeParams:
+        return _abi.RopeParams(float(self.base), float(self.factor), int(self.initial_context),
+                               int(self.rotary_dim), float(self.ntk_alpha), float(self.ntk_beta))
+
+    @staticmethod
+    def from_dict(d: dict, rotary_dim: int = 64) -> "RopeConfig":
+        return RopeConfig(d["base"], d["factor"], d["initial_context"], d["ntk_alpha"], d["ntk_beta"], rotary_dim)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _strides(t: torch.Tensor, thd: bool) -> _abi.Strides:
+    if t.stride(-1) != 1:
+        raise ValueError("head_dim must be contiguous")
+    if thd:
+        return _abi.Strides(0, t.stride(0), t.stride(1))
+    return _abi.Strides(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _check_dev(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+
+
+def gptoss_rope_qk(q, k, rope: RopeConfig, positions=None, cu_seqlens=None, q_out=None, k_out=None, stream=None):
+    """YaRN RoPE of q ``[B,S,Hq,D]`` / ``[T,Hq,D]`` and k (Hkv heads).
+    Returns ``(q_out, k_out)`` (new tensors unless given)."""
+    lib = _abi.load()
+    thd = cu_seqlens is not None
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    _check_dev(q, k, q_out, k_out, positions, cu_seqlens)
+    if thd:
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        B, S_or_T = cu_seqlens.numel() - 1, T
+    else:
+        B, S_or_T, Hq, D = q.shape
+        Hkv = k.shape[2]
+    r = rope.to_c()
+    st = lib.gptoss_rope_qk(_ptr(q), _strides(q, thd), _ptr(k), _strides(k, thd), _ptr(q_out),
+                            _strides(q_out, thd), _ptr(k_out), _strides(k_out, thd), _ptr(positions),
+                            _ptr(cu_seqlens), B, S_or_T, Hq, Hkv, D, ctypes.byref(r), _stream(stream))
+    _abi.check("gptoss_rope_qk", st)
+    return q_out, k_out
+
+
+def gptoss_attn_fwd(q, k, v, sinks, window: int = 0, softmax_scale: float | None = None,
+                    rope: RopeConfig | None = None, positions=None, cu_seqlens=None, max_seqlen: int | None = None,
+                    out=None, return_lse: bool = False, lse=None, stream=None):
+    """Prefill sink attention.  BSHD when q is 4-D, packed THD when q is 3-D
+    with ``cu_seqlens`` (then ``max_seqlen`` bounds the longest sequence).
+    Returns ``out`` or ``(out, lse)``."""
+    lib = _abi.load()
+    thd = cu_seqlens is not None
+    out = torch.empty_like(q) if out is None else out
+    if thd:
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            if cu_seqlens.is_cuda:
+                raise ValueError("max_seqlen is required when cu_seqlens lives on the device")
+            max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max()) if B > 0 else 0
+        S, total = int(max_seqlen), T
+        lse_shape = (Hq, T)
+    else:
+        B, S, Hq, D = q.shape
+        Hkv = k.shape[2]
+        total = B * S
+        lse_shape = (B, Hq, S)
+    if return_lse and lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    _check_dev(q, k, v, sinks, out, lse, positions, cu_seqlens)
+    scale = float(D) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    r = rope.to_c() if rope is not None else None
+    st = lib.gptoss_attn_fwd(_ptr(q), _strides(q, thd), _ptr(k), _strides(k, thd), _ptr(v), _strides(v, thd),
+                             _ptr(sinks), _ptr(positions), _ptr(cu_seqlens), B, S, total, Hq, Hkv, D, int(window),
+                             scale, ctypes.byref(r) if r is not None else None, _ptr(out), _strides(out, thd),
+                             _ptr(lse), _stream(stream))
+    _abi.check("gptoss_attn_fwd", st)
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def gptoss_attn_decode_workspace_size(B: int, Lmax: int, Hq: int, Hkv: int, D: int = 64) -> int:
+    return int(_abi.load().gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D))
+
+
+def gptoss_attn_decode(q, k_cache, v_cache, cache_seqlens, sinks, window: int = 0,
+                       softmax_scale: float | None = None, rope: RopeConfig | None = None, out=None,
+                       return_lse: bool = False, lse=None, workspace=None, stream=None):
+    """Single-token decode: q ``[B,Hq,D]`` raw, caches ``[B,Lmax,Hkv,D]`` (keys
+    rotated), ``cache_seqlens [B]`` int32 on the device."""
+    lib = _abi.load()
+    B, Hq, D = q.shape
+    _, Lmax, Hkv, _ = k_cache.shape
+    out = torch.empty_like(q) if out is None else out
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check_dev(q, k_cache, v_cache, cache_seqlens, sinks, out, lse, workspace)
+    for t in (q, k_cache, v_cache, out):
+        if not t.is_contiguous():
+            raise ValueError("decode tensors must be contiguous")
+    scale = float(D) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    r = rope.to_c() if rope is not None else None
+    st = lib.gptoss_attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens), _ptr(sinks), B, Lmax,
+                                Hq, Hkv, D, int(window), scale, ctypes.byref(r) if r is not None else None,
+                                _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream))
+    _abi.check("gptoss_attn_decode", st)
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def read_device_status(reset: bool = True, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _abi.check("gptoss_read_device_status",
+               _abi.load().gptoss_read_device_status(ctypes.byref(v), 1 if reset else 0, _stream(stream)))
+    return int(v.value)
+
+
+def set_wait_limit(microseconds: int) -> None:
+    _abi.check("gptoss_set_wait_limit", _abi.load().gptoss_set_wait_limit(int(microseconds)))
+
+
+def selftest_wait_timeout(limit_us: int, result_dev: torch.Tensor, stream=None) -> None:
+    _abi.check("gptoss_selftest_wait_timeout",
+               _abi.load().gptoss_selftest_wait_timeout(int(limit_us), _ptr(result_dev), _stream(stream)))

@@ -1,0 +1,510 @@
+#!/usr/bin/env python
+"""Benchmark of the GPT-OSS attention core on B200.
+
+Default workload (one "step"): the GPT-OSS-20b-shaped sliding-window layer
+prefill -- B=4, S=4096, 64 query / 8 kv heads, head_dim 64, window 128,
+YaRN RoPE (base 150000, factor 32, L0 4096, alpha 1, beta 32) fused into the
+attention kernel, per-head sinks -- one ``gptoss_attn_fwd`` launch.
+
+Prints ONE JSON line: ``value`` is whole-job sink-attention TFLOP/s (4*D
+FLOP per visible (query, key) pair per head, summed over all ranks),
+``e2e`` the same metric through the public API with pinned host buffers and
+the host<->device copies inside the timed region, ``roofline`` the dominant
+kernel against the measured HBM peak, ``cpu_baseline`` the float64 oracle on
+a bounded sample, and ``per_config`` the other workloads (full prefill, THD
+pair, decode) measured the same way.
+
+``--impl reference`` times the float64 CPU oracle on the same workload
+(bounded sample per step) and prints the same line with ``"impl":
+"reference"``.
+
+Multi-GPU (``torchrun --nproc-per-node N bench.py --gpus N``): one process per
+GPU, each running its own replica of the workload (the path has no exchange
+step, so there is no collective in the data path); the time is the max over
+ranks and ``value`` sums the work of all ranks (weak scaling).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sink-attn fwd TFLOP/s (prefill) & HBM GB/s (decode), % of B200 roofline"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def visible_pairs(lens, window):
+    """Number of visible (query, key) pairs of causal attention over sequences
+    of the given lengths (window 0 = full)."""
+    tot = 0
+    for n in lens:
+        n = int(n)
+        if window <= 0 or window >= n:
+            tot += n * (n + 1) // 2
+        else:
+            tot += window * (window + 1) // 2 + (n - window) * window
+    return tot
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        self.t0 = time.time()
+
+    def mark(self):
+        return time.time()
+
+    def stop(self, t_lo=None, t_hi=None):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "nvidia-smi unavailable"}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[5:]))
+                except Exception:
+                    continue
+        os.unlink(self.tmp.name)
+        window = "timed"
+        sel = [r for r in rows if t_lo is not None and t_lo - 1 <= r[0] <= t_hi + 1]
+        if not sel:
+            sel, window = rows, "warmup+timed"
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        mhz = sorted(r[1] for r in sel)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in sel:
+            flags = r[3][1:]
+            for n, f in zip(names, flags):
+                if f.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": max(r[2] for r in sel), "reasons": sorted(reasons),
+                "samples": len(sel), "window": window}
+
+
+# ----------------------------------------------------------------------------
+# timing helpers
+# ----------------------------------------------------------------------------
+def timed_steps(torch, fn, steps, stream, flush=None):
+    """Device time (ms) of `steps` calls of fn on `stream`, CUDA events on that
+    stream; with `flush`, L2 is overwritten between calls (outside the timing)."""
+    if flush is None:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(steps):
+            fn()
+        end.record(stream)
+        end.synchronize()
+        return start.elapsed_time(end)
+    total = 0.0
+    for _ in range(steps):
+        flush()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        fn()
+        end.record(stream)
+        end.synchronize()
+        total += start.elapsed_time(end)
+    return total
+
+
+# ----------------------------------------------------------------------------
+# workloads (our arm)
+# ----------------------------------------------------------------------------
+def prefill_case(torch, ops, cfg, device, seed_offset=0):
+    """Device inputs and a step closure for one prefill workload."""
+    from attention_yarn_rope_b200.workloads import make_prefill, to_torch_bf16
+
+    x = make_prefill(cfg, seed=cfg.seed + seed_offset)
+    q, k, v = (to_torch_bf16(a, device) for a in (x.q, x.k, x.v))
+    sinks = torch.from_numpy(x.sinks).to(device)
+    rope = ops.RopeConfig.from_dict(cfg.rope)
+    out = torch.empty_like(q)
+    if x.cu_seqlens is not None:
+        lens = [int(a) for a in (x.cu_seqlens[1:] - x.cu_seqlens[:-1])]
+        cu = torch.from_numpy(x.cu_seqlens).to(device)
+        max_len = max(lens)
+
+        def step():
+            ops.gptoss_attn_fwd(q, k, v, sinks, window=cfg.window, rope=rope, cu_seqlens=cu, max_seqlen=max_len,
+                                out=out)
+    else:
+        lens = [cfg.S] * cfg.B
+        cu = None
+
+        def step():
+            ops.gptoss_attn_fwd(q, k, v, sinks, window=cfg.window, rope=rope, out=out)
+    pairs = visible_pairs(lens, cfg.window) * cfg.Hq
+    flops = 4 * cfg.D * pairs
+    io_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, out))
+    return dict(x=x, q=q, k=k, v=v, sinks=sinks, out=out, cu=cu, step=step, flops=flops, bytes=io_bytes,
+                pairs=pairs, rope=rope, lens=lens)
+
+
+def decode_case(torch, ops, cfg, device):
+    from attention_yarn_rope_b200.workloads import make_decode_device
+
+    q, kc, vc, sinks, seqlens = make_decode_device(cfg, device)
+    rope = ops.RopeConfig.from_dict(cfg.rope)
+    out = torch.empty_like(q)
+    ws = torch.empty(ops.gptoss_attn_decode_workspace_size(cfg.B, cfg.L, cfg.Hq, cfg.Hkv, cfg.D),
+                     dtype=torch.uint8, device=device)
+
+    def step():
+        ops.gptoss_attn_decode(q, kc, vc, seqlens, sinks, window=cfg.window, rope=rope, out=out, workspace=ws)
+    span = cfg.L if cfg.window == 0 else min(cfg.window, cfg.L)
+    kv_bytes = 2 * cfg.B * span * cfg.Hkv * cfg.D * 2
+    io_bytes = kv_bytes + 2 * q.numel() * 2
+    return dict(step=step, bytes=io_bytes, kv_bytes=kv_bytes, flops=4 * cfg.D * cfg.B * cfg.Hq * span)
+
+
+def run_ours(args, torch, dist, rank, world, device):
+    from attention_yarn_rope_b200 import ops
+    from attention_yarn_rope_b200.workloads import (
+        DECODE_B8, DECODE_B8_W, DECODE_B64, DECODE_B64_W, FULL, SLIDING, THD_FULL, THD_WINDOW)
+
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    cfg = SLIDING
+    case = prefill_case(torch, ops, cfg, device, seed_offset=rank)
+    for _ in range(args.warmup):
+        case["step"]()
+    torch.cuda.synchronize()
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(torch.cuda.current_device())).split(",")[0]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else torch.cuda.current_device()
+    clk = ClockSampler(gpu_index if world == 1 else torch.cuda.current_device())
+    clk.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_lo = time.time()
+    ms = timed_steps(torch, case["step"], args.steps, stream)
+    torch.cuda.synchronize()
+    t_hi = time.time()
+    if world > 1:
+        dist.barrier()
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks = clk.stop(t_lo, t_hi)
+    per_step_ms = ms / args.steps
+    value = case["flops"] * world / (per_step_ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API, host buffers, copies inside ----
+    h_q = case["q"].cpu().pin_memory()
+    h_k = case["k"].cpu().pin_memory()
+    h_v = case["v"].cpu().pin_memory()
+    h_s = case["sinks"].cpu().pin_memory()
+    h_o = torch.empty(case["out"].shape, dtype=case["out"].dtype).pin_memory()
+    d_q, d_k, d_v, d_s, d_o = (torch.empty_like(t) for t in (case["q"], case["k"], case["v"], case["sinks"],
+                                                             case["out"]))
+
+    def e2e_step():
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        d_s.copy_(h_s, non_blocking=True)
+        ops.gptoss_attn_fwd(d_q, d_k, d_v, d_s, window=cfg.window, rope=case["rope"], out=d_o)
+        h_o.copy_(d_o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(3, min(args.steps, 50))
+    if world > 1:
+        dist.barrier()
+    ems = timed_steps(torch, e2e_step, e2e_steps, stream)
+    if world > 1:
+        t = torch.tensor([ems], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = case["flops"] * world / (ems / e2e_steps * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_s))
+    d2h = h_o.numel() * h_o.element_size()
+
+    achieved_gbs = case["bytes"] / (per_step_ms * 1e-3) / 1e9
+    roofline = {"kernel": "attn_fwd_kernel", "bound": "hbm", "achieved": round(achieved_gbs, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
+                "peak_source": peaks["source"], "traffic": read_traffic("attn_fwd_kernel", cfg.name),
+                "algorithmic_bytes_per_launch": case["bytes"],
+                "tflops": round(case["flops"] / (per_step_ms * 1e-3) / 1e12, 2)}
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "S": cfg.S, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D,
+                   "window": cfg.window, "rope": "yarn base 150000 factor 32 L0 4096 alpha 1 beta 32 (fused)",
+                   "global_batch": cfg.B * world, "seq_len": cfg.S, "parallelism": f"replicas{world}",
+                   "l2": f"inputs {case['bytes'] / 1e6:.0f} MB > L2 126 MB, no flush"},
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "roofline": roofline,
+    }
+    del h_q, h_k, h_v, h_o, d_q, d_k, d_v, d_o, case
+    torch.cuda.empty_cache()
+
+    if world == 1 and not args.no_extras:
+        line["per_config"] = per_config(torch, ops, device, stream, peaks,
+                                        [FULL, THD_FULL, THD_WINDOW],
+                                        [DECODE_B64, DECODE_B64_W, DECODE_B8, DECODE_B8_W], args)
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(SLIDING, budget_s=args.cpu_seconds)
+    return line
+
+
+def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, args):
+    res = {}
+    reps = max(3, min(args.steps, 20))
+    for cfg in prefill_cfgs:
+        case = prefill_case(torch, ops, cfg, device)
+        for _ in range(3):
+            case["step"]()
+        torch.cuda.synchronize()
+        ms = timed_steps(torch, case["step"], reps, stream) / reps
+        tf = case["flops"] / (ms * 1e-3) / 1e12
+        gbs = case["bytes"] / (ms * 1e-3) / 1e9
+        res[cfg.name] = {"ms": round(ms, 4), "tflops": round(tf, 2), "frac_of_measured_bf16": round(
+            tf / peaks["bf16_tflops"], 4), "frac_of_2250_spec": round(tf / 2250.0, 4), "gbs": round(gbs, 1),
+            "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "visible_pairs": case["pairs"],
+            "flops": case["flops"], "bytes": case["bytes"], "launches_per_call": 1}
+        del case
+        torch.cuda.empty_cache()
+    flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+    for cfg in decode_cfgs:
+        case = decode_case(torch, ops, cfg, device)
+        for _ in range(3):
+            case["step"]()
+        torch.cuda.synchronize()
+        small = case["kv_bytes"] < 4 * L2_BYTES
+        ms = timed_steps(torch, case["step"], reps, stream,
+                         flush=(lambda: flush_buf.fill_(1)) if small else None) / reps
+        gbs = case["bytes"] / (ms * 1e-3) / 1e9
+        res[cfg.name] = {"ms": round(ms, 4), "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+                         "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": case["kv_bytes"],
+                         "l2": "flushed between calls" if small else "cache > L2", "launches_per_call": 2}
+        del case
+        torch.cuda.empty_cache()
+    return res
+
+
+def read_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the kernel source as it is now (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = f"{kernel} {workload} "
+    src_hash = csrc_hash()
+    with open(path) as fh:
+        for line in fh:
+            if line.startswith(want):
+                parts = line.split()
+                if len(parts) >= 4 and parts[3] == src_hash:
+                    return int(parts[2])
+    return None
+
+
+def csrc_hash():
+    import hashlib
+
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "attention_yarn_rope_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+# ----------------------------------------------------------------------------
+# the float64 oracle on the host cores (cpu_baseline and the reference arm)
+# ----------------------------------------------------------------------------
+def _oracle_unit(x, cfg, b, g, tables):
+    """Oracle prefill of one (batch row, kv group): G query heads, all rows.
+    Returns the visible pairs it covered."""
+    import numpy as np
+
+    from oracle.attention import sink_attention_sequence
+    from oracle.rope import rope
+
+    G = cfg.Hq // cfg.Hkv
+    pos = np.arange(cfg.S)
+    qr = rope(x.q[b][:, g * G:(g + 1) * G], pos, *tables)
+    kr = rope(x.k[b][:, g:g + 1], pos, *tables)
+    sink_attention_sequence(qr, kr, x.v[b][:, g:g + 1], x.sinks[g * G:(g + 1) * G], cfg.softmax_scale, cfg.window)
+    return visible_pairs([cfg.S], cfg.window) * G
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    """Times the oracle as it stands on (batch row, kv group) units of the
+    workload until about `budget_s` seconds of CPU work; TFLOP/s of the sample."""
+    from attention_yarn_rope_b200.workloads import make_prefill
+    from oracle.yarn import yarn_inv_freq_and_concentration
+
+    x = make_prefill(cfg)
+    r = cfg.rope
+    tables = yarn_inv_freq_and_concentration(cfg.D, r["base"], r["factor"], r["initial_context"], r["ntk_alpha"],
+                                             r["ntk_beta"])
+    units = [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
+    done_pairs, n = 0, 0
+    t0 = time.perf_counter()
+    for b, g in units:
+        done_pairs += _oracle_unit(x, cfg, b, g, tables)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    tf = 4 * cfg.D * done_pairs / dt / 1e12
+    return {"value": round(tf, 6), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{n} of {len(units)} (batch row, kv-group) units of {cfg.name} "
+                      f"({n * cfg.Hq // cfg.Hkv} query heads x {cfg.S} rows), float64 NumPy, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The reference arm: the float64 oracle on this machine's host cores,
+    one (batch row, kv group) unit of the default workload per step."""
+    from attention_yarn_rope_b200.workloads import SLIDING, make_prefill
+    from oracle.yarn import yarn_inv_freq_and_concentration
+
+    cfg = SLIDING
+    x = make_prefill(cfg)
+    r = cfg.rope
+    tables = yarn_inv_freq_and_concentration(cfg.D, r["base"], r["factor"], r["initial_context"], r["ntk_alpha"],
+                                             r["ntk_beta"])
+    units = [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
+    for i in range(args.warmup):
+        _oracle_unit(x, cfg, *units[i % len(units)], tables)
+    pairs = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        pairs += _oracle_unit(x, cfg, *units[i % len(units)], tables)
+    dt = time.perf_counter() - t0
+    value = 4 * cfg.D * pairs / dt / 1e12
+    sample = (f"one (batch row, kv-group) unit per step: {cfg.Hq // cfg.Hkv} query heads x {cfg.S} rows of "
+              f"{cfg.name}, float64 NumPy")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / max(1, args.steps) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "S": cfg.S, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D,
+                   "window": cfg.window, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="skip the per-config measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import torch
+
+    dist = None
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = f"cuda:{local}"
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(device))
+    try:
+        line = run_ours(args, torch, dist, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

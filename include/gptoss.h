@@ -1,0 +1,185 @@
+/*
+ * gptoss.h -- C ABI of libgptoss_attn, the GPT-OSS attention core for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources by page title and section):
+ *   - YaRN rotary embedding of q and k: NeMo AutoModel
+ *     "nemo_automodel.components.models.gpt_oss.rope_utils", class
+ *     RotaryEmbedding (head_dim, base, initial_context_length, scaling_factor,
+ *     ntk_alpha, ntk_beta, partial_rotary_factor) and its method
+ *     _compute_concentration_and_inv_freq (YaRN paper, arXiv 2309.00071);
+ *     apply_rotary_emb / apply_rotary_emb_qk (half-split pairs, tables with
+ *     the concentration applied, BSHD or packed THD with cu_seqlens,
+ *     arbitrary strides, independently allocated outputs).
+ *   - Grouped-query causal softmax attention with a learned per-head sink
+ *     logit that adds exp(sink) to the softmax denominator only, full context
+ *     or a sliding window: NeMo AutoModel
+ *     "nemo_automodel.components.models.gpt_oss.layers", GptOssAttention
+ *     (sinks, sliding_window, softmax_scale = head_dim ** -0.5,
+ *     num_attention_heads, num_key_value_heads, _has_thd_metadata);
+ *     Transformers v4.55.0 release notes, "Architecture".
+ *
+ * Definitions used by every entry point (token i of a sequence, q-head h,
+ * kv-head g = h / (Hq / Hkv)):
+ *   theta(p, j) = p * inv_freq[j], j in [0, D/2), inv_freq from YaRN;
+ *   x'[j]       = c * (x[j] cos theta - x[j+D/2] sin theta)
+ *   x'[j+D/2]   = c * (x[j+D/2] cos theta + x[j] sin theta),  c = concentration;
+ *   s_ij  = softmax_scale * <q'_i[h], k'_j[g]>;
+ *   key j visible from query i iff j <= i (token order inside the sequence)
+ *         and (window == 0 or i - j < window);
+ *   M_i   = max(sink_h, max_visible s_ij);
+ *   Z_i   = exp(sink_h - M_i) + sum_visible exp(s_ij - M_i);
+ *   out_i = sum_visible exp(s_ij - M_i) v_j[g] / Z_i;   lse_i = M_i + ln Z_i.
+ * sink_h = -inf gives standard softmax attention.  Positions feed RoPE only.
+ *
+ * Conventions:
+ *   - Every tensor pointer is caller-owned DEVICE memory.  The library
+ *     allocates nothing; its only state is the wait limit below.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronises.
+ *   - Arguments are validated on the host before any launch; a failed check
+ *     returns GPTOSS_ERR_INVALID_ARG or GPTOSS_ERR_UNSUPPORTED and launches
+ *     nothing.  A failed launch returns GPTOSS_ERR_CUDA.
+ *   - Device-side conditions (a bounded pipeline wait that gave up) are
+ *     recorded in a device status word read by gptoss_read_device_status.
+ *   - bf16 tensors are IEEE bfloat16; head_dim D must be 64 and contiguous
+ *     (element stride 1); rotary_dim must equal D.
+ *   - No C++ exception crosses this ABI.
+ */
+#ifndef GPTOSS_H_
+#define GPTOSS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t == struct CUstream_st* */
+
+typedef enum gptoss_status {
+  GPTOSS_OK = 0,
+  GPTOSS_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad stride or alignment */
+  GPTOSS_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (D != 64, ...) */
+  GPTOSS_ERR_CUDA = 3,        /* a CUDA runtime call or a kernel launch failed */
+  GPTOSS_ERR_TIMEOUT = 4      /* a device-side bounded wait gave up (device status word) */
+} gptoss_status;
+
+/* YaRN parameters, as RotaryEmbedding on the rope_utils page names them.
+ * factor <= 1 means plain RoPE (inv_freq = base^(-2j/rotary_dim), c = 1).
+ * Otherwise c = 0.1 ln(factor) + 1 and pair j is kept (j <= d_lo), divided by
+ * factor (j >= d_hi) or blended linearly in j between the two correction
+ * dimensions d_lo / d_hi at which a pair makes ntk_beta / ntk_alpha turns
+ * over initial_context tokens. */
+typedef struct gptoss_rope_params {
+  double base;             /* 150000 for GPT-OSS */
+  double factor;           /* scaling_factor, 32 for GPT-OSS */
+  int32_t initial_context; /* initial_context_length, 4096 */
+  int32_t rotary_dim;      /* int(head_dim * partial_rotary_factor); must equal D */
+  double ntk_alpha;        /* 1 */
+  double ntk_beta;         /* 32 */
+} gptoss_rope_params;
+
+/* Strides in ELEMENTS.  BSHD element (b, s, h, d) sits at
+ * b*batch + s*tok + h*head + d; packed THD element (t, h, d) at
+ * t*tok + h*head + d (batch ignored).  tok and head must be multiples of 8
+ * (16 bytes) and every base pointer 16-byte aligned. */
+typedef struct gptoss_strides {
+  int64_t batch;
+  int64_t tok;
+  int64_t head;
+} gptoss_strides;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gptoss_status_string(gptoss_status status);
+
+/* gptoss_rope_qk -- YaRN RoPE of q and k, out of place (in place when an
+ * output aliases its input with the same strides).
+ *   q      [B,S,Hq,D] (BSHD) or [T,Hq,D] (THD) bf16, strides sq; k likewise
+ *          with Hkv heads, strides sk.
+ *   q_out, k_out: bf16, same logical shapes, own strides (k_out may point
+ *          into a KV cache slot: that is the cache-append use).
+ *   positions  int32 [B*S] (row-major over b, s) or [T]; NULL -> 0..S-1 per
+ *          batch row (BSHD) or restarting at 0 for every sequence (THD).
+ *   cu_seqlens int32 [nseq+1], nondecreasing, cu_seqlens[0] = 0,
+ *          cu_seqlens[nseq] = T; NULL -> BSHD.  With cu_seqlens, B = nseq and
+ *          S_or_T = T; otherwise S_or_T = S.
+ *   Angles are reduced in double precision and rotated in fp32; outputs are
+ *   rounded to bf16. */
+gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
+                             void* q_out, gptoss_strides sq_out, void* k_out, gptoss_strides sk_out,
+                             const int32_t* positions, const int32_t* cu_seqlens, int32_t B,
+                             int32_t S_or_T, int32_t Hq, int32_t Hkv, int32_t D,
+                             const gptoss_rope_params* rope, struct CUstream_st* stream);
+
+/* gptoss_attn_fwd -- prefill sink attention, causal, full (window = 0) or
+ * sliding window, BSHD or packed THD.
+ *   q [B,S,Hq,D] / [T,Hq,D], k and v [B,S,Hkv,D] / [T,Hkv,D], bf16, own
+ *          strides.  rope != NULL: q and k are raw and RoPE is applied inside
+ *          the kernel as the tiles are loaded; rope == NULL: q and k are
+ *          already rotated.
+ *   sinks  fp32 [Hq], in the units of the scaled logits (may be -inf).
+ *   positions / cu_seqlens as for gptoss_rope_qk (positions only used when
+ *          rope != NULL).
+ *   B      batch (BSHD) or number of sequences (THD).
+ *   S      sequence length (BSHD) or the longest sequence (THD, upper bound).
+ *   total_tokens  B*S (BSHD) or T (THD).
+ *   window 0 = full causal; w > 0 = the last w keys including the query.
+ *   softmax_scale  head_dim^-0.5 for GPT-OSS.
+ *   out    bf16, q's logical shape, strides so.
+ *   lse    fp32, nullable: [B,Hq,S] (BSHD) or [Hq,T] (THD), natural log. */
+gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
+                              const void* v, gptoss_strides sv, const float* sinks,
+                              const int32_t* positions, const int32_t* cu_seqlens, int32_t B,
+                              int32_t S, int32_t total_tokens, int32_t Hq, int32_t Hkv, int32_t D,
+                              int32_t window, float softmax_scale, const gptoss_rope_params* rope,
+                              void* out, gptoss_strides so, float* lse, struct CUstream_st* stream);
+
+/* Workspace bytes gptoss_attn_decode needs for these sizes (split-KV
+ * partial results).  0 when a size is out of range. */
+size_t gptoss_attn_decode_workspace_size(int32_t B, int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D);
+
+/* gptoss_attn_decode -- one new query token per sequence against a bf16 KV
+ * cache, split over the cache length, merged with the sink folded once.
+ *   q        [B,Hq,D] bf16 contiguous, raw: rotated here at position
+ *            cache_seqlens[b]-1 when rope != NULL.
+ *   k_cache, v_cache [B,Lmax,Hkv,D] bf16 contiguous; k_cache holds keys
+ *            already rotated, v_cache raw values; the new token's k/v are
+ *            already in slot cache_seqlens[b]-1.
+ *   cache_seqlens int32 [B], 1 <= len <= Lmax (device memory).
+ *   The query sees slots [len-window, len) (all of [0, len) when window = 0).
+ *   out      [B,Hq,D] bf16 contiguous; lse fp32 [B,Hq], nullable.
+ *   workspace  device memory of at least
+ *            gptoss_attn_decode_workspace_size(...) bytes, 16-byte aligned,
+ *            owned by the caller; contents need not be initialised. */
+gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* cache_seqlens, const float* sinks, int32_t B,
+                                 int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D, int32_t window,
+                                 float softmax_scale, const gptoss_rope_params* rope, void* out,
+                                 float* lse, void* workspace, size_t workspace_bytes,
+                                 struct CUstream_st* stream);
+
+/* Reads (and, if reset != 0, clears) the device status word of the current
+ * device: GPTOSS_OK or GPTOSS_ERR_TIMEOUT.  Synchronises `stream`. */
+gptoss_status gptoss_read_device_status(int32_t* status_out, int32_t reset, struct CUstream_st* stream);
+
+/* Time limit, in microseconds, of every device-side pipeline wait of later
+ * launches from this process (0 = the built-in default of 2 s).  A wait that
+ * exceeds it records GPTOSS_ERR_TIMEOUT in the device status word and the
+ * kernel winds down: it drains its own copies in flight, waits for its own
+ * tensor-core work and frees its tensor memory before returning.  This limit
+ * is the only state the library keeps between calls. */
+gptoss_status gptoss_set_wait_limit(uint32_t microseconds);
+
+/* Failure-path self test: launches one warp that waits, with the given limit
+ * (1..1000000 us), on a barrier nothing ever arrives at.  The wait gives up,
+ * records GPTOSS_ERR_TIMEOUT in the device status word and writes 0 to
+ * *result_dev (1 would mean the wait was satisfied).  No fault, no trap. */
+gptoss_status gptoss_selftest_wait_timeout(uint32_t limit_us, int32_t* result_dev, struct CUstream_st* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTOSS_H_ */

@@ -1,0 +1,51 @@
+"""Shared helpers of the GPU parity tests: upload seeded inputs, compare a
+kernel's output with the float64 oracle.
+
+Tolerance (stated for bf16 inputs with fp32 accumulation and outputs of unit
+scale): max-abs error <= 1e-2 and mean-abs error <= 1e-3 on every compared
+element.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from attention_yarn_rope_b200.workloads import to_torch_bf16
+
+MAX_ABS = 1e-2
+MEAN_ABS = 1e-3
+
+
+def dev(x, device="cuda:0"):
+    return to_torch_bf16(x, device)
+
+
+def f32(x: np.ndarray, device="cuda:0"):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(device)
+
+
+def i32(x, device="cuda:0"):
+    return torch.as_tensor(np.asarray(x, np.int32), device=device)
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_parity(got: np.ndarray, ref: np.ndarray, what: str, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = np.abs(got - ref)
+    mx, mean = float(err.max()), float(err.mean())
+    assert mx <= max_abs, f"{what}: max-abs {mx:.3e} > {max_abs} (mean {mean:.3e})"
+    assert mean <= mean_abs, f"{what}: mean-abs {mean:.3e} > {mean_abs}"
+    return mx, mean
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |x| (8 significand bits)."""
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(ax)) - 7)

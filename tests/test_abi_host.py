@@ -1,0 +1,142 @@
+"""Host-side checks of the C ABI (CPU only, no kernel launches).
+
+* the in-tree library loads and exports every function include/gptoss.h declares;
+* argument validation rejects bad calls before touching the GPU (each case
+  returns before any CUDA runtime call, so it runs on a machine without one);
+* the decode workspace size is consistent.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_yarn_rope_b200 import _abi, build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return _abi.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "gptoss.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptoss_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 8
+    assert sorted(_abi.EXPORTED) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code, name in _abi.STATUS_NAMES.items():
+        assert lib.gptoss_status_string(code).decode() == name
+    assert lib.gptoss_status_string(99).decode() == "GPTOSS_ERR_UNKNOWN"
+
+
+ROPE = _abi.RopeParams(150000.0, 32.0, 4096, 64, 1.0, 32.0)
+S_BSHD_Q = _abi.Strides(4096 * 64 * 64, 64 * 64, 64)
+S_BSHD_K = _abi.Strides(4096 * 8 * 64, 8 * 64, 64)
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case fails validation first
+
+
+def _fwd(lib, **kw):
+    a = dict(q=FAKE, sq=S_BSHD_Q, k=FAKE, sk=S_BSHD_K, v=FAKE, sv=S_BSHD_K, sinks=FAKE, pos=None, cu=None, B=1,
+             S=4096, T=4096, Hq=64, Hkv=8, D=64, window=0, scale=0.125, rope=ctypes.byref(ROPE), out=FAKE,
+             so=S_BSHD_Q, lse=None)
+    a.update(kw)
+    return lib.gptoss_attn_fwd(a["q"], a["sq"], a["k"], a["sk"], a["v"], a["sv"], a["sinks"], a["pos"], a["cu"],
+                               a["B"], a["S"], a["T"], a["Hq"], a["Hkv"], a["D"], a["window"], a["scale"],
+                               a["rope"], a["out"], a["so"], a["lse"], None)
+
+
+def test_attn_fwd_validation(lib):
+    assert _fwd(lib, D=128) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert _fwd(lib, Hkv=7) == _abi.GPTOSS_ERR_INVALID_ARG          # Hq % Hkv != 0
+    assert _fwd(lib, window=-1) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert _fwd(lib, scale=0.0) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan")) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert _fwd(lib, T=4095) == _abi.GPTOSS_ERR_INVALID_ARG          # B*S != total for BSHD
+    assert _fwd(lib, q=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert _fwd(lib, sinks=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert _fwd(lib, q=ctypes.c_void_p(0x10008)) == _abi.GPTOSS_ERR_INVALID_ARG  # not 16-byte aligned
+    assert _fwd(lib, sq=_abi.Strides(0, 4097, 64)) == _abi.GPTOSS_ERR_INVALID_ARG  # stride not 16 B multiple
+    bad_rope = _abi.RopeParams(150000.0, 32.0, 4096, 32, 1.0, 32.0)
+    assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_UNSUPPORTED  # partial rotary
+    bad_rope = _abi.RopeParams(150000.0, 32.0, 4096, 64, 32.0, 1.0)
+    assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_INVALID_ARG  # alpha >= beta
+    # empty inputs are a successful no-op (nothing launched)
+    assert _fwd(lib, B=0, T=0) == _abi.GPTOSS_OK
+    assert _fwd(lib, S=0, T=0) == _abi.GPTOSS_OK
+
+
+def test_rope_qk_validation(lib):
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, qo=FAKE, ko=FAKE, B=1, S=16, Hq=64, Hkv=8, D=64, rope=ctypes.byref(ROPE))
+        a.update(kw)
+        return lib.gptoss_rope_qk(a["q"], S_BSHD_Q, a["k"], S_BSHD_K, a["qo"], S_BSHD_Q, a["ko"], S_BSHD_K, None,
+                                  None, a["B"], a["S"], a["Hq"], a["Hkv"], a["D"], a["rope"], None)
+
+    assert call(rope=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(D=32) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert call(ko=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(B=-1) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(B=0) == _abi.GPTOSS_OK
+    assert call(S=0) == _abi.GPTOSS_OK
+
+
+def test_decode_validation_and_workspace(lib):
+    ws = lib.gptoss_attn_decode_workspace_size(64, 32768, 64, 8, 64)
+    assert ws > 0 and ws % 16 == 0
+    assert lib.gptoss_attn_decode_workspace_size(64, 32768, 64, 8, 128) == 0
+    assert lib.gptoss_attn_decode_workspace_size(1, 32768, 64, 7, 64) == 0
+
+    def call(**kw):
+        a = dict(B=64, L=32768, Hq=64, Hkv=8, D=64, window=0, ws=FAKE, wsb=ws, seq=FAKE)
+        a.update(kw)
+        return lib.gptoss_attn_decode(FAKE, FAKE, FAKE, a["seq"], FAKE, a["B"], a["L"], a["Hq"], a["Hkv"], a["D"],
+                                      a["window"], 0.125, ctypes.byref(ROPE), FAKE, None, a["ws"], a["wsb"], None)
+
+    assert call(wsb=ws - 16) == _abi.GPTOSS_ERR_INVALID_ARG   # workspace too small
+    assert call(ws=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(seq=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(Hq=64, Hkv=2) == _abi.GPTOSS_ERR_UNSUPPORTED   # 32 query heads per group
+    assert call(D=96) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert call(window=-5) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(B=0) == _abi.GPTOSS_OK
+
+
+def test_wait_limit_setter(lib):
+    assert lib.gptoss_set_wait_limit(1000) == _abi.GPTOSS_OK
+    assert lib.gptoss_set_wait_limit(0) == _abi.GPTOSS_OK  # back to the default
+    assert lib.gptoss_selftest_wait_timeout(0, FAKE, None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert lib.gptoss_selftest_wait_timeout(10, None, None) == _abi.GPTOSS_ERR_INVALID_ARG
+
+
+def test_product_path_never_imports_oracle():
+    pkg = os.path.join(ROOT, "attention_yarn_rope_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+
+
+def test_oracle_is_independent_of_the_cuda_path():
+    odir = os.path.join(ROOT, "oracle")
+    for f in os.listdir(odir):
+        if f.endswith(".py"):
+            txt = open(os.path.join(odir, f)).read()
+            for line in txt.splitlines():
+                if line.startswith(("import ", "from ")):
+                    mod = line.split()[1]
+                    assert mod.split(".")[0] in {"numpy", "math", "cmath", "__future__", ""} or mod.startswith("."), (f, line)
