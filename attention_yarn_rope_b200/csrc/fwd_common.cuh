@@ -1,0 +1,130 @@
+// fwd_common.cuh -- shared definitions of the prefill kernel (gptoss_attn_fwd).
+//
+// Rule: GptOssAttention on the NeMo AutoModel gpt_oss.layers page (sinks,
+// sliding_window, softmax_scale = head_dim^-0.5, grouped query heads), RoPE of
+// the gpt_oss.rope_utils page, sink in the denominator only (Transformers
+// v4.55.0 release notes, "Architecture").
+//
+// Design: persistent CTAs (one per SM), each walking a static, heaviest-first
+// list of work units.  A unit is one 128-query tile of TWO query heads that
+// share a kv head, so every K/V tile is loaded and rotated once for 256 query
+// rows.  16 warps (roles in fwd_softmax.cuh, fwd_rope.cuh, fwd_pipeline.cuh):
+//   warps 0-3 / 4-7   softmax of head A / head B (thread = query row = TMEM lane)
+//   warps 8-11        rope: next unit's Q tiles, every K tile in place
+//   warp 12           TMA producer (K, V tiles into a 4-stage ring)
+//   warp 13           TMEM allocation and tcgen05.mma issue
+//   warps 14-15       idle (complete the register split)
+// setmaxnreg moves registers from the rope / producer / MMA warpgroups to the
+// two softmax warpgroups: launch 512 threads x 128 registers = 65536, split
+// 2 x 128 x 192 + 128 x 88 + 128 x 40 = 65536.  The host refuses to launch if
+// the compiled kernel does not start at exactly 128 registers per thread.
+// TMEM columns (all 512): S_A [0,128) P_A [128,192) O_A [192,256),
+//                         S_B [256,384) P_B [384,448) O_B [448,512).
+#pragma once
+
+#include "host_util.cuh"
+#include "rope_qk.cuh"
+#include "sm100_ptx.cuh"
+
+namespace gptoss {
+
+constexpr int kFwdTile = 128;         // query rows and keys per tile
+constexpr int kFwdStages = 4;
+constexpr int kFwdThreads = 512;
+constexpr int kFwdLaunchRegs = 128;   // 65536 / 512
+constexpr int kFwdTileBytes = kFwdTile * kHeadDim * 2;  // 16 KB
+constexpr uint32_t kFwdTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kRegsSoftmax = 192, kRegsRope = 88, kRegsOther = 40;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsRope + 128 * kRegsOther == kFwdThreads * kFwdLaunchRegs,
+              "register split must add up to the launch allocation");
+
+struct FwdParams {
+  CUtensorMap tmap_k;  // dims (64, Hkv, S or T, B or 1), box (64, 1, 128, 1)
+  CUtensorMap tmap_v;
+  const __nv_bfloat16* q;
+  gptoss_strides sq;
+  __nv_bfloat16* out;
+  gptoss_strides so;
+  float* lse;
+  const float* sinks;
+  const int32_t* positions;
+  const int32_t* cu_seqlens;
+  int B, S, T, Hq, Hkv, G, HP, window, n_qtiles, n_units;
+  float scale_log2;
+  uint64_t wait_ns;
+  RopeTable tab;
+};
+
+struct __align__(1024) FwdSmem {
+  uint8_t q[2][2][kFwdTileBytes];  // [buffer][head A/B], rotated, 128B-swizzled
+  uint8_t k[kFwdStages][kFwdTileBytes];
+  uint8_t v[kFwdStages][kFwdTileBytes];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[kFwdStages], k_ready[kFwdStages], k_empty[kFwdStages];
+  uint64_t v_full[kFwdStages], v_empty[kFwdStages];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];  // per head slot A/B
+  uint64_t mma_final;
+  uint32_t tmem_base;
+};
+
+// One work unit: query tile q0 / 128 of heads (h0, h1) of sequence b.
+struct Unit {
+  int b, h0, h1, g, q0, L, seq_start, j_lo, n_kt;
+  bool dup;  // h1 repeats h0 (odd group size): computed, not stored
+};
+
+// Unit u of the static list (heaviest query tiles first).  Returns false for
+// a tile past the end of its packed sequence; every role skips the same units.
+__device__ __forceinline__ bool make_unit(const FwdParams& p, int u, Unit& w) {
+  const int per_tile = p.B * p.Hkv * p.HP;
+  const int qt = p.n_qtiles - 1 - u / per_tile;
+  int rest = u % per_tile;
+  const int hp = rest % p.HP;
+  rest /= p.HP;
+  w.g = rest % p.Hkv;
+  w.b = rest / p.Hkv;
+  w.h0 = w.g * p.G + 2 * hp;
+  w.dup = (2 * hp + 1) >= p.G;
+  w.h1 = w.dup ? w.h0 : w.h0 + 1;
+  const bool thd = p.cu_seqlens != nullptr;
+  w.seq_start = thd ? __ldg(p.cu_seqlens + w.b) : 0;
+  w.L = thd ? __ldg(p.cu_seqlens + w.b + 1) - w.seq_start : p.S;
+  w.q0 = qt * kFwdTile;
+  if (w.q0 >= w.L) return false;
+  const int q_last = min(w.q0 + kFwdTile, w.L) - 1;
+  const int j_hi = q_last / kFwdTile;
+  w.j_lo = p.window > 0 ? max(0, w.q0 - p.window + 1) / kFwdTile : 0;
+  w.n_kt = j_hi - w.j_lo + 1;
+  return true;
+}
+
+// Byte offset of the 32-bit word holding features (e, e+1) of row r in a
+// 128B-swizzled 128 x 64 bf16 tile (e even).
+__device__ __forceinline__ uint32_t sw128_word(int r, int e) {
+  return r * 128 + ((((e >> 3) ^ (r & 7))) << 4) + (e & 7) * 2;
+}
+
+// Rotates the two pairs held in words (lo, hi) = features (e, e+1), (e+32, e+33).
+__device__ __forceinline__ void rotate_words(uint32_t& lo, uint32_t& hi, float2 a, float2 b) {
+  const float x0 = bf16lo(lo), x1 = bf16hi(lo);
+  const float y0 = bf16lo(hi), y1 = bf16hi(hi);
+  lo = pack_bf16(x0 * a.x - y0 * a.y, x1 * b.x - y1 * b.y);
+  hi = pack_bf16(y0 * a.x + x0 * a.y, y1 * b.x + x1 * b.y);
+}
+
+// (c, s) * (cos d, sin d): advances an angle seed by a fixed step.
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+  return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+}  // namespace gptoss

@@ -1,0 +1,160 @@
+// fwd_softmax.cuh -- softmax warpgroups of the prefill kernel.
+//
+// Thread r of warpgroup X owns query row r of head slot X (TMEM lane r).  Per
+// key tile: read S from TMEM and release the S buffer at once (the next
+// QK^T overlaps the exponentials); classify each 32-key chunk for this warp
+// as hidden (skipped: its P is zero), partly visible (masked per element) or
+// fully visible; online softmax in log2 units where the sink is the initial
+// running max and its exp the initial running sum (sink = -inf starts from
+// an empty sum); P in bf16 into TMEM, one half at a time; O rescaled in TMEM
+// only when the running max grows by more than 2^8.  Epilogue: O / l in bf16
+// and LSE = (m + log2 l) ln 2.
+#pragma once
+
+#include "fwd_common.cuh"
+
+namespace gptoss {
+
+__device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem, int X) {
+  const int wq = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quarter
+  const int r = threadIdx.x & 127;        // query row of the tile
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const uint32_t colS = X * 256, colP = X * 256 + 128, colO = X * 256 + 192;
+  const bool thd = p.cu_seqlens != nullptr;
+  uint32_t t = 0;  // running tile count of this CTA
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    Unit w;
+    if (!make_unit(p, u, w)) continue;
+    const int h = X == 0 ? w.h0 : w.h1;
+    const int qi = w.q0 + r;
+    const int qw_lo = w.q0 + wq * 32, qw_hi = qw_lo + 31;  // rows of this warp
+    const float sink = __ldg(p.sinks + h) * kLog2e;
+    float m_run = sink;
+    float l_run = sink == -INFINITY ? 0.f : 1.f;
+    for (int j = 0; j < w.n_kt; ++j, ++t) {
+      const int k0 = (w.j_lo + j) * kFwdTile;
+      if (!mbar_wait_warp(&sm.s_full[X], t & 1, p.wait_ns)) return;
+      tc_fence_after();
+      // chunk classes for this warp: 0 hidden, 1 partly visible, 2 visible
+      int cls[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int kl = k0 + 32 * c, kh = kl + 31;
+        const bool hidden = kl > min(qw_hi, w.L - 1) || (p.window > 0 && kh < qw_lo - p.window + 1);
+        const bool full = kh <= qw_lo && kh <= w.L - 1 && (p.window == 0 || kl >= qw_hi - p.window + 1);
+        cls[c] = hidden ? 0 : (full ? 2 : 1);
+      }
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + colS + c * 32, sr[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[X]);
+      const int c_hi = min(qi, w.L - 1) - k0;  // visible columns of this row: [c_lo, c_hi]
+      const int c_lo = p.window > 0 ? qi - p.window + 1 - k0 : -1;
+      // mask only tiles that cross an edge for this warp (whole-tile, warp-uniform)
+      const bool edge = cls[0] != 2 || cls[1] != 2 || cls[2] != 2 || cls[3] != 2;
+      if (edge) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = c * 32 + e;
+            const float x = (col <= c_hi && col >= c_lo) ? __uint_as_float(sr[c][e]) : -INFINITY;
+            sr[c][e] = __float_as_uint(x);
+          }
+      }
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mt = fmaxf(mt, __uint_as_float(sr[c][e]));
+      const float m_cand = mt * p.scale_log2;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m_cand > m_run + kRescaleThreshold) {
+        alpha = ex2_approx(m_run - m_cand);  // 0 when m_run is -inf
+        m_run = m_cand;
+        rescale = true;
+      }
+      const float base = m_run == -INFINITY ? 0.f : m_run;
+      float rs = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
+          if (cls[c] == 0) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[cc * 16 + e] = 0u;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), p.scale_log2, -base));
+              const float x1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), p.scale_log2, -base));
+              rs += x0 + x1;
+              pk[cc * 16 + e] = pack_bf16(x0, x1);
+            }
+          }
+        }
+        if (half == 0) {
+          // P(t) overwrites P(t-1): the previous P V product must have completed
+          if (t > 0) {
+            if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
+            tc_fence_after();
+          }
+          if (rescale && j > 0) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t ov[32];
+              tmem_ld32(lane_base + colO + c * 32, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              tmem_st32(lane_base + colO + c * 32, ov);
+            }
+          }
+        }
+        tmem_st32(lane_base + colP + half * 32, pk);
+      }
+      l_run = l_run * alpha + rs;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[X]);
+    }
+    // ---- epilogue: O / l, LSE ----
+    if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
+    tc_fence_after();
+    uint32_t ov[2][32];
+    tmem_ld32(lane_base + colO, ov[0]);
+    tmem_ld32(lane_base + colO + 32, ov[1]);
+    tmem_wait_ld();
+    tc_fence_before();
+    if (qi < w.L && !(X == 1 && w.dup)) {
+      const float inv = 1.f / l_run;
+      const int64_t row = thd ? static_cast<int64_t>(w.seq_start + qi) * p.so.tok
+                              : static_cast<int64_t>(w.b) * p.so.batch + static_cast<int64_t>(qi) * p.so.tok;
+      __nv_bfloat16* dst = p.out + row + static_cast<int64_t>(h) * p.so.head;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint4 v;
+        const int c = c8 >> 2, e = (c8 & 3) * 8;
+        v.x = pack_bf16(__uint_as_float(ov[c][e + 0]) * inv, __uint_as_float(ov[c][e + 1]) * inv);
+        v.y = pack_bf16(__uint_as_float(ov[c][e + 2]) * inv, __uint_as_float(ov[c][e + 3]) * inv);
+        v.z = pack_bf16(__uint_as_float(ov[c][e + 4]) * inv, __uint_as_float(ov[c][e + 5]) * inv);
+        v.w = pack_bf16(__uint_as_float(ov[c][e + 6]) * inv, __uint_as_float(ov[c][e + 7]) * inv);
+        *reinterpret_cast<uint4*>(dst + c8 * 8) = v;
+      }
+      if (p.lse != nullptr) {
+        const float lse = (m_run + log2f(l_run)) * kLn2;
+        if (thd)
+          p.lse[static_cast<int64_t>(h) * p.T + w.seq_start + qi] = lse;
+        else
+          p.lse[(static_cast<int64_t>(w.b) * p.Hq + h) * p.S + qi] = lse;
+      }
+    }
+  }
+}
+
+}  // namespace gptoss

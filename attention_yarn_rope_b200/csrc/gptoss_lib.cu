@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 
 #include "attn_decode.cuh"
-#include "attn_fwd.cuh"
+#include "fwd_pipeline.cuh"
 #include "gptoss.h"
 #include "host_util.cuh"
 #include "rope_qk.cuh"
@@ -131,8 +131,24 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   if (!strides_ok(sq, !thd) || !strides_ok(sk, !thd) || !strides_ok(sv, !thd) || !strides_ok(so, !thd))
     return GPTOSS_ERR_INVALID_ARG;
   const int n_qtiles = (S + kFwdTile - 1) / kFwdTile;
-  const int64_t grid = static_cast<int64_t>(n_qtiles) * Hq * B;
-  if (grid > INT32_MAX) return GPTOSS_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  const int HP = (G + 1) / 2;  // head pairs per kv group
+  const int64_t n_units = static_cast<int64_t>(n_qtiles) * B * Hkv * HP;
+  if (n_units > INT32_MAX) return GPTOSS_ERR_UNSUPPORTED;
+  // The register split inside the kernel assumes exactly kFwdLaunchRegs
+  // registers per thread at launch; anything else could stall the split.
+  static int launch_regs = -1;
+  if (launch_regs < 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel) != cudaSuccess) return GPTOSS_ERR_CUDA;
+    launch_regs = fa.numRegs;
+  }
+  if (launch_regs != kFwdLaunchRegs) return GPTOSS_ERR_UNSUPPORTED;
+  int device = 0, n_sm = 0;
+  if (cudaGetDevice(&device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return GPTOSS_ERR_CUDA;
+  const int grid = static_cast<int>(n_units < n_sm ? n_units : n_sm);
 
   FwdParams p;
   memset(&p, 0, sizeof(p));
@@ -159,9 +175,11 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   p.T = total_tokens;
   p.Hq = Hq;
   p.Hkv = Hkv;
-  p.G = Hq / Hkv;
+  p.G = G;
+  p.HP = HP;
   p.window = window;
   p.n_qtiles = n_qtiles;
+  p.n_units = static_cast<int>(n_units);
   p.scale_log2 = softmax_scale * kLog2e;
   p.wait_ns = wait_limit_ns();
   if (rope != nullptr) yarn_table(*rope, &p.tab);
@@ -170,7 +188,7 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return GPTOSS_ERR_CUDA;
-  attn_fwd_kernel<<<static_cast<int>(grid), kFwdThreads, smem, as_stream(stream)>>>(p);
+  attn_fwd_kernel<<<grid, kFwdThreads, smem, as_stream(stream)>>>(p);
   return check_launch();
 }
 

@@ -137,6 +137,20 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # timing helpers
 # ----------------------------------------------------------------------------
+def aggregate_ranks(torch, dist, device, ms_local, work_local):
+    """Whole-job view of one timed region: the time is the max over ranks
+    (every rank waited at a barrier before and after it), the work the sum.
+    Single process: returned unchanged."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(ms_local), float(work_local)
+    dist.barrier()
+    t = torch.tensor([float(ms_local)], dtype=torch.float64, device=device)
+    w = torch.tensor([float(work_local)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(w, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(w.item())
+
+
 def timed_steps(torch, fn, steps, stream, flush=None):
     """Device time (ms) of `steps` calls of fn on `stream`, CUDA events on that
     stream; with `flush`, L2 is overwritten between calls (outside the timing)."""
@@ -236,14 +250,10 @@ def run_ours(args, torch, dist, rank, world, device):
     ms = timed_steps(torch, case["step"], args.steps, stream)
     torch.cuda.synchronize()
     t_hi = time.time()
-    if world > 1:
-        dist.barrier()
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, job_flops = aggregate_ranks(torch, dist, device, ms, case["flops"] * args.steps)
     clocks = clk.stop(t_lo, t_hi)
     per_step_ms = ms / args.steps
-    value = case["flops"] * world / (per_step_ms * 1e-3) / 1e12
+    value = job_flops / (ms * 1e-3) / 1e12
 
     # ---- end to end through the public API, host buffers, copies inside ----
     h_q = case["q"].cpu().pin_memory()
@@ -268,11 +278,8 @@ def run_ours(args, torch, dist, rank, world, device):
     if world > 1:
         dist.barrier()
     ems = timed_steps(torch, e2e_step, e2e_steps, stream)
-    if world > 1:
-        t = torch.tensor([ems], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e_value = case["flops"] * world / (ems / e2e_steps * 1e-3) / 1e12
+    ems, e2e_flops = aggregate_ranks(torch, dist, device, ems, case["flops"] * e2e_steps)
+    e2e_value = e2e_flops / (ems * 1e-3) / 1e12
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_s))
     d2h = h_o.numel() * h_o.element_size()
 
@@ -460,6 +467,33 @@ def run_reference(args):
     }
 
 
+def profile_case(args):
+    """Launch one workload's kernel(s) warmup + steps times and exit (a small,
+    self-contained target for ncu captures)."""
+    import dataclasses
+
+    import torch
+
+    from attention_yarn_rope_b200 import ops
+    from attention_yarn_rope_b200 import workloads as wl
+
+    cfgs = {c.name: c for c in wl.PREFILL_CONFIGS + wl.DECODE_CONFIGS}
+    cfg = cfgs[args.profile_case]
+    if args.profile_batch is not None:
+        cfg = dataclasses.replace(cfg, B=args.profile_batch)
+    device = "cuda:0"
+    if isinstance(cfg, wl.DecodeConfig):
+        case = decode_case(torch, ops, cfg, device)
+    else:
+        case = prefill_case(torch, ops, cfg, device)
+    for _ in range(args.warmup + args.steps):
+        case["step"]()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": cfg.name, "B": cfg.B, "launches": args.warmup + args.steps,
+                      "bytes_per_launch": case["bytes"], "flops_per_launch": case["flops"]}))
+    return 0
+
+
 # ----------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
@@ -470,7 +504,13 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the per-config measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile-case", default=None,
+                    help="only launch this workload's kernel warmup+steps times (for ncu), e.g. "
+                         "sliding_b4_s4096_w128, full_b2_s8192, decode_b64_l32768_full; no timing")
+    ap.add_argument("--profile-batch", type=int, default=None, help="smaller batch for --profile-case")
     args = ap.parse_args()
+    if args.profile_case:
+        return profile_case(args)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
 
