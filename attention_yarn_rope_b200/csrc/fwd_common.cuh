@@ -35,6 +35,12 @@ constexpr int kFwdLaunchRegs = 128;   // 65536 / 512
 constexpr int kFwdTileBytes = kFwdTile * kHeadDim * 2;  // 16 KB
 constexpr uint32_t kFwdTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Which of the 16 column pairs of every 32-key chunk take 2^x from the FMA-pipe
+// polynomial (bit e set) instead of the MUFU unit; balances the two pipes.
+#ifndef GPTOSS_POLY_MASK
+#define GPTOSS_POLY_MASK 0x0000u
+#endif
+constexpr uint32_t kPolyMask = GPTOSS_POLY_MASK;
 constexpr uint32_t kRegsSoftmax = 192, kRegsRope = 88, kRegsOther = 40;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsRope + 128 * kRegsOther == kFwdThreads * kFwdLaunchRegs,
               "register split must add up to the launch allocation");

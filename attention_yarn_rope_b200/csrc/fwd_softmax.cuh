@@ -64,11 +64,15 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
             sr[c][e] = __float_as_uint(x);
           }
       }
-      float mt = -INFINITY;
+      float mc[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
+        mc[c] = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mt = fmaxf(mt, __uint_as_float(sr[c][e]));
+        for (int e = 0; e < 32; e += 2)
+          mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+      }
+      const float mt = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
       const float m_cand = mt * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
@@ -78,7 +82,9 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
         rescale = true;
       }
       const float base = m_run == -INFINITY ? 0.f : m_run;
-      float rs = 0.f;
+      const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nb2 = make_float2(-base, -base);
+      float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -91,10 +97,17 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float x0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), p.scale_log2, -base));
-              const float x1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), p.scale_log2, -base));
-              rs += x0 + x1;
-              pk[cc * 16 + e] = pack_bf16(x0, x1);
+              const float2 s2 = make_float2(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1]));
+              const float2 x2 = ffma2(s2, sl2, nb2);
+              float2 p2;
+              if ((kPolyMask >> e) & 1u) {
+                p2 = exp2_poly2(x2);
+              } else {
+                p2.x = ex2_approx(x2.x);
+                p2.y = ex2_approx(x2.y);
+              }
+              rs2 = fadd2(rs2, p2);
+              pk[cc * 16 + e] = pack_bf16(p2.x, p2.y);
             }
           }
         }
@@ -104,7 +117,9 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
             if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
             tc_fence_after();
           }
-          if (rescale && j > 0) {
+          // warp-collective TMEM access: the whole warp rescales when any row
+          // needs it (alpha is 1 for the rows that do not)
+          if (__any_sync(0xffffffffu, rescale && j > 0)) {
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
               uint32_t ov[32];
@@ -118,7 +133,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
         }
         tmem_st32(lane_base + colP + half * 32, pk);
       }
-      l_run = l_run * alpha + rs;
+      l_run = l_run * alpha + (rs2.x + rs2.y);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[X]);
