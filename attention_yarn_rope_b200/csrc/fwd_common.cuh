@@ -111,12 +111,16 @@ __device__ __forceinline__ uint32_t sw128_word(int r, int e) {
   return r * 128 + ((((e >> 3) ^ (r & 7))) << 4) + (e & 7) * 2;
 }
 
-// Rotates the two pairs held in words (lo, hi) = features (e, e+1), (e+32, e+33).
+// Rotates the two pairs held in bf16 words (lo, hi) = features (e, e+1),
+// (e+32, e+33) and returns them as fp16: the rotated q / k feed the QK^T
+// product in fp16, whose 11-bit significand leaves eight times less rounding
+// in the concentration-scaled logits than bf16 would (the rotated values must
+// stay inside the fp16 range, |x| < 65504; GPT-OSS activations are O(10)).
 __device__ __forceinline__ void rotate_words(uint32_t& lo, uint32_t& hi, float2 a, float2 b) {
   const float x0 = bf16lo(lo), x1 = bf16hi(lo);
   const float y0 = bf16lo(hi), y1 = bf16hi(hi);
-  lo = pack_bf16(x0 * a.x - y0 * a.y, x1 * b.x - y1 * b.y);
-  hi = pack_bf16(y0 * a.x + x0 * a.y, y1 * b.x + x1 * b.y);
+  lo = pack_f16(x0 * a.x - y0 * a.y, x1 * b.x - y1 * b.y);
+  hi = pack_f16(y0 * a.x + x0 * a.y, y1 * b.x + x1 * b.y);
 }
 
 // (c, s) * (cos d, sin d): advances an angle seed by a fixed step.

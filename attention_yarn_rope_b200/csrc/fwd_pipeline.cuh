@@ -73,7 +73,8 @@ __device__ __forceinline__ bool fwd_issue_pv(const FwdParams& p, FwdSmem& sm, ui
 }
 
 __device__ __forceinline__ void fwd_mma_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem) {
-  constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+  // fused RoPE leaves Q and K in shared memory as fp16; pre-rotated inputs stay bf16
+  const uint32_t idesc_s = p.tab.enabled ? idesc_f16_f32(128, 128) : idesc_bf16_f32(128, 128, false);
   uint32_t t = 0, kv_it = 0, i = 0;
   bool have_prev = false, prev_first = false, ok = true;
   uint32_t prev_t = 0, prev_kv = 0;

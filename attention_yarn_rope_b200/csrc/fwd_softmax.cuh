@@ -4,11 +4,11 @@
 // key tile: read S from TMEM and release the S buffer at once (the next
 // QK^T overlaps the exponentials); classify each 32-key chunk for this warp
 // as hidden (skipped: its P is zero), partly visible (masked per element) or
-// fully visible; online softmax in log2 units where the sink is the initial
-// running max and its exp the initial running sum (sink = -inf starts from
-// an empty sum); P in bf16 into TMEM, one half at a time; O rescaled in TMEM
-// only when the running max grows by more than 2^8.  Epilogue: O / l in bf16
-// and LSE = (m + log2 l) ln 2.
+// fully visible; online softmax in log2 units (running max m, running sum l);
+// P in bf16 into TMEM, one half at a time; O rescaled in TMEM only when the
+// running max grows by more than 2^8.  Epilogue: the sink joins the max and
+// the sum once -- M = max(m, sink), l' = l 2^(m-M) + 2^(sink-M) (no term for
+// sink = -inf) -- then O 2^(m-M) / l' in bf16 and LSE = (M + log2 l') ln 2.
 #pragma once
 
 #include "fwd_common.cuh"
@@ -29,8 +29,11 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
     const int qi = w.q0 + r;
     const int qw_lo = w.q0 + wq * 32, qw_hi = qw_lo + 31;  // rows of this warp
     const float sink = __ldg(p.sinks + h) * kLog2e;
-    float m_run = sink;
-    float l_run = sink == -INFINITY ? 0.f : 1.f;
+    // The running max starts empty, so the first tile's largest P is exactly
+    // 1 (no bf16 rounding on the dominant key of short rows); the sink joins
+    // the max and the sum once, in the epilogue.
+    float m_run = -INFINITY;
+    float l_run = 0.f;
     for (int j = 0; j < w.n_kt; ++j, ++t) {
       const int k0 = (w.j_lo + j) * kFwdTile;
       if (!mbar_wait_warp(&sm.s_full[X], t & 1, p.wait_ns)) return;
@@ -147,7 +150,11 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
     tmem_wait_ld();
     tc_fence_before();
     if (qi < w.L && !(X == 1 && w.dup)) {
-      const float inv = 1.f / l_run;
+      // fold the sink: M = max(m, sink), l = l 2^(m - M) + 2^(sink - M)
+      const float M = fmaxf(m_run, sink);
+      const float a = m_run == -INFINITY ? 0.f : ex2_approx(m_run - M);
+      const float l_fin = l_run * a + (sink == -INFINITY ? 0.f : ex2_approx(sink - M));
+      const float inv = a / l_fin;
       const int64_t row = thd ? static_cast<int64_t>(w.seq_start + qi) * p.so.tok
                               : static_cast<int64_t>(w.b) * p.so.batch + static_cast<int64_t>(qi) * p.so.tok;
       __nv_bfloat16* dst = p.out + row + static_cast<int64_t>(h) * p.so.head;
@@ -162,7 +169,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
         *reinterpret_cast<uint4*>(dst + c8 * 8) = v;
       }
       if (p.lse != nullptr) {
-        const float lse = (m_run + log2f(l_run)) * kLn2;
+        const float lse = (M + log2f(l_fin)) * kLn2;
         if (thd)
           p.lse[static_cast<int64_t>(h) * p.T + w.seq_start + qi] = lse;
         else

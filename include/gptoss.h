@@ -117,8 +117,9 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
  * sliding window, BSHD or packed THD.
  *   q [B,S,Hq,D] / [T,Hq,D], k and v [B,S,Hkv,D] / [T,Hkv,D], bf16, own
  *          strides.  rope != NULL: q and k are raw and RoPE is applied inside
- *          the kernel as the tiles are loaded; rope == NULL: q and k are
- *          already rotated.
+ *          the kernel as the tiles are loaded (the rotated values enter the
+ *          QK^T product as fp16, so c * |x| must stay below 65504);
+ *          rope == NULL: q and k are already rotated (bf16 product).
  *   sinks  fp32 [Hq], in the units of the scaled logits (may be -inf).
  *   positions / cu_seqlens as for gptoss_rope_qk (positions only used when
  *          rope != NULL).

@@ -1,9 +1,12 @@
 """Shared helpers of the GPU parity tests: upload seeded inputs, compare a
 kernel's output with the float64 oracle.
 
-Tolerance (stated for bf16 inputs with fp32 accumulation and outputs of unit
-scale): max-abs error <= 1e-2 and mean-abs error <= 1e-3 on every compared
-element.
+Tolerance (bf16 inputs, fp32 accumulation, stated for outputs of unit scale):
+every element within 1e-2 of the oracle on the unit scale -- i.e.
+|got - ref| <= 1e-2 * max(1, |ref|) -- and mean-abs error <= 1e-3.  The
+scale factor only matters above |ref| = 1: a bf16 output of magnitude 2..4 is
+quantised in steps of 2^-6, so half a step (7.8e-3) of the 1e-2 budget is
+spent by the output format alone, and above 4 the step itself exceeds 1e-2.
 """
 
 from __future__ import annotations
@@ -39,8 +42,9 @@ def assert_parity(got: np.ndarray, ref: np.ndarray, what: str, max_abs=MAX_ABS, 
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     err = np.abs(got - ref)
-    mx, mean = float(err.max()), float(err.mean())
-    assert mx <= max_abs, f"{what}: max-abs {mx:.3e} > {max_abs} (mean {mean:.3e})"
+    scaled = err / np.maximum(1.0, np.abs(ref))
+    mx, mean, smx = float(err.max()), float(err.mean()), float(scaled.max())
+    assert smx <= max_abs, f"{what}: scaled max error {smx:.3e} > {max_abs} (max-abs {mx:.3e}, mean {mean:.3e})"
     assert mean <= mean_abs, f"{what}: mean-abs {mean:.3e} > {mean_abs}"
     return mx, mean
 

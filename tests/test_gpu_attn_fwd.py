@@ -14,6 +14,7 @@ import torch
 from attention_yarn_rope_b200 import ops
 from attention_yarn_rope_b200.workloads import GPTOSS_ROPE, PLAIN_ROPE, TINY, bf16_round, make_prefill
 from oracle.attention import attn_fwd_bshd, attn_fwd_thd
+from oracle.rope import rope
 from oracle.yarn import yarn_inv_freq_and_concentration
 from tests.gpu_util import assert_parity, dev, f32, host, i32
 
@@ -50,11 +51,16 @@ def test_bshd_multi_tile_ragged(cuda_device, window, fused_rope):
     if fused_rope:
         out, lse = ops.gptoss_attn_fwd(dev(q), dev(k), dev(v), f32(sinks), window=window,
                                        rope=ops.RopeConfig.from_dict(GPTOSS_ROPE), return_lse=True)
+        torch.cuda.synchronize()
+        ref, ref_lse = attn_fwd_bshd(q, k, v, sinks, 0.125, window, rope_tables=tabs)
     else:
-        qr, kr = ops.gptoss_rope_qk(dev(q), dev(k), ops.RopeConfig.from_dict(GPTOSS_ROPE))
-        out, lse = ops.gptoss_attn_fwd(qr, kr, dev(v), f32(sinks), window=window, return_lse=True)
-    torch.cuda.synchronize()
-    ref, ref_lse = attn_fwd_bshd(q, k, v, sinks, 0.125, window, rope_tables=tabs)
+        # pre-rotated bf16 inputs: both sides get the oracle's rotation rounded to bf16
+        pos = np.broadcast_to(np.arange(S), (B, S))
+        qr = np.stack([bf16_round(rope(q[b], pos[b], *tabs)) for b in range(B)])
+        kr = np.stack([bf16_round(rope(k[b], pos[b], *tabs)) for b in range(B)])
+        out, lse = ops.gptoss_attn_fwd(dev(qr), dev(kr), dev(v), f32(sinks), window=window, return_lse=True)
+        torch.cuda.synchronize()
+        ref, ref_lse = attn_fwd_bshd(qr, kr, v, sinks, 0.125, window, rope_tables=None)
     assert_parity(host(out), ref, f"out w={window}")
     assert_parity(host(lse), ref_lse, f"lse w={window}")
 
