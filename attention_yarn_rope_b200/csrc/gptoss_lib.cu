@@ -5,6 +5,8 @@
 
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "attn_decode.cuh"
 #include "fwd_pipeline.cuh"
 #include "gptoss.h"
@@ -267,3 +269,67 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they decode:
+// a serving loop that plans its memory once up front and may not call
+// cudaMalloc (which can synchronise the device or fail under memory pressure),
+// or a host runtime whose only device memory comes from its own fixed pools.
+// For them the split-KV partials live in one file-scope device array of fixed
+// size instead.  Every GPU that loads this library holds the array until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+// The array's name is a host-side stand-in in host code: its device address
+// comes from cudaGetSymbolAddress, once per device, with that device current.
+void* g_scratch_addr[kNoAllocMaxDevices];
+std::once_flag g_scratch_once[kNoAllocMaxDevices];
+cudaError_t g_scratch_err[kNoAllocMaxDevices];
+
+void* scratch_address(int device, gptoss_status* st) {
+  if (device < 0 || device >= kNoAllocMaxDevices) {
+    *st = GPTOSS_ERR_UNSUPPORTED;
+    return nullptr;
+  }
+  std::call_once(g_scratch_once[device], [device]() {
+    void* ptr = nullptr;
+    g_scratch_err[device] = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    g_scratch_addr[device] = ptr;
+  });
+  if (g_scratch_err[device] != cudaSuccess || g_scratch_addr[device] == nullptr) {
+    *st = GPTOSS_ERR_CUDA;
+    return nullptr;
+  }
+  *st = GPTOSS_OK;
+  return g_scratch_addr[device];
+}
+
+}  // namespace
+
+extern "C" gptoss_status gptoss_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                                    const int32_t* cache_seqlens, const float* sinks, int32_t B,
+                                                    int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D,
+                                                    int32_t window, float softmax_scale,
+                                                    const gptoss_rope_params* rope, void* out, float* lse,
+                                                    struct CUstream_st* stream) {
+  if (B == 0) return gptoss_attn_decode(q, k_cache, v_cache, cache_seqlens, sinks, B, Lmax, Hq, Hkv, D, window,
+                                        softmax_scale, rope, out, lse, nullptr, 0, stream);
+  const size_t need = gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D);
+  if (need == 0) return D != kHeadDim ? GPTOSS_ERR_UNSUPPORTED : GPTOSS_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) return GPTOSS_ERR_UNSUPPORTED;  // partials exceed the fixed array
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return GPTOSS_ERR_CUDA;
+  gptoss_status st = GPTOSS_OK;
+  void* ws = scratch_address(device, &st);
+  if (ws == nullptr) return st;
+  return gptoss_attn_decode(q, k_cache, v_cache, cache_seqlens, sinks, B, Lmax, Hq, Hkv, D, window, softmax_scale,
+                            rope, out, lse, ws, kNoAllocScratchBytes, stream);
+}

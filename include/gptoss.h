@@ -161,6 +161,32 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
                                  float* lse, void* workspace, size_t workspace_bytes,
                                  struct CUstream_st* stream);
 
+/* gptoss_attn_decode_noalloc -- gptoss_attn_decode for callers that cannot
+ * allocate device memory when they decode (a serving loop whose memory is
+ * planned once up front and must not call cudaMalloc, which may synchronise
+ * the device or fail under memory pressure; a runtime whose device memory
+ * comes only from its own fixed pools).  The pages have no counterpart: this
+ * is a packaging variant of the decode entry point, same arguments minus the
+ * workspace, same results.
+ *   The split-KV partials go to one file-scope device array of 16 MiB that
+ *   every GPU loading this library holds until the process exits.  Sizes
+ *   whose gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D) exceeds
+ *   16 MiB are rejected with GPTOSS_ERR_UNSUPPORTED (B=64 x 32768 needs
+ *   8.7 MB, B=8 x 131072 needs 5.0 MB).
+ *   The first call on a device looks the array's device address up
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  Nothing in the array needs to start at zero:
+ *   each call writes every partial it later reads.
+ *   All calls share the one array, which keeps the last call's contents:
+ *   calls whose executions overlap on the GPU (other streams, other host
+ *   threads) race and must be serialised by the caller.
+ *   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library. */
+gptoss_status gptoss_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* cache_seqlens, const float* sinks, int32_t B,
+                                         int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D, int32_t window,
+                                         float softmax_scale, const gptoss_rope_params* rope, void* out,
+                                         float* lse, struct CUstream_st* stream);
+
 /* Reads (and, if reset != 0, clears) the device status word of the current
  * device: GPTOSS_OK or GPTOSS_ERR_TIMEOUT.  Synchronises `stream`. */
 gptoss_status gptoss_read_device_status(int32_t* status_out, int32_t reset, struct CUstream_st* stream);
