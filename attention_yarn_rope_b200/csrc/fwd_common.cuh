@@ -10,8 +10,9 @@
 // share a kv head, so every K/V tile is loaded and rotated once for 256 query
 // rows.  16 warps (roles in fwd_softmax.cuh, fwd_rope.cuh, fwd_pipeline.cuh):
 //   warps 0-3 / 4-7   softmax of head A / head B (thread = query row = TMEM lane)
-//   warps 8-11        rope: next unit's Q tiles, every K tile in place
-//   warp 12           TMA producer (K, V tiles into a 4-stage ring)
+//   warps 8-11        rope: every Q and K tile rotated in place after TMA
+//   warp 12           TMA producer (two Q tiles per unit into a double
+//                     buffer, K / V tiles into a 4-stage ring)
 //   warp 13           TMEM allocation and tcgen05.mma issue
 //   warps 14-15       idle (complete the register split)
 // setmaxnreg moves registers from the rope / producer / MMA warpgroups to the
@@ -46,6 +47,7 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsRope + 128 * kRegsOther == kFw
               "register split must add up to the launch allocation");
 
 struct FwdParams {
+  CUtensorMap tmap_q;  // dims (64, Hq, S or T, B or 1), box (64, 1, 128, 1)
   CUtensorMap tmap_k;  // dims (64, Hkv, S or T, B or 1), box (64, 1, 128, 1)
   CUtensorMap tmap_v;
   const __nv_bfloat16* q;
@@ -66,7 +68,7 @@ struct __align__(1024) FwdSmem {
   uint8_t q[2][2][kFwdTileBytes];  // [buffer][head A/B], rotated, 128B-swizzled
   uint8_t k[kFwdStages][kFwdTileBytes];
   uint8_t v[kFwdStages][kFwdTileBytes];
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_loaded[2], q_full[2], q_empty[2];  // TMA landed / rotated / free again
   uint64_t k_full[kFwdStages], k_ready[kFwdStages], k_empty[kFwdStages];
   uint64_t v_full[kFwdStages], v_empty[kFwdStages];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];  // per head slot A/B

@@ -17,16 +17,24 @@ namespace gptoss {
 
 // =============================== TMA producer ===============================
 __device__ __forceinline__ void fwd_producer_role(const FwdParams& p, FwdSmem& sm) {
+  tma_prefetch_desc(&p.tmap_q);
   tma_prefetch_desc(&p.tmap_k);
   tma_prefetch_desc(&p.tmap_v);
   const bool thd = p.cu_seqlens != nullptr;
-  uint32_t kv_it = 0, k_issued = 0, v_issued = 0;
+  uint32_t kv_it = 0, k_issued = 0, v_issued = 0, i = 0, q_issued = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
     Unit wu;
     if (!make_unit(p, u, wu)) continue;
     const int tok0 = thd ? wu.seq_start : 0;
     const int bc = thd ? 0 : wu.b;
+    // the unit's two raw Q tiles into the free half of the Q double buffer
+    const int qb = i & 1;
+    if (!mbar_wait(&sm.q_empty[qb], ((i >> 1) & 1) ^ 1, p.wait_ns)) break;
+    mbar_arrive_expect_tx(&sm.q_loaded[qb], 2 * kFwdTileBytes);
+    tma_load_4d(sm.q[qb][0], &p.tmap_q, &sm.q_loaded[qb], 0, wu.h0, tok0 + wu.q0, bc);
+    tma_load_4d(sm.q[qb][1], &p.tmap_q, &sm.q_loaded[qb], 0, wu.h1, tok0 + wu.q0, bc);
+    q_issued = ++i;
     for (int j = 0; j < wu.n_kt; ++j, ++kv_it) {
       const int s = kv_it % kFwdStages;
       const uint32_t ph = ((kv_it / kFwdStages) & 1) ^ 1;
@@ -42,6 +50,8 @@ __device__ __forceinline__ void fwd_producer_role(const FwdParams& p, FwdSmem& s
     }
   }
   // the copies of the last stages must land before the CTA exits
+  for (uint32_t it = q_issued > 2 ? q_issued - 2 : 0; it < q_issued; ++it)
+    mbar_wait(&sm.q_loaded[it & 1], (it >> 1) & 1, p.wait_ns);
   for (uint32_t it = k_issued > kFwdStages ? k_issued - kFwdStages : 0; it < k_issued; ++it)
     mbar_wait(&sm.k_full[it % kFwdStages], (it / kFwdStages) & 1, p.wait_ns);
   for (uint32_t it = v_issued > kFwdStages ? v_issued - kFwdStages : 0; it < v_issued; ++it)
@@ -123,6 +133,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_loaded[i], 1);
       mbar_init(&sm.q_full[i], 128);
       mbar_init(&sm.q_empty[i], 1);
       mbar_init(&sm.s_full[i], 1);

@@ -55,25 +55,23 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
       mbar_arrive(&sm.s_free[X]);
       const int c_hi = min(qi, w.L - 1) - k0;  // visible columns of this row: [c_lo, c_hi]
       const int c_lo = p.window > 0 ? qi - p.window + 1 - k0 : -1;
-      // mask only tiles that cross an edge for this warp (whole-tile, warp-uniform)
-      const bool edge = cls[0] != 2 || cls[1] != 2 || cls[2] != 2 || cls[3] != 2;
-      if (edge) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = c * 32 + e;
-            const float x = (col <= c_hi && col >= c_lo) ? __uint_as_float(sr[c][e]) : -INFINITY;
-            sr[c][e] = __float_as_uint(x);
-          }
-      }
+      // mask only the chunks that are partly visible for this warp (warp-uniform
+      // branches); hidden chunks take no part in the max and get P = 0
       float mc[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        mc[c] = -INFINITY;
+        if (cls[c] == 1) {
+          const int lo_c = c_lo - 32 * c, hi_c = c_hi - 32 * c;  // visible e in [lo_c, hi_c]
 #pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+          for (int e = 0; e < 32; ++e)
+            if (e > hi_c || e < lo_c) sr[c][e] = __float_as_uint(-INFINITY);
+        }
+        mc[c] = -INFINITY;
+        if (cls[c] != 0) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+        }
       }
       const float mt = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
       const float m_cand = mt * p.scale_log2;

@@ -156,6 +156,10 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   memset(&p, 0, sizeof(p));
   const uint64_t dimS = thd ? static_cast<uint64_t>(total_tokens) : static_cast<uint64_t>(S);
   const uint64_t dimB = thd ? 1 : static_cast<uint64_t>(B);
+  const uint64_t qb_stride = thd ? dimS * sq.tok * 2 : static_cast<uint64_t>(sq.batch) * 2;
+  st = make_tmap_bf16_4d(&p.tmap_q, q, kHeadDim, Hq, dimS, dimB, sq.head * 2, sq.tok * 2,
+                         qb_stride == 0 ? 16 : qb_stride, kHeadDim, 1, kFwdTile, 1);
+  if (st != GPTOSS_OK) return st;
   const uint64_t kb_stride = thd ? dimS * sk.tok * 2 : static_cast<uint64_t>(sk.batch) * 2;
   const uint64_t vb_stride = thd ? dimS * sv.tok * 2 : static_cast<uint64_t>(sv.batch) * 2;
   st = make_tmap_bf16_4d(&p.tmap_k, k, kHeadDim, Hkv, dimS, dimB, sk.head * 2, sk.tok * 2,

@@ -62,14 +62,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits until the phase of `bar` with the given parity has completed, for at
-// most `limit_ns` nanoseconds.  On expiry records GPTOSS_ERR_TIMEOUT in the
-// device status word and returns false; the caller then stops its loop.
+// most about `limit_ns` nanoseconds.  On expiry records GPTOSS_ERR_TIMEOUT in
+// the device status word and returns false; the caller then stops its loop.
+// The bound is counted in SM clock cycles (2 per ns, i.e. exact at 2 GHz and
+// longer at lower clocks): the cycle counter is cheap to read, unlike the
+// global timer, whose read latency would delay every wake-up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
+  const long long limit_cycles = static_cast<long long>(limit_ns) * 2;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) {
+    if (clock64() - t0 > limit_cycles) {
       record_timeout();
       return false;
     }
@@ -304,6 +308,11 @@ __device__ __forceinline__ float2 bits_f2(uint64_t r) {
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
   return bits_f2(d);
 }
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
