@@ -116,6 +116,12 @@ __device__ __forceinline__ void fwd_mma_role(const FwdParams& p, FwdSmem& sm, ui
       prev_t = t;
       prev_kv = kv_it;
       prev_first = (j == 0);
+      if (j == wu.n_kt - 1) {
+        // close the unit now: its epilogue must not wait for the next unit's
+        // first QK^T (which needs that unit's Q and K tiles to be ready)
+        if (!fwd_issue_pv(p, sm, tmem, prev_t, prev_kv, prev_first)) { ok = false; break; }
+        have_prev = false;
+      }
     }
     ++i;
   }
