@@ -31,6 +31,7 @@ EXPORTED = (
     "gptoss_status_string",
     "gptoss_rope_qk",
     "gptoss_attn_fwd",
+    "gptoss_attn_fwd_workspace_size",
     "gptoss_attn_decode_workspace_size",
     "gptoss_attn_decode",
     "gptoss_attn_decode_noalloc",
@@ -66,7 +67,9 @@ _SIGNATURES = {
     "gptoss_rope_qk": (_st, [_vp, Strides, _vp, Strides, _vp, Strides, _vp, Strides, _vp, _vp, _i32, _i32, _i32,
                              _i32, _i32, ctypes.POINTER(RopeParams), _vp]),
     "gptoss_attn_fwd": (_st, [_vp, Strides, _vp, Strides, _vp, Strides, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
-                              _i32, _i32, _i32, _f32, ctypes.POINTER(RopeParams), _vp, Strides, _vp, _vp]),
+                              _i32, _i32, _i32, _f32, ctypes.POINTER(RopeParams), _vp, Strides, _vp, _vp,
+                              ctypes.c_size_t, _vp]),
+    "gptoss_attn_fwd_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32]),
     "gptoss_attn_decode_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
     "gptoss_attn_decode": (_st, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                  ctypes.POINTER(RopeParams), _vp, _vp, _vp, ctypes.c_size_t, _vp]),

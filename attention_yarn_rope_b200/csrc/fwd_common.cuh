@@ -7,17 +7,20 @@
 //
 // Design: persistent CTAs (one per SM), each walking a static, heaviest-first
 // list of work units.  A unit is one 128-query tile of TWO query heads that
-// share a kv head, so every K/V tile is loaded and rotated once for 256 query
-// rows.  16 warps (roles in fwd_softmax.cuh, fwd_rope.cuh, fwd_pipeline.cuh):
-//   warps 0-3 / 4-7   softmax of head A / head B (thread = query row = TMEM lane)
-//   warps 8-11        rope: every Q and K tile rotated in place after TMA
+// share a kv head, so every K/V tile is loaded once for 256 query rows.
+// 16 warps (roles in fwd_softmax.cuh, fwd_rope.cuh, fwd_pipeline.cuh):
+//   warps 0-3         rope: the Q tiles (and, without a workspace, the K
+//                     tiles) rotated in place after TMA
+//   warps 4-7 / 8-11  softmax of head A / head B (thread = query row; warp w
+//                     reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31)
 //   warp 12           TMA producer (two Q tiles per unit into a double
 //                     buffer, K / V tiles into a 4-stage ring)
-//   warp 13           TMEM allocation and tcgen05.mma issue
-//   warps 14-15       idle (complete the register split)
+//   warp 13           TMEM allocation; QK^T issue (fwd_mma_s_role)
+//   warp 14           P V issue (fwd_mma_pv_role)
+//   warp 15           idle (completes the register split)
 // setmaxnreg moves registers from the rope / producer / MMA warpgroups to the
 // two softmax warpgroups: launch 512 threads x 128 registers = 65536, split
-// 2 x 128 x 192 + 128 x 88 + 128 x 40 = 65536.  The host refuses to launch if
+// 2 x 128 x 208 + 128 x 56 + 128 x 40 = 65536.  The host refuses to launch if
 // the compiled kernel does not start at exactly 128 registers per thread.
 // TMEM columns (all 512): S_A [0,128) P_A [128,192) O_A [192,256),
 //                         S_B [256,384) P_B [384,448) O_B [448,512).
@@ -42,7 +45,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define GPTOSS_POLY_MASK 0x0000u
 #endif
 constexpr uint32_t kPolyMask = GPTOSS_POLY_MASK;
-constexpr uint32_t kRegsSoftmax = 192, kRegsRope = 88, kRegsOther = 40;
+constexpr uint32_t kRegsSoftmax = 208, kRegsRope = 56, kRegsOther = 40;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsRope + 128 * kRegsOther == kFwdThreads * kFwdLaunchRegs,
               "register split must add up to the launch allocation");
 
@@ -59,6 +62,7 @@ struct FwdParams {
   const int32_t* positions;
   const int32_t* cu_seqlens;
   int B, S, T, Hq, Hkv, G, HP, window, n_qtiles, n_units;
+  int k_in_kernel;  // 1: K tiles are rotated in shared memory; 0: k arrives rotated (or RoPE is off)
   float scale_log2;
   uint64_t wait_ns;
   RopeTable tab;
@@ -72,7 +76,7 @@ struct __align__(1024) FwdSmem {
   uint64_t k_full[kFwdStages], k_ready[kFwdStages], k_empty[kFwdStages];
   uint64_t v_full[kFwdStages], v_empty[kFwdStages];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];  // per head slot A/B
-  uint64_t mma_final;
+  uint64_t mma_final[2];  // the S and P V issuers' last products have completed
   uint32_t tmem_base;
 };
 

@@ -1,12 +1,10 @@
-// fwd_pipeline.cuh -- TMA producer, tcgen05 MMA issuer and the prefill
+// fwd_pipeline.cuh -- TMA producer, tcgen05 MMA issuers and the prefill
 // kernel itself (gptoss_attn_fwd).
 //
-// MMA order per key tile t (one thread issues everything):
-//   S_A(t) = Q_A K(t)^T, S_B(t) = Q_B K(t)^T   (SS, M128 N128, 4 x K16)
-//   O_A += P_A(t-1) V(t-1), O_B += P_B(t-1) V(t-1)   (TS: P from TMEM, V from
-//   shared memory read N-major, M128 N64, 8 x K16)
-// so the next tile's QK^T runs while the softmax warps exponentiate.  Each
-// consumer is signalled by tcgen05.commit on an mbarrier.
+// Products (each consumer is signalled by tcgen05.commit on an mbarrier):
+//   S_X(t) = Q_X K(t)^T   (SS, M128 N128, 4 x K16)
+//   O_X += P_X(t) V(t)    (TS: P from TMEM, V from shared memory read N-major,
+//                          M128 N64, 8 x K16)
 #pragma once
 
 #include "fwd_common.cuh"
@@ -58,47 +56,34 @@ __device__ __forceinline__ void fwd_producer_role(const FwdParams& p, FwdSmem& s
     mbar_wait(&sm.v_full[it % kFwdStages], (it / kFwdStages) & 1, p.wait_ns);
 }
 
-// ================================ MMA issuer ================================
-// O_X += P_X V for the tile with running index tt whose V sits in the stage of
-// kv iteration kv; `first` = the tile opens its unit (O starts from zero).
-__device__ __forceinline__ bool fwd_issue_pv(const FwdParams& p, FwdSmem& sm, uint32_t tmem, uint32_t tt,
-                                             uint32_t kv, bool first) {
-  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 64, true);
-  const int s = kv % kFwdStages;
-  if (!mbar_wait(&sm.v_full[s], (kv / kFwdStages) & 1, p.wait_ns)) return false;
-  const uint64_t vdesc = sw128_desc(smem_u32(sm.v[s]));
-#pragma unroll 1
-  for (int X = 0; X < 2; ++X) {
-    if (!mbar_wait(&sm.p_full[X], tt & 1, p.wait_ns)) return false;
-    tc_fence_after();
-    const uint32_t colP = X * 256 + 128, colO = X * 256 + 192;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_ts(tmem + colO, tmem + colP + kk * 8, vdesc + static_cast<uint64_t>(kk * 128), idesc_o,
-             (first && kk == 0) ? 0u : 1u);
-    mma_commit(&sm.o_done[X]);
-  }
-  mma_commit(&sm.v_empty[s]);
-  return true;
-}
+// ================================ MMA issuers ================================
+// Two threads issue the tensor-core work.  A tcgen05.mma blocks its issuing
+// thread until the tensor core takes it, and a product's completion reaches
+// its consumer roughly 450 cycles after issue; with one issuer, the next
+// QK^T would queue behind the previous tile's P V issue and wait for the
+// softmax's P.  Split, QK^T depends only on the softmax having read S (early
+// in each tile) and P V only on P: each is issued as soon as its inputs exist.
+// tcgen05.commit tracks the issuing thread's own products, so each thread
+// signals its own consumers.
 
-__device__ __forceinline__ void fwd_mma_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem) {
+// S_X(t) = Q_X K(t)^T for both head slots, tile by tile.
+__device__ __forceinline__ void fwd_mma_s_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem) {
   // fused RoPE leaves Q and K in shared memory as fp16; pre-rotated inputs stay bf16
   const uint32_t idesc_s = p.tab.enabled ? idesc_f16_f32(128, 128) : idesc_bf16_f32(128, 128, false);
   uint32_t t = 0, kv_it = 0, i = 0;
-  bool have_prev = false, prev_first = false, ok = true;
-  uint32_t prev_t = 0, prev_kv = 0;
+  bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
     Unit wu;
     if (!make_unit(p, u, wu)) continue;
     const int qb = i & 1;
-    if (!mbar_wait(&sm.q_full[qb], (i >> 1) & 1, p.wait_ns)) { ok = false; break; }
-    for (int j = 0; j < wu.n_kt && ok; ++j, ++t, ++kv_it) {
+    if (!mbar_wait(&sm.q_full[qb], (i >> 1) & 1, p.wait_ns)) break;
+    for (int j = 0; j < wu.n_kt; ++j, ++t, ++kv_it) {
       const int s = kv_it % kFwdStages;
-      if (!mbar_wait(&sm.k_ready[s], (kv_it / kFwdStages) & 1, p.wait_ns)) { ok = false; break; }
+      uint64_t* k_in = p.k_in_kernel ? &sm.k_ready[s] : &sm.k_full[s];  // rotated in place, or as copied
+      if (!mbar_wait(k_in, (kv_it / kFwdStages) & 1, p.wait_ns)) { ok = false; break; }
       const uint64_t kdesc = sw128_desc(smem_u32(sm.k[s]));
 #pragma unroll 1
-      for (int X = 0; X < 2 && ok; ++X) {
+      for (int X = 0; X < 2; ++X) {
         if (t > 0 && !mbar_wait(&sm.s_free[X], (t - 1) & 1, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint64_t qdesc = sw128_desc(smem_u32(sm.q[qb][X]));
@@ -111,24 +96,43 @@ __device__ __forceinline__ void fwd_mma_role(const FwdParams& p, FwdSmem& sm, ui
       if (!ok) break;
       mma_commit(&sm.k_empty[s]);
       if (j == wu.n_kt - 1) mma_commit(&sm.q_empty[qb]);
-      if (have_prev && !fwd_issue_pv(p, sm, tmem, prev_t, prev_kv, prev_first)) { ok = false; break; }
-      have_prev = true;
-      prev_t = t;
-      prev_kv = kv_it;
-      prev_first = (j == 0);
-      if (j == wu.n_kt - 1) {
-        // close the unit now: its epilogue must not wait for the next unit's
-        // first QK^T (which needs that unit's Q and K tiles to be ready)
-        if (!fwd_issue_pv(p, sm, tmem, prev_t, prev_kv, prev_first)) { ok = false; break; }
-        have_prev = false;
-      }
     }
     ++i;
   }
-  if (ok && have_prev) fwd_issue_pv(p, sm, tmem, prev_t, prev_kv, prev_first);
-  // every issued MMA must finish before TMEM is released
-  mma_commit(&sm.mma_final);
-  mbar_wait(&sm.mma_final, 0, p.wait_ns);
+  mma_commit(&sm.mma_final[0]);
+  mbar_wait(&sm.mma_final[0], 0, p.wait_ns);
+}
+
+// O_X += P_X(t) V(t) for both head slots (TS: P from TMEM, V N-major from
+// shared memory); the first tile of a unit starts O from zero.
+__device__ __forceinline__ void fwd_mma_pv_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem) {
+  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 64, true);
+  uint32_t t = 0, kv_it = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    Unit wu;
+    if (!make_unit(p, u, wu)) continue;
+    for (int j = 0; j < wu.n_kt; ++j, ++t, ++kv_it) {
+      const int s = kv_it % kFwdStages;
+      if (!mbar_wait(&sm.v_full[s], (kv_it / kFwdStages) & 1, p.wait_ns)) { ok = false; break; }
+      const uint64_t vdesc = sw128_desc(smem_u32(sm.v[s]));
+#pragma unroll 1
+      for (int X = 0; X < 2; ++X) {
+        if (!mbar_wait(&sm.p_full[X], t & 1, p.wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t colP = X * 256 + 128, colO = X * 256 + 192;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + colO, tmem + colP + kk * 8, vdesc + static_cast<uint64_t>(kk * 128), idesc_o,
+                 (j == 0 && kk == 0) ? 0u : 1u);
+        mma_commit(&sm.o_done[X]);
+      }
+      if (!ok) break;
+      mma_commit(&sm.v_empty[s]);
+    }
+  }
+  mma_commit(&sm.mma_final[1]);
+  mbar_wait(&sm.mma_final[1], 0, p.wait_ns);
 }
 
 // ================================== kernel ==================================
@@ -154,7 +158,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    mbar_init(&sm.mma_final, 1);
+    mbar_init(&sm.mma_final[0], 1);
+    mbar_init(&sm.mma_final[1], 1);
     fence_mbar_init();
   }
   if (warp == 13) {
@@ -166,16 +171,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const int wg = warp >> 2;
-  if (wg < 2) {
+  // the rope warpgroup takes the lowest warp numbers (measured: its Q
+  // rotation finishes sooner there, next to two busy softmax warpgroups)
+  if (wg == 1 || wg == 2) {
     reg_alloc<kRegsSoftmax>();
-    fwd_softmax_role(p, sm, tmem, wg);
-  } else if (wg == 2) {
+    fwd_softmax_role(p, sm, tmem, wg - 1);
+  } else if (wg == 0) {
     reg_dealloc<kRegsRope>();
     fwd_rope_role(p, sm);
   } else {
     reg_dealloc<kRegsOther>();
     if (warp == 12 && lane == 0) fwd_producer_role(p, sm);
-    else if (warp == 13 && lane == 0) fwd_mma_role(p, sm, tmem);
+    else if (warp == 13 && lane == 0) fwd_mma_s_role(p, sm, tmem);
+    else if (warp == 14 && lane == 0) fwd_mma_pv_role(p, sm, tmem);
   }
   tc_fence_before();
   __syncthreads();

@@ -57,7 +57,7 @@ __device__ __forceinline__ void rotate_tile(const FwdParams& p, const RopeLane& 
 }
 
 __device__ __forceinline__ void fwd_rope_role(const FwdParams& p, FwdSmem& sm) {
-  const int rt = threadIdx.x - 256;
+  const int rt = threadIdx.x;  // warps 0-3
   const int w = rt >> 5, l = rt & 31;
   const int pb = l & 15;
   RopeLane rl;
@@ -100,16 +100,18 @@ __device__ __forceinline__ void fwd_rope_role(const FwdParams& p, FwdSmem& sm) {
       fence_proxy_async_smem();
     }
     mbar_arrive(&sm.q_full[qb]);
+    ++i;
+    if (!p.k_in_kernel) continue;  // k arrives rotated (or RoPE is off): QK^T waits on the copy itself
     // ---- the unit's K tiles: consecutive, so one seed plus a fixed step each ----
     float2 k0s = one, k1s = one;
-    if (rot && !explicit_pos) {
+    if (!explicit_pos) {
       k0s = rope_cs(wu.j_lo * kFwdTile + rl.ro, rl.f0, p.tab.conc);
       k1s = rope_cs(wu.j_lo * kFwdTile + rl.ro, rl.f1, p.tab.conc);
     }
     for (int j = 0; j < wu.n_kt; ++j, ++kv_it) {
       const int s = kv_it % kFwdStages;
       if (!mbar_wait_warp(&sm.k_full[s], (kv_it / kFwdStages) & 1, p.wait_ns)) return;
-      if (rot) {
+      {
         const int k0 = (wu.j_lo + j) * kFwdTile;
         rotate_tile(p, rl, sm.k[s], k0s, k1s, min(kFwdTile, wu.L - k0), explicit_pos ? pos_seq + k0 : nullptr);
         fence_proxy_async_smem();
@@ -118,7 +120,6 @@ __device__ __forceinline__ void fwd_rope_role(const FwdParams& p, FwdSmem& sm) {
       }
       mbar_arrive(&sm.k_ready[s]);
     }
-    ++i;
   }
 }
 

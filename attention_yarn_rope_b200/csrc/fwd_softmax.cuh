@@ -4,16 +4,97 @@
 // key tile: read S from TMEM and release the S buffer at once (the next
 // QK^T overlaps the exponentials); classify each 32-key chunk for this warp
 // as hidden (skipped: its P is zero), partly visible (masked per element) or
-// fully visible; online softmax in log2 units (running max m, running sum l);
-// P in bf16 into TMEM, one half at a time; O rescaled in TMEM only when the
-// running max grows by more than 2^8.  Epilogue: the sink joins the max and
-// the sum once -- M = max(m, sink), l' = l 2^(m-M) + 2^(sink-M) (no term for
-// sink = -inf) -- then O 2^(m-M) / l' in bf16 and LSE = (M + log2 l') ln 2.
+// fully visible; online softmax in log2 units with a running base m and sum
+// l; P in bf16 into TMEM, one half at a time.
+//
+// The base.  A row's first visible tile sets m to its maximum, so that tile's
+// largest P is exactly 1.  Later tiles reuse m as it stands and skip the row
+// maximum: any base gives the same O / l, and bf16 P and fp32 sums keep their
+// relative precision at any scale.  The only risk is range, so the tile's
+// sum is checked afterwards: above 2^64 (or not finite) the warp recomputes
+// tile against its true maximum (the scores are still in registers) and
+// rescales l and O.  In attention the
+// scores after the first tile rarely exceed it by 64 (log2 units), so the
+// redo path is cold; a row whose first tile is fully masked keeps m = -inf
+// and takes the maximum path again on the next one.
+//
+// Epilogue: the sink joins the max and the sum once -- M = max(m, sink),
+// l' = l 2^(m-M) + 2^(sink-M) (no term for sink = -inf) -- then
+// O 2^(m-M) / l' in bf16 and LSE = (M + log2 l') ln 2.
 #pragma once
 
 #include "fwd_common.cuh"
 
 namespace gptoss {
+
+constexpr float kMaxTileSum = 18446744073709551616.0f;  // 2^64
+
+// Row maximum of the raw scores over the chunks this warp can see (masked
+// elements already hold -inf); -inf when none is visible.
+__device__ __forceinline__ float tile_max(const uint32_t (&sr)[4][32], const int (&cls)[4]) {
+  float mc[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    mc[c] = -INFINITY;
+    if (cls[c] != 0) {
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+    }
+  }
+  return fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
+}
+
+// Reads this warp's 32 rows x 128 scores of S from TMEM and sets the hidden
+// elements of partly visible chunks to -inf (row qi sees keys
+// [qi - window + 1, min(qi, L - 1)]; k0 is the tile's first key).
+__device__ __forceinline__ void load_masked_s(uint32_t taddr, const int (&cls)[4], int qi, int k0, int L,
+                                              int window, uint32_t (&sr)[4][32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, sr[c]);
+  tmem_wait_ld();
+  const int c_hi = min(qi, L - 1) - k0;  // visible columns of this row: [c_lo, c_hi]
+  const int c_lo = window > 0 ? qi - window + 1 - k0 : -1;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    if (cls[c] == 1) {  // warp-uniform branch
+      const int lo_c = c_lo - 32 * c, hi_c = c_hi - 32 * c;
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (e > hi_c || e < lo_c) sr[c][e] = __float_as_uint(-INFINITY);
+    }
+  }
+}
+
+// P = 2^(s sl - base) for chunks (2 half, 2 half + 1) as 32 packed bf16 pairs;
+// adds the fp32 values to (rs0, rs1).  Hidden chunks give zeros.
+__device__ __forceinline__ void exp_half(const uint32_t (&sr)[4][32], const int (&cls)[4], int half, float sl,
+                                         float nb, float& rs0, float& rs1, uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = 2 * half + cc;
+    if (cls[c] == 0) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) pk[cc * 16 + e] = 0u;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float x0 = fmaf(__uint_as_float(sr[c][2 * e]), sl, nb);
+        const float x1 = fmaf(__uint_as_float(sr[c][2 * e + 1]), sl, nb);
+        float p0, p1;
+        if ((kPolyMask >> e) & 1u) {
+          p0 = exp2_poly(x0);
+          p1 = exp2_poly(x1);
+        } else {
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+        }
+        rs0 += p0;
+        rs1 += p1;
+        pk[cc * 16 + e] = pack_bf16(p0, p1);
+      }
+    }
+  }
+}
 
 __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem, int X) {
   const int wq = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quarter
@@ -21,6 +102,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   const uint32_t colS = X * 256, colP = X * 256 + 128, colO = X * 256 + 192;
   const bool thd = p.cu_seqlens != nullptr;
+  const float sl = p.scale_log2;
   uint32_t t = 0;  // running tile count of this CTA
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     Unit w;
@@ -29,9 +111,6 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
     const int qi = w.q0 + r;
     const int qw_lo = w.q0 + wq * 32, qw_hi = qw_lo + 31;  // rows of this warp
     const float sink = __ldg(p.sinks + h) * kLog2e;
-    // The running max starts empty, so the first tile's largest P is exactly
-    // 1 (no bf16 rounding on the dominant key of short rows); the sink joins
-    // the max and the sum once, in the epilogue.
     float m_run = -INFINITY;
     float l_run = 0.f;
     for (int j = 0; j < w.n_kt; ++j, ++t) {
@@ -48,95 +127,71 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
         cls[c] = hidden ? 0 : (full ? 2 : 1);
       }
       uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + colS + c * 32, sr[c]);
-      tmem_wait_ld();
+      load_masked_s(lane_base + colS, cls, qi, k0, w.L, p.window, sr);
       tc_fence_before();
       mbar_arrive(&sm.s_free[X]);
-      const int c_hi = min(qi, w.L - 1) - k0;  // visible columns of this row: [c_lo, c_hi]
-      const int c_lo = p.window > 0 ? qi - p.window + 1 - k0 : -1;
-      // mask only the chunks that are partly visible for this warp (warp-uniform
-      // branches); hidden chunks take no part in the max and get P = 0
-      float mc[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (cls[c] == 1) {
-          const int lo_c = c_lo - 32 * c, hi_c = c_hi - 32 * c;  // visible e in [lo_c, hi_c]
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (e > hi_c || e < lo_c) sr[c][e] = __float_as_uint(-INFINITY);
-        }
-        mc[c] = -INFINITY;
-        if (cls[c] != 0) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 2)
-            mc[c] = fmax3(mc[c], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
-        }
-      }
-      const float mt = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
-      const float m_cand = mt * p.scale_log2;
       float alpha = 1.f;
       bool rescale = false;
-      if (m_cand > m_run + kRescaleThreshold) {
-        alpha = ex2_approx(m_run - m_cand);  // 0 when m_run is -inf
-        m_run = m_cand;
-        rescale = true;
+      // a row without a base yet takes its maximum (the whole warp does, so the
+      // branch stays uniform; rows that have a base keep it unless it grows by 2^8)
+      if (__any_sync(0xffffffffu, m_run == -INFINITY)) {
+        const float m_cand = tile_max(sr, cls) * sl;
+        if (m_cand > m_run + kRescaleThreshold) {
+          alpha = ex2_approx(m_run - m_cand);  // 0 when m_run is -inf
+          m_run = m_cand;
+          rescale = true;
+        }
       }
-      const float base = m_run == -INFINITY ? 0.f : m_run;
-      const float sl = p.scale_log2, nb = -base;
-      // scalar arithmetic: measured faster here than packed fp32x2
+      float nb = m_run == -INFINITY ? 0.f : -m_run;
       float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      {
         uint32_t pk[32];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = 2 * half + cc;
-          if (cls[c] == 0) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[cc * 16 + e] = 0u;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float x0 = fmaf(__uint_as_float(sr[c][2 * e]), sl, nb);
-              const float x1 = fmaf(__uint_as_float(sr[c][2 * e + 1]), sl, nb);
-              float p0, p1;
-              if ((kPolyMask >> e) & 1u) {
-                p0 = exp2_poly(x0);
-                p1 = exp2_poly(x1);
-              } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
-              }
-              rs0 += p0;
-              rs1 += p1;
-              pk[cc * 16 + e] = pack_bf16(p0, p1);
-            }
-          }
+        exp_half(sr, cls, 0, sl, nb, rs0, rs1, pk);
+        // P(t) overwrites P(t-1): the previous P V product must have completed
+        if (t > 0) {
+          if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
+          tc_fence_after();
         }
-        if (half == 0) {
-          // P(t) overwrites P(t-1): the previous P V product must have completed
-          if (t > 0) {
-            if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
-            tc_fence_after();
-          }
-          // warp-collective TMEM access: the whole warp rescales when any row
-          // needs it (alpha is 1 for the rows that do not)
-          if (__any_sync(0xffffffffu, rescale && j > 0)) {
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              uint32_t ov[32];
-              tmem_ld32(lane_base + colO + c * 32, ov);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-              tmem_st32(lane_base + colO + c * 32, ov);
-            }
-          }
-        }
-        tmem_st32(lane_base + colP + half * 32, pk);
+        tmem_st32(lane_base + colP, pk);
       }
-      l_run = l_run * alpha + (rs0 + rs1);
+      {
+        uint32_t pk[32];
+        exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
+        tmem_st32(lane_base + colP + 32, pk);
+      }
+      float rs = rs0 + rs1;
+      if (__any_sync(0xffffffffu, !(rs <= kMaxTileSum))) {
+        // cold: rebase on the tile maximum and redo both halves (P(t) is not
+        // consumed before p_full, so overwriting it is safe)
+        const float m_new = fmaxf(m_run, tile_max(sr, cls) * sl);
+        if (m_new > m_run) {
+          alpha *= ex2_approx(m_run - m_new);
+          m_run = m_new;
+          rescale = true;
+        }
+        nb = m_run == -INFINITY ? 0.f : -m_run;
+        rs0 = rs1 = 0.f;
+        uint32_t pk[32];
+        exp_half(sr, cls, 0, sl, nb, rs0, rs1, pk);
+        tmem_st32(lane_base + colP, pk);
+        exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
+        tmem_st32(lane_base + colP + 32, pk);
+        rs = rs0 + rs1;
+      }
+      // warp-collective TMEM access: the whole warp rescales O when any row
+      // needs it (alpha is 1 for the rows that do not)
+      if (__any_sync(0xffffffffu, rescale && j > 0)) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(lane_base + colO + c * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(lane_base + colO + c * 32, ov);
+        }
+      }
+      l_run = l_run * alpha + rs;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full[X]);

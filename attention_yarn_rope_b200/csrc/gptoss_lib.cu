@@ -109,8 +109,13 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
   p.Hkv = Hkv;
   yarn_table(*rope, &p.tab);
   const int grid = static_cast<int>((ntok + kRopeTokensPerCta - 1) / kRopeTokensPerCta);
-  rope_qk_kernel<<<grid, kRopeThreads, 0, as_stream(stream)>>>(p);
+  rope_qk_kernel<false><<<grid, kRopeThreads, 0, as_stream(stream)>>>(p);
   return check_launch();
+}
+
+size_t gptoss_attn_fwd_workspace_size(int32_t total_tokens, int32_t Hkv, int32_t D) {
+  if (total_tokens < 0 || Hkv <= 0 || D != kHeadDim) return 0;
+  return static_cast<size_t>(total_tokens) * Hkv * kHeadDim * 2;  // fp16
 }
 
 gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk, const void* v,
@@ -118,7 +123,7 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
                               const int32_t* cu_seqlens, int32_t B, int32_t S, int32_t total_tokens, int32_t Hq,
                               int32_t Hkv, int32_t D, int32_t window, float softmax_scale,
                               const gptoss_rope_params* rope, void* out, gptoss_strides so, float* lse,
-                              struct CUstream_st* stream) {
+                              void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
   if (B < 0 || S < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0 || window < 0) return GPTOSS_ERR_INVALID_ARG;
   if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
   if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
@@ -131,6 +136,11 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   if (!q || !k || !v || !sinks || !out) return GPTOSS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GPTOSS_ERR_INVALID_ARG;
   if (!strides_ok(sq, !thd) || !strides_ok(sk, !thd) || !strides_ok(sv, !thd) || !strides_ok(so, !thd))
+    return GPTOSS_ERR_INVALID_ARG;
+  // with RoPE and a workspace, k is rotated once into it (fp16) instead of
+  // once per work unit inside the kernel
+  const bool k_pre = rope != nullptr && workspace != nullptr;
+  if (k_pre && (workspace_bytes < gptoss_attn_fwd_workspace_size(total_tokens, Hkv, D) || !aligned16(workspace)))
     return GPTOSS_ERR_INVALID_ARG;
   const int n_qtiles = (S + kFwdTile - 1) / kFwdTile;
   const int G = Hq / Hkv;
@@ -157,15 +167,21 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   const uint64_t dimS = thd ? static_cast<uint64_t>(total_tokens) : static_cast<uint64_t>(S);
   const uint64_t dimB = thd ? 1 : static_cast<uint64_t>(B);
   const uint64_t qb_stride = thd ? dimS * sq.tok * 2 : static_cast<uint64_t>(sq.batch) * 2;
-  st = make_tmap_bf16_4d(&p.tmap_q, q, kHeadDim, Hq, dimS, dimB, sq.head * 2, sq.tok * 2,
+  st = make_tmap_4d(&p.tmap_q, q, kHeadDim, Hq, dimS, dimB, sq.head * 2, sq.tok * 2,
                          qb_stride == 0 ? 16 : qb_stride, kHeadDim, 1, kFwdTile, 1);
   if (st != GPTOSS_OK) return st;
   const uint64_t kb_stride = thd ? dimS * sk.tok * 2 : static_cast<uint64_t>(sk.batch) * 2;
   const uint64_t vb_stride = thd ? dimS * sv.tok * 2 : static_cast<uint64_t>(sv.batch) * 2;
-  st = make_tmap_bf16_4d(&p.tmap_k, k, kHeadDim, Hkv, dimS, dimB, sk.head * 2, sk.tok * 2,
-                         kb_stride == 0 ? 16 : kb_stride, kHeadDim, 1, kFwdTile, 1);
+  if (k_pre) {  // dense fp16 [B, S, Hkv, D] / [T, Hkv, D] in the workspace
+    const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
+    st = make_tmap_4d(&p.tmap_k, workspace, kHeadDim, Hkv, dimS, dimB, kHeadDim * 2, tok_b,
+                      thd ? dimS * tok_b : static_cast<uint64_t>(S) * tok_b, kHeadDim, 1, kFwdTile, 1, true);
+  } else {
+    st = make_tmap_4d(&p.tmap_k, k, kHeadDim, Hkv, dimS, dimB, sk.head * 2, sk.tok * 2,
+                      kb_stride == 0 ? 16 : kb_stride, kHeadDim, 1, kFwdTile, 1);
+  }
   if (st != GPTOSS_OK) return st;
-  st = make_tmap_bf16_4d(&p.tmap_v, v, kHeadDim, Hkv, dimS, dimB, sv.head * 2, sv.tok * 2,
+  st = make_tmap_4d(&p.tmap_v, v, kHeadDim, Hkv, dimS, dimB, sv.head * 2, sv.tok * 2,
                          vb_stride == 0 ? 16 : vb_stride, kHeadDim, 1, kFwdTile, 1);
   if (st != GPTOSS_OK) return st;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -190,6 +206,29 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   p.wait_ns = wait_limit_ns();
   if (rope != nullptr) yarn_table(*rope, &p.tab);
   else p.tab.enabled = 0;
+  p.k_in_kernel = rope != nullptr && !k_pre;
+  if (k_pre) {
+    RopeQkParams rp;
+    memset(&rp, 0, sizeof(rp));
+    rp.k = static_cast<const __nv_bfloat16*>(k);
+    rp.k_out = static_cast<__nv_bfloat16*>(workspace);  // fp16 bits (rope_qk_kernel<true>)
+    rp.sk = sk;
+    rp.sko.head = kHeadDim;
+    rp.sko.tok = static_cast<int64_t>(Hkv) * kHeadDim;
+    rp.sko.batch = thd ? 0 : static_cast<int64_t>(S) * Hkv * kHeadDim;
+    rp.tm.positions = positions;
+    rp.tm.cu_seqlens = cu_seqlens;
+    rp.tm.nseq = B;
+    rp.tm.S = thd ? 0 : S;
+    rp.tm.ntok = total_tokens;
+    rp.Hq = 0;
+    rp.Hkv = Hkv;
+    rp.tab = p.tab;
+    const int rgrid = (total_tokens + kRopeTokensPerCta - 1) / kRopeTokensPerCta;
+    rope_qk_kernel<true><<<rgrid, kRopeThreads, 0, as_stream(stream)>>>(rp);
+    st = check_launch();
+    if (st != GPTOSS_OK) return st;
+  }
   const size_t smem = sizeof(FwdSmem) + 1024;
   if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
@@ -231,10 +270,10 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
   memset(&p, 0, sizeof(p));
   const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
   const uint64_t bat_b = tok_b * Lmax;
-  st = make_tmap_bf16_4d(&p.tmap_k, k_cache, kHeadDim, Hkv, Lmax, B, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
+  st = make_tmap_4d(&p.tmap_k, k_cache, kHeadDim, Hkv, Lmax, B, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
                          kDecTileKeys, 1);
   if (st != GPTOSS_OK) return st;
-  st = make_tmap_bf16_4d(&p.tmap_v, v_cache, kHeadDim, Hkv, Lmax, B, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
+  st = make_tmap_4d(&p.tmap_v, v_cache, kHeadDim, Hkv, Lmax, B, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
                          kDecTileKeys, 1);
   if (st != GPTOSS_OK) return st;
   const int G = Hq / Hkv;

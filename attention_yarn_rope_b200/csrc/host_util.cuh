@@ -96,18 +96,20 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D bf16 map (dims innermost first: d, head, token, batch) with a 128-byte
+// 4-D bf16 (or fp16) map (dims innermost first: d, head, token, batch) with a 128-byte
 // swizzle; out-of-range rows read as zeros.
-inline gptoss_status make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+inline gptoss_status make_tmap_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                                        uint64_t d2, uint64_t d3, uint64_t s1_bytes, uint64_t s2_bytes,
-                                       uint64_t s3_bytes, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+                                       uint64_t s3_bytes, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3,
+                                       bool fp16 = false) {
   auto fn = encode_fn();
   if (fn == nullptr) return GPTOSS_ERR_CUDA;
   cuuint64_t dims[4] = {d0, d1, d2, d3};
   cuuint64_t strides[3] = {s1_bytes, s2_bytes, s3_bytes};
   cuuint32_t box[4] = {b0, b1, b2, b3};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GPTOSS_OK : GPTOSS_ERR_INVALID_ARG;

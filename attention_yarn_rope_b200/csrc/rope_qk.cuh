@@ -59,7 +59,10 @@ __device__ __forceinline__ float2 rope_cs(int pos, double f, float conc) {
 }
 
 // Rotates the 8 pairs held by (lo, hi): lo = features [8c, 8c+8), hi = the
-// partners [32+8c, 40+8c); cs[e] = (c cos, c sin) of pair 8c+e.
+// partners [32+8c, 40+8c); cs[e] = (c cos, c sin) of pair 8c+e.  The result
+// is rounded to bf16, or to fp16 when kF16Out (the QK^T operand format of the
+// prefill kernel under fused RoPE).
+template <bool kF16Out>
 __device__ __forceinline__ void rotate8(uint4& lo, uint4& hi, const float2* cs) {
   uint32_t* l = reinterpret_cast<uint32_t*>(&lo);
   uint32_t* h = reinterpret_cast<uint32_t*>(&hi);
@@ -68,8 +71,10 @@ __device__ __forceinline__ void rotate8(uint4& lo, uint4& hi, const float2* cs) 
     const float x0 = bf16lo(l[w]), x1 = bf16hi(l[w]);
     const float y0 = bf16lo(h[w]), y1 = bf16hi(h[w]);
     const float2 a = cs[2 * w], b = cs[2 * w + 1];
-    l[w] = pack_bf16(x0 * a.x - y0 * a.y, x1 * b.x - y1 * b.y);
-    h[w] = pack_bf16(y0 * a.x + x0 * a.y, y1 * b.x + x1 * b.y);
+    const float rx0 = x0 * a.x - y0 * a.y, rx1 = x1 * b.x - y1 * b.y;
+    const float ry0 = y0 * a.x + x0 * a.y, ry1 = y1 * b.x + x1 * b.y;
+    l[w] = kF16Out ? pack_f16(rx0, rx1) : pack_bf16(rx0, rx1);
+    h[w] = kF16Out ? pack_f16(ry0, ry1) : pack_bf16(ry0, ry1);
   }
 }
 
@@ -87,6 +92,9 @@ struct RopeQkParams {
 constexpr int kRopeTokensPerCta = 8;
 constexpr int kRopeThreads = 256;
 
+// q (Hq heads, may be 0) and k (Hkv heads) of TB tokens per CTA.  kF16Out:
+// fp16 results (k rotated once for the prefill kernel); otherwise bf16.
+template <bool kF16Out>
 __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_constant__ RopeQkParams p) {
   constexpr int TB = kRopeTokensPerCta;
   __shared__ float2 tab[TB][kPairs];
@@ -133,7 +141,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_cons
     }
     uint4 lo = *reinterpret_cast<const uint4*>(src + 8 * chunk);
     uint4 hi = *reinterpret_cast<const uint4*>(src + 32 + 8 * chunk);
-    rotate8(lo, hi, &tab[tt][8 * chunk]);
+    rotate8<kF16Out>(lo, hi, &tab[tt][8 * chunk]);
     *reinterpret_cast<uint4*>(dst + 8 * chunk) = lo;
     *reinterpret_cast<uint4*>(dst + 32 + 8 * chunk) = hi;
   }

@@ -116,9 +116,10 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
 /* gptoss_attn_fwd -- prefill sink attention, causal, full (window = 0) or
  * sliding window, BSHD or packed THD.
  *   q [B,S,Hq,D] / [T,Hq,D], k and v [B,S,Hkv,D] / [T,Hkv,D], bf16, own
- *          strides.  rope != NULL: q and k are raw and RoPE is applied inside
- *          the kernel as the tiles are loaded (the rotated values enter the
- *          QK^T product as fp16, so c * |x| must stay below 65504);
+ *          strides.  rope != NULL: q and k are raw; q is rotated inside the
+ *          kernel as its tiles are loaded, k likewise or once beforehand
+ *          (see workspace); the rotated values enter the QK^T product as
+ *          fp16, so c * |x| must stay below 65504;
  *          rope == NULL: q and k are already rotated (bf16 product).
  *   sinks  fp32 [Hq], in the units of the scaled logits (may be -inf).
  *   positions / cu_seqlens as for gptoss_rope_qk (positions only used when
@@ -129,13 +130,26 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
  *   window 0 = full causal; w > 0 = the last w keys including the query.
  *   softmax_scale  head_dim^-0.5 for GPT-OSS.
  *   out    bf16, q's logical shape, strides so.
- *   lse    fp32, nullable: [B,Hq,S] (BSHD) or [Hq,T] (THD), natural log. */
+ *   lse    fp32, nullable: [B,Hq,S] (BSHD) or [Hq,T] (THD), natural log.
+ *   workspace  nullable device memory of at least
+ *          gptoss_attn_fwd_workspace_size(total_tokens, Hkv, D) bytes, 16-byte
+ *          aligned, owned by the caller, contents need not be initialised;
+ *          only used when rope != NULL.  Given one, k is rotated once into it
+ *          (fp16, dense) by a first kernel on the same stream; without one,
+ *          every work unit rotates the k tiles it loads (same results, more
+ *          work per key).  A workspace that is too small or misaligned is
+ *          GPTOSS_ERR_INVALID_ARG. */
 gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
                               const void* v, gptoss_strides sv, const float* sinks,
                               const int32_t* positions, const int32_t* cu_seqlens, int32_t B,
                               int32_t S, int32_t total_tokens, int32_t Hq, int32_t Hkv, int32_t D,
                               int32_t window, float softmax_scale, const gptoss_rope_params* rope,
-                              void* out, gptoss_strides so, float* lse, struct CUstream_st* stream);
+                              void* out, gptoss_strides so, float* lse, void* workspace,
+                              size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Workspace bytes for gptoss_attn_fwd's rotated k: total_tokens x Hkv x D
+ * fp16 values.  0 when a size is out of range. */
+size_t gptoss_attn_fwd_workspace_size(int32_t total_tokens, int32_t Hkv, int32_t D);
 
 /* Workspace bytes gptoss_attn_decode needs for these sizes (split-KV
  * partial results).  0 when a size is out of range. */

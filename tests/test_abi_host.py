@@ -52,11 +52,11 @@ FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case fails validati
 def _fwd(lib, **kw):
     a = dict(q=FAKE, sq=S_BSHD_Q, k=FAKE, sk=S_BSHD_K, v=FAKE, sv=S_BSHD_K, sinks=FAKE, pos=None, cu=None, B=1,
              S=4096, T=4096, Hq=64, Hkv=8, D=64, window=0, scale=0.125, rope=ctypes.byref(ROPE), out=FAKE,
-             so=S_BSHD_Q, lse=None)
+             so=S_BSHD_Q, lse=None, ws=None, ws_bytes=0)
     a.update(kw)
     return lib.gptoss_attn_fwd(a["q"], a["sq"], a["k"], a["sk"], a["v"], a["sv"], a["sinks"], a["pos"], a["cu"],
                                a["B"], a["S"], a["T"], a["Hq"], a["Hkv"], a["D"], a["window"], a["scale"],
-                               a["rope"], a["out"], a["so"], a["lse"], None)
+                               a["rope"], a["out"], a["so"], a["lse"], a["ws"], a["ws_bytes"], None)
 
 
 def test_attn_fwd_validation(lib):
@@ -74,6 +74,11 @@ def test_attn_fwd_validation(lib):
     assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_UNSUPPORTED  # partial rotary
     bad_rope = _abi.RopeParams(150000.0, 32.0, 4096, 64, 32.0, 1.0)
     assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_INVALID_ARG  # alpha >= beta
+    # the rotated-k workspace: too small or misaligned
+    need = lib.gptoss_attn_fwd_workspace_size(4096, 8, 64)
+    assert need == 4096 * 8 * 64 * 2
+    assert _fwd(lib, ws=FAKE, ws_bytes=need - 16) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert _fwd(lib, ws=ctypes.c_void_p(0x10008), ws_bytes=need) == _abi.GPTOSS_ERR_INVALID_ARG
     # empty inputs are a successful no-op (nothing launched)
     assert _fwd(lib, B=0, T=0) == _abi.GPTOSS_OK
     assert _fwd(lib, S=0, T=0) == _abi.GPTOSS_OK

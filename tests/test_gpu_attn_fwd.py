@@ -41,16 +41,22 @@ def test_tiny_workload(cuda_device):
     assert_parity(host(lse), ref_lse, "tiny lse")
 
 
+# rope modes: k rotated once into the workspace, k tiles rotated inside the
+# kernel, or q and k rotated beforehand (no RoPE in the call)
+ROPE_MODES = ["k_once", "k_in_kernel", "prerotated"]
+
+
 @pytest.mark.parametrize("window", [0, 1, 128, 200, 1000])
-@pytest.mark.parametrize("fused_rope", [True, False])
-def test_bshd_multi_tile_ragged(cuda_device, window, fused_rope):
+@pytest.mark.parametrize("mode", ROPE_MODES)
+def test_bshd_multi_tile_ragged(cuda_device, window, mode):
     B, S, Hq, Hkv = 2, 300, 16, 2
     q, k, v = _rand((B, S, Hq, 64), 1), _rand((B, S, Hkv, 64), 2), _rand((B, S, Hkv, 64), 3)
     sinks = np.random.default_rng(4).standard_normal(Hq).astype(np.float32)
     tabs = _tables(GPTOSS_ROPE)
-    if fused_rope:
+    if mode != "prerotated":
         out, lse = ops.gptoss_attn_fwd(dev(q), dev(k), dev(v), f32(sinks), window=window,
-                                       rope=ops.RopeConfig.from_dict(GPTOSS_ROPE), return_lse=True)
+                                       rope=ops.RopeConfig.from_dict(GPTOSS_ROPE), return_lse=True,
+                                       rotate_k_once=mode == "k_once")
         torch.cuda.synchronize()
         ref, ref_lse = attn_fwd_bshd(q, k, v, sinks, 0.125, window, rope_tables=tabs)
     else:
@@ -78,7 +84,8 @@ def test_extreme_sinks(cuda_device, sink):
 
 
 @pytest.mark.parametrize("window", [0, 128])
-def test_thd_ragged_sequences(cuda_device, window):
+@pytest.mark.parametrize("k_once", [True, False])
+def test_thd_ragged_sequences(cuda_device, window, k_once):
     lens = [1, 129, 300, 77, 128, 256]
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     T, Hq, Hkv = int(cu[-1]), 16, 2
@@ -86,14 +93,15 @@ def test_thd_ragged_sequences(cuda_device, window):
     sinks = np.random.default_rng(24).standard_normal(Hq).astype(np.float32)
     out, lse = ops.gptoss_attn_fwd(dev(q), dev(k), dev(v), f32(sinks), window=window, cu_seqlens=i32(cu),
                                    max_seqlen=max(lens), rope=ops.RopeConfig.from_dict(GPTOSS_ROPE),
-                                   return_lse=True)
+                                   return_lse=True, rotate_k_once=k_once)
     torch.cuda.synchronize()
     ref, ref_lse = attn_fwd_thd(q, k, v, sinks, cu, 0.125, window, rope_tables=_tables(GPTOSS_ROPE))
     assert_parity(host(out), ref, "thd out")
     assert_parity(host(lse), ref_lse, "thd lse")
 
 
-def test_explicit_positions_and_strided_io(cuda_device):
+@pytest.mark.parametrize("k_once", [True, False])
+def test_explicit_positions_and_strided_io(cuda_device, k_once):
     # q/k/v as views of one fused buffer; output into a strided view; positions offset by a prefix
     B, S, Hq, Hkv = 2, 200, 8, 2
     qkv = _rand((B, S, Hq + 2 * Hkv, 64), 31)
@@ -104,7 +112,7 @@ def test_explicit_positions_and_strided_io(cuda_device):
     big = torch.zeros((B, S, Hq + 8, 64), dtype=torch.bfloat16, device=cuda_device)
     out = big[:, :, 4:4 + Hq]
     ops.gptoss_attn_fwd(q, k, v, f32(sinks), window=128, rope=ops.RopeConfig.from_dict(GPTOSS_ROPE),
-                        positions=i32(pos), out=out)
+                        positions=i32(pos), out=out, rotate_k_once=k_once)
     torch.cuda.synchronize()
     ref, _ = attn_fwd_bshd(qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:], sinks, 0.125, 128,
                            rope_tables=_tables(GPTOSS_ROPE), positions=pos)
