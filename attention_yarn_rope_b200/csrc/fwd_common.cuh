@@ -63,6 +63,7 @@ struct FwdParams {
   const int32_t* cu_seqlens;
   int B, S, T, Hq, Hkv, G, HP, window, n_qtiles, n_units;
   int k_in_kernel;  // 1: K tiles are rotated in shared memory; 0: k arrives rotated (or RoPE is off)
+  const float2* cs_tab;  // nullable: per-token (c cos, c sin) of the 32 pairs, [token][32]
   float scale_log2;
   uint64_t wait_ns;
   RopeTable tab;

@@ -56,6 +56,49 @@ __device__ __forceinline__ void rotate_tile(const FwdParams& p, const RopeLane& 
   }
 }
 
+// Rotates the 16 rows this thread owns in BOTH Q tiles of a unit: the two
+// heads share every row's angle, so each angle is formed once.  Angles as in
+// rotate_tile; with a per-token table (row_cs != nullptr, row r's 32
+// (c cos, c sin) pairs at row_cs[16 r .. 16 r + 15] as float4) explicit
+// positions read their row's angles instead of forming them.
+__device__ __forceinline__ void rotate_q_pair(const FwdParams& p, const RopeLane& rl, uint8_t* ta, uint8_t* tb,
+                                              float2 c0, float2 c1, int n_valid, const int32_t* pos_row0,
+                                              const float4* row_cs, int pb) {
+  const bool explicit_pos = pos_row0 != nullptr;
+#pragma unroll 4
+  for (int kk = 0; kk < 16; ++kk) {
+    const int r = rl.ro + 8 * kk;
+    if (r < n_valid) {
+      if (explicit_pos) {
+        if (row_cs != nullptr) {
+          const float4 v = __ldg(row_cs + 16 * r + pb);
+          c0 = make_float2(v.x, v.y);
+          c1 = make_float2(v.z, v.w);
+        } else {
+          const int pos = __ldg(pos_row0 + r);
+          c0 = rope_cs(pos, rl.f0, p.tab.conc);
+          c1 = rope_cs(pos, rl.f1, p.tab.conc);
+        }
+      }
+      uint32_t* pa_lo = reinterpret_cast<uint32_t*>(ta + rl.w_lo + kk * 1024);
+      uint32_t* pa_hi = reinterpret_cast<uint32_t*>(ta + rl.w_hi + kk * 1024);
+      uint32_t* pb_lo = reinterpret_cast<uint32_t*>(tb + rl.w_lo + kk * 1024);
+      uint32_t* pb_hi = reinterpret_cast<uint32_t*>(tb + rl.w_hi + kk * 1024);
+      uint32_t alo = *pa_lo, ahi = *pa_hi, blo = *pb_lo, bhi = *pb_hi;
+      rotate_words(alo, ahi, c0, c1);
+      rotate_words(blo, bhi, c0, c1);
+      *pa_lo = alo;
+      *pa_hi = ahi;
+      *pb_lo = blo;
+      *pb_hi = bhi;
+    }
+    if (!explicit_pos) {
+      c0 = cmul(c0, rl.step0);
+      c1 = cmul(c1, rl.step1);
+    }
+  }
+}
+
 __device__ __forceinline__ void fwd_rope_role(const FwdParams& p, FwdSmem& sm) {
   const int rt = threadIdx.x;  // warps 0-3
   const int w = rt >> 5, l = rt & 31;
@@ -90,13 +133,22 @@ __device__ __forceinline__ void fwd_rope_role(const FwdParams& p, FwdSmem& sm) {
     if (!mbar_wait_warp(&sm.q_loaded[qb], (i >> 1) & 1, p.wait_ns)) return;
     if (rot) {
       const int n_valid = min(kFwdTile, wu.L - wu.q0);
+      // the unit's first query token; its rows' angles in the per-token table
+      const int64_t tok_q0 = (thd ? wu.seq_start : static_cast<int64_t>(wu.b) * p.S) + wu.q0;
+      const float4* row_cs = p.cs_tab != nullptr ? reinterpret_cast<const float4*>(p.cs_tab + tok_q0 * kPairs) : nullptr;
       float2 c0 = one, c1 = one;
-      if (!explicit_pos) {  // one double-precision seed serves both heads' tiles
-        c0 = rope_cs(wu.q0 + rl.ro, rl.f0, p.tab.conc);
-        c1 = rope_cs(wu.q0 + rl.ro, rl.f1, p.tab.conc);
+      if (!explicit_pos && rl.ro < n_valid) {  // one seed for row ro serves both heads' tiles
+        if (row_cs != nullptr) {  // (a thread without a valid row rotates nothing and reads no table row)
+          const float4 v = __ldg(row_cs + 16 * rl.ro + pb);
+          c0 = make_float2(v.x, v.y);
+          c1 = make_float2(v.z, v.w);
+        } else {
+          c0 = rope_cs(wu.q0 + rl.ro, rl.f0, p.tab.conc);
+          c1 = rope_cs(wu.q0 + rl.ro, rl.f1, p.tab.conc);
+        }
       }
-      for (int X = 0; X < 2; ++X)
-        rotate_tile(p, rl, sm.q[qb][X], c0, c1, n_valid, explicit_pos ? pos_seq + wu.q0 : nullptr);
+      rotate_q_pair(p, rl, sm.q[qb][0], sm.q[qb][1], c0, c1, n_valid, explicit_pos ? pos_seq + wu.q0 : nullptr,
+                    row_cs, pb);
       fence_proxy_async_smem();
     }
     mbar_arrive(&sm.q_full[qb]);

@@ -92,6 +92,7 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
   if (!strides_ok(sq, !thd) || !strides_ok(sk, !thd) || !strides_ok(sq_out, !thd) || !strides_ok(sk_out, !thd))
     return GPTOSS_ERR_INVALID_ARG;
   RopeQkParams p;
+  memset(&p, 0, sizeof(p));  // no angle table output (cs_out = nullptr)
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k = static_cast<const __nv_bfloat16*>(k);
   p.q_out = static_cast<__nv_bfloat16*>(q_out);
@@ -113,9 +114,15 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
   return check_launch();
 }
 
+// Workspace of gptoss_attn_fwd: rotated k (fp16, [token][Hkv][64]), then at a
+// 256-byte boundary each token's 32 (c cos, c sin) pairs ([token][32] float2).
+static size_t fwd_ws_k_bytes(int32_t total_tokens, int32_t Hkv) {
+  return (static_cast<size_t>(total_tokens) * Hkv * kHeadDim * 2 + 255) & ~static_cast<size_t>(255);
+}
+
 size_t gptoss_attn_fwd_workspace_size(int32_t total_tokens, int32_t Hkv, int32_t D) {
   if (total_tokens < 0 || Hkv <= 0 || D != kHeadDim) return 0;
-  return static_cast<size_t>(total_tokens) * Hkv * kHeadDim * 2;  // fp16
+  return fwd_ws_k_bytes(total_tokens, Hkv) + static_cast<size_t>(total_tokens) * kPairs * sizeof(float2);
 }
 
 gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk, const void* v,
@@ -224,6 +231,8 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
     rp.Hq = 0;
     rp.Hkv = Hkv;
     rp.tab = p.tab;
+    rp.cs_out = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + fwd_ws_k_bytes(total_tokens, Hkv));
+    p.cs_tab = rp.cs_out;
     const int rgrid = (total_tokens + kRopeTokensPerCta - 1) / kRopeTokensPerCta;
     rope_qk_kernel<true><<<rgrid, kRopeThreads, 0, as_stream(stream)>>>(rp);
     st = check_launch();

@@ -87,6 +87,7 @@ struct RopeQkParams {
   TokenMap tm;
   int Hq, Hkv;
   RopeTable tab;
+  float2* cs_out;  // nullable: each token's 32 (c cos, c sin) pairs, [token][32]
 };
 
 constexpr int kRopeTokensPerCta = 8;
@@ -109,6 +110,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_cons
       token_coords(p.tm, t, seq, idx);
       const int pos = p.tm.positions ? __ldg(p.tm.positions + t) : idx;
       tab[tt][j] = rope_cs(pos, p.tab.inv_freq[j], p.tab.conc);
+      if (p.cs_out != nullptr) p.cs_out[static_cast<int64_t>(t) * kPairs + j] = tab[tt][j];
       if (j == 0) {
         const bool thd = p.tm.cu_seqlens != nullptr;
         const int64_t b = thd ? 0 : seq;

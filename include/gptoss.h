@@ -134,10 +134,12 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
  *   workspace  nullable device memory of at least
  *          gptoss_attn_fwd_workspace_size(total_tokens, Hkv, D) bytes, 16-byte
  *          aligned, owned by the caller, contents need not be initialised;
- *          only used when rope != NULL.  Given one, k is rotated once into it
- *          (fp16, dense) by a first kernel on the same stream; without one,
- *          every work unit rotates the k tiles it loads (same results, more
- *          work per key).  A workspace that is too small or misaligned is
+ *          only used when rope != NULL.  Given one, a first kernel on the
+ *          same stream rotates k once into it (fp16, dense) and stores every
+ *          token's 32 RoPE angles (c cos, c sin), which the attention kernel
+ *          reads for q; without one, every work unit rotates the k tiles it
+ *          loads and forms the angles itself (same results, more work per
+ *          key).  A workspace that is too small or misaligned is
  *          GPTOSS_ERR_INVALID_ARG. */
 gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
                               const void* v, gptoss_strides sv, const float* sinks,
@@ -147,8 +149,9 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
                               void* out, gptoss_strides so, float* lse, void* workspace,
                               size_t workspace_bytes, struct CUstream_st* stream);
 
-/* Workspace bytes for gptoss_attn_fwd's rotated k: total_tokens x Hkv x D
- * fp16 values.  0 when a size is out of range. */
+/* Workspace bytes for gptoss_attn_fwd: the rotated k (total_tokens x Hkv x D
+ * fp16 values, rounded up to 256 bytes) and the angle table (total_tokens x
+ * 32 fp32 pairs).  0 when a size is out of range. */
 size_t gptoss_attn_fwd_workspace_size(int32_t total_tokens, int32_t Hkv, int32_t D);
 
 /* Workspace bytes gptoss_attn_decode needs for these sizes (split-KV

@@ -76,7 +76,7 @@ def test_attn_fwd_validation(lib):
     assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_INVALID_ARG  # alpha >= beta
     # the rotated-k workspace: too small or misaligned
     need = lib.gptoss_attn_fwd_workspace_size(4096, 8, 64)
-    assert need == 4096 * 8 * 64 * 2
+    assert need == 4096 * 8 * 64 * 2 + 4096 * 32 * 8  # rotated k + per-token angle table
     assert _fwd(lib, ws=FAKE, ws_bytes=need - 16) == _abi.GPTOSS_ERR_INVALID_ARG
     assert _fwd(lib, ws=ctypes.c_void_p(0x10008), ws_bytes=need) == _abi.GPTOSS_ERR_INVALID_ARG
     # empty inputs are a successful no-op (nothing launched)
