@@ -15,7 +15,9 @@
 // heads as the 16-row M side), an online softmax per head with quad shuffles,
 // and fp32 accumulators in registers.  The CTA writes an unnormalised partial
 // (m, l, O) per head; a second kernel merges the splits of each (b, g) and
-// folds exp(sink) into the denominator exactly once.
+// folds exp(sink) into the denominator exactly once.  When every sequence has
+// a single split (a short window: 128 keys per sequence and kv head), the
+// split kernel folds the sink itself and writes the output: one launch.
 #pragma once
 
 #include "host_util.cuh"
@@ -44,6 +46,7 @@ struct DecodeParams {
   float* ws_o;             // [B, Hkv, nsplit, G, 64]
   float* ws_ml;            // [B, Hkv, nsplit, G, 2]
   int B, Lmax, Hq, Hkv, G, window, chunk, nsplit;
+  int direct;  // one split per sequence: fold the sink and write out / lse here, no merge launch
   float scale_log2;
   uint64_t wait_ns;
   RopeTable tab;
@@ -107,7 +110,16 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   const int lo = p.window > 0 ? max(0, n - p.window) : 0;
   const int k_begin = lo + split * p.chunk;
   const int k_end = min(n, k_begin + p.chunk);
-  if (k_begin >= k_end) return;  // this split is past the sequence: the merge skips it
+  if (k_begin >= k_end) {  // this split is past the sequence: the merge skips it
+    if (p.direct) {        // (only an empty cache reaches here): the sink alone, O = 0
+      for (int idx = threadIdx.x; idx < p.G * kHeadDim; idx += kDecThreads) {
+        const int head = g * p.G + idx / kHeadDim;
+        p.out[(static_cast<int64_t>(b) * p.Hq + head) * kHeadDim + idx % kHeadDim] = __float2bfloat16_rn(0.f);
+        if (p.lse != nullptr && idx % kHeadDim == 0) p.lse[static_cast<int64_t>(b) * p.Hq + head] = __ldg(p.sinks + head);
+      }
+    }
+    return;
+  }
   const int ntile = (k_end - k_begin + kDecTileKeys - 1) / kDecTileKeys;
   const int G = p.G;
 
@@ -296,6 +308,22 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       acc.y += wo[w][h][d4 + 1] * sc;
       acc.z += wo[w][h][d4 + 2] * sc;
       acc.w += wo[w][h][d4 + 3] * sc;
+    }
+    if (p.direct) {
+      // the only split of this (b, g): fold exp(sink) here as the merge would
+      const int head = g * G + h;
+      const float sink = __ldg(p.sinks + head) * kLog2e;
+      const float Mt = fmaxf(M, sink);
+      const float Mts = Mt == -INFINITY ? 0.f : Mt;
+      const float sc = M == -INFINITY ? 0.f : ex2_approx(M - Mts);
+      const float Lt = L * sc + ex2_approx(sink - Mts);
+      const float inv = sc / Lt;
+      uint2 r;
+      r.x = pack_bf16(acc.x * inv, acc.y * inv);
+      r.y = pack_bf16(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(p.out + (static_cast<int64_t>(b) * p.Hq + head) * kHeadDim + d4) = r;
+      if (p.lse != nullptr && d4 == 0) p.lse[static_cast<int64_t>(b) * p.Hq + head] = (Mt + log2f(Lt)) * kLn2;
+      continue;
     }
     const int64_t slot = ((static_cast<int64_t>(b) * p.Hkv + g) * p.nsplit + split) * G + h;
     *reinterpret_cast<float4*>(p.ws_o + slot * kHeadDim + d4) = acc;

@@ -130,7 +130,7 @@ __device__ __forceinline__ void fwd_rope_role(const FwdParams& p, FwdSmem& sm) {
     const int32_t* pos_seq =
         explicit_pos ? p.positions + (thd ? wu.seq_start : static_cast<int64_t>(wu.b) * p.S) : nullptr;
     // ---- the unit's two Q tiles ----
-    if (!mbar_wait_warp(&sm.q_loaded[qb], (i >> 1) & 1, p.wait_ns)) return;
+    if (!mbar_wait_warp_relaxed(&sm.q_loaded[qb], (i >> 1) & 1, p.wait_ns)) return;
     if (rot) {
       const int n_valid = min(kFwdTile, wu.L - wu.q0);
       // the unit's first query token; its rows' angles in the per-token table
@@ -162,7 +162,7 @@ __device__ __forceinline__ void fwd_rope_role(const FwdParams& p, FwdSmem& sm) {
     }
     for (int j = 0; j < wu.n_kt; ++j, ++kv_it) {
       const int s = kv_it % kFwdStages;
-      if (!mbar_wait_warp(&sm.k_full[s], (kv_it / kFwdStages) & 1, p.wait_ns)) return;
+      if (!mbar_wait_warp_relaxed(&sm.k_full[s], (kv_it / kFwdStages) & 1, p.wait_ns)) return;
       {
         const int k0 = (wu.j_lo + j) * kFwdTile;
         rotate_tile(p, rl, sm.k[s], k0s, k1s, min(kFwdTile, wu.L - k0), explicit_pos ? pos_seq + k0 : nullptr);

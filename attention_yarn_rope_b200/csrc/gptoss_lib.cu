@@ -305,6 +305,7 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
   p.window = window;
   p.chunk = chunk;
   p.nsplit = nsplit_max;
+  p.direct = nsplit == 1;  // e.g. window 128: one split per (sequence, kv head)
   p.scale_log2 = softmax_scale * kLog2e;
   p.wait_ns = wait_limit_ns();
   if (rope != nullptr) yarn_table(*rope, &p.tab);
@@ -316,6 +317,7 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
   cudaStream_t s = as_stream(stream);
   attn_decode_split_kernel<<<dim3(Hkv, nsplit, B), kDecThreads, smem, s>>>(p);
   if (check_launch() != GPTOSS_OK) return GPTOSS_ERR_CUDA;
+  if (p.direct) return GPTOSS_OK;
   attn_decode_merge_kernel<<<dim3(Hkv, B), 256, 0, s>>>(p);
   return check_launch();
 }

@@ -80,6 +80,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
   }
 }
 
+// mbar_wait for warps with slack (work queued well ahead of its consumer):
+// sleeps ~256 ns between polls so the poll leaves issue slots to the warps on
+// the critical path.  Measured on the prefill rope warps: 1-2 % faster.
+__device__ __forceinline__ bool mbar_wait_relaxed(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  const long long limit_cycles = static_cast<long long>(limit_ns) * 2;
+  while (true) {
+    __nanosleep(256);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > limit_cycles) {
+      record_timeout();
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ bool mbar_wait_warp_relaxed(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const bool ok = mbar_wait_relaxed(bar, parity, limit_ns);
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
 // Warp-uniform wait: every lane polls (each acquires the barrier) and the
 // warp proceeds only if all lanes saw the phase complete, so warp-collective
 // tcgen05 instructions after it always run converged.

@@ -350,7 +350,8 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
         gbs = case["bytes"] / (ms * 1e-3) / 1e9
         res[cfg.name] = {"ms": round(ms, 4), "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
                          "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": case["kv_bytes"],
-                         "l2": "flushed between calls" if small else "cache > L2", "launches_per_call": 2}
+                         "l2": "flushed between calls" if small else "cache > L2",
+                         "launches_per_call": 1 if cfg.window and cfg.window <= 256 else 2}
         del case
         torch.cuda.empty_cache()
     return res
