@@ -35,6 +35,8 @@ EXPORTED = (
     "gptoss_attn_decode_workspace_size",
     "gptoss_attn_decode",
     "gptoss_attn_decode_noalloc",
+    "gptoss_attn_decode_paged",
+    "gptoss_kv_append_paged",
     "gptoss_read_device_status",
     "gptoss_set_wait_limit",
     "gptoss_selftest_wait_timeout",
@@ -75,6 +77,11 @@ _SIGNATURES = {
                                  ctypes.POINTER(RopeParams), _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "gptoss_attn_decode_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                          ctypes.POINTER(RopeParams), _vp, _vp, _vp]),
+    "gptoss_attn_decode_paged": (_st, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32,
+                                       _i32, _f32, ctypes.POINTER(RopeParams), _vp, _vp, _vp, ctypes.c_size_t,
+                                       _vp]),
+    "gptoss_kv_append_paged": (_st, [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32,
+                                     ctypes.POINTER(RopeParams), _vp]),
     "gptoss_read_device_status": (_st, [ctypes.POINTER(_i32), _i32, _vp]),
     "gptoss_set_wait_limit": (_st, [_u32]),
     "gptoss_selftest_wait_timeout": (_st, [_u32, _vp, _vp]),

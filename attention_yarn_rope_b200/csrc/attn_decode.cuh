@@ -18,6 +18,9 @@
 // folds exp(sink) into the denominator exactly once.  When every sequence has
 // a single split (a short window: 128 keys per sequence and kv head), the
 // split kernel folds the sink itself and writes the output: one launch.
+// The same kernel reads a paged cache through a block table (the producer maps
+// each 64-key tile to its block's rows); kv_append_paged_kernel writes a new
+// token into such a cache.
 #pragma once
 
 #include "host_util.cuh"
@@ -47,6 +50,11 @@ struct DecodeParams {
   float* ws_ml;            // [B, Hkv, nsplit, G, 2]
   int B, Lmax, Hq, Hkv, G, window, chunk, nsplit;
   int direct;  // one split per sequence: fold the sink and write out / lse here, no merge launch
+  // paged cache (block_table != nullptr): the K / V tensor maps cover the pools
+  // [num_blocks * block_size, Hkv, 64]; token p of sequence b is row
+  // block_table[b * max_blocks + p / block_size] * block_size + p % block_size
+  const int32_t* block_table;
+  int max_blocks, block_size, num_blocks;
   float scale_log2;
   uint64_t wait_ns;
   RopeTable tab;
@@ -110,6 +118,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   const int lo = p.window > 0 ? max(0, n - p.window) : 0;
   const int k_begin = lo + split * p.chunk;
   const int k_end = min(n, k_begin + p.chunk);
+  // paged: tiles start on 64-key boundaries (block_size is a multiple of 64,
+  // so a tile never straddles two blocks); keys before k_begin are masked
+  const int k_tile0 = p.block_table != nullptr ? (k_begin & ~(kDecTileKeys - 1)) : k_begin;
   if (k_begin >= k_end) {  // this split is past the sequence: the merge skips it
     if (p.direct) {        // (only an empty cache reaches here): the sink alone, O = 0
       for (int idx = threadIdx.x; idx < p.G * kHeadDim; idx += kDecThreads) {
@@ -120,7 +131,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
     }
     return;
   }
-  const int ntile = (k_end - k_begin + kDecTileKeys - 1) / kDecTileKeys;
+  const int ntile = (k_end - k_tile0 + kDecTileKeys - 1) / kDecTileKeys;
   const int G = p.G;
 
   if (threadIdx.x == 0) {
@@ -160,9 +171,19 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
         const int s = it % kDecStages;
         if (!mbar_wait(&sm.empty[s], ((it / kDecStages) & 1) ^ 1, p.wait_ns)) break;
         mbar_arrive_expect_tx(&sm.full[s], 2 * kDecTileBytes);
-        const int key0 = k_begin + it * kDecTileKeys;
-        tma_load_4d(sm.k[s], &p.tmap_k, &sm.full[s], 0, g, key0, b);
-        tma_load_4d(sm.v[s], &p.tmap_v, &sm.full[s], 0, g, key0, b);
+        const int key0 = k_tile0 + it * kDecTileKeys;
+        int row = key0, bat = b;
+        if (p.block_table != nullptr) {
+          // a block index outside the pool (or a length past the table) reads
+          // the tensor map's zero fill: the row coordinate is put past its end
+          const int j = key0 / p.block_size;
+          const int blk = j < p.max_blocks ? __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks + j) : -1;
+          row = (blk >= 0 && blk < p.num_blocks) ? blk * p.block_size + key0 % p.block_size
+                                                  : p.num_blocks * p.block_size;
+          bat = 0;
+        }
+        tma_load_4d(sm.k[s], &p.tmap_k, &sm.full[s], 0, g, row, bat);
+        tma_load_4d(sm.v[s], &p.tmap_v, &sm.full[s], 0, g, row, bat);
       }
       // drain: every issued stage must land before the CTA may exit
       const int first = ntile > kDecStages ? ntile - kDecStages : 0;
@@ -210,14 +231,14 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
         mma_bf16_16816(sc[nb], qa[2 * kp + 1], b2, b3);
       }
     }
-    // mask keys past the chunk, scale into log2 units
-    const int key_base = k_begin + it * kDecTileKeys + r0;
+    // mask keys outside the chunk, scale into log2 units
+    const int key_base = k_tile0 + it * kDecTileKeys + r0;
 #pragma unroll
     for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int key = key_base + nb * 8 + 2 * tq + (e & 1);
-        sc[nb][e] = key < k_end ? sc[nb][e] * p.scale_log2 : -INFINITY;
+        sc[nb][e] = (key >= k_begin && key < k_end) ? sc[nb][e] * p.scale_log2 : -INFINITY;
       }
     // online softmax, rows gr (e = 0, 1) and gr + 8 (e = 2, 3)
     float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
@@ -249,6 +270,18 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       o[dt][2] *= a1;
       o[dt][3] *= a1;
     }
+    // Rows of this warp past the sequence end get P = 0, but 0 x NaN is NaN:
+    // those rows of a cache (a paged pool's unused rows above all) may hold
+    // anything, so the warp zeroes its own V rows there before P V.
+    const bool tail = key_base + 15 >= k_end;
+    if (tail) {
+      for (int idx = lane; idx < 16 * 8; idx += 32) {  // 16 rows x 8 chunks of 16 bytes
+        const int rr = idx >> 3, ch = idx & 7;
+        if (key_base + rr >= k_end)
+          *reinterpret_cast<uint4*>(sm.v[s] + (r0 + rr) * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
+    }
     // P as the A operand (16 heads x 16 keys)
     uint32_t pa[4];
     pa[0] = pack_bf16(pr[0][0], pr[0][1]);
@@ -264,6 +297,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       mma_bf16_16816(o[2 * dp], pa, v0, v1);
       mma_bf16_16816(o[2 * dp + 1], pa, v2, v3);
     }
+    if (tail) fence_proxy_async_smem();  // the zeroed rows before the next TMA write of the stage
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[s]);
   }
@@ -366,6 +400,48 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_con
     *reinterpret_cast<__nv_bfloat162*>(p.out + (static_cast<int64_t>(b) * p.Hq + head) * kHeadDim + d2) = r;
     if (p.lse != nullptr && d2 == 0) p.lse[static_cast<int64_t>(b) * p.Hq + head] = (M + log2f(L)) * kLn2;
   }
+}
+
+// KV-cache append: sequence b's new token (position cache_seqlens[b] - 1)
+// into a paged cache -- the key rotated (the cache holds post-RoPE keys,
+// bf16), the value as given.  Block (b), thread (g, j): pair j of kv head g.
+struct AppendParams {
+  const __nv_bfloat16* k_new;  // [B, Hkv, 64]
+  const __nv_bfloat16* v_new;
+  const int32_t* seqlens;      // [B]
+  const int32_t* block_table;  // [B, max_blocks]
+  __nv_bfloat16* k_pool;       // [num_blocks * block_size, Hkv, 64]
+  __nv_bfloat16* v_pool;
+  int B, Hkv, max_blocks, block_size, num_blocks;
+  RopeTable tab;
+};
+
+constexpr int kStatusBadIndex = 1;  // == GPTOSS_ERR_INVALID_ARG
+
+__global__ void kv_append_paged_kernel(const __grid_constant__ AppendParams p) {
+  const int b = blockIdx.x;
+  const int g = threadIdx.x / kPairs, j = threadIdx.x % kPairs;
+  const int pos = __ldg(p.seqlens + b) - 1;
+  const int jb = pos >= 0 ? pos / p.block_size : -1;
+  const int blk = (jb >= 0 && jb < p.max_blocks) ? __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks + jb) : -1;
+  if (blk < 0 || blk >= p.num_blocks) {  // nothing is written outside the pool
+    if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusBadIndex);
+    return;
+  }
+  const int64_t off = (static_cast<int64_t>(blk) * p.block_size + pos % p.block_size) * p.Hkv * kHeadDim +
+                      static_cast<int64_t>(g) * kHeadDim;
+  const int64_t src = (static_cast<int64_t>(b) * p.Hkv + g) * kHeadDim;
+  float x = __bfloat162float(p.k_new[src + j]), y = __bfloat162float(p.k_new[src + j + kPairs]);
+  if (p.tab.enabled) {
+    const float2 cs = rope_cs(pos, p.tab.inv_freq[j], p.tab.conc);
+    const float xr = x * cs.x - y * cs.y, yr = y * cs.x + x * cs.y;
+    x = xr;
+    y = yr;
+  }
+  p.k_pool[off + j] = __float2bfloat16_rn(x);
+  p.k_pool[off + j + kPairs] = __float2bfloat16_rn(y);
+  p.v_pool[off + j] = p.v_new[src + j];
+  p.v_pool[off + j + kPairs] = p.v_new[src + j + kPairs];
 }
 
 }  // namespace gptoss

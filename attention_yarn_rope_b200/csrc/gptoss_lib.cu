@@ -254,11 +254,23 @@ size_t gptoss_attn_decode_workspace_size(int32_t B, int32_t Lmax, int32_t Hq, in
   return static_cast<size_t>(slots * (kHeadDim + 2) * sizeof(float));
 }
 
-gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void* v_cache,
-                                 const int32_t* cache_seqlens, const float* sinks, int32_t B, int32_t Lmax,
-                                 int32_t Hq, int32_t Hkv, int32_t D, int32_t window, float softmax_scale,
-                                 const gptoss_rope_params* rope, void* out, float* lse, void* workspace,
-                                 size_t workspace_bytes, struct CUstream_st* stream) {
+}  // extern "C"
+
+namespace {
+
+// A paged cache: pools [num_blocks * block_size, Hkv, 64] and the block table.
+struct PagedLayout {
+  const int32_t* table;
+  int32_t max_blocks, block_size, num_blocks;
+};
+
+// Decode over a contiguous cache [B, Lmax, Hkv, 64] (paged == nullptr) or a
+// paged one (Lmax = max_blocks * block_size, the caches are the pools).
+gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_seqlens,
+                          const float* sinks, int32_t B, int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D,
+                          int32_t window, float softmax_scale, const gptoss_rope_params* rope, void* out,
+                          float* lse, void* workspace, size_t workspace_bytes, struct CUstream_st* stream,
+                          const PagedLayout* paged) {
   if (B < 0 || Lmax <= 0 || Hq <= 0 || Hkv <= 0 || window < 0) return GPTOSS_ERR_INVALID_ARG;
   if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
   if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
@@ -272,23 +284,29 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
     return GPTOSS_ERR_INVALID_ARG;
   const size_t need = gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D);
   if (need == 0 || workspace_bytes < need) return GPTOSS_ERR_INVALID_ARG;
-  const int64_t max_b = static_cast<int64_t>(B) * Lmax * Hkv * kHeadDim;
-  if (max_b > (int64_t(1) << 40)) return GPTOSS_ERR_UNSUPPORTED;
+  const int64_t rows = paged ? static_cast<int64_t>(paged->num_blocks) * paged->block_size
+                             : static_cast<int64_t>(B) * Lmax;
+  if (rows * Hkv * kHeadDim > (int64_t(1) << 40)) return GPTOSS_ERR_UNSUPPORTED;
 
   DecodeParams p;
   memset(&p, 0, sizeof(p));
   const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
-  const uint64_t bat_b = tok_b * Lmax;
-  st = make_tmap_4d(&p.tmap_k, k_cache, kHeadDim, Hkv, Lmax, B, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
-                         kDecTileKeys, 1);
+  // contiguous: (d, head, slot, sequence); paged: (d, head, pool row, 1)
+  const uint64_t d2 = paged ? static_cast<uint64_t>(rows) : static_cast<uint64_t>(Lmax);
+  const uint64_t d3 = paged ? 1 : static_cast<uint64_t>(B);
+  const uint64_t bat_b = paged ? tok_b * d2 : tok_b * Lmax;
+  st = make_tmap_4d(&p.tmap_k, k_cache, kHeadDim, Hkv, d2, d3, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
+                    kDecTileKeys, 1);
   if (st != GPTOSS_OK) return st;
-  st = make_tmap_4d(&p.tmap_v, v_cache, kHeadDim, Hkv, Lmax, B, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
-                         kDecTileKeys, 1);
+  st = make_tmap_4d(&p.tmap_v, v_cache, kHeadDim, Hkv, d2, d3, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
+                    kDecTileKeys, 1);
   if (st != GPTOSS_OK) return st;
   const int G = Hq / Hkv;
   const int chunk = decode_chunk(B, Lmax, Hkv);
   const int nsplit_max = (Lmax + chunk - 1) / chunk;
   const int span = window > 0 ? (window < Lmax ? window : Lmax) : Lmax;
+  // a window that does not start on a 64-key boundary may touch one more tile,
+  // still inside one split: chunks are multiples of 64 keys and at least 256
   const int nsplit = (span + chunk - 1) / chunk;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -306,6 +324,12 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
   p.chunk = chunk;
   p.nsplit = nsplit_max;
   p.direct = nsplit == 1;  // e.g. window 128: one split per (sequence, kv head)
+  if (paged) {
+    p.block_table = paged->table;
+    p.max_blocks = paged->max_blocks;
+    p.block_size = paged->block_size;
+    p.num_blocks = paged->num_blocks;
+  }
   p.scale_log2 = softmax_scale * kLog2e;
   p.wait_ns = wait_limit_ns();
   if (rope != nullptr) yarn_table(*rope, &p.tab);
@@ -319,6 +343,74 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
   if (check_launch() != GPTOSS_OK) return GPTOSS_ERR_CUDA;
   if (p.direct) return GPTOSS_OK;
   attn_decode_merge_kernel<<<dim3(Hkv, B), 256, 0, s>>>(p);
+  return check_launch();
+}
+
+gptoss_status check_paged(int32_t max_blocks, int32_t block_size, int32_t num_blocks) {
+  if (max_blocks <= 0 || block_size <= 0 || num_blocks <= 0) return GPTOSS_ERR_INVALID_ARG;
+  if (block_size % kDecTileKeys) return GPTOSS_ERR_UNSUPPORTED;  // 64-key tiles must not straddle blocks
+  if (static_cast<int64_t>(num_blocks) * block_size >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(max_blocks) * block_size >= (int64_t(1) << 31))
+    return GPTOSS_ERR_UNSUPPORTED;
+  return GPTOSS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* cache_seqlens, const float* sinks, int32_t B, int32_t Lmax,
+                                 int32_t Hq, int32_t Hkv, int32_t D, int32_t window, float softmax_scale,
+                                 const gptoss_rope_params* rope, void* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, struct CUstream_st* stream) {
+  return decode_impl(q, k_cache, v_cache, cache_seqlens, sinks, B, Lmax, Hq, Hkv, D, window, softmax_scale, rope,
+                     out, lse, workspace, workspace_bytes, stream, nullptr);
+}
+
+gptoss_status gptoss_attn_decode_paged(const void* q, const void* k_pool, const void* v_pool,
+                                       const int32_t* block_table, int32_t max_blocks, int32_t block_size,
+                                       int32_t num_blocks, const int32_t* cache_seqlens, const float* sinks,
+                                       int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t window,
+                                       float softmax_scale, const gptoss_rope_params* rope, void* out, float* lse,
+                                       void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
+  gptoss_status st = check_paged(max_blocks, block_size, num_blocks);
+  if (st != GPTOSS_OK) return st;
+  if (B > 0 && block_table == nullptr) return GPTOSS_ERR_INVALID_ARG;
+  const PagedLayout layout{block_table, max_blocks, block_size, num_blocks};
+  return decode_impl(q, k_pool, v_pool, cache_seqlens, sinks, B, max_blocks * block_size, Hq, Hkv, D, window,
+                     softmax_scale, rope, out, lse, workspace, workspace_bytes, stream, &layout);
+}
+
+gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const int32_t* cache_seqlens,
+                                     const int32_t* block_table, int32_t max_blocks, int32_t block_size,
+                                     void* k_pool, void* v_pool, int32_t num_blocks, int32_t B, int32_t Hkv,
+                                     int32_t D, const gptoss_rope_params* rope, struct CUstream_st* stream) {
+  if (B < 0 || Hkv <= 0) return GPTOSS_ERR_INVALID_ARG;
+  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (Hkv * kPairs > 1024) return GPTOSS_ERR_UNSUPPORTED;
+  gptoss_status st = check_paged(max_blocks, block_size, num_blocks);
+  if (st != GPTOSS_OK) return st;
+  st = check_rope(rope, D);
+  if (st != GPTOSS_OK) return st;
+  if (B == 0) return GPTOSS_OK;
+  if (!k_new || !v_new || !cache_seqlens || !block_table || !k_pool || !v_pool) return GPTOSS_ERR_INVALID_ARG;
+  AppendParams p;
+  memset(&p, 0, sizeof(p));
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.seqlens = cache_seqlens;
+  p.block_table = block_table;
+  p.k_pool = static_cast<__nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<__nv_bfloat16*>(v_pool);
+  p.B = B;
+  p.Hkv = Hkv;
+  p.max_blocks = max_blocks;
+  p.block_size = block_size;
+  p.num_blocks = num_blocks;
+  if (rope != nullptr) yarn_table(*rope, &p.tab);
+  else p.tab.enabled = 0;
+  kv_append_paged_kernel<<<B, Hkv * kPairs, 0, as_stream(stream)>>>(p);
   return check_launch();
 }
 

@@ -429,6 +429,32 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
                 res[cfg.name]["graph_error"] = str(e)[:200]
         del case
         torch.cuda.empty_cache()
+    # paged decode: the B=64 x 32768 cache seen as 256-token blocks behind a
+    # random block table (same bytes, read through the page indirection)
+    for cfg in decode_cfgs[:1]:
+        case = decode_case(torch, ops, cfg, device)
+        bs = 256
+        nblk = cfg.B * cfg.L // bs
+        gen = torch.Generator(device="cpu").manual_seed(7)
+        table = torch.randperm(nblk, generator=gen).reshape(cfg.B, cfg.L // bs).to(torch.int32).to(device)
+        kp = case["kc"].view(nblk, bs, cfg.Hkv, cfg.D)
+        vp = case["vc"].view(nblk, bs, cfg.Hkv, cfg.D)
+        lens = torch.full((cfg.B,), cfg.L, dtype=torch.int32, device=device)
+
+        def pstep():
+            ops.gptoss_attn_decode_paged(case["q"], kp, vp, table, lens, case["sinks"], window=cfg.window,
+                                         rope=case["rope"], out=case["out"], workspace=case["ws"])
+        for _ in range(3):
+            pstep()
+        torch.cuda.synchronize()
+        ms = timed_steps(torch, pstep, reps, stream) / reps
+        gbs = case["bytes"] / (ms * 1e-3) / 1e9
+        res[f"decode_paged_b{cfg.B}_l{cfg.L}_bs{bs}_full"] = {
+            "ms": round(ms, 4), "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+            "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": case["kv_bytes"],
+            "block_size": bs, "table": f"random permutation of the {nblk} blocks", "launches_per_call": 2}
+        del case, kp, vp
+        torch.cuda.empty_cache()
     return res
 
 

@@ -40,8 +40,9 @@
  *   - Arguments are validated on the host before any launch; a failed check
  *     returns GPTOSS_ERR_INVALID_ARG or GPTOSS_ERR_UNSUPPORTED and launches
  *     nothing.  A failed launch returns GPTOSS_ERR_CUDA.
- *   - Device-side conditions (a bounded pipeline wait that gave up) are
- *     recorded in a device status word read by gptoss_read_device_status.
+ *   - Device-side conditions (a bounded pipeline wait that gave up, a block
+ *     index outside a paged pool) are recorded in a device status word read
+ *     by gptoss_read_device_status.
  *   - bf16 tensors are IEEE bfloat16; head_dim D must be 64 and contiguous
  *     (element stride 1); rotary_dim must equal D.
  *   - No C++ exception crosses this ABI.
@@ -166,7 +167,8 @@ size_t gptoss_attn_decode_workspace_size(int32_t B, int32_t Lmax, int32_t Hq, in
  *            already rotated, v_cache raw values; the new token's k/v are
  *            already in slot cache_seqlens[b]-1.
  *   cache_seqlens int32 [B], 1 <= len <= Lmax (device memory).
- *   The query sees slots [len-window, len) (all of [0, len) when window = 0).
+ *   The query sees slots [len-window, len) (all of [0, len) when window = 0);
+ *   slots past len are never read into the result and may hold anything.
  *   out      [B,Hq,D] bf16 contiguous; lse fp32 [B,Hq], nullable.
  *   workspace  device memory of at least
  *            gptoss_attn_decode_workspace_size(...) bytes, 16-byte aligned,
@@ -177,6 +179,46 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
                                  float softmax_scale, const gptoss_rope_params* rope, void* out,
                                  float* lse, void* workspace, size_t workspace_bytes,
                                  struct CUstream_st* stream);
+
+/* gptoss_attn_decode_paged -- gptoss_attn_decode over a paged KV cache.  The
+ * pages describe generation with a key/value cache (Transformers v4.55.0
+ * release notes, the model.generate examples and the cache entries of the
+ * change list) but give no layout; this one is a block table over a pool of
+ * fixed-size blocks.
+ *   k_pool, v_pool [num_blocks, block_size, Hkv, D] bf16 contiguous; k_pool
+ *            holds rotated keys, v_pool raw values.
+ *   block_table int32 [B, max_blocks] (device memory): token p of sequence b
+ *            is row p % block_size of block block_table[b * max_blocks +
+ *            p / block_size].  A block index outside [0, num_blocks) reads as
+ *            zeros (it never faults).
+ *   block_size a multiple of 64 (whole 64-key tiles per block);
+ *            num_blocks * block_size and max_blocks * block_size < 2^31.
+ *   The other arguments as for gptoss_attn_decode with Lmax = max_blocks *
+ *   block_size (workspace: gptoss_attn_decode_workspace_size(B, max_blocks *
+ *   block_size, Hq, Hkv, D) bytes). */
+gptoss_status gptoss_attn_decode_paged(const void* q, const void* k_pool, const void* v_pool,
+                                       const int32_t* block_table, int32_t max_blocks, int32_t block_size,
+                                       int32_t num_blocks, const int32_t* cache_seqlens, const float* sinks,
+                                       int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t window,
+                                       float softmax_scale, const gptoss_rope_params* rope, void* out,
+                                       float* lse, void* workspace, size_t workspace_bytes,
+                                       struct CUstream_st* stream);
+
+/* gptoss_kv_append_paged -- writes each sequence's new token into a paged
+ * cache: its key rotated at position cache_seqlens[b] - 1 (RoPE as for
+ * gptoss_rope_qk, rounded to bf16; the cache holds post-RoPE keys) and its
+ * value as given.  Run it before gptoss_attn_decode_paged on the same stream.
+ *   k_new, v_new [B, Hkv, D] bf16 contiguous (raw key).
+ *   cache_seqlens int32 [B] (device memory), the new token included (>= 1).
+ *   block_table, max_blocks, block_size, k_pool, v_pool, num_blocks as for
+ *            gptoss_attn_decode_paged.  A sequence whose block index is
+ *            outside [0, num_blocks) is not written and the device status
+ *            word records GPTOSS_ERR_INVALID_ARG.
+ *   rope     NULL stores the key unrotated. */
+gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const int32_t* cache_seqlens,
+                                     const int32_t* block_table, int32_t max_blocks, int32_t block_size,
+                                     void* k_pool, void* v_pool, int32_t num_blocks, int32_t B, int32_t Hkv,
+                                     int32_t D, const gptoss_rope_params* rope, struct CUstream_st* stream);
 
 /* gptoss_attn_decode_noalloc -- gptoss_attn_decode for callers that cannot
  * allocate device memory when they decode (a serving loop whose memory is
@@ -205,7 +247,9 @@ gptoss_status gptoss_attn_decode_noalloc(const void* q, const void* k_cache, con
                                          float* lse, struct CUstream_st* stream);
 
 /* Reads (and, if reset != 0, clears) the device status word of the current
- * device: GPTOSS_OK or GPTOSS_ERR_TIMEOUT.  Synchronises `stream`. */
+ * device: GPTOSS_OK, GPTOSS_ERR_TIMEOUT (a bounded wait gave up) or
+ * GPTOSS_ERR_INVALID_ARG (gptoss_kv_append_paged skipped a block index outside
+ * the pool).  Synchronises `stream`. */
 gptoss_status gptoss_read_device_status(int32_t* status_out, int32_t reset, struct CUstream_st* stream);
 
 /* Time limit, in microseconds, of every device-side pipeline wait of later

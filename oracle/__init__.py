@@ -21,6 +21,10 @@ Contents
                ``GptOssAttention`` attributes ``sinks``, ``sliding_window``,
                ``softmax_scale``; Transformers v4.55.0 release notes,
                "Architecture").
+``paged``      Decode over a paged KV cache (block table over a pool of
+               fixed-size blocks) and appending a new token to it, reduced to
+               ``attention.attn_decode`` and ``rope.rope`` (the pages describe
+               generation with a cache but no cache layout).
 ``brute``      A second, independent formulation in scalar Python loops for
                tiny shapes (complex-multiply RoPE, softmax over the logits
                with the sink appended as one more column).

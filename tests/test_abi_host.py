@@ -120,6 +120,37 @@ def test_decode_validation_and_workspace(lib):
     assert call(B=0) == _abi.GPTOSS_OK
 
 
+def test_paged_validation(lib):
+    rp = ctypes.byref(ROPE)
+
+    def dec(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, table=FAKE, maxb=4, bs=64, nb=16, lens=FAKE, sinks=FAKE, B=2, Hq=64, Hkv=8,
+                 D=64, window=0, scale=0.125, out=FAKE, ws=FAKE, ws_bytes=1 << 30)
+        a.update(kw)
+        return lib.gptoss_attn_decode_paged(a["q"], a["k"], a["v"], a["table"], a["maxb"], a["bs"], a["nb"],
+                                            a["lens"], a["sinks"], a["B"], a["Hq"], a["Hkv"], a["D"], a["window"],
+                                            a["scale"], rp, a["out"], None, a["ws"], a["ws_bytes"], None)
+
+    assert dec(bs=48) == _abi.GPTOSS_ERR_UNSUPPORTED              # tiles would straddle blocks
+    assert dec(nb=1 << 25, bs=128) == _abi.GPTOSS_ERR_UNSUPPORTED  # pool rows >= 2^31
+    assert dec(maxb=0) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert dec(table=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert dec(ws_bytes=16) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert dec(B=0) == _abi.GPTOSS_OK
+
+    def app(**kw):
+        a = dict(kn=FAKE, vn=FAKE, lens=FAKE, table=FAKE, maxb=4, bs=64, kp=FAKE, vp=FAKE, nb=16, B=2, Hkv=8, D=64)
+        a.update(kw)
+        return lib.gptoss_kv_append_paged(a["kn"], a["vn"], a["lens"], a["table"], a["maxb"], a["bs"], a["kp"],
+                                          a["vp"], a["nb"], a["B"], a["Hkv"], a["D"], rp, None)
+
+    assert app(bs=100) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert app(Hkv=33) == _abi.GPTOSS_ERR_UNSUPPORTED  # one thread per (head, pair): 33 x 32 > 1024
+    assert app(D=128) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert app(kp=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert app(B=0) == _abi.GPTOSS_OK
+
+
 def test_wait_limit_setter(lib):
     assert lib.gptoss_set_wait_limit(1000) == _abi.GPTOSS_OK
     assert lib.gptoss_set_wait_limit(0) == _abi.GPTOSS_OK  # back to the default
