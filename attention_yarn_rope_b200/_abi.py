@@ -78,9 +78,9 @@ _SIGNATURES = {
     "gptoss_attn_decode_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                          ctypes.POINTER(RopeParams), _vp, _vp, _vp]),
     "gptoss_attn_decode_paged": (_st, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32,
-                                       _i32, _f32, ctypes.POINTER(RopeParams), _vp, _vp, _vp, ctypes.c_size_t,
-                                       _vp]),
-    "gptoss_kv_append_paged": (_st, [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32,
+                                       _i32, _i32, _f32, ctypes.POINTER(RopeParams), _vp, _vp, _vp,
+                                       ctypes.c_size_t, _vp]),
+    "gptoss_kv_append_paged": (_st, [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                      ctypes.POINTER(RopeParams), _vp]),
     "gptoss_read_device_status": (_st, [ctypes.POINTER(_i32), _i32, _vp]),
     "gptoss_set_wait_limit": (_st, [_u32]),

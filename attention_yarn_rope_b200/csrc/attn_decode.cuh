@@ -3,7 +3,8 @@
 // Rule: the sink attention of GptOssAttention (NeMo AutoModel gpt_oss.layers
 // page: sinks, sliding_window, softmax_scale) for one new query per sequence
 // at position len-1 (RoPE rule of the gpt_oss.rope_utils page), keys already
-// rotated in the cache.
+// rotated in the cache; with q_len new tokens, token i at position
+// len - q_len + i sees the keys up to its own (causal).
 //
 // Design: the op streams the cache once, so it is HBM-bound (8 FLOP per cache
 // byte at 8 q-heads per kv-head).  Split-KV: CTA (g, split, b) owns one kv
@@ -19,8 +20,11 @@
 // a single split (a short window: 128 keys per sequence and kv head), the
 // split kernel folds the sink itself and writes the output: one launch.
 // The same kernel reads a paged cache through a block table (the producer maps
-// each 64-key tile to its block's rows); kv_append_paged_kernel writes a new
-// token into such a cache.
+// each 64-key tile to its block's rows); kv_append_paged_kernel writes new
+// tokens into such a cache.  Several new tokens of one sequence share a CTA:
+// the M side holds (token, head) rows -- two tokens fill the 16 rows at G = 8,
+// four fill two M fragments -- each row masking keys past its own position, so
+// the cache is streamed once per CTA, not once per token.
 #pragma once
 
 #include "host_util.cuh"
@@ -34,9 +38,8 @@ constexpr int kDecStages = 6;
 constexpr int kDecConsumerWarps = 4;   // 16 keys of a stage each
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
 constexpr int kDecTileBytes = kDecTileKeys * kHeadDim * 2;  // 8 KB
-constexpr int kDecMaxGroup = 16;
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kDecMaxGroup = 16;  // query heads per kv head
+constexpr int kDecMaxRows = 32;   // query rows of a CTA: two 16-row M fragments
 
 struct DecodeParams {
   CUtensorMap tmap_k;  // dims (64, Hkv, Lmax, B), box (64, 1, 64, 1)
@@ -50,6 +53,12 @@ struct DecodeParams {
   float* ws_ml;            // [B, Hkv, nsplit, G, 2]
   int B, Lmax, Hq, Hkv, G, window, chunk, nsplit;
   int direct;  // one split per sequence: fold the sink and write out / lse here, no merge launch
+  // query tokens per sequence: query token i of cache row b is the virtual
+  // sequence b * q_len + i (q / out / lse row, workspace slot); it sees the
+  // first len_b - (q_len - 1 - i) keys (causal among the new tokens).  One CTA
+  // serves tpc consecutive tokens of a sequence (tpc * G query rows), so the
+  // grid's z runs over B * n_slices, n_slices = ceil(q_len / tpc).
+  int q_len, tpc, n_slices;
   // paged cache (block_table != nullptr): the K / V tensor maps cover the pools
   // [num_blocks * block_size, Hkv, 64]; token p of sequence b is row
   // block_table[b * max_blocks + p / block_size] * block_size + p % block_size
@@ -101,38 +110,61 @@ __device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int r, int c) {
 struct __align__(1024) DecodeSmem {
   uint8_t k[kDecStages][kDecTileBytes];
   uint8_t v[kDecStages][kDecTileBytes];
-  __nv_bfloat16 q[kDecMaxGroup][kHeadDim + 8];  // rotated query rows, padded
-  float wm[kDecConsumerWarps][kDecMaxGroup];
-  float wl[kDecConsumerWarps][kDecMaxGroup];
+  __nv_bfloat16 q[kDecMaxRows][kHeadDim + 8];  // rotated query rows, padded
+  float wm[kDecConsumerWarps][kDecMaxRows];
+  float wl[kDecConsumerWarps][kDecMaxRows];
   uint64_t full[kDecStages];
   uint64_t empty[kDecStages];
 };
 
+// The query tokens one CTA serves and the keys they see.  CTA z = (b, slice)
+// takes new tokens tok0 .. tok0 + ntok - 1 of sequence b; its query rows are
+// (token t, head h) -> row t * G + h.  Token t sees keys [lo_t, n_t) with
+// n_t = n_first + t; the CTA streams the union [lo_first, n_last) split into
+// chunks, and each row masks the keys outside its own range.
+struct DecodeRows {
+  int b, tok0, ntok, n_first, lo_first;
+};
+
+__device__ __forceinline__ DecodeRows decode_rows(const DecodeParams& p, int z) {
+  DecodeRows r;
+  r.b = z / p.n_slices;
+  r.tok0 = (z - r.b * p.n_slices) * p.tpc;
+  r.ntok = min(p.tpc, p.q_len - r.tok0);
+  r.n_first = __ldg(p.seqlens + r.b) - (p.q_len - 1 - r.tok0);
+  r.lo_first = p.window > 0 ? max(0, r.n_first - p.window) : 0;
+  return r;
+}
+
+// RM = 16-row M fragments of query rows (1: up to 16 rows, 2: up to 32).
+template <int RM>
 __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  const int g = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+  const int g = blockIdx.x, split = blockIdx.y;
+  const DecodeRows cr = decode_rows(p, blockIdx.z);
+  const int b = cr.b;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = __ldg(p.seqlens + b);
-  const int lo = p.window > 0 ? max(0, n - p.window) : 0;
-  const int k_begin = lo + split * p.chunk;
-  const int k_end = min(n, k_begin + p.chunk);
+  const int G = p.G;
+  const int n_last = cr.n_first + cr.ntok - 1;
+  const int k_begin = cr.lo_first + split * p.chunk;
+  const int k_end = min(n_last, k_begin + p.chunk);
   // paged: tiles start on 64-key boundaries (block_size is a multiple of 64,
   // so a tile never straddles two blocks); keys before k_begin are masked
   const int k_tile0 = p.block_table != nullptr ? (k_begin & ~(kDecTileKeys - 1)) : k_begin;
   if (k_begin >= k_end) {  // this split is past the sequence: the merge skips it
     if (p.direct) {        // (only an empty cache reaches here): the sink alone, O = 0
-      for (int idx = threadIdx.x; idx < p.G * kHeadDim; idx += kDecThreads) {
-        const int head = g * p.G + idx / kHeadDim;
-        p.out[(static_cast<int64_t>(b) * p.Hq + head) * kHeadDim + idx % kHeadDim] = __float2bfloat16_rn(0.f);
-        if (p.lse != nullptr && idx % kHeadDim == 0) p.lse[static_cast<int64_t>(b) * p.Hq + head] = __ldg(p.sinks + head);
+      for (int idx = threadIdx.x; idx < cr.ntok * G * kHeadDim; idx += kDecThreads) {
+        const int row = idx / kHeadDim, t = row / G, head = g * G + row % G;
+        const int64_t vb = static_cast<int64_t>(b) * p.q_len + cr.tok0 + t;
+        p.out[(vb * p.Hq + head) * kHeadDim + idx % kHeadDim] = __float2bfloat16_rn(0.f);
+        if (p.lse != nullptr && idx % kHeadDim == 0) p.lse[vb * p.Hq + head] = __ldg(p.sinks + head);
       }
     }
     return;
   }
   const int ntile = (k_end - k_tile0 + kDecTileKeys - 1) / kDecTileKeys;
-  const int G = p.G;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
@@ -141,24 +173,27 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
     }
     fence_mbar_init();
   }
-  // rotated query rows of this group (zero rows past G)
-  for (int idx = threadIdx.x; idx < kDecMaxGroup * kPairs; idx += kDecThreads) {
-    const int h = idx / kPairs, j = idx % kPairs;
+  // rotated query rows of this CTA (zero rows past its tokens); token t's
+  // query sits at position n_first + t - 1
+  for (int idx = threadIdx.x; idx < 16 * RM * kPairs; idx += kDecThreads) {
+    const int row = idx / kPairs, j = idx % kPairs;
+    const int t = row / G;
     float x = 0.f, y = 0.f;
-    if (h < G) {
-      const __nv_bfloat16* qr = p.q + (static_cast<int64_t>(b) * p.Hq + g * G + h) * kHeadDim;
+    if (t < cr.ntok) {
+      const int64_t vb = static_cast<int64_t>(b) * p.q_len + cr.tok0 + t;
+      const __nv_bfloat16* qr = p.q + (vb * p.Hq + g * G + row % G) * kHeadDim;
       x = __bfloat162float(qr[j]);
       y = __bfloat162float(qr[j + kPairs]);
       if (p.tab.enabled) {
-        const float2 cs = rope_cs(n - 1, p.tab.inv_freq[j], p.tab.conc);
+        const float2 cs = rope_cs(cr.n_first + t - 1, p.tab.inv_freq[j], p.tab.conc);
         const float xr = x * cs.x - y * cs.y;
         const float yr = y * cs.x + x * cs.y;
         x = xr;
         y = yr;
       }
     }
-    sm.q[h][j] = __float2bfloat16_rn(x);
-    sm.q[h][j + kPairs] = __float2bfloat16_rn(y);
+    sm.q[row][j] = __float2bfloat16_rn(x);
+    sm.q[row][j + kPairs] = __float2bfloat16_rn(y);
   }
   __syncthreads();
 
@@ -195,21 +230,39 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
 
   // ---------------- consumer warps ----------------
   const int gr = lane >> 2, tq = lane & 3;  // fragment row / column-pair index
-  // query A fragments: rows gr and gr+8, k-tiles of 16 features
-  uint32_t qa[4][4];
+  // query A fragments of M fragment mi: rows 16 mi + gr and 16 mi + gr + 8
+  uint32_t qa[RM][4][4];
+  // each of this thread's rows (mi, half) sees keys [klo, khi): its token's
+  // range cut to this split; rows past the CTA's tokens see none
+  int klo[RM][2], khi[RM][2];
 #pragma unroll
-  for (int kt = 0; kt < 4; ++kt) {
-    const int c0 = kt * 16 + 2 * tq;
-    qa[kt][0] = *reinterpret_cast<const uint32_t*>(&sm.q[gr][c0]);
-    qa[kt][1] = *reinterpret_cast<const uint32_t*>(&sm.q[gr + 8][c0]);
-    qa[kt][2] = *reinterpret_cast<const uint32_t*>(&sm.q[gr][c0 + 8]);
-    qa[kt][3] = *reinterpret_cast<const uint32_t*>(&sm.q[gr + 8][c0 + 8]);
+  for (int mi = 0; mi < RM; ++mi) {
+#pragma unroll
+    for (int kt = 0; kt < 4; ++kt) {
+      const int c0 = kt * 16 + 2 * tq;
+      qa[mi][kt][0] = *reinterpret_cast<const uint32_t*>(&sm.q[16 * mi + gr][c0]);
+      qa[mi][kt][1] = *reinterpret_cast<const uint32_t*>(&sm.q[16 * mi + gr + 8][c0]);
+      qa[mi][kt][2] = *reinterpret_cast<const uint32_t*>(&sm.q[16 * mi + gr][c0 + 8]);
+      qa[mi][kt][3] = *reinterpret_cast<const uint32_t*>(&sm.q[16 * mi + gr + 8][c0 + 8]);
+    }
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int t = (16 * mi + gr + 8 * hf) / G;
+      const int n_t = cr.n_first + t;
+      const int lo_t = p.window > 0 ? max(0, n_t - p.window) : 0;
+      klo[mi][hf] = max(k_begin, lo_t);
+      khi[mi][hf] = t < cr.ntok ? min(k_end, n_t) : k_begin;
+    }
   }
-  float o[8][4];
+  float o[RM][8][4];
+  float m[RM][2], l[RM][2];  // running max (log2 units) and this thread's share of the sums
 #pragma unroll
-  for (int dt = 0; dt < 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of rows gr, gr+8
-  float l0 = 0.f, l1 = 0.f;              // this thread's share of the running sums
+  for (int mi = 0; mi < RM; ++mi) {
+#pragma unroll
+    for (int dt = 0; dt < 8; ++dt) o[mi][dt][0] = o[mi][dt][1] = o[mi][dt][2] = o[mi][dt][3] = 0.f;
+    m[mi][0] = m[mi][1] = -INFINITY;
+    l[mi][0] = l[mi][1] = 0.f;
+  }
 
   for (int it = 0; it < ntile; ++it) {
     const int s = it % kDecStages;
@@ -217,58 +270,66 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
     const uint32_t kb = smem_u32(sm.k[s]);
     const uint32_t vb = smem_u32(sm.v[s]);
     const int r0 = warp * 16;  // first key row of this warp in the tile
-    // S = Q K^T for two 8-key blocks
-    float sc[2][4];
+    // S = Q K^T for two 8-key blocks; each K fragment serves every M fragment
+    float sc[RM][2][4];
 #pragma unroll
     for (int nb = 0; nb < 2; ++nb) {
-      sc[nb][0] = sc[nb][1] = sc[nb][2] = sc[nb][3] = 0.f;
+#pragma unroll
+      for (int mi = 0; mi < RM; ++mi) sc[mi][nb][0] = sc[mi][nb][1] = sc[mi][nb][2] = sc[mi][nb][3] = 0.f;
       const int row = r0 + nb * 8 + (lane & 7);
 #pragma unroll
       for (int kp = 0; kp < 2; ++kp) {
         uint32_t b0, b1, b2, b3;
         ldsm_x4(sw128_addr(kb, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
-        mma_bf16_16816(sc[nb], qa[2 * kp], b0, b1);
-        mma_bf16_16816(sc[nb], qa[2 * kp + 1], b2, b3);
+#pragma unroll
+        for (int mi = 0; mi < RM; ++mi) {
+          mma_bf16_16816(sc[mi][nb], qa[mi][2 * kp], b0, b1);
+          mma_bf16_16816(sc[mi][nb], qa[mi][2 * kp + 1], b2, b3);
+        }
       }
     }
-    // mask keys outside the chunk, scale into log2 units
     const int key_base = k_tile0 + it * kDecTileKeys + r0;
+    float pr[RM][2][4];
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb)
+    for (int mi = 0; mi < RM; ++mi) {
+      // mask keys outside each row's range, scale into log2 units
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = key_base + nb * 8 + 2 * tq + (e & 1);
-        sc[nb][e] = (key >= k_begin && key < k_end) ? sc[nb][e] * p.scale_log2 : -INFINITY;
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = key_base + nb * 8 + 2 * tq + (e & 1);
+          const int hf = e >> 1;
+          sc[mi][nb][e] = (key >= klo[mi][hf] && key < khi[mi][hf]) ? sc[mi][nb][e] * p.scale_log2 : -INFINITY;
+        }
+      // online softmax, rows gr (e = 0, 1) and gr + 8 (e = 2, 3)
+      float mx0 = fmaxf(fmaxf(sc[mi][0][0], sc[mi][0][1]), fmaxf(sc[mi][1][0], sc[mi][1][1]));
+      float mx1 = fmaxf(fmaxf(sc[mi][0][2], sc[mi][0][3]), fmaxf(sc[mi][1][2], sc[mi][1][3]));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float n0 = fmaxf(m[mi][0], mx0), n1 = fmaxf(m[mi][1], mx1);
+      const float b0s = n0 == -INFINITY ? 0.f : n0;  // safe subtrahends
+      const float b1s = n1 == -INFINITY ? 0.f : n1;
+      const float a0 = ex2_approx(m[mi][0] - b0s), a1 = ex2_approx(m[mi][1] - b1s);
+      m[mi][0] = n0;
+      m[mi][1] = n1;
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb) {
+        pr[mi][nb][0] = ex2_approx(sc[mi][nb][0] - b0s);
+        pr[mi][nb][1] = ex2_approx(sc[mi][nb][1] - b0s);
+        pr[mi][nb][2] = ex2_approx(sc[mi][nb][2] - b1s);
+        pr[mi][nb][3] = ex2_approx(sc[mi][nb][3] - b1s);
       }
-    // online softmax, rows gr (e = 0, 1) and gr + 8 (e = 2, 3)
-    float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-    float mx1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-    const float b0s = n0 == -INFINITY ? 0.f : n0;  // safe subtrahends
-    const float b1s = n1 == -INFINITY ? 0.f : n1;
-    const float a0 = ex2_approx(m0 - b0s), a1 = ex2_approx(m1 - b1s);
-    m0 = n0;
-    m1 = n1;
-    float pr[2][4];
+      l[mi][0] = l[mi][0] * a0 + (pr[mi][0][0] + pr[mi][0][1] + pr[mi][1][0] + pr[mi][1][1]);
+      l[mi][1] = l[mi][1] * a1 + (pr[mi][0][2] + pr[mi][0][3] + pr[mi][1][2] + pr[mi][1][3]);
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-      pr[nb][0] = ex2_approx(sc[nb][0] - b0s);
-      pr[nb][1] = ex2_approx(sc[nb][1] - b0s);
-      pr[nb][2] = ex2_approx(sc[nb][2] - b1s);
-      pr[nb][3] = ex2_approx(sc[nb][3] - b1s);
-    }
-    l0 = l0 * a0 + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
-    l1 = l1 * a1 + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
-#pragma unroll
-    for (int dt = 0; dt < 8; ++dt) {
-      o[dt][0] *= a0;
-      o[dt][1] *= a0;
-      o[dt][2] *= a1;
-      o[dt][3] *= a1;
+      for (int dt = 0; dt < 8; ++dt) {
+        o[mi][dt][0] *= a0;
+        o[mi][dt][1] *= a0;
+        o[mi][dt][2] *= a1;
+        o[mi][dt][3] *= a1;
+      }
     }
     // Rows of this warp past the sequence end get P = 0, but 0 x NaN is NaN:
     // those rows of a cache (a paged pool's unused rows above all) may hold
@@ -282,20 +343,26 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       }
       __syncwarp();
     }
-    // P as the A operand (16 heads x 16 keys)
-    uint32_t pa[4];
-    pa[0] = pack_bf16(pr[0][0], pr[0][1]);
-    pa[1] = pack_bf16(pr[0][2], pr[0][3]);
-    pa[2] = pack_bf16(pr[1][0], pr[1][1]);
-    pa[3] = pack_bf16(pr[1][2], pr[1][3]);
-    // O += P V over 8 feature blocks of 8
+    // P as the A operand (16 query rows x 16 keys per M fragment)
+    uint32_t pa[RM][4];
+#pragma unroll
+    for (int mi = 0; mi < RM; ++mi) {
+      pa[mi][0] = pack_bf16(pr[mi][0][0], pr[mi][0][1]);
+      pa[mi][1] = pack_bf16(pr[mi][0][2], pr[mi][0][3]);
+      pa[mi][2] = pack_bf16(pr[mi][1][0], pr[mi][1][1]);
+      pa[mi][3] = pack_bf16(pr[mi][1][2], pr[mi][1][3]);
+    }
+    // O += P V over 8 feature blocks of 8; each V fragment serves every M fragment
 #pragma unroll
     for (int dp = 0; dp < 4; ++dp) {
       uint32_t v0, v1, v2, v3;
       const int row = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
       ldsm_x4_t(sw128_addr(vb, row, 2 * dp + (lane >> 4)), v0, v1, v2, v3);
-      mma_bf16_16816(o[2 * dp], pa, v0, v1);
-      mma_bf16_16816(o[2 * dp + 1], pa, v2, v3);
+#pragma unroll
+      for (int mi = 0; mi < RM; ++mi) {
+        mma_bf16_16816(o[mi][2 * dp], pa[mi], v0, v1);
+        mma_bf16_16816(o[mi][2 * dp + 1], pa[mi], v2, v3);
+      }
     }
     if (tail) fence_proxy_async_smem();  // the zeroed rows before the next TMA write of the stage
     __syncwarp();
@@ -303,45 +370,51 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   }
 
   // ---------------- merge the four warps ----------------
-  // The per-warp accumulators reuse the K stages once every warp is done.
+  // The per-warp accumulators reuse the K stages once every warp is done
+  // (4 warps x 32 rows x 64 floats = 32 KB of the 48 KB).
   named_barrier_sync(1, kDecConsumerWarps * 32);
-  float(*wo)[kDecMaxGroup][kHeadDim] = reinterpret_cast<float(*)[kDecMaxGroup][kHeadDim]>(&sm.k[0][0]);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  if (tq == 0) {
-    sm.wm[warp][gr] = m0;
-    sm.wm[warp][gr + 8] = m1;
-    sm.wl[warp][gr] = l0;
-    sm.wl[warp][gr + 8] = l1;
-  }
+  float(*wo)[kDecMaxRows][kHeadDim] = reinterpret_cast<float(*)[kDecMaxRows][kHeadDim]>(&sm.k[0][0]);
 #pragma unroll
-  for (int dt = 0; dt < 8; ++dt) {
-    wo[warp][gr][dt * 8 + 2 * tq] = o[dt][0];
-    wo[warp][gr][dt * 8 + 2 * tq + 1] = o[dt][1];
-    wo[warp][gr + 8][dt * 8 + 2 * tq] = o[dt][2];
-    wo[warp][gr + 8][dt * 8 + 2 * tq + 1] = o[dt][3];
+  for (int mi = 0; mi < RM; ++mi) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      float lv = l[mi][hf];
+      lv += __shfl_xor_sync(0xffffffffu, lv, 1);
+      lv += __shfl_xor_sync(0xffffffffu, lv, 2);
+      if (tq == 0) {
+        sm.wm[warp][16 * mi + gr + 8 * hf] = m[mi][hf];
+        sm.wl[warp][16 * mi + gr + 8 * hf] = lv;
+      }
+    }
+#pragma unroll
+    for (int dt = 0; dt < 8; ++dt) {
+      wo[warp][16 * mi + gr][dt * 8 + 2 * tq] = o[mi][dt][0];
+      wo[warp][16 * mi + gr][dt * 8 + 2 * tq + 1] = o[mi][dt][1];
+      wo[warp][16 * mi + gr + 8][dt * 8 + 2 * tq] = o[mi][dt][2];
+      wo[warp][16 * mi + gr + 8][dt * 8 + 2 * tq + 1] = o[mi][dt][3];
+    }
   }
   named_barrier_sync(1, kDecConsumerWarps * 32);
-  const int tid = threadIdx.x;  // 128 consumer threads: (head, 4 features) x 2 passes
-  for (int idx = tid; idx < kDecMaxGroup * 16; idx += kDecConsumerWarps * 32) {
-    const int h = idx >> 4, d4 = (idx & 15) * 4;
-    if (h >= G) continue;
+  const int tid = threadIdx.x;  // 128 consumer threads: (row, 4 features)
+  for (int idx = tid; idx < 16 * RM * 16; idx += kDecConsumerWarps * 32) {
+    const int row = idx >> 4, d4 = (idx & 15) * 4;
+    const int t = row / G, h = row - t * G;
+    if (t >= cr.ntok) continue;
+    const int64_t vbq = static_cast<int64_t>(b) * p.q_len + cr.tok0 + t;  // virtual sequence of the row
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, sm.wm[w][h]);
+    for (int w = 0; w < kDecConsumerWarps; ++w) M = fmaxf(M, sm.wm[w][row]);
     const float Ms = M == -INFINITY ? 0.f : M;
     float L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < kDecConsumerWarps; ++w) {
-      const float sc = ex2_approx(sm.wm[w][h] - Ms);
-      L += sm.wl[w][h] * sc;
-      acc.x += wo[w][h][d4] * sc;
-      acc.y += wo[w][h][d4 + 1] * sc;
-      acc.z += wo[w][h][d4 + 2] * sc;
-      acc.w += wo[w][h][d4 + 3] * sc;
+      const float sc = ex2_approx(sm.wm[w][row] - Ms);
+      L += sm.wl[w][row] * sc;
+      acc.x += wo[w][row][d4] * sc;
+      acc.y += wo[w][row][d4 + 1] * sc;
+      acc.z += wo[w][row][d4 + 2] * sc;
+      acc.w += wo[w][row][d4 + 3] * sc;
     }
     if (p.direct) {
       // the only split of this (b, g): fold exp(sink) here as the merge would
@@ -355,11 +428,11 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       uint2 r;
       r.x = pack_bf16(acc.x * inv, acc.y * inv);
       r.y = pack_bf16(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(p.out + (static_cast<int64_t>(b) * p.Hq + head) * kHeadDim + d4) = r;
-      if (p.lse != nullptr && d4 == 0) p.lse[static_cast<int64_t>(b) * p.Hq + head] = (Mt + log2f(Lt)) * kLn2;
+      *reinterpret_cast<uint2*>(p.out + (vbq * p.Hq + head) * kHeadDim + d4) = r;
+      if (p.lse != nullptr && d4 == 0) p.lse[vbq * p.Hq + head] = (Mt + log2f(Lt)) * kLn2;
       continue;
     }
-    const int64_t slot = ((static_cast<int64_t>(b) * p.Hkv + g) * p.nsplit + split) * G + h;
+    const int64_t slot = ((vbq * p.Hkv + g) * p.nsplit + split) * G + h;
     *reinterpret_cast<float4*>(p.ws_o + slot * kHeadDim + d4) = acc;
     if (d4 == 0) {
       p.ws_ml[slot * 2] = M;
@@ -368,18 +441,21 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   }
 }
 
-// Merge the splits of one (b, g): fold exp(sink) once, normalise, write bf16.
+// Merge the splits of one (virtual sequence, g): fold exp(sink) once,
+// normalise, write bf16.  The splits are those of the sequence's CTA group:
+// chunks of the union of its tokens' key ranges.
 __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_constant__ DecodeParams p) {
-  const int g = blockIdx.x, b = blockIdx.y;
-  const int n = __ldg(p.seqlens + b);
-  const int lo = p.window > 0 ? max(0, n - p.window) : 0;
-  const int nsp = min(p.nsplit, (n - lo + p.chunk - 1) / p.chunk);
+  const int g = blockIdx.x, vb = blockIdx.y;  // virtual sequence (cache row, query token)
+  const int b = vb / p.q_len, tok = vb - b * p.q_len;
+  const DecodeRows cr = decode_rows(p, b * p.n_slices + tok / p.tpc);
+  const int n_last = cr.n_first + cr.ntok - 1;
+  const int nsp = min(p.nsplit, (n_last - cr.lo_first + p.chunk - 1) / p.chunk);
   const int G = p.G;
   for (int idx = threadIdx.x; idx < G * 32; idx += 256) {
     const int h = idx >> 5, d2 = (idx & 31) * 2;
     const int head = g * G + h;
     const float sink = __ldg(p.sinks + head) * kLog2e;
-    const int64_t base = (static_cast<int64_t>(b) * p.Hkv + g) * p.nsplit;
+    const int64_t base = (static_cast<int64_t>(vb) * p.Hkv + g) * p.nsplit;
     float M = sink;
     for (int s = 0; s < nsp; ++s) M = fmaxf(M, p.ws_ml[((base + s) * G + h) * 2]);
     const float Ms = M == -INFINITY ? 0.f : M;
@@ -397,31 +473,32 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_con
     __nv_bfloat162 r;
     r.x = __float2bfloat16_rn(ox * inv);
     r.y = __float2bfloat16_rn(oy * inv);
-    *reinterpret_cast<__nv_bfloat162*>(p.out + (static_cast<int64_t>(b) * p.Hq + head) * kHeadDim + d2) = r;
-    if (p.lse != nullptr && d2 == 0) p.lse[static_cast<int64_t>(b) * p.Hq + head] = (M + log2f(L)) * kLn2;
+    *reinterpret_cast<__nv_bfloat162*>(p.out + (static_cast<int64_t>(vb) * p.Hq + head) * kHeadDim + d2) = r;
+    if (p.lse != nullptr && d2 == 0) p.lse[static_cast<int64_t>(vb) * p.Hq + head] = (M + log2f(L)) * kLn2;
   }
 }
 
-// KV-cache append: sequence b's new token (position cache_seqlens[b] - 1)
-// into a paged cache -- the key rotated (the cache holds post-RoPE keys,
-// bf16), the value as given.  Block (b), thread (g, j): pair j of kv head g.
+// KV-cache append: sequence b's q_len new tokens (positions cache_seqlens[b]
+// - q_len .. cache_seqlens[b] - 1) into a paged cache -- the keys rotated
+// (the cache holds post-RoPE keys, bf16), the values as given.  Block (b, i):
+// new token i of sequence b; thread (g, j): pair j of kv head g.
 struct AppendParams {
-  const __nv_bfloat16* k_new;  // [B, Hkv, 64]
+  const __nv_bfloat16* k_new;  // [B, q_len, Hkv, 64]
   const __nv_bfloat16* v_new;
   const int32_t* seqlens;      // [B]
   const int32_t* block_table;  // [B, max_blocks]
   __nv_bfloat16* k_pool;       // [num_blocks * block_size, Hkv, 64]
   __nv_bfloat16* v_pool;
-  int B, Hkv, max_blocks, block_size, num_blocks;
+  int B, q_len, Hkv, max_blocks, block_size, num_blocks;
   RopeTable tab;
 };
 
 constexpr int kStatusBadIndex = 1;  // == GPTOSS_ERR_INVALID_ARG
 
 __global__ void kv_append_paged_kernel(const __grid_constant__ AppendParams p) {
-  const int b = blockIdx.x;
+  const int b = blockIdx.x, tok = blockIdx.y;
   const int g = threadIdx.x / kPairs, j = threadIdx.x % kPairs;
-  const int pos = __ldg(p.seqlens + b) - 1;
+  const int pos = __ldg(p.seqlens + b) - p.q_len + tok;
   const int jb = pos >= 0 ? pos / p.block_size : -1;
   const int blk = (jb >= 0 && jb < p.max_blocks) ? __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks + jb) : -1;
   if (blk < 0 || blk >= p.num_blocks) {  // nothing is written outside the pool
@@ -430,7 +507,7 @@ __global__ void kv_append_paged_kernel(const __grid_constant__ AppendParams p) {
   }
   const int64_t off = (static_cast<int64_t>(blk) * p.block_size + pos % p.block_size) * p.Hkv * kHeadDim +
                       static_cast<int64_t>(g) * kHeadDim;
-  const int64_t src = (static_cast<int64_t>(b) * p.Hkv + g) * kHeadDim;
+  const int64_t src = ((static_cast<int64_t>(b) * p.q_len + tok) * p.Hkv + g) * kHeadDim;
   float x = __bfloat162float(p.k_new[src + j]), y = __bfloat162float(p.k_new[src + j + kPairs]);
   if (p.tab.enabled) {
     const float2 cs = rope_cs(pos, p.tab.inv_freq[j], p.tab.conc);

@@ -1,0 +1,272 @@
+// decode_host.cuh -- host side of the decode entry points of libgptoss_attn
+// (declared in include/gptoss.h): split-KV decode over a contiguous or paged
+// cache, appending new tokens to a paged cache, and decode without a
+// caller-provided workspace.  Included once, at the end of gptoss_lib.cu (the
+// library is one translation unit, so the device status word is shared).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "attn_decode.cuh"
+#include "gptoss.h"
+#include "host_util.cuh"
+
+using namespace gptoss;
+
+extern "C" {
+
+size_t gptoss_attn_decode_workspace_size(int32_t B, int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D) {
+  if (B <= 0 || Lmax <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D != kHeadDim) return 0;
+  const int chunk = decode_chunk(B, Lmax, Hkv);
+  const int64_t nsplit = (Lmax + chunk - 1) / chunk;
+  const int64_t slots = static_cast<int64_t>(B) * Hkv * nsplit * (Hq / Hkv);
+  return static_cast<size_t>(slots * (kHeadDim + 2) * sizeof(float));
+}
+
+}  // extern "C"
+
+namespace {
+
+// A paged cache: pools [num_blocks * block_size, Hkv, 64] and the block table.
+struct PagedLayout {
+  const int32_t* table;
+  int32_t max_blocks, block_size, num_blocks;
+};
+
+// Decode over a contiguous cache [B, Lmax, Hkv, 64] (paged == nullptr) or a
+// paged one (Lmax = max_blocks * block_size, the caches are the pools).
+gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_seqlens,
+                          const float* sinks, int32_t B, int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D,
+                          int32_t window, float softmax_scale, const gptoss_rope_params* rope, void* out,
+                          float* lse, void* workspace, size_t workspace_bytes, struct CUstream_st* stream,
+                          const PagedLayout* paged, int32_t q_len) {
+  if (q_len <= 0) return GPTOSS_ERR_INVALID_ARG;
+  // B x q_len virtual sequences (query token i of cache row b)
+  const int64_t BQ = static_cast<int64_t>(B) * q_len;
+  if (BQ > 65535) return GPTOSS_ERR_UNSUPPORTED;  // grid z / y limit
+  if (B < 0 || Lmax <= 0 || Hq <= 0 || Hkv <= 0 || window < 0) return GPTOSS_ERR_INVALID_ARG;
+  if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
+  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (Hq / Hkv > kDecMaxGroup) return GPTOSS_ERR_UNSUPPORTED;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
+  gptoss_status st = check_rope(rope, D);
+  if (st != GPTOSS_OK) return st;
+  if (B == 0) return GPTOSS_OK;
+  if (!q || !k_cache || !v_cache || !cache_seqlens || !sinks || !out || !workspace) return GPTOSS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(workspace))
+    return GPTOSS_ERR_INVALID_ARG;
+  const size_t need = gptoss_attn_decode_workspace_size(static_cast<int32_t>(BQ), Lmax, Hq, Hkv, D);
+  if (need == 0 || workspace_bytes < need) return GPTOSS_ERR_INVALID_ARG;
+  const int64_t rows = paged ? static_cast<int64_t>(paged->num_blocks) * paged->block_size
+                             : static_cast<int64_t>(B) * Lmax;
+  if (rows * Hkv * kHeadDim > (int64_t(1) << 40)) return GPTOSS_ERR_UNSUPPORTED;
+
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
+  // contiguous: (d, head, slot, sequence); paged: (d, head, pool row, 1)
+  const uint64_t d2 = paged ? static_cast<uint64_t>(rows) : static_cast<uint64_t>(Lmax);
+  const uint64_t d3 = paged ? 1 : static_cast<uint64_t>(B);
+  const uint64_t bat_b = paged ? tok_b * d2 : tok_b * Lmax;
+  st = make_tmap_4d(&p.tmap_k, k_cache, kHeadDim, Hkv, d2, d3, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
+                    kDecTileKeys, 1);
+  if (st != GPTOSS_OK) return st;
+  st = make_tmap_4d(&p.tmap_v, v_cache, kHeadDim, Hkv, d2, d3, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
+                    kDecTileKeys, 1);
+  if (st != GPTOSS_OK) return st;
+  const int G = Hq / Hkv;
+  // tokens per CTA: as many as fill one 16-row M fragment, or two when q_len
+  // needs more than one fragment's worth
+  const int rm = q_len > 16 / G ? 2 : 1;
+  const int tpc = q_len < 16 * rm / G ? q_len : 16 * rm / G;
+  const int n_slices = (q_len + tpc - 1) / tpc;
+  const int chunk = decode_chunk(static_cast<int>(BQ), Lmax, Hkv);
+  const int nsplit_max = (Lmax + chunk - 1) / chunk;
+  // a CTA's tokens see the union of their key ranges: window + tpc - 1 keys
+  const int64_t span_w = static_cast<int64_t>(window) + tpc - 1;
+  const int span = window > 0 ? (span_w < Lmax ? static_cast<int>(span_w) : Lmax) : Lmax;
+  // a window that does not start on a 64-key boundary may touch one more tile,
+  // still inside one split: chunks are multiples of 64 keys and at least 256
+  const int nsplit = (span + chunk - 1) / chunk;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.seqlens = cache_seqlens;
+  p.sinks = sinks;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = p.ws_o + BQ * Hkv * nsplit_max * G * kHeadDim;
+  p.B = B;
+  p.q_len = q_len;
+  p.tpc = tpc;
+  p.n_slices = n_slices;
+  p.Lmax = Lmax;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.window = window;
+  p.chunk = chunk;
+  p.nsplit = nsplit_max;
+  p.direct = nsplit == 1;  // e.g. window 128: one split per (sequence, kv head)
+  if (paged) {
+    p.block_table = paged->table;
+    p.max_blocks = paged->max_blocks;
+    p.block_size = paged->block_size;
+    p.num_blocks = paged->num_blocks;
+  }
+  p.scale_log2 = softmax_scale * kLog2e;
+  p.wait_ns = wait_limit_ns();
+  if (rope != nullptr) yarn_table(*rope, &p.tab);
+  else p.tab.enabled = 0;
+  const size_t smem = sizeof(DecodeSmem) + 1024;
+  auto kernel = rm == 1 ? attn_decode_split_kernel<1> : attn_decode_split_kernel<2>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return GPTOSS_ERR_CUDA;
+  cudaStream_t s = as_stream(stream);
+  const dim3 grid(Hkv, nsplit, static_cast<unsigned>(static_cast<int64_t>(B) * n_slices));
+  kernel<<<grid, kDecThreads, smem, s>>>(p);
+  if (check_launch() != GPTOSS_OK) return GPTOSS_ERR_CUDA;
+  if (p.direct) return GPTOSS_OK;
+  attn_decode_merge_kernel<<<dim3(Hkv, static_cast<unsigned>(BQ)), 256, 0, s>>>(p);
+  return check_launch();
+}
+
+gptoss_status check_paged(int32_t max_blocks, int32_t block_size, int32_t num_blocks) {
+  if (max_blocks <= 0 || block_size <= 0 || num_blocks <= 0) return GPTOSS_ERR_INVALID_ARG;
+  if (block_size % kDecTileKeys) return GPTOSS_ERR_UNSUPPORTED;  // 64-key tiles must not straddle blocks
+  if (static_cast<int64_t>(num_blocks) * block_size >= (int64_t(1) << 31) ||
+      static_cast<int64_t>(max_blocks) * block_size >= (int64_t(1) << 31))
+    return GPTOSS_ERR_UNSUPPORTED;
+  return GPTOSS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                                 const int32_t* cache_seqlens, const float* sinks, int32_t B, int32_t Lmax,
+                                 int32_t Hq, int32_t Hkv, int32_t D, int32_t window, float softmax_scale,
+                                 const gptoss_rope_params* rope, void* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, struct CUstream_st* stream) {
+  return decode_impl(q, k_cache, v_cache, cache_seqlens, sinks, B, Lmax, Hq, Hkv, D, window, softmax_scale, rope,
+                     out, lse, workspace, workspace_bytes, stream, nullptr, 1);
+}
+
+gptoss_status gptoss_attn_decode_paged(const void* q, const void* k_pool, const void* v_pool,
+                                       const int32_t* block_table, int32_t max_blocks, int32_t block_size,
+                                       int32_t num_blocks, const int32_t* cache_seqlens, const float* sinks,
+                                       int32_t B, int32_t q_len, int32_t Hq, int32_t Hkv, int32_t D,
+                                       int32_t window, float softmax_scale, const gptoss_rope_params* rope,
+                                       void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                       struct CUstream_st* stream) {
+  gptoss_status st = check_paged(max_blocks, block_size, num_blocks);
+  if (st != GPTOSS_OK) return st;
+  if (B > 0 && block_table == nullptr) return GPTOSS_ERR_INVALID_ARG;
+  const PagedLayout layout{block_table, max_blocks, block_size, num_blocks};
+  return decode_impl(q, k_pool, v_pool, cache_seqlens, sinks, B, max_blocks * block_size, Hq, Hkv, D, window,
+                     softmax_scale, rope, out, lse, workspace, workspace_bytes, stream, &layout, q_len);
+}
+
+gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const int32_t* cache_seqlens,
+                                     const int32_t* block_table, int32_t max_blocks, int32_t block_size,
+                                     void* k_pool, void* v_pool, int32_t num_blocks, int32_t B, int32_t q_len,
+                                     int32_t Hkv, int32_t D, const gptoss_rope_params* rope,
+                                     struct CUstream_st* stream) {
+  if (B < 0 || q_len <= 0 || Hkv <= 0) return GPTOSS_ERR_INVALID_ARG;
+  if (q_len > 65535) return GPTOSS_ERR_UNSUPPORTED;
+  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (Hkv * kPairs > 1024) return GPTOSS_ERR_UNSUPPORTED;
+  gptoss_status st = check_paged(max_blocks, block_size, num_blocks);
+  if (st != GPTOSS_OK) return st;
+  st = check_rope(rope, D);
+  if (st != GPTOSS_OK) return st;
+  if (B == 0) return GPTOSS_OK;
+  if (!k_new || !v_new || !cache_seqlens || !block_table || !k_pool || !v_pool) return GPTOSS_ERR_INVALID_ARG;
+  AppendParams p;
+  memset(&p, 0, sizeof(p));
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.seqlens = cache_seqlens;
+  p.block_table = block_table;
+  p.k_pool = static_cast<__nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<__nv_bfloat16*>(v_pool);
+  p.B = B;
+  p.q_len = q_len;
+  p.Hkv = Hkv;
+  p.max_blocks = max_blocks;
+  p.block_size = block_size;
+  p.num_blocks = num_blocks;
+  if (rope != nullptr) yarn_table(*rope, &p.tab);
+  else p.tab.enabled = 0;
+  kv_append_paged_kernel<<<dim3(B, q_len), Hkv * kPairs, 0, as_stream(stream)>>>(p);
+  return check_launch();
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they decode:
+// a serving loop that plans its memory once up front and may not call
+// cudaMalloc (which can synchronise the device or fail under memory pressure),
+// or a host runtime whose only device memory comes from its own fixed pools.
+// For them the split-KV partials live in one file-scope device array of fixed
+// size instead.  Every GPU that loads this library holds the array until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+// The array's name is a host-side stand-in in host code: its device address
+// comes from cudaGetSymbolAddress, once per device, with that device current.
+void* g_scratch_addr[kNoAllocMaxDevices];
+std::once_flag g_scratch_once[kNoAllocMaxDevices];
+cudaError_t g_scratch_err[kNoAllocMaxDevices];
+
+void* scratch_address(int device, gptoss_status* st) {
+  if (device < 0 || device >= kNoAllocMaxDevices) {
+    *st = GPTOSS_ERR_UNSUPPORTED;
+    return nullptr;
+  }
+  std::call_once(g_scratch_once[device], [device]() {
+    void* ptr = nullptr;
+    g_scratch_err[device] = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    g_scratch_addr[device] = ptr;
+  });
+  if (g_scratch_err[device] != cudaSuccess || g_scratch_addr[device] == nullptr) {
+    *st = GPTOSS_ERR_CUDA;
+    return nullptr;
+  }
+  *st = GPTOSS_OK;
+  return g_scratch_addr[device];
+}
+
+}  // namespace
+
+extern "C" gptoss_status gptoss_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                                    const int32_t* cache_seqlens, const float* sinks, int32_t B,
+                                                    int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D,
+                                                    int32_t window, float softmax_scale,
+                                                    const gptoss_rope_params* rope, void* out, float* lse,
+                                                    struct CUstream_st* stream) {
+  if (B == 0) return gptoss_attn_decode(q, k_cache, v_cache, cache_seqlens, sinks, B, Lmax, Hq, Hkv, D, window,
+                                        softmax_scale, rope, out, lse, nullptr, 0, stream);
+  const size_t need = gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D);
+  if (need == 0) return D != kHeadDim ? GPTOSS_ERR_UNSUPPORTED : GPTOSS_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) return GPTOSS_ERR_UNSUPPORTED;  // partials exceed the fixed array
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return GPTOSS_ERR_CUDA;
+  gptoss_status st = GPTOSS_OK;
+  void* ws = scratch_address(device, &st);
+  if (ws == nullptr) return st;
+  return gptoss_attn_decode(q, k_cache, v_cache, cache_seqlens, sinks, B, Lmax, Hq, Hkv, D, window, softmax_scale,
+                            rope, out, lse, ws, kNoAllocScratchBytes, stream);
+}

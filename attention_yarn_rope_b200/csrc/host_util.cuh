@@ -15,6 +15,8 @@ namespace gptoss {
 
 constexpr int kHeadDim = 64;
 constexpr int kPairs = kHeadDim / 2;
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
+constexpr float kLn2 = 0.6931471805599453f;     // ln(2)
 
 // Per-launch rotary table: inverse frequencies in double plus the
 // concentration.  Passed to kernels by value (268 bytes).

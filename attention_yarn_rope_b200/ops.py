@@ -175,17 +175,24 @@ def gptoss_attn_decode(q, k_cache, v_cache, cache_seqlens, sinks, window: int = 
 def gptoss_attn_decode_paged(q, k_pool, v_pool, block_table, cache_seqlens, sinks, window: int = 0,
                              softmax_scale: float | None = None, rope: RopeConfig | None = None, out=None,
                              return_lse: bool = False, lse=None, workspace=None, stream=None):
-    """Single-token decode over a paged cache: pools ``[num_blocks, block_size,
-    Hkv, D]`` (keys rotated), ``block_table [B, max_blocks]`` int32 and
-    ``cache_seqlens [B]`` int32 on the device."""
+    """Decode over a paged cache: pools ``[num_blocks, block_size, Hkv, D]``
+    (keys rotated), ``block_table [B, max_blocks]`` int32 and ``cache_seqlens
+    [B]`` int32 on the device.  ``q`` is ``[B, Hq, D]`` (one new token per
+    sequence) or ``[B, q_len, Hq, D]`` (q_len new tokens, already in the cache,
+    each attending causally: token i sees ``cache_seqlens[b] - q_len + 1 + i``
+    keys); ``out`` and ``lse`` take q's leading shape."""
     lib = _abi.load()
-    B, Hq, D = q.shape
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        q_len = 1
+    else:
+        B, q_len, Hq, D = q.shape
     num_blocks, block_size, Hkv, _ = k_pool.shape
     max_blocks = block_table.shape[1]
     out = torch.empty_like(q) if out is None else out
     if return_lse and lse is None:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    need = gptoss_attn_decode_workspace_size(B, max_blocks * block_size, Hq, Hkv, D)
+        lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    need = gptoss_attn_decode_workspace_size(B * q_len, max_blocks * block_size, Hq, Hkv, D)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     _check_dev(q, k_pool, v_pool, block_table, cache_seqlens, sinks, out, lse, workspace)
@@ -195,8 +202,8 @@ def gptoss_attn_decode_paged(q, k_pool, v_pool, block_table, cache_seqlens, sink
     scale = float(D) ** -0.5 if softmax_scale is None else float(softmax_scale)
     r = rope.to_c() if rope is not None else None
     st = lib.gptoss_attn_decode_paged(_ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), max_blocks, block_size,
-                                      num_blocks, _ptr(cache_seqlens), _ptr(sinks), B, Hq, Hkv, D, int(window), scale,
-                                      ctypes.byref(r) if r is not None else None, _ptr(out), _ptr(lse),
+                                      num_blocks, _ptr(cache_seqlens), _ptr(sinks), B, q_len, Hq, Hkv, D, int(window),
+                                      scale, ctypes.byref(r) if r is not None else None, _ptr(out), _ptr(lse),
                                       _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _abi.check("gptoss_attn_decode_paged", st)
     return (out, lse) if (return_lse or lse is not None) else out
@@ -204,10 +211,15 @@ def gptoss_attn_decode_paged(q, k_pool, v_pool, block_table, cache_seqlens, sink
 
 def gptoss_kv_append_paged(k_new, v_new, cache_seqlens, block_table, k_pool, v_pool, rope: RopeConfig | None,
                            stream=None):
-    """Write each sequence's new token (``k_new``, ``v_new`` ``[B, Hkv, D]``) into
-    the paged pools in place: the key rotated at position ``cache_seqlens[b] - 1``."""
+    """Write each sequence's new tokens into the paged pools in place: ``k_new``,
+    ``v_new`` ``[B, Hkv, D]`` (one token) or ``[B, q_len, Hkv, D]``; token i's key
+    is rotated at position ``cache_seqlens[b] - q_len + i``."""
     lib = _abi.load()
-    B, Hkv, D = k_new.shape
+    if k_new.dim() == 3:
+        B, Hkv, D = k_new.shape
+        q_len = 1
+    else:
+        B, q_len, Hkv, D = k_new.shape
     num_blocks, block_size = k_pool.shape[0], k_pool.shape[1]
     _check_dev(k_new, v_new, cache_seqlens, block_table, k_pool, v_pool)
     for t in (k_new, v_new, k_pool, v_pool, block_table):
@@ -215,8 +227,8 @@ def gptoss_kv_append_paged(k_new, v_new, cache_seqlens, block_table, k_pool, v_p
             raise ValueError("append tensors must be contiguous")
     r = rope.to_c() if rope is not None else None
     st = lib.gptoss_kv_append_paged(_ptr(k_new), _ptr(v_new), _ptr(cache_seqlens), _ptr(block_table),
-                                    block_table.shape[1], block_size, _ptr(k_pool), _ptr(v_pool), num_blocks, B, Hkv,
-                                    D, ctypes.byref(r) if r is not None else None, _stream(stream))
+                                    block_table.shape[1], block_size, _ptr(k_pool), _ptr(v_pool), num_blocks, B,
+                                    q_len, Hkv, D, ctypes.byref(r) if r is not None else None, _stream(stream))
     _abi.check("gptoss_kv_append_paged", st)
 
 

@@ -352,9 +352,13 @@ def run_ours(args, torch, dist, rank, world, device):
     d2h = h_os[0].numel() * h_os[0].element_size()
 
     achieved_gbs = case["bytes"] / (per_step_ms * 1e-3) / 1e9
+    # DRAM bytes of the step's two kernels (one ncu capture each, taken on
+    # their current sources), summed like the duration they are set against
+    by_kernel = {k: read_traffic(k, cfg.name) for k in ("rope_qk_kernel<true>", "attn_fwd_kernel")}
+    traffic = None if None in by_kernel.values() else sum(by_kernel.values())
     roofline = {"kernel": "attn_fwd_kernel", "bound": "hbm", "achieved": round(achieved_gbs, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-                "peak_source": peaks["source"], "traffic": read_traffic("attn_fwd_kernel", cfg.name),
+                "peak_source": peaks["source"], "traffic": traffic, "traffic_by_kernel": by_kernel,
                 "algorithmic_bytes_per_launch": case["bytes"],
                 "duration": "whole step: k rotation into the workspace + attention kernel",
                 "tflops": round(case["flops"] / (per_step_ms * 1e-3) / 1e12, 2)}
@@ -453,19 +457,38 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
             "ms": round(ms, 4), "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
             "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": case["kv_bytes"],
             "block_size": bs, "table": f"random permutation of the {nblk} blocks", "launches_per_call": 2}
-        del case, kp, vp
+        # four new tokens per sequence (draft tokens checked in one call): the
+        # four share each CTA's pass over the cache (32 query rows per kv head)
+        q_len = 4
+        q4 = case["q"][:, None].repeat(1, q_len, 1, 1).contiguous()  # the seeded queries, one per new token
+        o4 = torch.empty_like(q4)
+        ws4 = torch.empty(ops.gptoss_attn_decode_workspace_size(cfg.B * q_len, cfg.L, cfg.Hq, cfg.Hkv, cfg.D),
+                          dtype=torch.uint8, device=device)
+
+        def mstep():
+            ops.gptoss_attn_decode_paged(q4, kp, vp, table, lens, case["sinks"], window=cfg.window,
+                                         rope=case["rope"], out=o4, workspace=ws4)
+        for _ in range(3):
+            mstep()
+        torch.cuda.synchronize()
+        ms4 = timed_steps(torch, mstep, reps, stream) / reps
+        res[f"decode_paged_b{cfg.B}_l{cfg.L}_bs{bs}_qlen{q_len}_full"] = {
+            "ms": round(ms4, 4), "us": round(ms4 * 1e3, 2), "q_len": q_len,
+            "cache_read_once_gbs": round(case["bytes"] / (ms4 * 1e-3) / 1e9, 1),
+            "x_single_token_time": round(ms4 / ms, 3), "launches_per_call": 2}
+        del case, kp, vp, q4, o4, ws4
         torch.cuda.empty_cache()
     return res
 
 
 def read_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the kernel source as it is now (else None)."""
+    on the kernel's sources as they are now (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
     want = f"{kernel} {workload} "
-    src_hash = csrc_hash()
+    src_hash = kernel_src_hash(kernel)
     with open(path) as fh:
         for line in fh:
             if line.startswith(want):
@@ -475,14 +498,37 @@ def read_traffic(kernel, workload):
     return None
 
 
-def csrc_hash():
-    import hashlib
+# The sources each measured kernel is built from: the include closure of the
+# header that defines it, plus the host file that launches it (its own text
+# only: the library source also includes the other kernels' headers).
+_KERNEL_SOURCES = {
+    "attn_fwd_kernel": ("fwd_pipeline.cuh", "gptoss_lib.cu"),
+    "rope_qk_kernel<true>": ("rope_qk.cuh", "gptoss_lib.cu"),
+    "attn_decode_split_kernel": ("attn_decode.cuh", "decode_host.cuh"),
+}
 
+
+def kernel_src_hash(kernel):
+    import hashlib
+    import re
+
+    csrc = os.path.join(ROOT, "attention_yarn_rope_b200", "csrc")
+    inc = os.path.join(ROOT, "include")
+    root, launcher = _KERNEL_SOURCES[kernel]
+    seen, todo = [], [root]
+    while todo:
+        f = todo.pop()
+        if f in seen:
+            continue
+        seen.append(f)
+        path = os.path.join(csrc, f) if os.path.exists(os.path.join(csrc, f)) else os.path.join(inc, f)
+        with open(path) as fh:
+            todo += re.findall(r'^#include "([^"]+)"', fh.read(), flags=re.M)
     h = hashlib.sha256()
-    d = os.path.join(ROOT, "attention_yarn_rope_b200", "csrc")
-    for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(fh.read())
+    for f in sorted(seen) + [launcher]:
+        path = os.path.join(csrc, f) if os.path.exists(os.path.join(csrc, f)) else os.path.join(inc, f)
+        with open(path, "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:12]
 
 

@@ -193,23 +193,36 @@ gptoss_status gptoss_attn_decode(const void* q, const void* k_cache, const void*
  *            zeros (it never faults).
  *   block_size a multiple of 64 (whole 64-key tiles per block);
  *            num_blocks * block_size and max_blocks * block_size < 2^31.
+ *   q_len    query tokens per sequence (>= 1; B * q_len <= 65535): several
+ *            new tokens decoded in one call, as when draft tokens are
+ *            verified.  q [B, q_len, Hq, D] (rotated by the caller, or by
+ *            `rope` at positions cache_seqlens[b] - q_len + i), out
+ *            [B, q_len, Hq, D], lse [B, q_len, Hq].  Token i of sequence b
+ *            attends to the first cache_seqlens[b] - (q_len - 1 - i) cache
+ *            rows (causal among the new tokens, which the cache must already
+ *            hold); a sequence needs cache_seqlens[b] >= q_len.  The new
+ *            tokens of a sequence share one pass over its cache (up to
+ *            32 / (Hq / Hkv) tokens per pass: 4 at Hq / Hkv = 8).
  *   The other arguments as for gptoss_attn_decode with Lmax = max_blocks *
- *   block_size (workspace: gptoss_attn_decode_workspace_size(B, max_blocks *
- *   block_size, Hq, Hkv, D) bytes). */
+ *   block_size (workspace: gptoss_attn_decode_workspace_size(B * q_len,
+ *   max_blocks * block_size, Hq, Hkv, D) bytes). */
 gptoss_status gptoss_attn_decode_paged(const void* q, const void* k_pool, const void* v_pool,
                                        const int32_t* block_table, int32_t max_blocks, int32_t block_size,
                                        int32_t num_blocks, const int32_t* cache_seqlens, const float* sinks,
-                                       int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t window,
-                                       float softmax_scale, const gptoss_rope_params* rope, void* out,
-                                       float* lse, void* workspace, size_t workspace_bytes,
+                                       int32_t B, int32_t q_len, int32_t Hq, int32_t Hkv, int32_t D,
+                                       int32_t window, float softmax_scale, const gptoss_rope_params* rope,
+                                       void* out, float* lse, void* workspace, size_t workspace_bytes,
                                        struct CUstream_st* stream);
 
-/* gptoss_kv_append_paged -- writes each sequence's new token into a paged
- * cache: its key rotated at position cache_seqlens[b] - 1 (RoPE as for
- * gptoss_rope_qk, rounded to bf16; the cache holds post-RoPE keys) and its
- * value as given.  Run it before gptoss_attn_decode_paged on the same stream.
- *   k_new, v_new [B, Hkv, D] bf16 contiguous (raw key).
- *   cache_seqlens int32 [B] (device memory), the new token included (>= 1).
+/* gptoss_kv_append_paged -- writes each sequence's q_len new tokens into a
+ * paged cache: the key of token i rotated at position cache_seqlens[b] -
+ * q_len + i (RoPE as for gptoss_rope_qk, rounded to bf16; the cache holds
+ * post-RoPE keys) and the values as given.  Run it before
+ * gptoss_attn_decode_paged on the same stream.
+ *   k_new, v_new [B, q_len, Hkv, D] bf16 contiguous (raw keys).
+ *   q_len    new tokens per sequence (1 .. 65535).
+ *   cache_seqlens int32 [B] (device memory), the new tokens included
+ *            (>= q_len).
  *   block_table, max_blocks, block_size, k_pool, v_pool, num_blocks as for
  *            gptoss_attn_decode_paged.  A sequence whose block index is
  *            outside [0, num_blocks) is not written and the device status
@@ -217,8 +230,9 @@ gptoss_status gptoss_attn_decode_paged(const void* q, const void* k_pool, const 
  *   rope     NULL stores the key unrotated. */
 gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const int32_t* cache_seqlens,
                                      const int32_t* block_table, int32_t max_blocks, int32_t block_size,
-                                     void* k_pool, void* v_pool, int32_t num_blocks, int32_t B, int32_t Hkv,
-                                     int32_t D, const gptoss_rope_params* rope, struct CUstream_st* stream);
+                                     void* k_pool, void* v_pool, int32_t num_blocks, int32_t B, int32_t q_len,
+                                     int32_t Hkv, int32_t D, const gptoss_rope_params* rope,
+                                     struct CUstream_st* stream);
 
 /* gptoss_attn_decode_noalloc -- gptoss_attn_decode for callers that cannot
  * allocate device memory when they decode (a serving loop whose memory is

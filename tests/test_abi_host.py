@@ -124,30 +124,41 @@ def test_paged_validation(lib):
     rp = ctypes.byref(ROPE)
 
     def dec(**kw):
-        a = dict(q=FAKE, k=FAKE, v=FAKE, table=FAKE, maxb=4, bs=64, nb=16, lens=FAKE, sinks=FAKE, B=2, Hq=64, Hkv=8,
-                 D=64, window=0, scale=0.125, out=FAKE, ws=FAKE, ws_bytes=1 << 30)
+        a = dict(q=FAKE, k=FAKE, v=FAKE, table=FAKE, maxb=4, bs=64, nb=16, lens=FAKE, sinks=FAKE, B=2, q_len=1,
+                 Hq=64, Hkv=8, D=64, window=0, scale=0.125, out=FAKE, ws=FAKE, ws_bytes=1 << 30)
         a.update(kw)
         return lib.gptoss_attn_decode_paged(a["q"], a["k"], a["v"], a["table"], a["maxb"], a["bs"], a["nb"],
-                                            a["lens"], a["sinks"], a["B"], a["Hq"], a["Hkv"], a["D"], a["window"],
-                                            a["scale"], rp, a["out"], None, a["ws"], a["ws_bytes"], None)
+                                            a["lens"], a["sinks"], a["B"], a["q_len"], a["Hq"], a["Hkv"], a["D"],
+                                            a["window"], a["scale"], rp, a["out"], None, a["ws"], a["ws_bytes"],
+                                            None)
 
     assert dec(bs=48) == _abi.GPTOSS_ERR_UNSUPPORTED              # tiles would straddle blocks
     assert dec(nb=1 << 25, bs=128) == _abi.GPTOSS_ERR_UNSUPPORTED  # pool rows >= 2^31
     assert dec(maxb=0) == _abi.GPTOSS_ERR_INVALID_ARG
     assert dec(table=None) == _abi.GPTOSS_ERR_INVALID_ARG
     assert dec(ws_bytes=16) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert dec(q_len=0) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert dec(B=300, q_len=300) == _abi.GPTOSS_ERR_UNSUPPORTED   # 90000 query tokens > one grid dimension
+    # the workspace holds every query token's partials: B x q_len sequences
+    ws1 = lib.gptoss_attn_decode_workspace_size(2, 256, 64, 8, 64)
+    ws4 = lib.gptoss_attn_decode_workspace_size(8, 256, 64, 8, 64)
+    assert ws4 > ws1
+    assert dec(q_len=4, ws_bytes=ws1) == _abi.GPTOSS_ERR_INVALID_ARG
     assert dec(B=0) == _abi.GPTOSS_OK
 
     def app(**kw):
-        a = dict(kn=FAKE, vn=FAKE, lens=FAKE, table=FAKE, maxb=4, bs=64, kp=FAKE, vp=FAKE, nb=16, B=2, Hkv=8, D=64)
+        a = dict(kn=FAKE, vn=FAKE, lens=FAKE, table=FAKE, maxb=4, bs=64, kp=FAKE, vp=FAKE, nb=16, B=2, q_len=1,
+                 Hkv=8, D=64)
         a.update(kw)
         return lib.gptoss_kv_append_paged(a["kn"], a["vn"], a["lens"], a["table"], a["maxb"], a["bs"], a["kp"],
-                                          a["vp"], a["nb"], a["B"], a["Hkv"], a["D"], rp, None)
+                                          a["vp"], a["nb"], a["B"], a["q_len"], a["Hkv"], a["D"], rp, None)
 
     assert app(bs=100) == _abi.GPTOSS_ERR_UNSUPPORTED
     assert app(Hkv=33) == _abi.GPTOSS_ERR_UNSUPPORTED  # one thread per (head, pair): 33 x 32 > 1024
     assert app(D=128) == _abi.GPTOSS_ERR_UNSUPPORTED
     assert app(kp=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert app(q_len=0) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert app(q_len=70000) == _abi.GPTOSS_ERR_UNSUPPORTED
     assert app(B=0) == _abi.GPTOSS_OK
 
 

@@ -156,3 +156,78 @@ def test_rows_past_the_end_may_hold_nan(cuda_device, paged):
     got = host(out)
     assert np.all(np.isfinite(got))
     assert_parity(got, ref, f"nan-padded cache paged={paged}")
+
+
+# (q_len, query heads, kv heads): the tokens of a sequence share a CTA --
+# G = 8: two tokens fill one 16-row fragment (q_len 2), up to four fill two
+# (q_len 3), q_len 5 takes two CTAs of 4 + 1 tokens; G = 16: one token per
+# fragment, two per CTA (q_len 3: 2 + 1)
+@pytest.mark.parametrize("window", [0, 128])
+@pytest.mark.parametrize("q_len,Hq,Hkv", [(1, 16, 2), (2, 16, 2), (3, 16, 2), (5, 16, 2), (3, 32, 2)])
+def test_multi_token_decode_matches_oracle(cuda_device, window, q_len, Hq, Hkv):
+    # q_len new tokens per sequence (already in the cache), each attending
+    # causally; the shortest sequence holds only its new tokens
+    lens = [q_len, 77, 300, 1000, 256]
+    bs = 64
+    q1, kp, vp, table, sinks = _paged_case(lens, bs, Hq=Hq, Hkv=Hkv, seed=43)
+    rng = np.random.default_rng(47)
+    q = bf16_round(rng.standard_normal((len(lens), q_len, Hq, 64)))
+    out, lse = ops.gptoss_attn_decode_paged(dev(q), dev(kp), dev(vp), i32(table), i32(lens), f32(sinks),
+                                            window=window, rope=ROPE, return_lse=True)
+    torch.cuda.synchronize()
+    assert out.shape == (len(lens), q_len, Hq, 64) and lse.shape == (len(lens), q_len, Hq)
+    ref, ref_lse = attn_decode_paged(q, kp, vp, table, bs, lens, sinks, 0.125, window, TABLES)
+    assert_parity(host(out), ref, f"multi-token out q_len={q_len} G={Hq // Hkv} w={window}")
+    assert_parity(host(lse), ref_lse, f"multi-token lse q_len={q_len} G={Hq // Hkv} w={window}")
+
+
+def test_multi_token_many_splits(cuda_device):
+    # long sequences, few of them: several splits per sequence, so the merge
+    # combines partials of the union range for every token
+    lens = [5000, 4100, 9000]
+    q_len, bs = 4, 256
+    q1, kp, vp, table, sinks = _paged_case(lens, bs, seed=67)
+    rng = np.random.default_rng(71)
+    q = bf16_round(rng.standard_normal((len(lens), q_len, 16, 64)))
+    out = ops.gptoss_attn_decode_paged(dev(q), dev(kp), dev(vp), i32(table), i32(lens), f32(sinks), rope=ROPE)
+    torch.cuda.synchronize()
+    ref, _ = attn_decode_paged(q, kp, vp, table, bs, lens, sinks, 0.125, 0, TABLES)
+    assert_parity(host(out), ref, "multi-token, several splits")
+
+
+def test_multi_token_append_then_decode(cuda_device):
+    rng = np.random.default_rng(53)
+    q_len, bs = 4, 64
+    lens = [4, 131, 2000]  # new tokens straddle a block edge in sequence 1 (positions 127..130)
+    q1, kp, vp, table, sinks = _paged_case(lens, bs, seed=59)
+    B = len(lens)
+    k_new = bf16_round(rng.standard_normal((B, q_len, 2, 64)))
+    v_new = bf16_round(rng.standard_normal((B, q_len, 2, 64)))
+    q = bf16_round(rng.standard_normal((B, q_len, 16, 64)))
+    kd, vd = dev(kp), dev(vp)
+    ops.read_device_status()
+    ops.gptoss_kv_append_paged(dev(k_new), dev(v_new), i32(lens), i32(table), kd, vd, ROPE)
+    out = ops.gptoss_attn_decode_paged(dev(q), kd, vd, i32(table), i32(lens), f32(sinks), window=128, rope=ROPE)
+    torch.cuda.synchronize()
+    assert ops.read_device_status() == 0
+    ref_k, ref_v = kv_append_paged(k_new, v_new, lens, table, bs, kp, vp, TABLES)
+    written = np.zeros(kp.shape[:2], bool)
+    for b, n in enumerate(lens):
+        for p in range(n - q_len, n):
+            written[table[b, p // bs], p % bs] = True
+    got_k = host(kd)
+    np.testing.assert_array_equal(got_k[~written], kp[~written])
+    np.testing.assert_array_equal(host(vd), ref_v)
+    spacing = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref_k[written]), 1e-30))) - 7)
+    assert np.all(np.abs(got_k[written] - ref_k[written]) <= spacing + 1e-30)
+    ref, _ = attn_decode_paged(q, got_k, host(vd), table, bs, lens, sinks, 0.125, 128, TABLES)
+    assert_parity(host(out), ref, "multi-token append then decode")
+
+
+def test_multi_token_of_one_equals_single_token(cuda_device):
+    lens = [1000, 64, 513]
+    q, kp, vp, table, sinks = _paged_case(lens, 128, seed=61)
+    a = ops.gptoss_attn_decode_paged(dev(q), dev(kp), dev(vp), i32(table), i32(lens), f32(sinks), rope=ROPE)
+    m = ops.gptoss_attn_decode_paged(dev(q[:, None]), dev(kp), dev(vp), i32(table), i32(lens), f32(sinks), rope=ROPE)
+    torch.cuda.synchronize()
+    assert torch.equal(m[:, 0], a)

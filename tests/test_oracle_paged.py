@@ -2,12 +2,14 @@
 with any block permutation decodes exactly like the contiguous cache it was
 scattered from; the appended key sits in the right block row and equals an
 independent (complex-multiply) rotation; append-then-decode equals decode over
-the contiguous cache that holds the rotated new key."""
+the contiguous cache that holds the rotated new key; several new tokens per
+sequence, appended and decoded, reproduce the last rows of a causal prefill
+over the whole sequence (a different code path: the prefill's row mask)."""
 
 import numpy as np
 import pytest
 
-from oracle.attention import attn_decode
+from oracle.attention import attn_decode, attn_fwd_bshd
 from oracle.brute import rope_complex
 from oracle.paged import attn_decode_paged, gather_paged, kv_append_paged
 from oracle.yarn import yarn_inv_freq_and_concentration
@@ -97,3 +99,53 @@ def test_append_then_decode_equals_contiguous():
         vc[b, lens[b] - 1] = v_new[b]
     ref, _ = attn_decode(q, kc, vc, lens, sinks, 0.125, 0, TABLES)
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("window", [0, 5, 128])
+def test_multi_token_append_and_decode_equal_prefill_rows(window):
+    # a sequence of L tokens whose first L - q_len keys are already cached
+    # (rotated by the brute-force complex rotation); append the last q_len raw
+    # keys, decode the last q_len raw queries: the result is the causal prefill
+    # of all L tokens at rows L - q_len .. L - 1
+    rng = np.random.default_rng(19)
+    B, L, q_len, Hq, Hkv, D, bs = 2, 70, 4, 4, 2, 64, 16
+    q = rng.standard_normal((B, L, Hq, D))
+    k = rng.standard_normal((B, L, Hkv, D))
+    v = rng.standard_normal((B, L, Hkv, D))
+    sinks = rng.standard_normal(Hq)
+    ref_o, ref_l = attn_fwd_bshd(q, k, v, sinks, 0.125, window, rope_tables=TABLES)
+    nb_seq = -(-L // bs)
+    table = rng.permutation(B * nb_seq + 2)[:B * nb_seq].reshape(B, nb_seq)
+    kp = rng.standard_normal((B * nb_seq + 2, bs, Hkv, D))
+    vp = rng.standard_normal((B * nb_seq + 2, bs, Hkv, D))
+    inv, c = TABLES
+    for b in range(B):
+        for p in range(L - q_len):
+            for g in range(Hkv):
+                kp[table[b, p // bs], p % bs, g] = rope_complex(k[b, p, g], p, inv, c)
+            vp[table[b, p // bs], p % bs] = v[b, p]
+    lens = [L] * B
+    kp, vp = kv_append_paged(k[:, L - q_len:], v[:, L - q_len:], lens, table, bs, kp, vp, TABLES)
+    got_o, got_l = attn_decode_paged(q[:, L - q_len:], kp, vp, table, bs, lens, sinks, 0.125, window, TABLES)
+    assert got_o.shape == (B, q_len, Hq, D) and got_l.shape == (B, q_len, Hq)
+    np.testing.assert_allclose(got_o, ref_o[:, L - q_len:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got_l, np.transpose(ref_l, (0, 2, 1))[:, L - q_len:], rtol=0, atol=1e-12)
+
+
+def test_multi_token_with_one_token_is_single_token_decode():
+    rng = np.random.default_rng(21)
+    B, Hq, Hkv, D, bs = 2, 4, 2, 64, 32
+    lens = [33, 64]
+    table = np.array([[1, 0], [3, 2]])
+    kp, vp = rng.standard_normal((4, bs, Hkv, D)), rng.standard_normal((4, bs, Hkv, D))
+    q, sinks = rng.standard_normal((B, Hq, D)), rng.standard_normal(Hq)
+    a = attn_decode_paged(q, kp, vp, table, bs, lens, sinks, 0.125, 0, TABLES)
+    m = attn_decode_paged(q[:, None], kp, vp, table, bs, lens, sinks, 0.125, 0, TABLES)
+    np.testing.assert_array_equal(m[0][:, 0], a[0])
+    np.testing.assert_array_equal(m[1][:, 0], a[1])
+
+
+def test_multi_token_needs_its_tokens_in_the_cache():
+    z = np.zeros((2, 32, 1, 64))
+    with pytest.raises(ValueError):
+        attn_decode_paged(np.zeros((1, 3, 1, 64)), z, z, np.array([[0]]), 32, [2], np.zeros(1), 0.125, 0)
