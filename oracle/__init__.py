@@ -25,6 +25,11 @@ Contents
                fixed-size blocks) and appending a new token to it, reduced to
                ``attention.attn_decode`` and ``rope.rope`` (the pages describe
                generation with a cache but no cache layout).
+``backward``   Gradients of the sink attention with RoPE (dq, dk, dv and the
+               sink gradient): the exact derivative of ``attention``'s
+               definition by the chain rule, and the RoPE adjoint
+               ``rope_transpose``.  The pages define the forward and describe
+               training with it; they print no backward formula.
 ``brute``      A second, independent formulation in scalar Python loops for
                tiny shapes (complex-multiply RoPE, softmax over the logits
                with the sink appended as one more column).
@@ -35,7 +40,9 @@ no online softmax and no reordering beyond what a library matmul does.
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 against closed forms, invariants, a library routine
 (``torch.nn.functional.scaled_dot_product_attention`` in float64) and the
-brute-force formulation.  The one reading the pages leave open and no
+brute-force formulation; ``backward`` against central finite differences
+of the forward oracle and float64 ``torch.autograd`` of a separately written
+forward.  The one reading the pages leave open and no
 invariant can decide -- the shape of the YaRN ramp between the two correction
 dimensions -- is selectable (``ramp="index"`` is the adopted reading,
 ``ramp="paper"`` the YaRN paper's gamma(r)); the choice between them is
