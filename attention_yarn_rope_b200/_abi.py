@@ -37,6 +37,8 @@ EXPORTED = (
     "gptoss_attn_decode_noalloc",
     "gptoss_attn_decode_paged",
     "gptoss_kv_append_paged",
+    "gptoss_attn_bwd_workspace_size",
+    "gptoss_attn_bwd",
     "gptoss_read_device_status",
     "gptoss_set_wait_limit",
     "gptoss_selftest_wait_timeout",
@@ -82,6 +84,10 @@ _SIGNATURES = {
                                        ctypes.c_size_t, _vp]),
     "gptoss_kv_append_paged": (_st, [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                      ctypes.POINTER(RopeParams), _vp]),
+    "gptoss_attn_bwd_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32]),
+    "gptoss_attn_bwd": (_st, [_vp, Strides, _vp, Strides, _vp, Strides, _vp, Strides, _vp, Strides, _vp, _vp, _vp,
+                              _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, ctypes.POINTER(RopeParams), _vp,
+                              _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "gptoss_read_device_status": (_st, [ctypes.POINTER(_i32), _i32, _vp]),
     "gptoss_set_wait_limit": (_st, [_u32]),
     "gptoss_selftest_wait_timeout": (_st, [_u32, _vp, _vp]),

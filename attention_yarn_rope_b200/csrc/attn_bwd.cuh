@@ -1,0 +1,452 @@
+// attn_bwd.cuh -- gradients of the sink attention with RoPE (gptoss_attn_bwd).
+//
+// Rule: the derivative of GptOssAttention's forward (NeMo AutoModel
+// gpt_oss.layers page: sinks, sliding_window, softmax_scale; RoPE of the
+// gpt_oss.rope_utils page) for L = sum(dout * out), given the forward's
+// log-sum-exp per row (lse includes the sink term).  With P_ij = exp(s_ij -
+// lse_i) over the visible pairs and a_i = exp(sink_h - lse_i):
+//   D_i = <dout_i, out_i>,  dP_ij = <dout_i, v_j>,  dS_ij = P_ij (dP_ij - D_i)
+//   dv_j = sum_i P_ij dout_i,  dq'_i = scale sum_j dS_ij k'_j,
+//   dk'_j = scale sum_i dS_ij q'_i,  dsink_h = -sum_i a_i D_i,
+// and dq = c R(theta)^T dq', dk = c R(theta)^T dk' (RoPE is linear).
+//
+// Launches (all on the caller's stream):
+//   1. rope_qk_kernel<true>: q and k rotated once into the workspace (fp16,
+//      the forward's QK^T operand format) plus each token's 32 (c cos, c sin)
+//      pairs; without RoPE the same kernel converts them with the identity.
+//   2. attn_bwd_preprocess_kernel: D for every (row, head) into the workspace,
+//      and the sink gradient (one atomic add per head and CTA).
+//   3. attn_bwd_dkdv_kernel: CTA (key tile, kv head, sequence); its 4 warps
+//      own 16 keys each and keep K and V as mma.sync A fragments in registers
+//      while they sweep every (query head of the group, query tile) that sees
+//      the key tile, with the q and dout tiles double-buffered through shared
+//      memory by cp.async.  Per step: S^T = K Q^T, dP^T = V dout^T, P^T and
+//      dS^T in registers, dV += P^T dout, dK += dS^T Q.  The epilogue applies
+//      scale and c R^T to dK and writes bf16: no atomics, one writer per row.
+//   4. attn_bwd_dq_kernel: CTA (query tile, head, sequence); 4 warps of 16
+//      queries keep Q and dout as A fragments and sweep the key tiles the
+//      query tile sees (K and V double-buffered): S, dP, dS recomputed, dQ +=
+//      dS K, then scale and c R^T.  Recomputing S and dP here (3 products per
+//      step instead of atomics on a float dQ) keeps every output written once.
+// Operands: rotated q / k in fp16, v / dout in bf16, P rounded to bf16 for
+// P^T dout and dS to fp16 for the products with q and k; fp32 accumulation.
+#pragma once
+
+#include "host_util.cuh"
+#include "sm100_ptx.cuh"
+#include "warp_mma.cuh"
+
+namespace gptoss {
+
+constexpr int kBwdTile = 64;       // queries / keys per tile
+constexpr int kBwdThreads = 128;   // 4 warps x 16 rows
+constexpr int kBwdMaxHeads = 1024; // query heads the preprocess kernel reduces in shared memory
+
+struct BwdParams {
+  const __nv_bfloat16* qh;  // rotated q, fp16 bits, dense [T, Hq, 64]
+  const __nv_bfloat16* kh;  // rotated k, fp16 bits, dense [T, Hkv, 64]
+  const __nv_bfloat16* v;
+  const __nv_bfloat16* out;
+  const __nv_bfloat16* dout;
+  gptoss_strides sv, so, sdo;  // elements; BSHD uses batch, THD ignores it
+  const float* lse;            // the forward's: BSHD [B, Hq, S], THD [Hq, T]
+  float* dsum;                 // D, same layout as lse
+  const float2* cs;            // [T][32] (c cos, c sin) of every token's pairs
+  const float* sinks;          // [Hq]
+  float* dsinks;               // [Hq], accumulated (zeroed before the launches)
+  __nv_bfloat16* dq;           // dense [T, Hq, 64]
+  __nv_bfloat16* dk;           // dense [T, Hkv, 64]
+  __nv_bfloat16* dv;           // dense [T, Hkv, 64]
+  const int32_t* cu_seqlens;   // nullable -> BSHD
+  int B, S, T, Hq, Hkv, G, window;
+  int n_tiles;                 // tiles of the longest sequence
+  float scale, scale_log2;
+};
+
+struct BwdSeq {
+  int64_t tok0;  // dense index of the sequence's first token
+  int L;         // its length
+};
+
+__device__ __forceinline__ BwdSeq bwd_seq(const BwdParams& p, int b) {
+  BwdSeq s;
+  if (p.cu_seqlens != nullptr) {
+    const int a = __ldg(p.cu_seqlens + b);
+    s.tok0 = a;
+    s.L = __ldg(p.cu_seqlens + b + 1) - a;
+  } else {
+    s.tok0 = static_cast<int64_t>(b) * p.S;
+    s.L = p.S;
+  }
+  return s;
+}
+
+// Index of (sequence b, head h, row i) in the lse / D layout.
+__device__ __forceinline__ int64_t bwd_row_index(const BwdParams& p, int b, int h, int i, int64_t tok0) {
+  return p.cu_seqlens != nullptr ? static_cast<int64_t>(h) * p.T + tok0 + i
+                                 : (static_cast<int64_t>(b) * p.Hq + h) * p.S + i;
+}
+
+// Row i of head h of sequence b in a strided bf16 tensor.
+__device__ __forceinline__ const __nv_bfloat16* bwd_row(const __nv_bfloat16* base, const gptoss_strides& s, int b,
+                                                        int64_t tok0, int i, int h, bool thd) {
+  return thd ? base + (tok0 + i) * s.tok + static_cast<int64_t>(h) * s.head
+             : base + static_cast<int64_t>(b) * s.batch + static_cast<int64_t>(i) * s.tok +
+                   static_cast<int64_t>(h) * s.head;
+}
+
+__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(&a);
+  const uint32_t* y = reinterpret_cast<const uint32_t*>(&b);
+  float acc = 0.f;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) acc += bf16lo(x[w]) * bf16lo(y[w]) + bf16hi(x[w]) * bf16hi(y[w]);
+  return acc;
+}
+
+// D = <dout, out> for 64 rows x every head of one sequence, and the sink
+// gradient -sum_i exp(sink_h - lse_i) D_i of those rows.  Grid (tiles, B).
+__global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const __grid_constant__ BwdParams p) {
+  __shared__ float part[kBwdMaxHeads];
+  const int b = blockIdx.y;
+  const BwdSeq sq = bwd_seq(p, b);
+  const int i0 = blockIdx.x * kBwdTile;
+  if (i0 >= sq.L) return;
+  for (int h = threadIdx.x; h < p.Hq; h += blockDim.x) part[h] = 0.f;
+  __syncthreads();
+  const bool thd = p.cu_seqlens != nullptr;
+  const int rows = min(kBwdTile, sq.L - i0);
+  for (int it = threadIdx.x; it < rows * p.Hq; it += blockDim.x) {
+    const int r = it / p.Hq, h = it - r * p.Hq;
+    const int i = i0 + r;
+    const uint4* o = reinterpret_cast<const uint4*>(bwd_row(p.out, p.so, b, sq.tok0, i, h, thd));
+    const uint4* d = reinterpret_cast<const uint4*>(bwd_row(p.dout, p.sdo, b, sq.tok0, i, h, thd));
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc += dot8_bf16(__ldg(o + c), __ldg(d + c));
+    const int64_t ri = bwd_row_index(p, b, h, i, sq.tok0);
+    p.dsum[ri] = acc;
+    const float share = ex2_approx((__ldg(p.sinks + h) - __ldg(p.lse + ri)) * kLog2e);
+    atomicAdd(&part[h], -share * acc);
+  }
+  __syncthreads();
+  for (int h = threadIdx.x; h < p.Hq; h += blockDim.x) atomicAdd(p.dsinks + h, part[h]);
+}
+
+// Is query row i allowed to see key j (both inside a sequence of length L)?
+__device__ __forceinline__ bool bwd_visible(int i, int j, int L, int window) {
+  return j <= i && i < L && (window == 0 || i - j < window);
+}
+
+// Rows (gr, gr + 8) of an mma.sync A fragment from global memory: 16 rows
+// starting at row0 (stride `row_stride` elements between rows), invalid rows
+// (>= n_valid) zero.
+__device__ __forceinline__ void load_a_frag(uint32_t (&a)[4][4], const __nv_bfloat16* row_lo,
+                                            const __nv_bfloat16* row_hi, bool lo_ok, bool hi_ok, int tq) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const int c = kk * 16 + 2 * tq;
+    a[kk][0] = lo_ok ? *reinterpret_cast<const uint32_t*>(row_lo + c) : 0u;
+    a[kk][1] = hi_ok ? *reinterpret_cast<const uint32_t*>(row_hi + c) : 0u;
+    a[kk][2] = lo_ok ? *reinterpret_cast<const uint32_t*>(row_lo + c + 8) : 0u;
+    a[kk][3] = hi_ok ? *reinterpret_cast<const uint32_t*>(row_hi + c + 8) : 0u;
+  }
+}
+
+// Writes a 16 x 64 fp32 accumulator (C fragments, rows gr / gr + 8) as bf16
+// rows, optionally scaled and taken back through RoPE: for pair (d, d + 32),
+// (x, y) -> (x cc + y cs, y cc - x cs) with (cc, cs) = the row's (c cos, c sin).
+__device__ __forceinline__ void store_rows(const float (&acc)[8][4], __nv_bfloat16* row_lo, __nv_bfloat16* row_hi,
+                                           const float2* cs_lo, const float2* cs_hi, bool lo_ok, bool hi_ok,
+                                           float scale, bool rotate, int tq) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const bool ok = half == 0 ? lo_ok : hi_ok;
+    if (!ok) continue;
+    __nv_bfloat16* row = half == 0 ? row_lo : row_hi;
+    const float2* cs = half == 0 ? cs_lo : cs_hi;
+    const int e0 = 2 * half;
+    if (!rotate) {
+#pragma unroll
+      for (int nf = 0; nf < 8; ++nf)
+        *reinterpret_cast<uint32_t*>(row + 8 * nf + 2 * tq) =
+            pack_bf16(acc[nf][e0] * scale, acc[nf][e0 + 1] * scale);
+      continue;
+    }
+#pragma unroll
+    for (int nf = 0; nf < 4; ++nf) {
+      const int d = 8 * nf + 2 * tq;  // pairs d, d + 1 and their partners d + 32, d + 33
+      float xr[2], yr[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float x = acc[nf][e0 + e] * scale, y = acc[nf + 4][e0 + e] * scale;
+        const float2 c = __ldg(cs + d + e);
+        xr[e] = x * c.x + y * c.y;
+        yr[e] = y * c.x - x * c.y;
+      }
+      *reinterpret_cast<uint32_t*>(row + d) = pack_bf16(xr[0], xr[1]);
+      *reinterpret_cast<uint32_t*>(row + d + 32) = pack_bf16(yr[0], yr[1]);
+    }
+  }
+}
+
+struct __align__(128) BwdKvSmem {
+  uint8_t q[2][kBwdTile * 128];     // rotated q tile (fp16), 128B-swizzled rows
+  uint8_t dout[2][kBwdTile * 128];  // dout tile (bf16)
+  float lse[2][kBwdTile];
+  float dsum[2][kBwdTile];
+};
+
+__global__ void __launch_bounds__(kBwdThreads) attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
+  __shared__ BwdKvSmem sm;
+  const int kt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const BwdSeq sq = bwd_seq(p, b);
+  const int k0 = kt * kBwdTile;
+  if (k0 >= sq.L) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, tq = lane & 3;
+  const bool thd = p.cu_seqlens != nullptr;
+  const int L = sq.L, W = p.window, G = p.G;
+  // query tiles that see this key tile: [kt, last row that sees key k0 + 63]
+  const int q_last = W > 0 ? min(L - 1, k0 + kBwdTile - 1 + W - 1) : L - 1;
+  const int n_qt = q_last / kBwdTile - kt + 1;
+  const int n_it = G * n_qt;
+
+  // this warp's 16 keys as A fragments: rotated K (fp16) and V (bf16)
+  const int j0 = k0 + warp * 16;
+  const int jl = j0 + gr, jh = j0 + gr + 8;
+  const bool jl_ok = jl < L, jh_ok = jh < L;
+  uint32_t ka[4][4], va[4][4];
+  load_a_frag(ka, p.kh + ((sq.tok0 + jl) * p.Hkv + g) * kHeadDim, p.kh + ((sq.tok0 + jh) * p.Hkv + g) * kHeadDim,
+              jl_ok, jh_ok, tq);
+  load_a_frag(va, bwd_row(p.v, p.sv, b, sq.tok0, jl, g, thd), bwd_row(p.v, p.sv, b, sq.tok0, jh, g, thd), jl_ok,
+              jh_ok, tq);
+
+  auto load = [&](int it, int buf) {
+    const int h = g * G + it / n_qt;
+    const int i0 = (kt + it % n_qt) * kBwdTile;
+    const uint32_t qs = smem_u32(sm.q[buf]), os = smem_u32(sm.dout[buf]);
+    for (int c = tid; c < kBwdTile * 8; c += kBwdThreads) {
+      const int r = c >> 3, ch = c & 7, i = i0 + r;
+      if (i < L) {
+        cp_async16(sw128_addr(qs, r, ch), p.qh + ((sq.tok0 + i) * p.Hq + h) * kHeadDim + 8 * ch);
+        cp_async16(sw128_addr(os, r, ch), bwd_row(p.dout, p.sdo, b, sq.tok0, i, h, thd) + 8 * ch);
+      } else {
+        st_shared_zero16(sw128_addr(qs, r, ch));
+        st_shared_zero16(sw128_addr(os, r, ch));
+      }
+    }
+    const int r = tid & (kBwdTile - 1), i = i0 + r;
+    float* dst = tid < kBwdTile ? &sm.lse[buf][r] : &sm.dsum[buf][r];
+    const float* src = tid < kBwdTile ? p.lse : p.dsum;
+    if (i < L) cp_async4(smem_u32(dst), src + bwd_row_index(p, b, h, i, sq.tok0));
+    else *dst = 0.f;
+  };
+
+  float dk[8][4], dv[8][4];
+#pragma unroll
+  for (int nf = 0; nf < 8; ++nf)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dk[nf][e] = dv[nf][e] = 0.f;
+
+  load(0, 0);
+  cp_async_commit();
+  for (int it = 0; it < n_it; ++it) {
+    const int buf = it & 1;
+    if (it + 1 < n_it) {
+      load(it + 1, buf ^ 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const int i0 = (kt + it % n_qt) * kBwdTile;
+    const uint32_t qs = smem_u32(sm.q[buf]), os = smem_u32(sm.dout[buf]);
+    // S^T = K Q^T and dP^T = V dout^T: this warp's 16 keys x 64 queries
+    float st[8][4], dpt[8][4];
+#pragma unroll
+    for (int nf = 0; nf < 8; ++nf) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) st[nf][e] = dpt[nf][e] = 0.f;
+      const int row = 8 * nf + (lane & 7);
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sw128_addr(qs, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
+        mma_f16_16816(st[nf], ka[2 * kp], b0, b1);
+        mma_f16_16816(st[nf], ka[2 * kp + 1], b2, b3);
+        ldsm_x4(sw128_addr(os, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
+        mma_bf16_16816(dpt[nf], va[2 * kp], b0, b1);
+        mma_bf16_16816(dpt[nf], va[2 * kp + 1], b2, b3);
+      }
+    }
+    // P^T = exp(S^T scale - lse) on the visible pairs, dS^T = P^T (dP^T - D)
+#pragma unroll
+    for (int nf = 0; nf < 8; ++nf)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int col = 8 * nf + 2 * tq + (e & 1);
+        const int i = i0 + col, j = (e < 2 ? jl : jh);
+        const bool vis = j < L && bwd_visible(i, j, L, W);
+        const float pv = vis ? ex2_approx(st[nf][e] * p.scale_log2 - sm.lse[buf][col] * kLog2e) : 0.f;
+        st[nf][e] = pv;
+        dpt[nf][e] = pv * (dpt[nf][e] - sm.dsum[buf][col]);
+      }
+    // dV += P^T dout, dK += dS^T Q (contraction over the 64 queries)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t pa[4], sa[4];
+      pa[0] = pack_bf16(st[2 * kk][0], st[2 * kk][1]);
+      pa[1] = pack_bf16(st[2 * kk][2], st[2 * kk][3]);
+      pa[2] = pack_bf16(st[2 * kk + 1][0], st[2 * kk + 1][1]);
+      pa[3] = pack_bf16(st[2 * kk + 1][2], st[2 * kk + 1][3]);
+      sa[0] = pack_f16(dpt[2 * kk][0], dpt[2 * kk][1]);
+      sa[1] = pack_f16(dpt[2 * kk][2], dpt[2 * kk][3]);
+      sa[2] = pack_f16(dpt[2 * kk + 1][0], dpt[2 * kk + 1][1]);
+      sa[3] = pack_f16(dpt[2 * kk + 1][2], dpt[2 * kk + 1][3]);
+      const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int dp = 0; dp < 4; ++dp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sw128_addr(os, row, 2 * dp + (lane >> 4)), b0, b1, b2, b3);
+        mma_bf16_16816(dv[2 * dp], pa, b0, b1);
+        mma_bf16_16816(dv[2 * dp + 1], pa, b2, b3);
+        ldsm_x4_t(sw128_addr(qs, row, 2 * dp + (lane >> 4)), b0, b1, b2, b3);
+        mma_f16_16816(dk[2 * dp], sa, b0, b1);
+        mma_f16_16816(dk[2 * dp + 1], sa, b2, b3);
+      }
+    }
+    __syncthreads();  // the buffer is refilled two iterations on
+  }
+  const int64_t tl = sq.tok0 + jl, th = sq.tok0 + jh;
+  store_rows(dv, p.dv + (tl * p.Hkv + g) * kHeadDim, p.dv + (th * p.Hkv + g) * kHeadDim, nullptr, nullptr, jl_ok,
+             jh_ok, 1.f, false, tq);
+  store_rows(dk, p.dk + (tl * p.Hkv + g) * kHeadDim, p.dk + (th * p.Hkv + g) * kHeadDim, p.cs + tl * kPairs,
+             p.cs + th * kPairs, jl_ok, jh_ok, p.scale, true, tq);
+}
+
+struct __align__(128) BwdQSmem {
+  uint8_t k[2][kBwdTile * 128];  // rotated k tile (fp16), 128B-swizzled rows
+  uint8_t v[2][kBwdTile * 128];  // v tile (bf16)
+};
+
+__global__ void __launch_bounds__(kBwdThreads) attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+  __shared__ BwdQSmem sm;
+  const int qt = p.n_tiles - 1 - static_cast<int>(blockIdx.x);  // the longest sweeps start first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / p.G;
+  const BwdSeq sq = bwd_seq(p, b);
+  const int i0 = qt * kBwdTile;
+  if (i0 >= sq.L) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, tq = lane & 3;
+  const bool thd = p.cu_seqlens != nullptr;
+  const int L = sq.L, W = p.window;
+  // key tiles this query tile sees
+  const int j_first = W > 0 ? max(0, i0 - W + 1) : 0;
+  const int kt_lo = j_first / kBwdTile, kt_hi = min(L - 1, i0 + kBwdTile - 1) / kBwdTile;
+  const int n_it = kt_hi - kt_lo + 1;
+
+  // this warp's 16 queries: rotated Q (fp16) and dout (bf16) as A fragments
+  const int il = i0 + warp * 16 + gr, ih = il + 8;
+  const bool il_ok = il < L, ih_ok = ih < L;
+  uint32_t qa[4][4], da[4][4];
+  load_a_frag(qa, p.qh + ((sq.tok0 + il) * p.Hq + h) * kHeadDim, p.qh + ((sq.tok0 + ih) * p.Hq + h) * kHeadDim,
+              il_ok, ih_ok, tq);
+  load_a_frag(da, bwd_row(p.dout, p.sdo, b, sq.tok0, il, h, thd), bwd_row(p.dout, p.sdo, b, sq.tok0, ih, h, thd),
+              il_ok, ih_ok, tq);
+  const float lse_l = il_ok ? __ldg(p.lse + bwd_row_index(p, b, h, il, sq.tok0)) * kLog2e : 0.f;
+  const float lse_h = ih_ok ? __ldg(p.lse + bwd_row_index(p, b, h, ih, sq.tok0)) * kLog2e : 0.f;
+  const float d_l = il_ok ? __ldg(p.dsum + bwd_row_index(p, b, h, il, sq.tok0)) : 0.f;
+  const float d_h = ih_ok ? __ldg(p.dsum + bwd_row_index(p, b, h, ih, sq.tok0)) : 0.f;
+
+  auto load = [&](int it, int buf) {
+    const int j0 = (kt_lo + it) * kBwdTile;
+    const uint32_t ks = smem_u32(sm.k[buf]), vs = smem_u32(sm.v[buf]);
+    for (int c = tid; c < kBwdTile * 8; c += kBwdThreads) {
+      const int r = c >> 3, ch = c & 7, j = j0 + r;
+      if (j < L) {
+        cp_async16(sw128_addr(ks, r, ch), p.kh + ((sq.tok0 + j) * p.Hkv + g) * kHeadDim + 8 * ch);
+        cp_async16(sw128_addr(vs, r, ch), bwd_row(p.v, p.sv, b, sq.tok0, j, g, thd) + 8 * ch);
+      } else {
+        st_shared_zero16(sw128_addr(ks, r, ch));
+        st_shared_zero16(sw128_addr(vs, r, ch));
+      }
+    }
+  };
+
+  float dq[8][4];
+#pragma unroll
+  for (int nf = 0; nf < 8; ++nf)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dq[nf][e] = 0.f;
+
+  load(0, 0);
+  cp_async_commit();
+  for (int it = 0; it < n_it; ++it) {
+    const int buf = it & 1;
+    if (it + 1 < n_it) {
+      load(it + 1, buf ^ 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const int j0 = (kt_lo + it) * kBwdTile;
+    const uint32_t ks = smem_u32(sm.k[buf]), vs = smem_u32(sm.v[buf]);
+    // S = Q K^T and dP = dout V^T: this warp's 16 queries x 64 keys
+    float s[8][4], dpv[8][4];
+#pragma unroll
+    for (int nf = 0; nf < 8; ++nf) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[nf][e] = dpv[nf][e] = 0.f;
+      const int row = 8 * nf + (lane & 7);
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sw128_addr(ks, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
+        mma_f16_16816(s[nf], qa[2 * kp], b0, b1);
+        mma_f16_16816(s[nf], qa[2 * kp + 1], b2, b3);
+        ldsm_x4(sw128_addr(vs, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
+        mma_bf16_16816(dpv[nf], da[2 * kp], b0, b1);
+        mma_bf16_16816(dpv[nf], da[2 * kp + 1], b2, b3);
+      }
+    }
+    // dS = P (dP - D) on the visible pairs
+#pragma unroll
+    for (int nf = 0; nf < 8; ++nf)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = j0 + 8 * nf + 2 * tq + (e & 1);
+        const int i = e < 2 ? il : ih;
+        const bool vis = j < L && bwd_visible(i, j, L, W);
+        const float pv = vis ? ex2_approx(s[nf][e] * p.scale_log2 - (e < 2 ? lse_l : lse_h)) : 0.f;
+        dpv[nf][e] = pv * (dpv[nf][e] - (e < 2 ? d_l : d_h));
+      }
+    // dQ += dS K (contraction over the 64 keys)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t sa[4];
+      sa[0] = pack_f16(dpv[2 * kk][0], dpv[2 * kk][1]);
+      sa[1] = pack_f16(dpv[2 * kk][2], dpv[2 * kk][3]);
+      sa[2] = pack_f16(dpv[2 * kk + 1][0], dpv[2 * kk + 1][1]);
+      sa[3] = pack_f16(dpv[2 * kk + 1][2], dpv[2 * kk + 1][3]);
+      const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int dp = 0; dp < 4; ++dp) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sw128_addr(ks, row, 2 * dp + (lane >> 4)), b0, b1, b2, b3);
+        mma_f16_16816(dq[2 * dp], sa, b0, b1);
+        mma_f16_16816(dq[2 * dp + 1], sa, b2, b3);
+      }
+    }
+    __syncthreads();  // the buffer is refilled two iterations on
+  }
+  const int64_t tl = sq.tok0 + il, th = sq.tok0 + ih;
+  store_rows(dq, p.dq + (tl * p.Hq + h) * kHeadDim, p.dq + (th * p.Hq + h) * kHeadDim, p.cs + tl * kPairs,
+             p.cs + th * kPairs, il_ok, ih_ok, p.scale, true, tq);
+}
+
+}  // namespace gptoss

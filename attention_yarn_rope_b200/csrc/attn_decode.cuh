@@ -30,6 +30,7 @@
 #include "host_util.cuh"
 #include "rope_qk.cuh"
 #include "sm100_ptx.cuh"
+#include "warp_mma.cuh"
 
 namespace gptoss {
 
@@ -80,31 +81,6 @@ __host__ __device__ inline int decode_chunk(int B, int Lmax, int Hkv) {
   if (c < 256) c = 256;
   if (c > 4096) c = 4096;
   return static_cast<int>(c);
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Address of 16-byte chunk `c` of row `r` in a 128B-swizzled tile at `base`.
-__device__ __forceinline__ uint32_t sw128_addr(uint32_t base, int r, int c) {
-  return base + r * 128 + ((c ^ (r & 7)) << 4);
 }
 
 struct __align__(1024) DecodeSmem {

@@ -1,0 +1,157 @@
+// bwd_host.cuh -- host side of the backward entry points of libgptoss_attn
+// (declared in include/gptoss.h): gptoss_attn_bwd_workspace_size and
+// gptoss_attn_bwd.  Included once by gptoss_lib.cu (one translation unit).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "attn_bwd.cuh"
+#include "gptoss.h"
+#include "host_util.cuh"
+#include "rope_qk.cuh"
+
+using namespace gptoss;
+
+namespace {
+
+inline size_t bwd_round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace: rotated q (fp16) | rotated k (fp16) | per-token (c cos, c sin)
+// table | D = <dout, out> (fp32, lse layout), each 256-byte aligned.
+struct BwdWorkspace {
+  size_t q, k, cs, d, total;
+};
+
+inline BwdWorkspace bwd_workspace(int64_t T, int Hq, int Hkv) {
+  BwdWorkspace w;
+  w.q = 0;
+  w.k = w.q + bwd_round256(static_cast<size_t>(T) * Hq * kHeadDim * 2);
+  w.cs = w.k + bwd_round256(static_cast<size_t>(T) * Hkv * kHeadDim * 2);
+  w.d = w.cs + bwd_round256(static_cast<size_t>(T) * kPairs * sizeof(float2));
+  w.total = w.d + bwd_round256(static_cast<size_t>(T) * Hq * sizeof(float));
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gptoss_attn_bwd_workspace_size(int32_t total_tokens, int32_t Hq, int32_t Hkv, int32_t D) {
+  if (total_tokens <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D != kHeadDim) return 0;
+  return bwd_workspace(total_tokens, Hq, Hkv).total;
+}
+
+gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk, const void* v,
+                              gptoss_strides sv, const void* out, gptoss_strides so, const void* dout,
+                              gptoss_strides sdo, const float* lse, const float* sinks, const int32_t* positions,
+                              const int32_t* cu_seqlens, int32_t B, int32_t S, int32_t total_tokens, int32_t Hq,
+                              int32_t Hkv, int32_t D, int32_t window, float softmax_scale,
+                              const gptoss_rope_params* rope, void* dq, void* dk, void* dv, float* dsinks,
+                              void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
+  if (B < 0 || S < 0 || total_tokens < 0 || Hq <= 0 || Hkv <= 0 || window < 0) return GPTOSS_ERR_INVALID_ARG;
+  if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
+  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (Hq > kBwdMaxHeads || B > 65535) return GPTOSS_ERR_UNSUPPORTED;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
+  gptoss_status st = check_rope(rope, D);
+  if (st != GPTOSS_OK) return st;
+  const bool thd = cu_seqlens != nullptr;
+  if (!thd && static_cast<int64_t>(B) * S != total_tokens) return GPTOSS_ERR_INVALID_ARG;
+  if (dsinks == nullptr) return GPTOSS_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (total_tokens == 0 || B == 0 || S == 0) {  // no rows: the sink gradient is zero
+    return cudaMemsetAsync(dsinks, 0, sizeof(float) * Hq, s) == cudaSuccess ? GPTOSS_OK : GPTOSS_ERR_CUDA;
+  }
+  if (!q || !k || !v || !out || !dout || !lse || !sinks || !dq || !dk || !dv || !workspace)
+    return GPTOSS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return GPTOSS_ERR_INVALID_ARG;
+  if (!strides_ok(sq, !thd) || !strides_ok(sk, !thd) || !strides_ok(sv, !thd) || !strides_ok(so, !thd) ||
+      !strides_ok(sdo, !thd))
+    return GPTOSS_ERR_INVALID_ARG;
+  const BwdWorkspace ws = bwd_workspace(total_tokens, Hq, Hkv);
+  if (workspace_bytes < ws.total) return GPTOSS_ERR_INVALID_ARG;
+  uint8_t* wsb = static_cast<uint8_t*>(workspace);
+
+  // 1. q and k rotated once (fp16) with every token's angle table; without
+  //    RoPE the identity table (angle 0, concentration 1) converts them
+  RopeQkParams rp;
+  memset(&rp, 0, sizeof(rp));
+  rp.q = static_cast<const __nv_bfloat16*>(q);
+  rp.k = static_cast<const __nv_bfloat16*>(k);
+  rp.q_out = reinterpret_cast<__nv_bfloat16*>(wsb + ws.q);  // fp16 bits
+  rp.k_out = reinterpret_cast<__nv_bfloat16*>(wsb + ws.k);
+  rp.sq = sq;
+  rp.sk = sk;
+  rp.sqo.head = kHeadDim;
+  rp.sqo.tok = static_cast<int64_t>(Hq) * kHeadDim;
+  rp.sqo.batch = thd ? 0 : static_cast<int64_t>(S) * Hq * kHeadDim;
+  rp.sko.head = kHeadDim;
+  rp.sko.tok = static_cast<int64_t>(Hkv) * kHeadDim;
+  rp.sko.batch = thd ? 0 : static_cast<int64_t>(S) * Hkv * kHeadDim;
+  rp.tm.positions = positions;
+  rp.tm.cu_seqlens = cu_seqlens;
+  rp.tm.nseq = B;
+  rp.tm.S = thd ? 0 : S;
+  rp.tm.ntok = total_tokens;
+  rp.Hq = Hq;
+  rp.Hkv = Hkv;
+  if (rope != nullptr) {
+    yarn_table(*rope, &rp.tab);
+  } else {
+    memset(&rp.tab, 0, sizeof(rp.tab));  // every inverse frequency 0: cos 1, sin 0
+    rp.tab.conc = 1.f;
+  }
+  rp.cs_out = reinterpret_cast<float2*>(wsb + ws.cs);
+  const int rgrid = (total_tokens + kRopeTokensPerCta - 1) / kRopeTokensPerCta;
+  rope_qk_kernel<true><<<rgrid, kRopeThreads, 0, s>>>(rp);
+  st = check_launch();
+  if (st != GPTOSS_OK) return st;
+
+  // 2. D = <dout, out> and the sink gradient
+  if (cudaMemsetAsync(dsinks, 0, sizeof(float) * Hq, s) != cudaSuccess) return GPTOSS_ERR_CUDA;
+  BwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.qh = rp.q_out;
+  p.kh = rp.k_out;
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.out = static_cast<const __nv_bfloat16*>(out);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.sv = sv;
+  p.so = so;
+  p.sdo = sdo;
+  p.lse = lse;
+  p.dsum = reinterpret_cast<float*>(wsb + ws.d);
+  p.cs = rp.cs_out;
+  p.sinks = sinks;
+  p.dsinks = dsinks;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.cu_seqlens = cu_seqlens;
+  p.B = B;
+  p.S = S;
+  p.T = total_tokens;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.window = window;
+  p.n_tiles = (S + kBwdTile - 1) / kBwdTile;
+  p.scale = softmax_scale;
+  p.scale_log2 = softmax_scale * kLog2e;
+  attn_bwd_preprocess_kernel<<<dim3(p.n_tiles, B), 256, 0, s>>>(p);
+  st = check_launch();
+  if (st != GPTOSS_OK) return st;
+
+  // 3. dK, dV (one CTA per key tile and kv head) and 4. dQ (one per query tile and head)
+  attn_bwd_dkdv_kernel<<<dim3(p.n_tiles, Hkv, B), kBwdThreads, 0, s>>>(p);
+  st = check_launch();
+  if (st != GPTOSS_OK) return st;
+  attn_bwd_dq_kernel<<<dim3(p.n_tiles, Hq, B), kBwdThreads, 0, s>>>(p);
+  return check_launch();
+}
+
+}  // extern "C"

@@ -140,6 +140,54 @@ def gptoss_attn_fwd(q, k, v, sinks, window: int = 0, softmax_scale: float | None
     return (out, lse) if (return_lse or lse is not None) else out
 
 
+def gptoss_attn_bwd_workspace_size(total_tokens: int, Hq: int, Hkv: int, D: int = 64) -> int:
+    return int(_abi.load().gptoss_attn_bwd_workspace_size(total_tokens, Hq, Hkv, D))
+
+
+def gptoss_attn_bwd(q, k, v, sinks, out, dout, lse, window: int = 0, softmax_scale: float | None = None,
+                    rope: RopeConfig | None = None, positions=None, cu_seqlens=None, max_seqlen: int | None = None,
+                    dq=None, dk=None, dv=None, dsinks=None, workspace=None, stream=None):
+    """Gradients of :func:`gptoss_attn_fwd` for ``L = sum(dout * out)``: q, k,
+    v, sinks, window, scale, rope, positions and cu_seqlens exactly as given to
+    the forward, ``out`` and ``lse`` from it.  Returns ``(dq, dk, dv, dsinks)``
+    (dq / dk / dv bf16 contiguous in q / k / v's logical shapes, dsinks fp32)."""
+    lib = _abi.load()
+    thd = cu_seqlens is not None
+    if thd:
+        T, Hq, D = q.shape
+        Hkv = k.shape[1]
+        B = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            if cu_seqlens.is_cuda:
+                raise ValueError("max_seqlen is required when cu_seqlens lives on the device")
+            max_seqlen = int((cu_seqlens[1:] - cu_seqlens[:-1]).max()) if B > 0 else 0
+        S, total = int(max_seqlen), T
+    else:
+        B, S, Hq, D = q.shape
+        Hkv = k.shape[2]
+        total = B * S
+    dq = torch.empty(q.shape, dtype=q.dtype, device=q.device) if dq is None else dq
+    dk = torch.empty(k.shape, dtype=k.dtype, device=k.device) if dk is None else dk
+    dv = torch.empty(v.shape, dtype=v.dtype, device=v.device) if dv is None else dv
+    dsinks = torch.empty(Hq, dtype=torch.float32, device=q.device) if dsinks is None else dsinks
+    for t in (dq, dk, dv, dsinks):
+        if not t.is_contiguous():
+            raise ValueError("gradient outputs must be contiguous")
+    need = gptoss_attn_bwd_workspace_size(total, Hq, Hkv, D) if total > 0 else 0
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check_dev(q, k, v, sinks, out, dout, lse, positions, cu_seqlens, dq, dk, dv, dsinks, workspace)
+    scale = float(D) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    r = rope.to_c() if rope is not None else None
+    st = lib.gptoss_attn_bwd(_ptr(q), _strides(q, thd), _ptr(k), _strides(k, thd), _ptr(v), _strides(v, thd),
+                             _ptr(out), _strides(out, thd), _ptr(dout), _strides(dout, thd), _ptr(lse), _ptr(sinks),
+                             _ptr(positions), _ptr(cu_seqlens), B, S, total, Hq, Hkv, D, int(window), scale,
+                             ctypes.byref(r) if r is not None else None, _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dsinks),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _abi.check("gptoss_attn_bwd", st)
+    return dq, dk, dv, dsinks
+
+
 def gptoss_attn_decode_workspace_size(B: int, Lmax: int, Hq: int, Hkv: int, D: int = 64) -> int:
     return int(_abi.load().gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D))
 

@@ -385,13 +385,14 @@ def run_ours(args, torch, dist, rank, world, device):
     if world == 1 and not args.no_extras:
         line["per_config"] = per_config(torch, ops, device, stream, peaks,
                                         [FULL, THD_FULL, THD_WINDOW],
-                                        [DECODE_B64, DECODE_B64_W, DECODE_B8, DECODE_B8_W], args)
+                                        [DECODE_B64, DECODE_B64_W, DECODE_B8, DECODE_B8_W], args,
+                                        bwd_cfgs=[SLIDING, FULL])
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(SLIDING, budget_s=args.cpu_seconds)
     return line
 
 
-def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, args):
+def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, args, bwd_cfgs=()):
     res = {}
     reps = max(3, min(args.steps, 20))
     for cfg in prefill_cfgs:
@@ -407,6 +408,37 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
             "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "visible_pairs": case["pairs"],
             "flops": case["flops"], "bytes": case["bytes"], "launches_per_call": 2}
         del case
+        torch.cuda.empty_cache()
+    # backward (training): dq, dk, dv, dsinks of the forward's output; 5
+    # products per visible pair and head (S and dP recomputed, dV, dK, dQ)
+    for cfg in bwd_cfgs:
+        case = prefill_case(torch, ops, cfg, device)
+        out, lse = ops.gptoss_attn_fwd(case["q"], case["k"], case["v"], case["sinks"], window=cfg.window,
+                                       rope=case["rope"], return_lse=True)
+        gen = torch.Generator(device=device).manual_seed(cfg.seed + 100)
+        dout = torch.randn(case["q"].shape, generator=gen, device=device).to(torch.bfloat16)
+        total = case["q"].shape[0] * case["q"].shape[1]
+        ws = torch.empty(ops.gptoss_attn_bwd_workspace_size(total, cfg.Hq, cfg.Hkv, cfg.D), dtype=torch.uint8,
+                         device=device)
+        dq, dk, dv = torch.empty_like(case["q"]), torch.empty_like(case["k"]), torch.empty_like(case["v"])
+        dsinks = torch.empty(cfg.Hq, dtype=torch.float32, device=device)
+
+        def bstep():
+            ops.gptoss_attn_bwd(case["q"], case["k"], case["v"], case["sinks"], out, dout, lse, window=cfg.window,
+                                rope=case["rope"], dq=dq, dk=dk, dv=dv, dsinks=dsinks, workspace=ws)
+        for _ in range(3):
+            bstep()
+        torch.cuda.synchronize()
+        ms = timed_steps(torch, bstep, reps, stream) / reps
+        flops = 2.5 * case["flops"]
+        tf = flops / (ms * 1e-3) / 1e12
+        io = sum(t.numel() * t.element_size() for t in (case["q"], case["k"], case["v"], out, dout, dq, dk, dv))
+        res["bwd_" + cfg.name] = {"ms": round(ms, 4), "tflops": round(tf, 2),
+                                  "frac_of_measured_bf16": round(tf / peaks["bf16_tflops"], 4),
+                                  "gbs_io": round(io / (ms * 1e-3) / 1e9, 1), "flops": flops, "io_bytes": io,
+                                  "launches_per_call": 4,
+                                  "note": "mma.sync kernels; dq recomputes S and dP instead of atomics"}
+        del case, out, lse, dout, ws, dq, dk, dv
         torch.cuda.empty_cache()
     flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
     for cfg in decode_cfgs:
@@ -502,8 +534,8 @@ def read_traffic(kernel, workload):
 # header that defines it, plus the host file that launches it (its own text
 # only: the library source also includes the other kernels' headers).
 _KERNEL_SOURCES = {
-    "attn_fwd_kernel": ("fwd_pipeline.cuh", "gptoss_lib.cu"),
-    "rope_qk_kernel<true>": ("rope_qk.cuh", "gptoss_lib.cu"),
+    "attn_fwd_kernel": ("fwd_pipeline.cuh", "fwd_host.cuh"),
+    "rope_qk_kernel<true>": ("rope_qk.cuh", "fwd_host.cuh"),
     "attn_decode_split_kernel": ("attn_decode.cuh", "decode_host.cuh"),
 }
 

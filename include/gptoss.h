@@ -155,6 +155,49 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
  * 32 fp32 pairs).  0 when a size is out of range. */
 size_t gptoss_attn_fwd_workspace_size(int32_t total_tokens, int32_t Hkv, int32_t D);
 
+/* Workspace bytes gptoss_attn_bwd needs: q and k rotated once (fp16), every
+ * token's 32 RoPE angles, and <dout, out> per row and head (fp32).  0 when a
+ * size is out of range. */
+size_t gptoss_attn_bwd_workspace_size(int32_t total_tokens, int32_t Hq, int32_t Hkv, int32_t D);
+
+/* gptoss_attn_bwd -- gradients of gptoss_attn_fwd for L = sum(dout * out):
+ * the derivative of the sink attention (GptOssAttention on the NeMo
+ * AutoModel gpt_oss.layers page, with RoPE of the gpt_oss.rope_utils page;
+ * the pages define the forward and train with it) by the chain rule:
+ *   D_i = <dout_i, out_i>, dS_ij = P_ij (<dout_i, v_j> - D_i) over the
+ *   visible pairs, dv_j = sum_i P_ij dout_i, dq'_i = scale sum_j dS_ij k'_j,
+ *   dk'_j = scale sum_i dS_ij q'_i, dsink_h = -sum_i exp(sink_h - lse_i) D_i
+ *   (summed over every row of every sequence), and through RoPE
+ *   dq = c R(theta)^T dq', dk = c R(theta)^T dk'.
+ *   q, k, v, sinks, positions, cu_seqlens, B, S, total_tokens, Hq, Hkv, D,
+ *          window, softmax_scale, rope: exactly as given to gptoss_attn_fwd
+ *          (q and k raw with rope != NULL, already rotated with rope == NULL).
+ *   out, dout  bf16, q's logical shape, own strides: the forward's output
+ *          and the gradient arriving at it.
+ *   lse    fp32 from the same forward call: [B,Hq,S] (BSHD) / [Hq,T] (THD).
+ *   dq     [B,S,Hq,D] / [T,Hq,D] bf16 contiguous (written).
+ *   dk, dv [B,S,Hkv,D] / [T,Hkv,D] bf16 contiguous (written; the sums over
+ *          the query heads of each kv group).
+ *   dsinks fp32 [Hq] (written, not accumulated into; zero when there are no
+ *          rows).
+ *   workspace  device memory of gptoss_attn_bwd_workspace_size(total_tokens,
+ *          Hq, Hkv, D) bytes, 16-byte aligned, owned by the caller, contents
+ *          need not be initialised.
+ * Four kernels on `stream`: q / k rotation, D and dsinks, dk / dv (one CTA
+ * per key tile and kv head), dq (one CTA per query tile and head).  The
+ * rotated q / k enter the products as fp16 like the forward's; P is rounded
+ * to bf16 and dS to fp16 for the products, accumulation is fp32.  dsinks is
+ * summed with floating-point atomics (order not fixed); every other output
+ * element has one writer. */
+gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
+                              const void* v, gptoss_strides sv, const void* out, gptoss_strides so,
+                              const void* dout, gptoss_strides sdo, const float* lse, const float* sinks,
+                              const int32_t* positions, const int32_t* cu_seqlens, int32_t B, int32_t S,
+                              int32_t total_tokens, int32_t Hq, int32_t Hkv, int32_t D, int32_t window,
+                              float softmax_scale, const gptoss_rope_params* rope, void* dq, void* dk,
+                              void* dv, float* dsinks, void* workspace, size_t workspace_bytes,
+                              struct CUstream_st* stream);
+
 /* Workspace bytes gptoss_attn_decode needs for these sizes (split-KV
  * partial results).  0 when a size is out of range. */
 size_t gptoss_attn_decode_workspace_size(int32_t B, int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D);

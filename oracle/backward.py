@@ -12,7 +12,8 @@ For one sequence, query head h (kv head g), with the forward's weights
 
     dv_j[g]   += sum_i w_ij dout_i[h]
     dP_ij      = <dout_i[h], v_j[g]>
-    D_i        = sum_j w_ij dP_ij  (= <dout_i[h], o_i[h]>)
+    D_i        = sum_j w_ij dP_ij  (= <dout_i[h], o_i[h]>; formed from a
+                                      stored output when one is given)
     dS_ij      = w_ij (dP_ij - D_i)
     dsink_h   += -sum_i a_i D_i          (the sink column has no value row)
     dq'_i[h]   = scale * sum_j dS_ij k'_j[g]
@@ -21,14 +22,15 @@ For one sequence, query head h (kv head g), with the forward's weights
 and through RoPE, which is linear (``x' = c R(theta) x`` per pair), the raw
 gradients are ``dq = c R(theta)^T dq'`` and ``dk = c R(theta)^T dk'``
 (:func:`rope_transpose`).  The weights are recomputed here from the
-definition; nothing is tiled or reordered.
+definition; as in the forward oracle, rows go in blocks, each evaluated over
+the keys it can see, and nothing else is tiled or reordered.
 """
 
 from __future__ import annotations
 
 import numpy as np
 
-from .attention import _visible_mask
+from .attention import _ROW_BLOCK, _visible_mask
 from .rope import default_positions_bshd, default_positions_thd, rope
 
 
@@ -50,15 +52,23 @@ def rope_transpose(g: np.ndarray, positions: np.ndarray, inv_freq: np.ndarray, c
     return out
 
 
-def sink_attention_sequence_bwd(q_rot, k_rot, v, sinks, scale, window, dout):
+def sink_attention_sequence_bwd(q_rot, k_rot, v, sinks, scale, window, dout, out=None):
     """One sequence.  q_rot / dout ``[L, Hq, D]``, k_rot / v ``[L, Hkv, D]``.
     Returns ``dq_rot [L, Hq, D]``, ``dk_rot [L, Hkv, D]``, ``dv [L, Hkv, D]``,
-    ``dsink [Hq]``."""
+    ``dsink [Hq]``.  ``out`` (``[L, Hq, D]``), when given, is the forward
+    output as the caller stores it, and ``D_i = <dout_i, out_i>`` is formed
+    from it (with the exact output this is the same number as
+    ``sum_j w_ij dP_ij``); otherwise D comes from the exact weights.  Rows are
+    taken in blocks of the forward's size, each over the key range it can see
+    (masked pairs contribute nothing); the key-side gradients add up over the
+    blocks."""
     q_rot = np.asarray(q_rot, np.float64)
     k_rot = np.asarray(k_rot, np.float64)
     v = np.asarray(v, np.float64)
     dout = np.asarray(dout, np.float64)
     sinks = np.asarray(sinks, np.float64)
+    if out is not None:
+        out = np.asarray(out, np.float64)
     L, Hq, D = q_rot.shape
     Hkv = k_rot.shape[1]
     G = Hq // Hkv
@@ -66,44 +76,48 @@ def sink_attention_sequence_bwd(q_rot, k_rot, v, sinks, scale, window, dout):
     dk = np.zeros_like(k_rot)
     dv = np.zeros_like(v)
     dsink = np.zeros(Hq, np.float64)
-    if L == 0:
-        return dq, dk, dv, dsink
-    rows = np.arange(L)
-    vis = _visible_mask(rows, rows, window)
-    for h in range(Hq):
-        g = h // G
-        s = scale * (q_rot[:, h, :] @ k_rot[:, g, :].T)
-        s = np.where(vis, s, -np.inf)
-        m = np.maximum(sinks[h], s.max(axis=1))
-        e = np.exp(s - m[:, None])
-        z = np.exp(sinks[h] - m) + e.sum(axis=1)
-        w = e / z[:, None]                       # weights of the visible pairs
-        share = np.exp(sinks[h] - m) / z         # the sink's share a_i
-        dv[:, g, :] += w.T @ dout[:, h, :]
-        dP = dout[:, h, :] @ v[:, g, :].T
-        Drow = (w * dP).sum(axis=1)
-        dS = w * (dP - Drow[:, None])
-        dsink[h] = -(share * Drow).sum()
-        dq[:, h, :] = scale * (dS @ k_rot[:, g, :])
-        dk[:, g, :] += scale * (dS.T @ q_rot[:, h, :])
+    for r0 in range(0, L, _ROW_BLOCK):
+        r1 = min(L, r0 + _ROW_BLOCK)
+        k0 = max(0, r0 - window + 1) if window > 0 else 0
+        vis = _visible_mask(np.arange(r0, r1), np.arange(k0, r1), window)
+        for h in range(Hq):
+            g = h // G
+            s = scale * (q_rot[r0:r1, h, :] @ k_rot[k0:r1, g, :].T)
+            s = np.where(vis, s, -np.inf)
+            m = np.maximum(sinks[h], s.max(axis=1))
+            e = np.exp(s - m[:, None])
+            z = np.exp(sinks[h] - m) + e.sum(axis=1)
+            w = e / z[:, None]                       # weights of the visible pairs
+            share = np.exp(sinks[h] - m) / z         # the sink's share a_i
+            dv[k0:r1, g, :] += w.T @ dout[r0:r1, h, :]
+            dP = dout[r0:r1, h, :] @ v[k0:r1, g, :].T
+            if out is None:
+                Drow = (w * dP).sum(axis=1)
+            else:
+                Drow = (dout[r0:r1, h, :] * out[r0:r1, h, :]).sum(axis=1)
+            dS = w * (dP - Drow[:, None])
+            dsink[h] -= (share * Drow).sum()
+            dq[r0:r1, h, :] = scale * (dS @ k_rot[k0:r1, g, :])
+            dk[k0:r1, g, :] += scale * (dS.T @ q_rot[r0:r1, h, :])
     return dq, dk, dv, dsink
 
 
-def _grads_of_sequence(q, k, v, sinks, scale, window, dout, pos, rope_tables):
+def _grads_of_sequence(q, k, v, sinks, scale, window, dout, pos, rope_tables, out):
     if rope_tables is None:
-        dq, dk, dv, ds = sink_attention_sequence_bwd(q, k, v, sinks, scale, window, dout)
+        dq, dk, dv, ds = sink_attention_sequence_bwd(q, k, v, sinks, scale, window, dout, out)
         return dq, dk, dv, ds
     inv_freq, conc = rope_tables
     qr = rope(q, pos, inv_freq, conc)
     kr = rope(k, pos, inv_freq, conc)
-    dqr, dkr, dv, ds = sink_attention_sequence_bwd(qr, kr, v, sinks, scale, window, dout)
+    dqr, dkr, dv, ds = sink_attention_sequence_bwd(qr, kr, v, sinks, scale, window, dout, out)
     return rope_transpose(dqr, pos, inv_freq, conc), rope_transpose(dkr, pos, inv_freq, conc), dv, ds
 
 
-def attn_bwd_bshd(q, k, v, sinks, scale, window, dout, rope_tables=None, positions=None):
+def attn_bwd_bshd(q, k, v, sinks, scale, window, dout, rope_tables=None, positions=None, out=None):
     """Gradients of ``sum(dout * attn_fwd_bshd(q, k, v, ...).out)``: ``dq [B, S,
     Hq, D]``, ``dk``, ``dv [B, S, Hkv, D]``, ``dsinks [Hq]`` (summed over the
-    batch).  ``rope_tables`` and ``positions`` as for the forward."""
+    batch).  ``rope_tables`` and ``positions`` as for the forward; ``out``
+    optional, the stored forward output D is formed from."""
     B, S = q.shape[:2]
     if positions is None:
         positions = default_positions_bshd(B, S)
@@ -113,14 +127,15 @@ def attn_bwd_bshd(q, k, v, sinks, scale, window, dout, rope_tables=None, positio
     dsinks = np.zeros(q.shape[2], np.float64)
     for b in range(B):
         dq[b], dk[b], dv[b], ds = _grads_of_sequence(q[b], k[b], v[b], sinks, scale, window, dout[b], positions[b],
-                                                     rope_tables)
+                                                     rope_tables, None if out is None else out[b])
         dsinks += ds
     return dq, dk, dv, dsinks
 
 
-def attn_bwd_thd(q, k, v, sinks, cu_seqlens, scale, window, dout, rope_tables=None, positions=None):
+def attn_bwd_thd(q, k, v, sinks, cu_seqlens, scale, window, dout, rope_tables=None, positions=None, out=None):
     """Packed THD gradients: ``dq [T, Hq, D]``, ``dk``, ``dv [T, Hkv, D]``,
-    ``dsinks [Hq]`` (summed over the sequences)."""
+    ``dsinks [Hq]`` (summed over the sequences); ``out`` as for
+    :func:`attn_bwd_bshd`."""
     cu = np.asarray(cu_seqlens, np.int64)
     if positions is None:
         positions = default_positions_thd(cu)
@@ -133,6 +148,7 @@ def attn_bwd_thd(q, k, v, sinks, cu_seqlens, scale, window, dout, rope_tables=No
         if b == a:
             continue
         dq[a:b], dk[a:b], dv[a:b], ds = _grads_of_sequence(q[a:b], k[a:b], v[a:b], sinks, scale, window, dout[a:b],
-                                                           positions[a:b], rope_tables)
+                                                           positions[a:b], rope_tables,
+                                                           None if out is None else out[a:b])
         dsinks += ds
     return dq, dk, dv, dsinks

@@ -84,6 +84,37 @@ def test_attn_fwd_validation(lib):
     assert _fwd(lib, S=0, T=0) == _abi.GPTOSS_OK
 
 
+def test_attn_bwd_validation(lib):
+    need = lib.gptoss_attn_bwd_workspace_size(4096, 64, 8, 64)
+    # rotated q and k (fp16) + per-token angle table + <dout, out> per row and head
+    assert need == 4096 * 64 * 64 * 2 + 4096 * 8 * 64 * 2 + 4096 * 32 * 8 + 4096 * 64 * 4
+    assert lib.gptoss_attn_bwd_workspace_size(4096, 64, 7, 64) == 0
+    assert lib.gptoss_attn_bwd_workspace_size(4096, 64, 8, 128) == 0
+
+    def call(**kw):
+        a = dict(q=FAKE, dout=FAKE, lse=FAKE, dq=FAKE, dsinks=FAKE, B=1, S=4096, T=4096, Hq=64, Hkv=8, D=64,
+                 window=0, scale=0.125, ws=FAKE, wsb=need, sq=S_BSHD_Q)
+        a.update(kw)
+        return lib.gptoss_attn_bwd(a["q"], a["sq"], FAKE, S_BSHD_K, FAKE, S_BSHD_K, FAKE, S_BSHD_Q, a["dout"],
+                                   S_BSHD_Q, a["lse"], FAKE, None, None, a["B"], a["S"], a["T"], a["Hq"], a["Hkv"],
+                                   a["D"], a["window"], a["scale"], ctypes.byref(ROPE), a["dq"], FAKE, FAKE,
+                                   a["dsinks"], a["ws"], a["wsb"], None)
+
+    assert call(D=128) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert call(Hq=2048, Hkv=8) == _abi.GPTOSS_ERR_UNSUPPORTED      # more heads than the sink reduction holds
+    assert call(Hkv=7) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(window=-1) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(T=4000) == _abi.GPTOSS_ERR_INVALID_ARG              # B*S != total for BSHD
+    assert call(dsinks=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(lse=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(dout=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(dq=ctypes.c_void_p(0x10008)) == _abi.GPTOSS_ERR_INVALID_ARG  # not 16-byte aligned
+    assert call(sq=_abi.Strides(0, 4097, 64)) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(wsb=need - 256) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(ws=None) == _abi.GPTOSS_ERR_INVALID_ARG
+
+
 def test_rope_qk_validation(lib):
     def call(**kw):
         a = dict(q=FAKE, k=FAKE, qo=FAKE, ko=FAKE, B=1, S=16, Hq=64, Hkv=8, D=64, rope=ctypes.byref(ROPE))

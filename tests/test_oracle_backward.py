@@ -137,6 +137,20 @@ def test_torch_autograd(window):
         np.testing.assert_allclose(got, ref.numpy(), rtol=1e-10, atol=1e-10)
 
 
+@pytest.mark.parametrize("window", [0, 200])
+def test_torch_autograd_several_row_blocks(window):
+    # 1100 rows: three of the oracle's row blocks, key ranges cut by the window
+    rng = np.random.default_rng(17)
+    q, k, v, sinks, dout = _case(rng, 1, 1100, 2, 1)
+    dq, dk, dv, ds = attn_bwd_bshd(q, k, v, sinks, SCALE, window, dout, rope_tables=TABLES)
+    tq, tk, tv, ts = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v, sinks))
+    out = _torch_forward(tq, tk, tv, ts, window, torch.tensor(TABLES[0]), TABLES[1],
+                         torch.tensor(default_positions_bshd(1, 1100)))
+    (out * torch.tensor(dout)).sum().backward()
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad), (ds, ts.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), rtol=1e-9, atol=1e-9)
+
+
 def test_rope_transpose_is_the_adjoint():
     rng = np.random.default_rng(9)
     x = rng.standard_normal((5, 3, 64))
@@ -168,3 +182,17 @@ def test_sink_minus_inf_has_zero_gradient():
     sinks[1] = -np.inf
     _, _, _, ds = attn_bwd_bshd(q, k, v, sinks, SCALE, 0, dout, rope_tables=TABLES)
     assert ds[1] == 0.0 and ds[0] != 0.0
+
+
+def test_given_exact_output_changes_nothing():
+    # D formed from the exact forward output equals D from the weights
+    rng = np.random.default_rng(19)
+    q, k, v, sinks, dout = _case(rng, 2, 40, 4, 2)
+    out, _ = attn_fwd_bshd(q, k, v, sinks, SCALE, 7, rope_tables=TABLES)
+    a = attn_bwd_bshd(q, k, v, sinks, SCALE, 7, dout, rope_tables=TABLES)
+    b = attn_bwd_bshd(q, k, v, sinks, SCALE, 7, dout, rope_tables=TABLES, out=out)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, rtol=0, atol=1e-12)
+    # a perturbed output moves D and, through dS, every gradient but dv
+    c = attn_bwd_bshd(q, k, v, sinks, SCALE, 7, dout, rope_tables=TABLES, out=out * (1 + 1e-3))
+    assert np.abs(c[0] - a[0]).max() > 1e-6 and np.array_equal(c[2], a[2])
