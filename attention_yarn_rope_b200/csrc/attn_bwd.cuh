@@ -23,6 +23,11 @@
 //      memory by cp.async.  Per step: S^T = K Q^T, dP^T = V dout^T, P^T and
 //      dS^T in registers, dV += P^T dout, dK += dS^T Q.  The epilogue applies
 //      scale and c R^T to dK and writes bf16: no atomics, one writer per row.
+//      A sweep longer than kBwdChunkIt steps (full causal: key tile 0 sees
+//      every query tile of every head) would leave a few CTAs running long
+//      after the rest, so when the longest sweep is longer the sweeps are cut
+//      into chunks, one CTA each, that add into fp32 dK / dV accumulators;
+//      attn_bwd_dkdv_finish_kernel then applies scale and c R^T and writes bf16.
 //   4. attn_bwd_dq_kernel: CTA (query tile, head, sequence); 4 warps of 16
 //      queries keep Q and dout as A fragments and sweep the key tiles the
 //      query tile sees (K and V double-buffered): S, dP, dS recomputed, dQ +=
@@ -41,6 +46,7 @@ namespace gptoss {
 constexpr int kBwdTile = 64;       // queries / keys per tile
 constexpr int kBwdThreads = 128;   // 4 warps x 16 rows
 constexpr int kBwdMaxHeads = 1024; // query heads the preprocess kernel reduces in shared memory
+constexpr int kBwdChunkIt = 128;   // (query head, query tile) steps of one dK / dV CTA when sweeps are split
 
 struct BwdParams {
   const __nv_bfloat16* qh;  // rotated q, fp16 bits, dense [T, Hq, 64]
@@ -57,6 +63,13 @@ struct BwdParams {
   __nv_bfloat16* dq;           // dense [T, Hq, 64]
   __nv_bfloat16* dk;           // dense [T, Hkv, 64]
   __nv_bfloat16* dv;           // dense [T, Hkv, 64]
+  // Split sweeps (max_chunks > 1): a (key tile, kv head) sweep longer than
+  // kBwdChunkIt steps is cut into chunks, one CTA each, which add their
+  // unscaled dK (rotated space) and dV into these fp32 accumulators (zeroed
+  // first); attn_bwd_dkdv_finish_kernel then writes dk / dv.
+  float* dk_acc;               // [T, Hkv, 64]
+  float* dv_acc;               // [T, Hkv, 64]
+  int max_chunks;
   const int32_t* cu_seqlens;   // nullable -> BSHD
   int B, S, T, Hq, Hkv, G, window;
   int n_tiles;                 // tiles of the longest sequence
@@ -197,9 +210,14 @@ struct __align__(128) BwdKvSmem {
   float dsum[2][kBwdTile];
 };
 
+// kSplit: grid z = (sequence, chunk); the CTA takes steps [chunk kBwdChunkIt,
+// (chunk + 1) kBwdChunkIt) of its sweep and adds into the fp32 accumulators.
+template <bool kSplit>
 __global__ void __launch_bounds__(kBwdThreads) attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
   __shared__ BwdKvSmem sm;
-  const int kt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int kt = blockIdx.x, g = blockIdx.y;
+  const int b = kSplit ? static_cast<int>(blockIdx.z) / p.max_chunks : static_cast<int>(blockIdx.z);
+  const int chunk = kSplit ? static_cast<int>(blockIdx.z) - b * p.max_chunks : 0;
   const BwdSeq sq = bwd_seq(p, b);
   const int k0 = kt * kBwdTile;
   if (k0 >= sq.L) return;
@@ -210,7 +228,10 @@ __global__ void __launch_bounds__(kBwdThreads) attn_bwd_dkdv_kernel(const __grid
   // query tiles that see this key tile: [kt, last row that sees key k0 + 63]
   const int q_last = W > 0 ? min(L - 1, k0 + kBwdTile - 1 + W - 1) : L - 1;
   const int n_qt = q_last / kBwdTile - kt + 1;
-  const int n_it = G * n_qt;
+  // this CTA's steps [it0, it1) of the sweep over (query head, query tile)
+  const int it0 = chunk * kBwdChunkIt;
+  if (it0 >= G * n_qt) return;
+  const int it1 = kSplit ? min(G * n_qt, it0 + kBwdChunkIt) : G * n_qt;
 
   // this warp's 16 keys as A fragments: rotated K (fp16) and V (bf16)
   const int j0 = k0 + warp * 16;
@@ -249,11 +270,11 @@ __global__ void __launch_bounds__(kBwdThreads) attn_bwd_dkdv_kernel(const __grid
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[nf][e] = dv[nf][e] = 0.f;
 
-  load(0, 0);
+  load(it0, 0);
   cp_async_commit();
-  for (int it = 0; it < n_it; ++it) {
-    const int buf = it & 1;
-    if (it + 1 < n_it) {
+  for (int it = it0; it < it1; ++it) {
+    const int buf = (it - it0) & 1;
+    if (it + 1 < it1) {
       load(it + 1, buf ^ 1);
       cp_async_commit();
       cp_async_wait<1>();
@@ -320,10 +341,42 @@ __global__ void __launch_bounds__(kBwdThreads) attn_bwd_dkdv_kernel(const __grid
     __syncthreads();  // the buffer is refilled two iterations on
   }
   const int64_t tl = sq.tok0 + jl, th = sq.tok0 + jh;
+  if (kSplit) {  // partial sums of this chunk: unscaled dK (rotated space) and dV
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      if (!(half == 0 ? jl_ok : jh_ok)) continue;
+      const int64_t row = ((half == 0 ? tl : th) * p.Hkv + g) * kHeadDim;
+      const int e0 = 2 * half;
+#pragma unroll
+      for (int nf = 0; nf < 8; ++nf) {
+        const int64_t o = row + 8 * nf + 2 * tq;
+        atomicAdd(reinterpret_cast<float2*>(p.dk_acc + o), make_float2(dk[nf][e0], dk[nf][e0 + 1]));
+        atomicAdd(reinterpret_cast<float2*>(p.dv_acc + o), make_float2(dv[nf][e0], dv[nf][e0 + 1]));
+      }
+    }
+    return;
+  }
   store_rows(dv, p.dv + (tl * p.Hkv + g) * kHeadDim, p.dv + (th * p.Hkv + g) * kHeadDim, nullptr, nullptr, jl_ok,
              jh_ok, 1.f, false, tq);
   store_rows(dk, p.dk + (tl * p.Hkv + g) * kHeadDim, p.dk + (th * p.Hkv + g) * kHeadDim, p.cs + tl * kPairs,
              p.cs + th * kPairs, jl_ok, jh_ok, p.scale, true, tq);
+}
+
+// Split sweeps: dk = c R^T (scale dK_acc) and dv = dV_acc as bf16.  Thread
+// (token, kv head, pair j) handles features j and j + 32.
+__global__ void __launch_bounds__(256) attn_bwd_dkdv_finish_kernel(const __grid_constant__ BwdParams p) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<int64_t>(p.T) * p.Hkv * kPairs) return;
+  const int j = static_cast<int>(idx % kPairs);
+  const int64_t tg = idx / kPairs;  // token * Hkv + kv head
+  const int64_t t = tg / p.Hkv;
+  const int64_t row = tg * kHeadDim;
+  const float x = p.dk_acc[row + j] * p.scale, y = p.dk_acc[row + j + kPairs] * p.scale;
+  const float2 c = __ldg(p.cs + t * kPairs + j);
+  p.dk[row + j] = __float2bfloat16_rn(x * c.x + y * c.y);
+  p.dk[row + j + kPairs] = __float2bfloat16_rn(y * c.x - x * c.y);
+  p.dv[row + j] = __float2bfloat16_rn(p.dv_acc[row + j]);
+  p.dv[row + j + kPairs] = __float2bfloat16_rn(p.dv_acc[row + j + kPairs]);
 }
 
 struct __align__(128) BwdQSmem {
@@ -331,7 +384,8 @@ struct __align__(128) BwdQSmem {
   uint8_t v[2][kBwdTile * 128];  // v tile (bf16)
 };
 
-__global__ void __launch_bounds__(kBwdThreads) attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+// 3 CTAs per SM: at most 170 registers a thread.
+__global__ void __launch_bounds__(kBwdThreads, 3) attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   __shared__ BwdQSmem sm;
   const int qt = p.n_tiles - 1 - static_cast<int>(blockIdx.x);  // the longest sweeps start first
   const int h = blockIdx.y, b = blockIdx.z;

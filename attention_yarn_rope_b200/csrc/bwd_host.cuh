@@ -5,6 +5,7 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstring>
 
 #include "attn_bwd.cuh"
@@ -19,9 +20,10 @@ namespace {
 inline size_t bwd_round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace: rotated q (fp16) | rotated k (fp16) | per-token (c cos, c sin)
-// table | D = <dout, out> (fp32, lse layout), each 256-byte aligned.
+// table | D = <dout, out> (fp32, lse layout) | dK and dV fp32 accumulators of
+// split sweeps (adjacent, zeroed with one memset), each 256-byte aligned.
 struct BwdWorkspace {
-  size_t q, k, cs, d, total;
+  size_t q, k, cs, d, acc, acc_bytes, total;
 };
 
 inline BwdWorkspace bwd_workspace(int64_t T, int Hq, int Hkv) {
@@ -30,7 +32,9 @@ inline BwdWorkspace bwd_workspace(int64_t T, int Hq, int Hkv) {
   w.k = w.q + bwd_round256(static_cast<size_t>(T) * Hq * kHeadDim * 2);
   w.cs = w.k + bwd_round256(static_cast<size_t>(T) * Hkv * kHeadDim * 2);
   w.d = w.cs + bwd_round256(static_cast<size_t>(T) * kPairs * sizeof(float2));
-  w.total = w.d + bwd_round256(static_cast<size_t>(T) * Hq * sizeof(float));
+  w.acc = w.d + bwd_round256(static_cast<size_t>(T) * Hq * sizeof(float));
+  w.acc_bytes = 2 * static_cast<size_t>(T) * Hkv * kHeadDim * sizeof(float);
+  w.total = w.acc + bwd_round256(w.acc_bytes);
   return w;
 }
 
@@ -142,12 +146,32 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   p.n_tiles = (S + kBwdTile - 1) / kBwdTile;
   p.scale = softmax_scale;
   p.scale_log2 = softmax_scale * kLog2e;
+  // The longest dK / dV sweep (key tile 0 of the longest sequence): split it
+  // into chunks of kBwdChunkIt steps when it has more, so no CTA runs far
+  // longer than the rest; the chunks add into fp32 accumulators.
+  const int64_t q_last0 = window > 0 ? std::min<int64_t>(S - 1, kBwdTile - 1 + window - 1) : S - 1;
+  const int64_t max_it = static_cast<int64_t>(p.G) * (q_last0 / kBwdTile + 1);
+  const int64_t max_chunks = (max_it + kBwdChunkIt - 1) / kBwdChunkIt;
+  const bool split = max_chunks > 1 && static_cast<int64_t>(B) * max_chunks <= 65535;
+  p.max_chunks = split ? static_cast<int>(max_chunks) : 1;
+  p.dk_acc = reinterpret_cast<float*>(wsb + ws.acc);
+  p.dv_acc = p.dk_acc + static_cast<int64_t>(total_tokens) * Hkv * kHeadDim;
+  if (split && cudaMemsetAsync(wsb + ws.acc, 0, ws.acc_bytes, s) != cudaSuccess) return GPTOSS_ERR_CUDA;
   attn_bwd_preprocess_kernel<<<dim3(p.n_tiles, B), 256, 0, s>>>(p);
   st = check_launch();
   if (st != GPTOSS_OK) return st;
 
-  // 3. dK, dV (one CTA per key tile and kv head) and 4. dQ (one per query tile and head)
-  attn_bwd_dkdv_kernel<<<dim3(p.n_tiles, Hkv, B), kBwdThreads, 0, s>>>(p);
+  // 3. dK, dV (one CTA per key tile and kv head, or per chunk of its sweep)
+  //    and 4. dQ (one per query tile and head)
+  if (split) {
+    attn_bwd_dkdv_kernel<true><<<dim3(p.n_tiles, Hkv, B * p.max_chunks), kBwdThreads, 0, s>>>(p);
+    st = check_launch();
+    if (st != GPTOSS_OK) return st;
+    const int64_t n = static_cast<int64_t>(total_tokens) * Hkv * kPairs;
+    attn_bwd_dkdv_finish_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
+  } else {
+    attn_bwd_dkdv_kernel<false><<<dim3(p.n_tiles, Hkv, B), kBwdThreads, 0, s>>>(p);
+  }
   st = check_launch();
   if (st != GPTOSS_OK) return st;
   attn_bwd_dq_kernel<<<dim3(p.n_tiles, Hq, B), kBwdThreads, 0, s>>>(p);

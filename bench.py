@@ -212,6 +212,30 @@ def prefill_case(torch, ops, cfg, device, seed_offset=0):
                 pairs=pairs, rope=rope, lens=lens, ws=ws)
 
 
+def bwd_case(torch, ops, cfg, device):
+    """The backward of one prefill workload: the forward runs once outside the
+    step for out / lse; the step is one gptoss_attn_bwd call (dq, dk, dv,
+    dsinks) with a preallocated workspace.  FLOP = 2.5 x the forward's (5
+    products of 2 D per visible pair and head)."""
+    case = prefill_case(torch, ops, cfg, device)
+    q, k, v, sinks, rope = case["q"], case["k"], case["v"], case["sinks"], case["rope"]
+    kw = {} if case["cu"] is None else dict(cu_seqlens=case["cu"], max_seqlen=max(case["lens"]))
+    out, lse = ops.gptoss_attn_fwd(q, k, v, sinks, window=cfg.window, rope=rope, return_lse=True, **kw)
+    gen = torch.Generator(device=device).manual_seed(cfg.seed + 100)
+    dout = torch.randn(q.shape, generator=gen, device=device).to(torch.bfloat16)
+    total = q.shape[0] * q.shape[1] if q.dim() == 4 else q.shape[0]
+    ws = torch.empty(ops.gptoss_attn_bwd_workspace_size(total, cfg.Hq, cfg.Hkv, cfg.D), dtype=torch.uint8,
+                     device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dsinks = torch.empty(cfg.Hq, dtype=torch.float32, device=device)
+
+    def step():
+        ops.gptoss_attn_bwd(q, k, v, sinks, out, dout, lse, window=cfg.window, rope=rope, dq=dq, dk=dk, dv=dv,
+                            dsinks=dsinks, workspace=ws, **kw)
+    io = sum(t.numel() * t.element_size() for t in (q, k, v, out, dout, dq, dk, dv))
+    return dict(step=step, flops=2.5 * case["flops"], bytes=io)
+
+
 def decode_case(torch, ops, cfg, device):
     from attention_yarn_rope_b200.workloads import make_decode_device
 
@@ -412,33 +436,18 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
     # backward (training): dq, dk, dv, dsinks of the forward's output; 5
     # products per visible pair and head (S and dP recomputed, dV, dK, dQ)
     for cfg in bwd_cfgs:
-        case = prefill_case(torch, ops, cfg, device)
-        out, lse = ops.gptoss_attn_fwd(case["q"], case["k"], case["v"], case["sinks"], window=cfg.window,
-                                       rope=case["rope"], return_lse=True)
-        gen = torch.Generator(device=device).manual_seed(cfg.seed + 100)
-        dout = torch.randn(case["q"].shape, generator=gen, device=device).to(torch.bfloat16)
-        total = case["q"].shape[0] * case["q"].shape[1]
-        ws = torch.empty(ops.gptoss_attn_bwd_workspace_size(total, cfg.Hq, cfg.Hkv, cfg.D), dtype=torch.uint8,
-                         device=device)
-        dq, dk, dv = torch.empty_like(case["q"]), torch.empty_like(case["k"]), torch.empty_like(case["v"])
-        dsinks = torch.empty(cfg.Hq, dtype=torch.float32, device=device)
-
-        def bstep():
-            ops.gptoss_attn_bwd(case["q"], case["k"], case["v"], case["sinks"], out, dout, lse, window=cfg.window,
-                                rope=case["rope"], dq=dq, dk=dk, dv=dv, dsinks=dsinks, workspace=ws)
+        case = bwd_case(torch, ops, cfg, device)
         for _ in range(3):
-            bstep()
+            case["step"]()
         torch.cuda.synchronize()
-        ms = timed_steps(torch, bstep, reps, stream) / reps
-        flops = 2.5 * case["flops"]
-        tf = flops / (ms * 1e-3) / 1e12
-        io = sum(t.numel() * t.element_size() for t in (case["q"], case["k"], case["v"], out, dout, dq, dk, dv))
+        ms = timed_steps(torch, case["step"], reps, stream) / reps
+        tf = case["flops"] / (ms * 1e-3) / 1e12
         res["bwd_" + cfg.name] = {"ms": round(ms, 4), "tflops": round(tf, 2),
                                   "frac_of_measured_bf16": round(tf / peaks["bf16_tflops"], 4),
-                                  "gbs_io": round(io / (ms * 1e-3) / 1e9, 1), "flops": flops, "io_bytes": io,
-                                  "launches_per_call": 4,
+                                  "gbs_io": round(case["bytes"] / (ms * 1e-3) / 1e9, 1), "flops": case["flops"],
+                                  "io_bytes": case["bytes"], "launches_per_call": 4,
                                   "note": "mma.sync kernels; dq recomputes S and dP instead of atomics"}
-        del case, out, lse, dout, ws, dq, dk, dv
+        del case
         torch.cuda.empty_cache()
     flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
     for cfg in decode_cfgs:
@@ -669,6 +678,8 @@ def profile_case(args):
     device = "cuda:0"
     if isinstance(cfg, wl.DecodeConfig):
         case = decode_case(torch, ops, cfg, device)
+    elif args.profile_bwd:
+        case = bwd_case(torch, ops, cfg, device)
     else:
         case = prefill_case(torch, ops, cfg, device)
     for _ in range(args.warmup + args.steps):
@@ -693,6 +704,8 @@ def main():
                     help="only launch this workload's kernel warmup+steps times (for ncu), e.g. "
                          "sliding_b4_s4096_w128, full_b2_s8192, decode_b64_l32768_full; no timing")
     ap.add_argument("--profile-batch", type=int, default=None, help="smaller batch for --profile-case")
+    ap.add_argument("--profile-bwd", action="store_true",
+                    help="with --profile-case of a prefill workload: launch its backward instead")
     args = ap.parse_args()
     if args.profile_case:
         return profile_case(args)

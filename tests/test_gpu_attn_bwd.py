@@ -197,6 +197,59 @@ def test_bwd_no_rows(cuda_device):
     assert torch.all(ds == 0)
 
 
+# Split sweeps: with G = 8 query heads per kv head, a key tile whose sweep
+# covers more than 16 query tiles (more than 128 (head, tile) steps) is cut
+# into chunks whose partial dK / dV add up in fp32 -- 1100 rows give key tile
+# 0 eighteen query tiles (two chunks); window 1000 seventeen.
+@pytest.mark.parametrize("window", [0, 1000])
+def test_bwd_split_sweeps(cuda_device, window):
+    rng = np.random.default_rng(137)
+    B, S, Hq, Hkv = 1, 1100, 16, 2
+    q, k, v, dout, sinks = _inputs(rng, (B, S), (B, S), Hq, Hkv)
+    out, lse = _oracle_fwd(q, k, v, sinks, window, TABLES)
+    got = _bwd(q, k, v, sinks, dout, out, lse, window, ROPE)
+    ref = attn_bwd_bshd(q, k, v, sinks.astype(np.float64), SCALE, window, dout, rope_tables=TABLES, out=out)
+    _check_all(got, ref, f"split sweeps w={window}")
+
+
+def test_bwd_split_sweeps_thd(cuda_device):
+    rng = np.random.default_rng(139)
+    cu = np.array([0, 5, 1105, 1200], np.int64)  # lengths 5, 1100, 95
+    T, Hq, Hkv = int(cu[-1]), 16, 2
+    q, k, v, dout, sinks = _inputs(rng, (T,), (T,), Hq, Hkv)
+    out, lse = _oracle_fwd(q, k, v, sinks, 0, TABLES, cu=cu)
+    got = _bwd(q, k, v, sinks, dout, out, lse, 0, ROPE, cu_seqlens=i32(cu), max_seqlen=1100)
+    ref = attn_bwd_thd(q, k, v, sinks.astype(np.float64), cu, SCALE, 0, dout, rope_tables=TABLES, out=out)
+    _check_all(got, ref, "split sweeps thd")
+
+
+def test_bwd_full_size_full_causal_slice(cuda_device):
+    # the full-causal workload (B=2, S=8192, 64 / 8 heads): key tile 0 sweeps
+    # 128 query tiles x 8 heads, cut into 8 chunks.  The GPU forward supplies
+    # out / lse everywhere except the checked slice (batch row 1, kv group 2),
+    # where the oracle's stored output and lse stand in; that slice's dq / dk /
+    # dv depend on nothing else
+    from attention_yarn_rope_b200.workloads import FULL, make_prefill
+
+    x = make_prefill(FULL)
+    dout = bf16_round(np.random.default_rng(149).standard_normal(x.q.shape, dtype=np.float32))
+    b, g, G = 1, 2, 8
+    heads = slice(g * G, (g + 1) * G)
+    sinks = x.sinks.astype(np.float64)[heads]
+    qs, ks, vs, ds_ = x.q[b:b + 1, :, heads], x.k[b:b + 1, :, g:g + 1], x.v[b:b + 1, :, g:g + 1], dout[b:b + 1, :, heads]
+    o_sl, l_sl = _oracle_fwd(qs, ks, vs, x.sinks[heads], 0, TABLES)
+    qd, kd, vd, sd = dev(x.q), dev(x.k), dev(x.v), f32(x.sinks)
+    out, lse = ops.gptoss_attn_fwd(qd, kd, vd, sd, window=0, rope=ROPE, return_lse=True)
+    out[b, :, heads] = dev(o_sl[0])
+    lse[b, heads, :] = f32(l_sl[0])
+    dq, dk, dv, _ = ops.gptoss_attn_bwd(qd, kd, vd, sd, out, dev(dout), lse, window=0, rope=ROPE)
+    torch.cuda.synchronize()
+    rq, rk, rv, _ = attn_bwd_bshd(qs, ks, vs, sinks, SCALE, 0, ds_, rope_tables=TABLES, out=o_sl)
+    assert_grad_parity(host(dq[b:b + 1, :, heads]), rq, "full causal dq")
+    assert_grad_parity(host(dk[b:b + 1, :, g:g + 1]), rk, "full causal dk")
+    assert_grad_parity(host(dv[b:b + 1, :, g:g + 1]), rv, "full causal dv")
+
+
 @pytest.mark.parametrize("window", [0, 1, 128])
 def test_bwd_end_to_end(cuda_device, window):
     # GPU forward -> GPU backward against the exact gradient
