@@ -16,18 +16,15 @@
 //      pairs; without RoPE the same kernel converts them with the identity.
 //   2. attn_bwd_preprocess_kernel: D for every (row, head) into the workspace,
 //      and the sink gradient (one atomic add per head and CTA).
-//   3. attn_bwd_dkdv_kernel: CTA (key tile, kv head, sequence); its 4 warps
-//      own 16 keys each and keep K and V as mma.sync A fragments in registers
-//      while they sweep every (query head of the group, query tile) that sees
-//      the key tile, with the q and dout tiles double-buffered through shared
-//      memory by cp.async.  Per step: S^T = K Q^T, dP^T = V dout^T, P^T and
-//      dS^T in registers, dV += P^T dout, dK += dS^T Q.  The epilogue applies
-//      scale and c R^T to dK and writes bf16: no atomics, one writer per row.
-//      A sweep longer than kBwdChunkIt steps (full causal: key tile 0 sees
-//      every query tile of every head) would leave a few CTAs running long
-//      after the rest, so when the longest sweep is longer the sweeps are cut
-//      into chunks, one CTA each, that add into fp32 dK / dV accumulators;
-//      attn_bwd_dkdv_finish_kernel then applies scale and c R^T and writes bf16.
+//   3. attn_bwd_dkdv_tc_kernel (attn_bwd_tc.cuh): dK and dV on the tcgen05
+//      tensor cores, one CTA per (128-key tile, kv head, sequence) sweeping
+//      every (query head of the group, 64-query tile) that sees the key tile:
+//      S^T = K Q^T, dP^T = V dout^T, P^T and dS^T through tensor memory, dV +=
+//      P^T dout, dK += dS^T Q, then scale and c R^T.  A sweep longer than one
+//      chunk (full causal: key tile 0 sees every query tile of every head)
+//      would leave a few CTAs running long after the rest, so long sweeps are
+//      cut into chunks, one CTA each, adding into fp32 dK / dV accumulators;
+//      attn_bwd_dkdv_finish_kernel then applies scale and c R^T, writes bf16.
 //   4. attn_bwd_dq_kernel: CTA (query tile, head, sequence); 4 warps of 16
 //      queries keep Q and dout as A fragments and sweep the key tiles the
 //      query tile sees (K and V double-buffered): S, dP, dS recomputed, dQ +=
@@ -46,9 +43,12 @@ namespace gptoss {
 constexpr int kBwdTile = 64;       // queries / keys per tile
 constexpr int kBwdThreads = 128;   // 4 warps x 16 rows
 constexpr int kBwdMaxHeads = 1024; // query heads the preprocess kernel reduces in shared memory
-constexpr int kBwdChunkIt = 128;   // (query head, query tile) steps of one dK / dV CTA when sweeps are split
 
 struct BwdParams {
+  // tensor maps of the tcgen05 dK / dV kernel (dims d, head, token, batch;
+  // 128B swizzle): rotated k / q in the workspace (fp16), v and dout (bf16)
+  CUtensorMap tmap_k, tmap_v, tmap_q, tmap_do;
+  uint64_t wait_ns;         // bound of every device-side wait
   const __nv_bfloat16* qh;  // rotated q, fp16 bits, dense [T, Hq, 64]
   const __nv_bfloat16* kh;  // rotated k, fp16 bits, dense [T, Hkv, 64]
   const __nv_bfloat16* v;
@@ -64,7 +64,7 @@ struct BwdParams {
   __nv_bfloat16* dk;           // dense [T, Hkv, 64]
   __nv_bfloat16* dv;           // dense [T, Hkv, 64]
   // Split sweeps (max_chunks > 1): a (key tile, kv head) sweep longer than
-  // kBwdChunkIt steps is cut into chunks, one CTA each, which add their
+  // kBwdTcChunkIt steps is cut into chunks, one CTA each, which add their
   // unscaled dK (rotated space) and dV into these fp32 accumulators (zeroed
   // first); attn_bwd_dkdv_finish_kernel then writes dk / dv.
   float* dk_acc;               // [T, Hkv, 64]
@@ -201,165 +201,6 @@ __device__ __forceinline__ void store_rows(const float (&acc)[8][4], __nv_bfloat
       *reinterpret_cast<uint32_t*>(row + d + 32) = pack_bf16(yr[0], yr[1]);
     }
   }
-}
-
-struct __align__(128) BwdKvSmem {
-  uint8_t q[2][kBwdTile * 128];     // rotated q tile (fp16), 128B-swizzled rows
-  uint8_t dout[2][kBwdTile * 128];  // dout tile (bf16)
-  float lse[2][kBwdTile];
-  float dsum[2][kBwdTile];
-};
-
-// kSplit: grid z = (sequence, chunk); the CTA takes steps [chunk kBwdChunkIt,
-// (chunk + 1) kBwdChunkIt) of its sweep and adds into the fp32 accumulators.
-template <bool kSplit>
-__global__ void __launch_bounds__(kBwdThreads) attn_bwd_dkdv_kernel(const __grid_constant__ BwdParams p) {
-  __shared__ BwdKvSmem sm;
-  const int kt = blockIdx.x, g = blockIdx.y;
-  const int b = kSplit ? static_cast<int>(blockIdx.z) / p.max_chunks : static_cast<int>(blockIdx.z);
-  const int chunk = kSplit ? static_cast<int>(blockIdx.z) - b * p.max_chunks : 0;
-  const BwdSeq sq = bwd_seq(p, b);
-  const int k0 = kt * kBwdTile;
-  if (k0 >= sq.L) return;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gr = lane >> 2, tq = lane & 3;
-  const bool thd = p.cu_seqlens != nullptr;
-  const int L = sq.L, W = p.window, G = p.G;
-  // query tiles that see this key tile: [kt, last row that sees key k0 + 63]
-  const int q_last = W > 0 ? min(L - 1, k0 + kBwdTile - 1 + W - 1) : L - 1;
-  const int n_qt = q_last / kBwdTile - kt + 1;
-  // this CTA's steps [it0, it1) of the sweep over (query head, query tile)
-  const int it0 = chunk * kBwdChunkIt;
-  if (it0 >= G * n_qt) return;
-  const int it1 = kSplit ? min(G * n_qt, it0 + kBwdChunkIt) : G * n_qt;
-
-  // this warp's 16 keys as A fragments: rotated K (fp16) and V (bf16)
-  const int j0 = k0 + warp * 16;
-  const int jl = j0 + gr, jh = j0 + gr + 8;
-  const bool jl_ok = jl < L, jh_ok = jh < L;
-  uint32_t ka[4][4], va[4][4];
-  load_a_frag(ka, p.kh + ((sq.tok0 + jl) * p.Hkv + g) * kHeadDim, p.kh + ((sq.tok0 + jh) * p.Hkv + g) * kHeadDim,
-              jl_ok, jh_ok, tq);
-  load_a_frag(va, bwd_row(p.v, p.sv, b, sq.tok0, jl, g, thd), bwd_row(p.v, p.sv, b, sq.tok0, jh, g, thd), jl_ok,
-              jh_ok, tq);
-
-  auto load = [&](int it, int buf) {
-    const int h = g * G + it / n_qt;
-    const int i0 = (kt + it % n_qt) * kBwdTile;
-    const uint32_t qs = smem_u32(sm.q[buf]), os = smem_u32(sm.dout[buf]);
-    for (int c = tid; c < kBwdTile * 8; c += kBwdThreads) {
-      const int r = c >> 3, ch = c & 7, i = i0 + r;
-      if (i < L) {
-        cp_async16(sw128_addr(qs, r, ch), p.qh + ((sq.tok0 + i) * p.Hq + h) * kHeadDim + 8 * ch);
-        cp_async16(sw128_addr(os, r, ch), bwd_row(p.dout, p.sdo, b, sq.tok0, i, h, thd) + 8 * ch);
-      } else {
-        st_shared_zero16(sw128_addr(qs, r, ch));
-        st_shared_zero16(sw128_addr(os, r, ch));
-      }
-    }
-    const int r = tid & (kBwdTile - 1), i = i0 + r;
-    float* dst = tid < kBwdTile ? &sm.lse[buf][r] : &sm.dsum[buf][r];
-    const float* src = tid < kBwdTile ? p.lse : p.dsum;
-    if (i < L) cp_async4(smem_u32(dst), src + bwd_row_index(p, b, h, i, sq.tok0));
-    else *dst = 0.f;
-  };
-
-  float dk[8][4], dv[8][4];
-#pragma unroll
-  for (int nf = 0; nf < 8; ++nf)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dk[nf][e] = dv[nf][e] = 0.f;
-
-  load(it0, 0);
-  cp_async_commit();
-  for (int it = it0; it < it1; ++it) {
-    const int buf = (it - it0) & 1;
-    if (it + 1 < it1) {
-      load(it + 1, buf ^ 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int i0 = (kt + it % n_qt) * kBwdTile;
-    const uint32_t qs = smem_u32(sm.q[buf]), os = smem_u32(sm.dout[buf]);
-    // S^T = K Q^T and dP^T = V dout^T: this warp's 16 keys x 64 queries
-    float st[8][4], dpt[8][4];
-#pragma unroll
-    for (int nf = 0; nf < 8; ++nf) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st[nf][e] = dpt[nf][e] = 0.f;
-      const int row = 8 * nf + (lane & 7);
-#pragma unroll
-      for (int kp = 0; kp < 2; ++kp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(sw128_addr(qs, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
-        mma_f16_16816(st[nf], ka[2 * kp], b0, b1);
-        mma_f16_16816(st[nf], ka[2 * kp + 1], b2, b3);
-        ldsm_x4(sw128_addr(os, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
-        mma_bf16_16816(dpt[nf], va[2 * kp], b0, b1);
-        mma_bf16_16816(dpt[nf], va[2 * kp + 1], b2, b3);
-      }
-    }
-    // P^T = exp(S^T scale - lse) on the visible pairs, dS^T = P^T (dP^T - D)
-#pragma unroll
-    for (int nf = 0; nf < 8; ++nf)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = 8 * nf + 2 * tq + (e & 1);
-        const int i = i0 + col, j = (e < 2 ? jl : jh);
-        const bool vis = j < L && bwd_visible(i, j, L, W);
-        const float pv = vis ? ex2_approx(st[nf][e] * p.scale_log2 - sm.lse[buf][col] * kLog2e) : 0.f;
-        st[nf][e] = pv;
-        dpt[nf][e] = pv * (dpt[nf][e] - sm.dsum[buf][col]);
-      }
-    // dV += P^T dout, dK += dS^T Q (contraction over the 64 queries)
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t pa[4], sa[4];
-      pa[0] = pack_bf16(st[2 * kk][0], st[2 * kk][1]);
-      pa[1] = pack_bf16(st[2 * kk][2], st[2 * kk][3]);
-      pa[2] = pack_bf16(st[2 * kk + 1][0], st[2 * kk + 1][1]);
-      pa[3] = pack_bf16(st[2 * kk + 1][2], st[2 * kk + 1][3]);
-      sa[0] = pack_f16(dpt[2 * kk][0], dpt[2 * kk][1]);
-      sa[1] = pack_f16(dpt[2 * kk][2], dpt[2 * kk][3]);
-      sa[2] = pack_f16(dpt[2 * kk + 1][0], dpt[2 * kk + 1][1]);
-      sa[3] = pack_f16(dpt[2 * kk + 1][2], dpt[2 * kk + 1][3]);
-      const int row = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int dp = 0; dp < 4; ++dp) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sw128_addr(os, row, 2 * dp + (lane >> 4)), b0, b1, b2, b3);
-        mma_bf16_16816(dv[2 * dp], pa, b0, b1);
-        mma_bf16_16816(dv[2 * dp + 1], pa, b2, b3);
-        ldsm_x4_t(sw128_addr(qs, row, 2 * dp + (lane >> 4)), b0, b1, b2, b3);
-        mma_f16_16816(dk[2 * dp], sa, b0, b1);
-        mma_f16_16816(dk[2 * dp + 1], sa, b2, b3);
-      }
-    }
-    __syncthreads();  // the buffer is refilled two iterations on
-  }
-  const int64_t tl = sq.tok0 + jl, th = sq.tok0 + jh;
-  if (kSplit) {  // partial sums of this chunk: unscaled dK (rotated space) and dV
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      if (!(half == 0 ? jl_ok : jh_ok)) continue;
-      const int64_t row = ((half == 0 ? tl : th) * p.Hkv + g) * kHeadDim;
-      const int e0 = 2 * half;
-#pragma unroll
-      for (int nf = 0; nf < 8; ++nf) {
-        const int64_t o = row + 8 * nf + 2 * tq;
-        atomicAdd(reinterpret_cast<float2*>(p.dk_acc + o), make_float2(dk[nf][e0], dk[nf][e0 + 1]));
-        atomicAdd(reinterpret_cast<float2*>(p.dv_acc + o), make_float2(dv[nf][e0], dv[nf][e0 + 1]));
-      }
-    }
-    return;
-  }
-  store_rows(dv, p.dv + (tl * p.Hkv + g) * kHeadDim, p.dv + (th * p.Hkv + g) * kHeadDim, nullptr, nullptr, jl_ok,
-             jh_ok, 1.f, false, tq);
-  store_rows(dk, p.dk + (tl * p.Hkv + g) * kHeadDim, p.dk + (th * p.Hkv + g) * kHeadDim, p.cs + tl * kPairs,
-             p.cs + th * kPairs, jl_ok, jh_ok, p.scale, true, tq);
 }
 
 // Split sweeps: dk = c R^T (scale dK_acc) and dv = dV_acc as bf16.  Thread

@@ -1,0 +1,352 @@
+// attn_bwd_tc.cuh -- dK and dV of the sink attention backward on the 5th-
+// generation tensor cores (tcgen05, accumulators in tensor memory).
+//
+// Rule: as attn_bwd.cuh (the derivative of GptOssAttention's forward, NeMo
+// AutoModel gpt_oss.layers page, with the RoPE of gpt_oss.rope_utils): for a
+// key tile of kv head g, dV = sum over the query heads h of the group and
+// every query row i that sees the key of P_ij dout_i, and dK' = scale * sum
+// dS_ij q'_i, dS_ij = P_ij (dP_ij - D_i), P_ij = exp(s_ij - lse_i).
+//
+// CTA = (128-key tile, kv head, sequence[, chunk of its sweep]), 10 warps:
+//   warps 0-7  softmax: warp w reads TMEM lanes 32 (w % 4) .. + 31 (key rows)
+//              and query columns 32 (w / 4) .. + 31 of the step; per step each
+//              thread reads its half row of S^T and dP^T from tensor memory,
+//              forms P^T (bf16) and dS^T (fp16) for those 32 queries and stores
+//              them back to tensor memory for the gradient products; at the
+//              end warps 0-3 read and write dV, warps 4-7 dK (scale and c R^T),
+//              or add them into fp32 accumulators when sweeps are split;
+//   warp 8     TMA producer: K and V tiles once, then per step the step's
+//              rotated q tile (fp16) and dout tile (bf16), kBwdTcStages ahead;
+//   warp 9     MMA issuer (one thread) and tensor-memory owner.
+// Per step (query head h, 64-query tile), all M = 128, N = 64, K = 4 x 16:
+//   S^T  = K Q^T            (SS, fp16, both K-major)
+//   dP^T = V dout^T         (SS, bf16, both K-major)
+//   dV  += P^T dout         (TS: P^T from tensor memory, dout read N-major)
+//   dK  += dS^T Q           (TS: dS^T from tensor memory, Q read N-major)
+// S^T / dP^T / P^T / dS^T have two tensor-memory sets, so step t's S^T and
+// dP^T products run while the softmax warps work on step t-1; the gradient
+// products of step t-1 are issued right after step t's S^T / dP^T.
+// Tensor memory (512 columns): set X at 192 X: S^T [0, 64), dP^T [64, 128),
+// P^T [128, 160), dS^T [160, 192); dV [384, 448), dK [448, 512).
+#pragma once
+
+#include "attn_bwd.cuh"
+#include "host_util.cuh"
+#include "sm100_ptx.cuh"
+
+namespace gptoss {
+
+constexpr int kBwdTcKeys = 128;      // keys per CTA (the M side)
+constexpr int kBwdTcQ = 64;          // queries per step (the N side)
+constexpr int kBwdTcStages = 4;      // q / dout buffers: loads run 3 steps ahead of their use
+constexpr int kBwdTcSoftmax = 256;   // 8 softmax warps
+constexpr int kBwdTcThreads = kBwdTcSoftmax + 64;  // + producer warp, MMA warp
+constexpr int kBwdTcChunkIt = 64;    // steps of one CTA when sweeps are split
+constexpr uint32_t kBwdTcTmemCols = 512;
+constexpr uint32_t kColSet = 192, kColDP = 64, kColP = 128, kColDS = 160, kColDV = 384, kColDK = 448;
+
+struct __align__(1024) BwdTcSmem {
+  uint8_t k[kBwdTcKeys * 128];                 // rotated K tile (fp16), 128B-swizzled rows
+  uint8_t v[kBwdTcKeys * 128];                 // V tile (bf16)
+  uint8_t q[kBwdTcStages][kBwdTcQ * 128];      // rotated q tiles (fp16)
+  uint8_t dout[kBwdTcStages][kBwdTcQ * 128];   // dout tiles (bf16)
+  float lsd[2][2 * kBwdTcQ];                   // per step: lse * log2(e) [0, 64), D [64, 128)
+  uint64_t kv_full;
+  uint64_t qd_full[kBwdTcStages], qd_empty[kBwdTcStages];
+  uint64_t s_full[2], s_free[2], p_full[2];
+  uint64_t lsd_ready[2];  // the softmax threads have written lsd[X] (a bounded wait, unlike bar.sync)
+  uint64_t mma_done;
+  uint32_t tmem_base;
+};
+
+// 32 lanes x 16 consecutive 32-bit columns (thread i writes lane base + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// fp16 A and B with B read N-major (the q tile in dK += dS^T Q).
+__host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) { return idesc_f16_f32(M, N) | (1u << 16); }
+
+// The CTA's sweep: steps [it0, it1) over (query head of the group, query
+// tile), query tiles [qt0, qt0 + n_qt) of the sequence.
+struct BwdTcWork {
+  int b, kt, k0, qt0, n_qt, it0, it1;
+  BwdSeq sq;
+};
+
+template <bool kSplit>
+__device__ __forceinline__ bool bwd_tc_work(const BwdParams& p, BwdTcWork& w) {
+  w.kt = blockIdx.x;
+  w.b = kSplit ? static_cast<int>(blockIdx.z) / p.max_chunks : static_cast<int>(blockIdx.z);
+  const int chunk = kSplit ? static_cast<int>(blockIdx.z) - w.b * p.max_chunks : 0;
+  w.sq = bwd_seq(p, w.b);
+  w.k0 = w.kt * kBwdTcKeys;
+  if (w.k0 >= w.sq.L) return false;
+  const int L = w.sq.L, W = p.window;
+  // queries that see a key of the tile: [k0, last row that sees key k0 + 127]
+  const int q_last = W > 0 ? min(L - 1, w.k0 + kBwdTcKeys - 1 + W - 1) : L - 1;
+  w.qt0 = w.k0 / kBwdTcQ;
+  w.n_qt = q_last / kBwdTcQ - w.qt0 + 1;
+  const int n_it = p.G * w.n_qt;
+  w.it0 = chunk * kBwdTcChunkIt;
+  if (w.it0 >= n_it) return false;
+  w.it1 = kSplit ? min(n_it, w.it0 + kBwdTcChunkIt) : n_it;
+  return true;
+}
+
+__device__ __forceinline__ void bwd_tc_producer(const BwdParams& p, BwdTcSmem& sm, const BwdTcWork& w, int g) {
+  tma_prefetch_desc(&p.tmap_k);
+  tma_prefetch_desc(&p.tmap_v);
+  tma_prefetch_desc(&p.tmap_q);
+  tma_prefetch_desc(&p.tmap_do);
+  const bool thd = p.cu_seqlens != nullptr;
+  const int row0 = thd ? static_cast<int>(w.sq.tok0) : 0;  // token row of the sequence's first token
+  const int bc = thd ? 0 : w.b;
+  mbar_arrive_expect_tx(&sm.kv_full, 2 * kBwdTcKeys * 128);
+  tma_load_4d(sm.k, &p.tmap_k, &sm.kv_full, 0, g, row0 + w.k0, bc);
+  tma_load_4d(sm.v, &p.tmap_v, &sm.kv_full, 0, g, row0 + w.k0, bc);
+  int issued = 0;
+  for (int it = w.it0; it < w.it1; ++it, ++issued) {
+    const int t = it - w.it0, s = t % kBwdTcStages;
+    if (!mbar_wait(&sm.qd_empty[s], ((t / kBwdTcStages) & 1) ^ 1, p.wait_ns)) break;
+    const int h = g * p.G + it / w.n_qt;
+    const int i0 = (w.qt0 + it % w.n_qt) * kBwdTcQ;
+    mbar_arrive_expect_tx(&sm.qd_full[s], 2 * kBwdTcQ * 128);
+    tma_load_4d(sm.q[s], &p.tmap_q, &sm.qd_full[s], 0, h, row0 + i0, bc);
+    tma_load_4d(sm.dout[s], &p.tmap_do, &sm.qd_full[s], 0, h, row0 + i0, bc);
+  }
+  // every issued copy must land before the CTA may exit
+  mbar_wait(&sm.kv_full, 0, p.wait_ns);
+  for (int t = issued > kBwdTcStages ? issued - kBwdTcStages : 0; t < issued; ++t)
+    mbar_wait(&sm.qd_full[t % kBwdTcStages], (t / kBwdTcStages) & 1, p.wait_ns);
+}
+
+__device__ __forceinline__ void bwd_tc_mma(const BwdParams& p, BwdTcSmem& sm, const BwdTcWork& w, uint32_t tmem) {
+  constexpr uint32_t idesc_s = idesc_f16_f32(128, 64);          // K (fp16) x Q^T
+  constexpr uint32_t idesc_dp = idesc_bf16_f32(128, 64, false);  // V (bf16) x dout^T
+  constexpr uint32_t idesc_dv = idesc_bf16_f32(128, 64, true);   // P^T (TMEM) x dout, dout N-major
+  constexpr uint32_t idesc_dk = idesc_f16_f32_bmn(128, 64);      // dS^T (TMEM) x Q, Q N-major
+  const int n = w.it1 - w.it0;
+  const uint64_t kdesc = sw128_desc(smem_u32(sm.k));
+  const uint64_t vdesc = sw128_desc(smem_u32(sm.v));
+  bool ok = mbar_wait(&sm.kv_full, 0, p.wait_ns);
+  // dV += P^T(u) dout(u), dK += dS^T(u) Q(u) for step u, once its P^T / dS^T exist
+  auto grads = [&](int u) -> bool {
+    const uint32_t X = u & 1, s = u % kBwdTcStages;
+    if (!mbar_wait(&sm.p_full[X], (u >> 1) & 1, p.wait_ns)) return false;
+    tc_fence_after();
+    const uint64_t odesc = sw128_desc(smem_u32(sm.dout[s]));
+    const uint64_t qdesc = sw128_desc(smem_u32(sm.q[s]));
+    const uint32_t set = tmem + X * kColSet;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t acc = (u == 0 && kk == 0) ? 0u : 1u;
+      mma_ts(tmem + kColDV, set + kColP + kk * 8, odesc + static_cast<uint64_t>(kk * 128), idesc_dv, acc);
+      mma_ts(tmem + kColDK, set + kColDS + kk * 8, qdesc + static_cast<uint64_t>(kk * 128), idesc_dk, acc);
+    }
+    mma_commit(&sm.qd_empty[s]);  // the step's q / dout tiles are free once these complete
+    return true;
+  };
+  for (int t = 0; t < n && ok; ++t) {
+    const uint32_t X = t & 1, s = t % kBwdTcStages;
+    if (!mbar_wait(&sm.qd_full[s], (t / kBwdTcStages) & 1, p.wait_ns)) { ok = false; break; }
+    if (t >= 2 && !mbar_wait(&sm.s_free[X], ((t - 2) >> 1) & 1, p.wait_ns)) { ok = false; break; }
+    tc_fence_after();
+    const uint64_t qdesc = sw128_desc(smem_u32(sm.q[s]));
+    const uint64_t odesc = sw128_desc(smem_u32(sm.dout[s]));
+    const uint32_t set = tmem + X * kColSet;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ss(set, kdesc + static_cast<uint64_t>(kk * 2), qdesc + static_cast<uint64_t>(kk * 2), idesc_s,
+             kk > 0 ? 1u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ss(set + kColDP, vdesc + static_cast<uint64_t>(kk * 2), odesc + static_cast<uint64_t>(kk * 2), idesc_dp,
+             kk > 0 ? 1u : 0u);
+    mma_commit(&sm.s_full[X]);
+    if (t >= 1 && !grads(t - 1)) ok = false;
+  }
+  if (ok && n > 0) grads(n - 1);
+  // dV and dK are final once every product above has completed
+  mma_commit(&sm.mma_done);
+  mbar_wait(&sm.mma_done, 0, p.wait_ns);
+}
+
+// lse * log2(e) (slot r < 64) or D (slot r >= 64) of query column r % 64 of
+// step `it` for head group g; 0 past the sequence.
+__device__ __forceinline__ float bwd_tc_lsd(const BwdParams& p, const BwdTcWork& w, int g, int it, int r) {
+  const int h = g * p.G + it / w.n_qt;
+  const int i = (w.qt0 + it % w.n_qt) * kBwdTcQ + (r & (kBwdTcQ - 1));
+  if (i >= w.sq.L) return 0.f;
+  const int64_t ri = bwd_row_index(p, w.b, h, i, w.sq.tok0);
+  return r < kBwdTcQ ? __ldg(p.lse + ri) * kLog2e : __ldg(p.dsum + ri);
+}
+
+template <bool kSplit>
+__device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm, const BwdTcWork& w, int g,
+                                               uint32_t tmem) {
+  const int tid = threadIdx.x;         // 0 .. 255
+  const int wq = (tid >> 5) & 3;       // TMEM lane quarter
+  const int ch = tid >> 7;             // query-column half of the step
+  const int r = wq * 32 + (tid & 31);  // key row of the tile = TMEM lane
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const int L = w.sq.L, W = p.window;
+  const int j = w.k0 + r;              // this thread's key
+  const bool j_ok = j < L;
+  const float sl = p.scale_log2;
+  const int n = w.it1 - w.it0;
+  // the lse / D value this thread stages for the next step, loaded a step ahead
+  float lsd_next = tid < 2 * kBwdTcQ ? bwd_tc_lsd(p, w, g, w.it0, tid) : 0.f;
+  for (int t = 0; t < n; ++t) {
+    const int it = w.it0 + t;
+    const int i0 = (w.qt0 + it % w.n_qt) * kBwdTcQ + ch * 32;  // this thread's first query column
+    const uint32_t X = t & 1;
+    if (tid < 2 * kBwdTcQ) sm.lsd[X][tid] = lsd_next;
+    // lsd[X] is rewritten two steps on, after every thread passed step t+1's
+    // lsd_ready wait -- i.e. after every thread finished reading it here
+    mbar_arrive(&sm.lsd_ready[X]);
+    if (tid < 2 * kBwdTcQ && t + 1 < n) lsd_next = bwd_tc_lsd(p, w, g, it + 1, tid);
+    if (!mbar_wait_warp(&sm.lsd_ready[X], (t >> 1) & 1, p.wait_ns)) return;
+    if (!mbar_wait_warp(&sm.s_full[X], (t >> 1) & 1, p.wait_ns)) return;
+    tc_fence_after();
+    const uint32_t set = lane_base + X * kColSet;
+    uint32_t sv[32], dv[32];
+    tmem_ld32(set + ch * 32, sv);
+    tmem_ld32(set + kColDP + ch * 32, dv);
+    tmem_wait_ld();
+    tc_fence_before();
+    mbar_arrive(&sm.s_free[X]);  // S^T / dP^T of set X may be overwritten
+    const float* lse2 = &sm.lsd[X][ch * 32];
+    const float* dsum = &sm.lsd[X][kBwdTcQ + ch * 32];
+    // every pair of this warp's 32 keys x 32 queries visible: no mask
+    const int jw = w.k0 + wq * 32;
+    const bool all_vis = jw + 31 <= i0 && i0 + 31 < L && jw + 31 < L && (W == 0 || i0 + 31 - jw < W);
+    uint32_t pk[16], dk[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      const float4 l4 = *reinterpret_cast<const float4*>(lse2 + e);
+      const float4 d4 = *reinterpret_cast<const float4*>(dsum + e);
+      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+      const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+      float pv[4], ds[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool vis = all_vis || (j_ok && bwd_visible(i0 + e + u, j, L, W));
+        pv[u] = vis ? ex2_approx(__uint_as_float(sv[e + u]) * sl - lv[u]) : 0.f;
+        ds[u] = pv[u] * (__uint_as_float(dv[e + u]) - dd[u]);
+      }
+      pk[e / 2] = pack_bf16(pv[0], pv[1]);
+      pk[e / 2 + 1] = pack_bf16(pv[2], pv[3]);
+      dk[e / 2] = pack_f16(ds[0], ds[1]);
+      dk[e / 2 + 1] = pack_f16(ds[2], ds[3]);
+    }
+    // P^T / dS^T of set X were last read by step t-2's gradient products,
+    // which completed before step t's S^T (s_full covers all earlier products)
+    tmem_st16(set + kColP + ch * 16, pk);
+    tmem_st16(set + kColDS + ch * 16, dk);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&sm.p_full[X]);
+  }
+  // ---- epilogue: warps 0-3 write dV, warps 4-7 dK, one key row per thread ----
+  if (!mbar_wait_warp(&sm.mma_done, 0, p.wait_ns)) return;
+  tc_fence_after();
+  const int which = ch;  // 0: dV, 1: dK
+  const int64_t tok = w.sq.tok0 + j;
+  const int64_t row = (tok * p.Hkv + g) * kHeadDim;
+  uint32_t a[32], bb[32];
+  const uint32_t col = which == 0 ? kColDV : kColDK;
+  tmem_ld32(lane_base + col, a);        // features [0, 32)
+  tmem_ld32(lane_base + col + 32, bb);  // features [32, 64)
+  tmem_wait_ld();
+  if (!j_ok) return;
+  if (kSplit) {
+    float* acc = (which == 0 ? p.dv_acc : p.dk_acc) + row;
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      atomicAdd(reinterpret_cast<float2*>(acc + e), make_float2(__uint_as_float(a[e]), __uint_as_float(a[e + 1])));
+      atomicAdd(reinterpret_cast<float2*>(acc + 32 + e),
+                make_float2(__uint_as_float(bb[e]), __uint_as_float(bb[e + 1])));
+    }
+    return;
+  }
+  __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + row;
+  uint32_t lo[16], hi[16];
+  if (which == 0) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      lo[e] = pack_bf16(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
+      hi[e] = pack_bf16(__uint_as_float(bb[2 * e]), __uint_as_float(bb[2 * e + 1]));
+    }
+  } else {  // pair (d, d + 32): (x, y) -> (x cc + y cs, y cc - x cs), after the scale
+    const float2* cs = p.cs + tok * kPairs;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float xr[2], yr[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float x = __uint_as_float(a[2 * e + u]) * p.scale, y = __uint_as_float(bb[2 * e + u]) * p.scale;
+        const float2 c = __ldg(cs + 2 * e + u);
+        xr[u] = x * c.x + y * c.y;
+        yr[u] = y * c.x - x * c.y;
+      }
+      lo[e] = pack_bf16(xr[0], xr[1]);
+      hi[e] = pack_bf16(yr[0], yr[1]);
+    }
+  }
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    reinterpret_cast<uint4*>(dst)[q4] = make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
+    reinterpret_cast<uint4*>(dst + 32)[q4] = make_uint4(hi[4 * q4], hi[4 * q4 + 1], hi[4 * q4 + 2], hi[4 * q4 + 3]);
+  }
+}
+
+template <bool kSplit>
+__global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dkdv_tc_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  BwdTcSmem& sm = *reinterpret_cast<BwdTcSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  BwdTcWork w;
+  if (!bwd_tc_work<kSplit>(p, w)) return;  // uniform over the CTA, before any barrier
+  const int g = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.kv_full, 1);
+    for (int s = 0; s < kBwdTcStages; ++s) {
+      mbar_init(&sm.qd_full[s], 1);
+      mbar_init(&sm.qd_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.s_free[x], kBwdTcSoftmax);
+      mbar_init(&sm.p_full[x], kBwdTcSoftmax);
+      mbar_init(&sm.lsd_ready[x], kBwdTcSoftmax);
+    }
+    mbar_init(&sm.mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&sm.tmem_base, kBwdTcTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (warp < 8) bwd_tc_softmax<kSplit>(p, sm, w, g, tmem);
+  else if (warp == 8 && lane == 0) bwd_tc_producer(p, sm, w, g);
+  else if (warp == 9 && lane == 0) bwd_tc_mma(p, sm, w, tmem);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBwdTcTmemCols);
+  }
+}
+
+}  // namespace gptoss

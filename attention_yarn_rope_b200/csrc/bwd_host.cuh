@@ -9,6 +9,7 @@
 #include <cstring>
 
 #include "attn_bwd.cuh"
+#include "attn_bwd_tc.cuh"
 #include "gptoss.h"
 #include "host_util.cuh"
 #include "rope_qk.cuh"
@@ -146,12 +147,34 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   p.n_tiles = (S + kBwdTile - 1) / kBwdTile;
   p.scale = softmax_scale;
   p.scale_log2 = softmax_scale * kLog2e;
+  p.wait_ns = wait_limit_ns();
+  // tensor maps of the tcgen05 dK / dV kernel: (d, head, token, batch); THD
+  // is one batch of total_tokens rows (the batch stride is then unused)
+  {
+    const uint64_t dimS = thd ? static_cast<uint64_t>(total_tokens) : static_cast<uint64_t>(S);
+    const uint64_t dimB = thd ? 1 : static_cast<uint64_t>(B);
+    const uint64_t kt_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2, qt_b = static_cast<uint64_t>(Hq) * kHeadDim * 2;
+    st = make_tmap_4d(&p.tmap_k, p.kh, kHeadDim, Hkv, dimS, dimB, kHeadDim * 2, kt_b, dimS * kt_b, kHeadDim, 1,
+                      kBwdTcKeys, 1, true);
+    if (st != GPTOSS_OK) return st;
+    st = make_tmap_4d(&p.tmap_q, p.qh, kHeadDim, Hq, dimS, dimB, kHeadDim * 2, qt_b, dimS * qt_b, kHeadDim, 1,
+                      kBwdTcQ, 1, true);
+    if (st != GPTOSS_OK) return st;
+    const uint64_t vb = thd ? dimS * sv.tok * 2 : static_cast<uint64_t>(sv.batch) * 2;
+    st = make_tmap_4d(&p.tmap_v, v, kHeadDim, Hkv, dimS, dimB, sv.head * 2, sv.tok * 2, vb == 0 ? 16 : vb,
+                      kHeadDim, 1, kBwdTcKeys, 1);
+    if (st != GPTOSS_OK) return st;
+    const uint64_t db = thd ? dimS * sdo.tok * 2 : static_cast<uint64_t>(sdo.batch) * 2;
+    st = make_tmap_4d(&p.tmap_do, dout, kHeadDim, Hq, dimS, dimB, sdo.head * 2, sdo.tok * 2, db == 0 ? 16 : db,
+                      kHeadDim, 1, kBwdTcQ, 1);
+    if (st != GPTOSS_OK) return st;
+  }
   // The longest dK / dV sweep (key tile 0 of the longest sequence): split it
-  // into chunks of kBwdChunkIt steps when it has more, so no CTA runs far
+  // into chunks of kBwdTcChunkIt steps when it has more, so no CTA runs far
   // longer than the rest; the chunks add into fp32 accumulators.
-  const int64_t q_last0 = window > 0 ? std::min<int64_t>(S - 1, kBwdTile - 1 + window - 1) : S - 1;
-  const int64_t max_it = static_cast<int64_t>(p.G) * (q_last0 / kBwdTile + 1);
-  const int64_t max_chunks = (max_it + kBwdChunkIt - 1) / kBwdChunkIt;
+  const int64_t q_last0 = window > 0 ? std::min<int64_t>(S - 1, kBwdTcKeys - 1 + window - 1) : S - 1;
+  const int64_t max_it = static_cast<int64_t>(p.G) * (q_last0 / kBwdTcQ + 1);
+  const int64_t max_chunks = (max_it + kBwdTcChunkIt - 1) / kBwdTcChunkIt;
   const bool split = max_chunks > 1 && static_cast<int64_t>(B) * max_chunks <= 65535;
   p.max_chunks = split ? static_cast<int>(max_chunks) : 1;
   p.dk_acc = reinterpret_cast<float*>(wsb + ws.acc);
@@ -163,14 +186,18 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
 
   // 3. dK, dV (one CTA per key tile and kv head, or per chunk of its sweep)
   //    and 4. dQ (one per query tile and head)
+  const int n_ktiles = (S + kBwdTcKeys - 1) / kBwdTcKeys;
+  const size_t tc_smem = sizeof(BwdTcSmem) + 1024;
+  auto dkdv = split ? attn_bwd_dkdv_tc_kernel<true> : attn_bwd_dkdv_tc_kernel<false>;
+  if (cudaFuncSetAttribute(dkdv, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(tc_smem)) !=
+      cudaSuccess)
+    return GPTOSS_ERR_CUDA;
+  dkdv<<<dim3(n_ktiles, Hkv, B * p.max_chunks), kBwdTcThreads, tc_smem, s>>>(p);
   if (split) {
-    attn_bwd_dkdv_kernel<true><<<dim3(p.n_tiles, Hkv, B * p.max_chunks), kBwdThreads, 0, s>>>(p);
     st = check_launch();
     if (st != GPTOSS_OK) return st;
     const int64_t n = static_cast<int64_t>(total_tokens) * Hkv * kPairs;
     attn_bwd_dkdv_finish_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
-  } else {
-    attn_bwd_dkdv_kernel<false><<<dim3(p.n_tiles, Hkv, B), kBwdThreads, 0, s>>>(p);
   }
   st = check_launch();
   if (st != GPTOSS_OK) return st;
