@@ -25,11 +25,13 @@
 //      would leave a few CTAs running long after the rest, so long sweeps are
 //      cut into chunks, one CTA each, adding into fp32 dK / dV accumulators;
 //      attn_bwd_dkdv_finish_kernel then applies scale and c R^T, writes bf16.
-//   4. attn_bwd_dq_kernel: CTA (query tile, head, sequence); 4 warps of 16
-//      queries keep Q and dout as A fragments and sweep the key tiles the
-//      query tile sees (K and V double-buffered): S, dP, dS recomputed, dQ +=
-//      dS K, then scale and c R^T.  Recomputing S and dP here (3 products per
-//      step instead of atomics on a float dQ) keeps every output written once.
+//   4. dQ: attn_bwd_dq_tc_kernel (attn_bwd_tc.cuh, tcgen05) for long sweeps,
+//      or attn_bwd_dq_kernel here for short ones (a sliding window): CTA
+//      (query tile, head, sequence); 4 warps of 16 queries keep Q and dout as
+//      mma.sync A fragments and sweep the key tiles the query tile sees (K and
+//      V double-buffered): S, dP, dS recomputed, dQ += dS K, then scale and
+//      c R^T.  Recomputing S and dP (3 products per step instead of atomics on
+//      a float dQ) keeps every output written once.
 // Operands: rotated q / k in fp16, v / dout in bf16, P rounded to bf16 for
 // P^T dout and dS to fp16 for the products with q and k; fp32 accumulation.
 #pragma once

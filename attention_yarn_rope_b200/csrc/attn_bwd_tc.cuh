@@ -107,9 +107,13 @@ __device__ __forceinline__ void bwd_tc_producer(const BwdParams& p, BwdTcSmem& s
   const bool thd = p.cu_seqlens != nullptr;
   const int row0 = thd ? static_cast<int>(w.sq.tok0) : 0;  // token row of the sequence's first token
   const int bc = thd ? 0 : w.b;
+  // the 128-row K and V tiles as two 64-row boxes each (every map's box is
+  // 64 rows; the swizzle repeats every 8 rows, so the halves line up)
   mbar_arrive_expect_tx(&sm.kv_full, 2 * kBwdTcKeys * 128);
-  tma_load_4d(sm.k, &p.tmap_k, &sm.kv_full, 0, g, row0 + w.k0, bc);
-  tma_load_4d(sm.v, &p.tmap_v, &sm.kv_full, 0, g, row0 + w.k0, bc);
+  for (int hf = 0; hf < 2; ++hf) {
+    tma_load_4d(sm.k + hf * 64 * 128, &p.tmap_k, &sm.kv_full, 0, g, row0 + w.k0 + 64 * hf, bc);
+    tma_load_4d(sm.v + hf * 64 * 128, &p.tmap_v, &sm.kv_full, 0, g, row0 + w.k0 + 64 * hf, bc);
+  }
   int issued = 0;
   for (int it = w.it0; it < w.it1; ++it, ++issued) {
     const int t = it - w.it0, s = t % kBwdTcStages;
@@ -341,6 +345,249 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dkdv_tc_kernel(cons
   if (warp < 8) bwd_tc_softmax<kSplit>(p, sm, w, g, tmem);
   else if (warp == 8 && lane == 0) bwd_tc_producer(p, sm, w, g);
   else if (warp == 9 && lane == 0) bwd_tc_mma(p, sm, w, tmem);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBwdTcTmemCols);
+  }
+}
+
+// ============================================================================
+// dQ on the tensor cores.  CTA = (128-query tile, head, sequence), 10 warps:
+// 8 softmax warps (TMEM lanes 32 (w % 4) .. = query rows, key columns
+// 32 (w / 4) .. of the step), a TMA producer (Q and dout tiles once, then each
+// step's 64-key K and V tiles, 4 stages ahead), an MMA issuer.  Per step:
+//   S  = Q K^T, dP = dout V^T   (SS, K-major; M = 128 queries, N = 64 keys)
+//   dS = P (dP - D) -> tensor memory (fp16), P = exp(S scale - lse)
+//   dQ += dS K                  (TS: dS from tensor memory, K read N-major)
+// lse and D belong to the thread's own row, so they are loaded once.  TMEM:
+// set X at 192 X: S [0, 64), dP [64, 128), dS [128, 160); dQ [384, 448).
+// ============================================================================
+constexpr uint32_t kColDQ = 384;
+
+struct __align__(1024) BwdTcQSmem {
+  uint8_t q[128 * 128];                        // rotated Q tile (fp16), 128B-swizzled rows
+  uint8_t dout[128 * 128];                     // dout tile (bf16)
+  uint8_t k[kBwdTcStages][kBwdTcQ * 128];      // rotated K tiles (fp16), 64 keys
+  uint8_t v[kBwdTcStages][kBwdTcQ * 128];      // V tiles (bf16)
+  uint64_t qd_full;
+  uint64_t kv_full[kBwdTcStages], kv_empty[kBwdTcStages];
+  uint64_t s_full[2], s_free[2], p_full[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+};
+
+struct BwdTcQWork {
+  int b, h, q0, kt0, n;  // query tile start, first key tile (64 keys), steps
+  BwdSeq sq;
+};
+
+__device__ __forceinline__ bool bwd_tcq_work(const BwdParams& p, BwdTcQWork& w) {
+  const int n_qt = (p.S + 127) / 128;
+  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x);  // the longest sweeps start first
+  w.h = blockIdx.y;
+  w.b = blockIdx.z;
+  w.sq = bwd_seq(p, w.b);
+  w.q0 = qt * 128;
+  if (w.q0 >= w.sq.L) return false;
+  const int L = w.sq.L, W = p.window;
+  const int j_first = W > 0 ? max(0, w.q0 - W + 1) : 0;
+  const int j_last = min(L - 1, w.q0 + 127);
+  w.kt0 = j_first / kBwdTcQ;
+  w.n = j_last / kBwdTcQ - w.kt0 + 1;
+  return true;
+}
+
+__device__ __forceinline__ void bwd_tcq_producer(const BwdParams& p, BwdTcQSmem& sm, const BwdTcQWork& w) {
+  tma_prefetch_desc(&p.tmap_k);
+  tma_prefetch_desc(&p.tmap_v);
+  tma_prefetch_desc(&p.tmap_q);
+  tma_prefetch_desc(&p.tmap_do);
+  const bool thd = p.cu_seqlens != nullptr;
+  const int row0 = thd ? static_cast<int>(w.sq.tok0) : 0;
+  const int bc = thd ? 0 : w.b;
+  const int g = w.h / p.G;
+  mbar_arrive_expect_tx(&sm.qd_full, 2 * 128 * 128);
+  for (int hf = 0; hf < 2; ++hf) {
+    tma_load_4d(sm.q + hf * 64 * 128, &p.tmap_q, &sm.qd_full, 0, w.h, row0 + w.q0 + 64 * hf, bc);
+    tma_load_4d(sm.dout + hf * 64 * 128, &p.tmap_do, &sm.qd_full, 0, w.h, row0 + w.q0 + 64 * hf, bc);
+  }
+  int issued = 0;
+  for (int t = 0; t < w.n; ++t, ++issued) {
+    const int s = t % kBwdTcStages;
+    if (!mbar_wait(&sm.kv_empty[s], ((t / kBwdTcStages) & 1) ^ 1, p.wait_ns)) break;
+    const int j0 = (w.kt0 + t) * kBwdTcQ;
+    mbar_arrive_expect_tx(&sm.kv_full[s], 2 * kBwdTcQ * 128);
+    tma_load_4d(sm.k[s], &p.tmap_k, &sm.kv_full[s], 0, g, row0 + j0, bc);
+    tma_load_4d(sm.v[s], &p.tmap_v, &sm.kv_full[s], 0, g, row0 + j0, bc);
+  }
+  // every issued copy must land before the CTA may exit
+  mbar_wait(&sm.qd_full, 0, p.wait_ns);
+  for (int t = issued > kBwdTcStages ? issued - kBwdTcStages : 0; t < issued; ++t)
+    mbar_wait(&sm.kv_full[t % kBwdTcStages], (t / kBwdTcStages) & 1, p.wait_ns);
+}
+
+__device__ __forceinline__ void bwd_tcq_mma(const BwdParams& p, BwdTcQSmem& sm, const BwdTcQWork& w, uint32_t tmem) {
+  constexpr uint32_t idesc_s = idesc_f16_f32(128, 64);          // Q (fp16) x K^T
+  constexpr uint32_t idesc_dp = idesc_bf16_f32(128, 64, false);  // dout (bf16) x V^T
+  constexpr uint32_t idesc_dq = idesc_f16_f32_bmn(128, 64);      // dS (TMEM) x K, K N-major
+  const uint64_t qdesc = sw128_desc(smem_u32(sm.q));
+  const uint64_t odesc = sw128_desc(smem_u32(sm.dout));
+  bool ok = mbar_wait(&sm.qd_full, 0, p.wait_ns);
+  auto grads = [&](int u) -> bool {  // dQ += dS(u) K(u)
+    const uint32_t X = u & 1, s = u % kBwdTcStages;
+    if (!mbar_wait(&sm.p_full[X], (u >> 1) & 1, p.wait_ns)) return false;
+    tc_fence_after();
+    const uint64_t kdesc = sw128_desc(smem_u32(sm.k[s]));
+    const uint32_t set = tmem + X * kColSet;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ts(tmem + kColDQ, set + kColP + kk * 8, kdesc + static_cast<uint64_t>(kk * 128), idesc_dq,
+             (u == 0 && kk == 0) ? 0u : 1u);
+    mma_commit(&sm.kv_empty[s]);  // the step's K / V tiles are free once these complete
+    return true;
+  };
+  for (int t = 0; t < w.n && ok; ++t) {
+    const uint32_t X = t & 1, s = t % kBwdTcStages;
+    if (!mbar_wait(&sm.kv_full[s], (t / kBwdTcStages) & 1, p.wait_ns)) { ok = false; break; }
+    if (t >= 2 && !mbar_wait(&sm.s_free[X], ((t - 2) >> 1) & 1, p.wait_ns)) { ok = false; break; }
+    tc_fence_after();
+    const uint64_t kdesc = sw128_desc(smem_u32(sm.k[s]));
+    const uint64_t vdesc = sw128_desc(smem_u32(sm.v[s]));
+    const uint32_t set = tmem + X * kColSet;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ss(set, qdesc + static_cast<uint64_t>(kk * 2), kdesc + static_cast<uint64_t>(kk * 2), idesc_s,
+             kk > 0 ? 1u : 0u);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ss(set + kColDP, odesc + static_cast<uint64_t>(kk * 2), vdesc + static_cast<uint64_t>(kk * 2), idesc_dp,
+             kk > 0 ? 1u : 0u);
+    mma_commit(&sm.s_full[X]);
+    if (t >= 1 && !grads(t - 1)) ok = false;
+  }
+  if (ok && w.n > 0) grads(w.n - 1);
+  mma_commit(&sm.mma_done);
+  mbar_wait(&sm.mma_done, 0, p.wait_ns);
+}
+
+__device__ __forceinline__ void bwd_tcq_softmax(const BwdParams& p, BwdTcQSmem& sm, const BwdTcQWork& w,
+                                                uint32_t tmem) {
+  const int tid = threadIdx.x;         // 0 .. 255
+  const int wq = (tid >> 5) & 3;       // TMEM lane quarter
+  const int ch = tid >> 7;             // key-column half of the step
+  const int r = wq * 32 + (tid & 31);  // query row of the tile = TMEM lane
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const int L = w.sq.L, W = p.window;
+  const int i = w.q0 + r;              // this thread's query
+  const bool i_ok = i < L;
+  const float sl = p.scale_log2;
+  float lse2 = 0.f, dd = 0.f;
+  if (i_ok) {
+    const int64_t ri = bwd_row_index(p, w.b, w.h, i, w.sq.tok0);
+    lse2 = __ldg(p.lse + ri) * kLog2e;
+    dd = __ldg(p.dsum + ri);
+  }
+  const int iw = w.q0 + wq * 32;  // this warp's first query row
+  for (int t = 0; t < w.n; ++t) {
+    const uint32_t X = t & 1;
+    const int j0 = (w.kt0 + t) * kBwdTcQ + ch * 32;  // this thread's first key column
+    if (!mbar_wait_warp(&sm.s_full[X], (t >> 1) & 1, p.wait_ns)) return;
+    tc_fence_after();
+    const uint32_t set = lane_base + X * kColSet;
+    uint32_t sv[32], dv[32];
+    tmem_ld32(set + ch * 32, sv);
+    tmem_ld32(set + kColDP + ch * 32, dv);
+    tmem_wait_ld();
+    tc_fence_before();
+    mbar_arrive(&sm.s_free[X]);  // S / dP of set X may be overwritten
+    // every pair of this warp's 32 queries x 32 keys visible: no mask
+    const bool all_vis = j0 + 31 <= iw && iw + 31 < L && (W == 0 || iw + 31 - j0 < W);
+    uint32_t dk[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float ds[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const bool vis = all_vis || (i_ok && bwd_visible(i, j0 + e + u, L, W));
+        const float pv = vis ? ex2_approx(__uint_as_float(sv[e + u]) * sl - lse2) : 0.f;
+        ds[u] = pv * (__uint_as_float(dv[e + u]) - dd);
+      }
+      dk[e / 2] = pack_f16(ds[0], ds[1]);
+    }
+    // dS of set X was last read by step t-2's dQ product, which completed
+    // before step t's S (s_full covers all earlier products)
+    tmem_st16(set + kColP + ch * 16, dk);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(&sm.p_full[X]);
+  }
+  // ---- epilogue: warps 0-3 write this query row of dq (scale, c R^T) ----
+  if (!mbar_wait_warp(&sm.mma_done, 0, p.wait_ns)) return;
+  tc_fence_after();
+  if (ch != 0) return;  // warp-uniform
+  uint32_t a[32], bb[32];
+  tmem_ld32(lane_base + kColDQ, a);        // features [0, 32)
+  tmem_ld32(lane_base + kColDQ + 32, bb);  // features [32, 64)
+  tmem_wait_ld();
+  if (!i_ok) return;
+  const int64_t tok = w.sq.tok0 + i;
+  __nv_bfloat16* dst = p.dq + (tok * p.Hq + w.h) * kHeadDim;
+  const float2* cs = p.cs + tok * kPairs;
+  uint32_t lo[16], hi[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float xr[2], yr[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float x = __uint_as_float(a[2 * e + u]) * p.scale, y = __uint_as_float(bb[2 * e + u]) * p.scale;
+      const float2 c = __ldg(cs + 2 * e + u);
+      xr[u] = x * c.x + y * c.y;
+      yr[u] = y * c.x - x * c.y;
+    }
+    lo[e] = pack_bf16(xr[0], xr[1]);
+    hi[e] = pack_bf16(yr[0], yr[1]);
+  }
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    reinterpret_cast<uint4*>(dst)[q4] = make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
+    reinterpret_cast<uint4*>(dst + 32)[q4] = make_uint4(hi[4 * q4], hi[4 * q4 + 1], hi[4 * q4 + 2], hi[4 * q4 + 3]);
+  }
+}
+
+__global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dq_tc_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  BwdTcQSmem& sm = *reinterpret_cast<BwdTcQSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  BwdTcQWork w;
+  if (!bwd_tcq_work(p, w)) return;  // uniform over the CTA, before any barrier
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.qd_full, 1);
+    for (int s = 0; s < kBwdTcStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.s_free[x], kBwdTcSoftmax);
+      mbar_init(&sm.p_full[x], kBwdTcSoftmax);
+    }
+    mbar_init(&sm.mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&sm.tmem_base, kBwdTcTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (warp < 8) bwd_tcq_softmax(p, sm, w, tmem);
+  else if (warp == 8 && lane == 0) bwd_tcq_producer(p, sm, w);
+  else if (warp == 9 && lane == 0) bwd_tcq_mma(p, sm, w, tmem);
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {

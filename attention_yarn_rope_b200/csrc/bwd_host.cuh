@@ -148,21 +148,21 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   p.scale = softmax_scale;
   p.scale_log2 = softmax_scale * kLog2e;
   p.wait_ns = wait_limit_ns();
-  // tensor maps of the tcgen05 dK / dV kernel: (d, head, token, batch); THD
-  // is one batch of total_tokens rows (the batch stride is then unused)
+  // tensor maps of the tcgen05 kernels: (d, head, token, batch), 64-row
+  // boxes; THD is one batch of total_tokens rows (its batch stride unused)
   {
     const uint64_t dimS = thd ? static_cast<uint64_t>(total_tokens) : static_cast<uint64_t>(S);
     const uint64_t dimB = thd ? 1 : static_cast<uint64_t>(B);
     const uint64_t kt_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2, qt_b = static_cast<uint64_t>(Hq) * kHeadDim * 2;
     st = make_tmap_4d(&p.tmap_k, p.kh, kHeadDim, Hkv, dimS, dimB, kHeadDim * 2, kt_b, dimS * kt_b, kHeadDim, 1,
-                      kBwdTcKeys, 1, true);
+                      kBwdTcQ, 1, true);
     if (st != GPTOSS_OK) return st;
     st = make_tmap_4d(&p.tmap_q, p.qh, kHeadDim, Hq, dimS, dimB, kHeadDim * 2, qt_b, dimS * qt_b, kHeadDim, 1,
                       kBwdTcQ, 1, true);
     if (st != GPTOSS_OK) return st;
     const uint64_t vb = thd ? dimS * sv.tok * 2 : static_cast<uint64_t>(sv.batch) * 2;
     st = make_tmap_4d(&p.tmap_v, v, kHeadDim, Hkv, dimS, dimB, sv.head * 2, sv.tok * 2, vb == 0 ? 16 : vb,
-                      kHeadDim, 1, kBwdTcKeys, 1);
+                      kHeadDim, 1, kBwdTcQ, 1);
     if (st != GPTOSS_OK) return st;
     const uint64_t db = thd ? dimS * sdo.tok * 2 : static_cast<uint64_t>(sdo.batch) * 2;
     st = make_tmap_4d(&p.tmap_do, dout, kHeadDim, Hq, dimS, dimB, sdo.head * 2, sdo.tok * 2, db == 0 ? 16 : db,
@@ -201,7 +201,21 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   }
   st = check_launch();
   if (st != GPTOSS_OK) return st;
-  attn_bwd_dq_kernel<<<dim3(p.n_tiles, Hq, B), kBwdThreads, 0, s>>>(p);
+  // dQ: the tcgen05 kernel owns all tensor memory of its SM (one CTA at a
+  // time), so its fixed cost per CTA -- allocation, first loads, filling and
+  // draining the pipeline -- only pays off over long sweeps (full context or
+  // windows of 1024+ keys: 16+ key tiles per query tile).  Short sweeps (a
+  // 128-key window: 4-5 tiles) run faster on the mma.sync kernel, three
+  // CTAs to an SM (measured, B=4 S=4096 W=128: 1.27 against 1.66 ms).
+  if (window == 0 || window >= 1024) {
+    const size_t q_smem = sizeof(BwdTcQSmem) + 1024;
+    if (cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(q_smem)) != cudaSuccess)
+      return GPTOSS_ERR_CUDA;
+    attn_bwd_dq_tc_kernel<<<dim3((S + 127) / 128, Hq, B), kBwdTcThreads, q_smem, s>>>(p);
+  } else {
+    attn_bwd_dq_kernel<<<dim3(p.n_tiles, Hq, B), kBwdThreads, 0, s>>>(p);
+  }
   return check_launch();
 }
 

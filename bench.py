@@ -446,7 +446,7 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
                                   "frac_of_measured_bf16": round(tf / peaks["bf16_tflops"], 4),
                                   "gbs_io": round(case["bytes"] / (ms * 1e-3) / 1e9, 1), "flops": case["flops"],
                                   "io_bytes": case["bytes"], "launches_per_call": "4 (5 with split sweeps)",
-                                  "note": "dK / dV on tcgen05 (TMEM), dQ on mma.sync recomputing S and dP"}
+                                  "note": "dK / dV on tcgen05 (TMEM); dQ on tcgen05 for long sweeps, mma.sync for short ones"}
         del case
         torch.cuda.empty_cache()
     flush_buf = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
