@@ -15,8 +15,10 @@
 //              them back to tensor memory for the gradient products; at the
 //              end warps 0-3 read and write dV, warps 4-7 dK (scale and c R^T),
 //              or add them into fp32 accumulators when sweeps are split;
-//   warp 8     TMA producer: K and V tiles once, then per step the step's
-//              rotated q tile (fp16) and dout tile (bf16), kBwdTcStages ahead;
+//   warp 8     producer: K and V tiles once (TMA), then per step the step's
+//              rotated q tile (fp16) and dout tile (bf16) by TMA and its 64
+//              lse and 64 D values by cp.async, kBwdTcStages ahead, all
+//              completing on the stage's qd_full barrier;
 //   warp 9     MMA issuer (one thread) and tensor-memory owner.
 // Per step (query head h, 64-query tile), all M = 128, N = 64, K = 4 x 16:
 //   S^T  = K Q^T            (SS, fp16, both K-major)
@@ -50,11 +52,10 @@ struct __align__(1024) BwdTcSmem {
   uint8_t v[kBwdTcKeys * 128];                 // V tile (bf16)
   uint8_t q[kBwdTcStages][kBwdTcQ * 128];      // rotated q tiles (fp16)
   uint8_t dout[kBwdTcStages][kBwdTcQ * 128];   // dout tiles (bf16)
-  float lsd[2][2 * kBwdTcQ];                   // per step: lse * log2(e) [0, 64), D [64, 128)
+  float lsd[kBwdTcStages][2 * kBwdTcQ];        // per stage: lse [0, 64) and D [64, 128) of its queries
   uint64_t kv_full;
   uint64_t qd_full[kBwdTcStages], qd_empty[kBwdTcStages];
   uint64_t s_full[2], s_free[2], p_full[2];
-  uint64_t lsd_ready[2];  // the softmax threads have written lsd[X] (a bounded wait, unlike bar.sync)
   uint64_t mma_done;
   uint32_t tmem_base;
 };
@@ -67,6 +68,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+// Arrive on `bar` once this thread's earlier cp.async copies have completed,
+// without adding to the barrier's expected count (it was initialised with
+// one arrival per thread that does this).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // fp16 A and B with B read N-major (the q tile in dK += dS^T Q).
@@ -99,30 +107,50 @@ __device__ __forceinline__ bool bwd_tc_work(const BwdParams& p, BwdTcWork& w) {
   return true;
 }
 
+// The whole producer warp runs this: lane 0 issues the TMA copies, every lane
+// copies 4 of the step's 128 lse / D values.
 __device__ __forceinline__ void bwd_tc_producer(const BwdParams& p, BwdTcSmem& sm, const BwdTcWork& w, int g) {
-  tma_prefetch_desc(&p.tmap_k);
-  tma_prefetch_desc(&p.tmap_v);
-  tma_prefetch_desc(&p.tmap_q);
-  tma_prefetch_desc(&p.tmap_do);
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) {
+    tma_prefetch_desc(&p.tmap_k);
+    tma_prefetch_desc(&p.tmap_v);
+    tma_prefetch_desc(&p.tmap_q);
+    tma_prefetch_desc(&p.tmap_do);
+  }
   const bool thd = p.cu_seqlens != nullptr;
   const int row0 = thd ? static_cast<int>(w.sq.tok0) : 0;  // token row of the sequence's first token
   const int bc = thd ? 0 : w.b;
-  // the 128-row K and V tiles as two 64-row boxes each (every map's box is
-  // 64 rows; the swizzle repeats every 8 rows, so the halves line up)
-  mbar_arrive_expect_tx(&sm.kv_full, 2 * kBwdTcKeys * 128);
-  for (int hf = 0; hf < 2; ++hf) {
-    tma_load_4d(sm.k + hf * 64 * 128, &p.tmap_k, &sm.kv_full, 0, g, row0 + w.k0 + 64 * hf, bc);
-    tma_load_4d(sm.v + hf * 64 * 128, &p.tmap_v, &sm.kv_full, 0, g, row0 + w.k0 + 64 * hf, bc);
+  const int L = w.sq.L;
+  if (lane == 0) {
+    // the 128-row K and V tiles as two 64-row boxes each (every map's box is
+    // 64 rows; the swizzle repeats every 8 rows, so the halves line up)
+    mbar_arrive_expect_tx(&sm.kv_full, 2 * kBwdTcKeys * 128);
+    for (int hf = 0; hf < 2; ++hf) {
+      tma_load_4d(sm.k + hf * 64 * 128, &p.tmap_k, &sm.kv_full, 0, g, row0 + w.k0 + 64 * hf, bc);
+      tma_load_4d(sm.v + hf * 64 * 128, &p.tmap_v, &sm.kv_full, 0, g, row0 + w.k0 + 64 * hf, bc);
+    }
   }
   int issued = 0;
   for (int it = w.it0; it < w.it1; ++it, ++issued) {
     const int t = it - w.it0, s = t % kBwdTcStages;
-    if (!mbar_wait(&sm.qd_empty[s], ((t / kBwdTcStages) & 1) ^ 1, p.wait_ns)) break;
+    if (!mbar_wait_warp(&sm.qd_empty[s], ((t / kBwdTcStages) & 1) ^ 1, p.wait_ns)) break;
     const int h = g * p.G + it / w.n_qt;
     const int i0 = (w.qt0 + it % w.n_qt) * kBwdTcQ;
-    mbar_arrive_expect_tx(&sm.qd_full[s], 2 * kBwdTcQ * 128);
-    tma_load_4d(sm.q[s], &p.tmap_q, &sm.qd_full[s], 0, h, row0 + i0, bc);
-    tma_load_4d(sm.dout[s], &p.tmap_do, &sm.qd_full[s], 0, h, row0 + i0, bc);
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.qd_full[s], 2 * kBwdTcQ * 128);
+      tma_load_4d(sm.q[s], &p.tmap_q, &sm.qd_full[s], 0, h, row0 + i0, bc);
+      tma_load_4d(sm.dout[s], &p.tmap_do, &sm.qd_full[s], 0, h, row0 + i0, bc);
+    }
+    // slots 4 lane .. 4 lane + 3: lse of queries [0, 64), D of [64, 128); a
+    // query past the sequence copies the last row's (finite, masked anyway)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int slot = 4 * lane + u;
+      const int i = min(i0 + (slot & (kBwdTcQ - 1)), L - 1);
+      const int64_t ri = bwd_row_index(p, w.b, h, i, w.sq.tok0);
+      cp_async4(smem_u32(&sm.lsd[s][slot]), (slot < kBwdTcQ ? p.lse : p.dsum) + ri);
+    }
+    cp_async_mbar_arrive_noinc(&sm.qd_full[s]);
   }
   // every issued copy must land before the CTA may exit
   mbar_wait(&sm.kv_full, 0, p.wait_ns);
@@ -181,16 +209,6 @@ __device__ __forceinline__ void bwd_tc_mma(const BwdParams& p, BwdTcSmem& sm, co
   mbar_wait(&sm.mma_done, 0, p.wait_ns);
 }
 
-// lse * log2(e) (slot r < 64) or D (slot r >= 64) of query column r % 64 of
-// step `it` for head group g; 0 past the sequence.
-__device__ __forceinline__ float bwd_tc_lsd(const BwdParams& p, const BwdTcWork& w, int g, int it, int r) {
-  const int h = g * p.G + it / w.n_qt;
-  const int i = (w.qt0 + it % w.n_qt) * kBwdTcQ + (r & (kBwdTcQ - 1));
-  if (i >= w.sq.L) return 0.f;
-  const int64_t ri = bwd_row_index(p, w.b, h, i, w.sq.tok0);
-  return r < kBwdTcQ ? __ldg(p.lse + ri) * kLog2e : __ldg(p.dsum + ri);
-}
-
 template <bool kSplit>
 __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm, const BwdTcWork& w, int g,
                                                uint32_t tmem) {
@@ -204,18 +222,15 @@ __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm
   const bool j_ok = j < L;
   const float sl = p.scale_log2;
   const int n = w.it1 - w.it0;
-  // the lse / D value this thread stages for the next step, loaded a step ahead
-  float lsd_next = tid < 2 * kBwdTcQ ? bwd_tc_lsd(p, w, g, w.it0, tid) : 0.f;
   for (int t = 0; t < n; ++t) {
     const int it = w.it0 + t;
     const int i0 = (w.qt0 + it % w.n_qt) * kBwdTcQ + ch * 32;  // this thread's first query column
     const uint32_t X = t & 1;
-    if (tid < 2 * kBwdTcQ) sm.lsd[X][tid] = lsd_next;
-    // lsd[X] is rewritten two steps on, after every thread passed step t+1's
-    // lsd_ready wait -- i.e. after every thread finished reading it here
-    mbar_arrive(&sm.lsd_ready[X]);
-    if (tid < 2 * kBwdTcQ && t + 1 < n) lsd_next = bwd_tc_lsd(p, w, g, it + 1, tid);
-    if (!mbar_wait_warp(&sm.lsd_ready[X], (t >> 1) & 1, p.wait_ns)) return;
+    const int stg = t % kBwdTcStages;
+    // the step's lse / D landed with its tiles (cp.async on qd_full); they
+    // stay until this step's gradient products free the stage (qd_empty),
+    // which follows this thread's p_full arrival below
+    if (!mbar_wait_warp(&sm.qd_full[stg], (t / kBwdTcStages) & 1, p.wait_ns)) return;
     if (!mbar_wait_warp(&sm.s_full[X], (t >> 1) & 1, p.wait_ns)) return;
     tc_fence_after();
     const uint32_t set = lane_base + X * kColSet;
@@ -225,17 +240,17 @@ __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm
     tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(&sm.s_free[X]);  // S^T / dP^T of set X may be overwritten
-    const float* lse2 = &sm.lsd[X][ch * 32];
-    const float* dsum = &sm.lsd[X][kBwdTcQ + ch * 32];
+    const float* lse = &sm.lsd[stg][ch * 32];
+    const float* dsum = &sm.lsd[stg][kBwdTcQ + ch * 32];
     // every pair of this warp's 32 keys x 32 queries visible: no mask
     const int jw = w.k0 + wq * 32;
     const bool all_vis = jw + 31 <= i0 && i0 + 31 < L && jw + 31 < L && (W == 0 || i0 + 31 - jw < W);
     uint32_t pk[16], dk[16];
 #pragma unroll
     for (int e = 0; e < 32; e += 4) {
-      const float4 l4 = *reinterpret_cast<const float4*>(lse2 + e);
+      const float4 l4 = *reinterpret_cast<const float4*>(lse + e);
       const float4 d4 = *reinterpret_cast<const float4*>(dsum + e);
-      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+      const float lv[4] = {l4.x * kLog2e, l4.y * kLog2e, l4.z * kLog2e, l4.w * kLog2e};
       const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
       float pv[4], ds[4];
 #pragma unroll
@@ -322,14 +337,13 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dkdv_tc_kernel(cons
   if (threadIdx.x == 0) {
     mbar_init(&sm.kv_full, 1);
     for (int s = 0; s < kBwdTcStages; ++s) {
-      mbar_init(&sm.qd_full[s], 1);
+      mbar_init(&sm.qd_full[s], 1 + 32);  // the TMA arrival + one cp.async arrival per producer lane
       mbar_init(&sm.qd_empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sm.s_full[x], 1);
       mbar_init(&sm.s_free[x], kBwdTcSoftmax);
       mbar_init(&sm.p_full[x], kBwdTcSoftmax);
-      mbar_init(&sm.lsd_ready[x], kBwdTcSoftmax);
     }
     mbar_init(&sm.mma_done, 1);
     fence_mbar_init();
@@ -343,7 +357,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dkdv_tc_kernel(cons
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   if (warp < 8) bwd_tc_softmax<kSplit>(p, sm, w, g, tmem);
-  else if (warp == 8 && lane == 0) bwd_tc_producer(p, sm, w, g);
+  else if (warp == 8) bwd_tc_producer(p, sm, w, g);
   else if (warp == 9 && lane == 0) bwd_tc_mma(p, sm, w, tmem);
   tc_fence_before();
   __syncthreads();
