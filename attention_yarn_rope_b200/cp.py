@@ -1,0 +1,205 @@
+"""Context parallelism for the sliding-window layers: one sequence split
+along its length over the ranks of a process group.
+
+The NeMo AutoModel gpt_oss.rope_utils page gives ``apply_rotary_emb_qk``
+``cp_size`` / ``cp_rank`` arguments, with the local context-parallel shard in
+the leading dimensions of q and k; it does not give the shards' layout.
+Here rank r of R holds the contiguous tokens [r S_loc, (r + 1) S_loc) of
+every sequence (BSHD ``[B, S_loc, H, D]``), so RoPE takes the global position
+r S_loc + i.
+
+GPT-OSS alternates full-context and 128-token sliding-window layers
+(Transformers v4.55.0 release notes, "Architecture").  With a window of W
+keys, query row i sees keys [i - W + 1, i]: the rows of rank r reach into
+rank r - 1 by at most W - 1 keys, and no further while S_loc >= W - 1.  So
+the forward needs one exchange -- rank r - 1 sends its last W - 1 rows of k
+and v to rank r (a halo) -- after which rank r runs the ordinary prefill on
+[halo | shard] with the halo's query rows left zero and their outputs
+dropped.  Every query row of the shard then sees exactly its keys, the sink
+once, so the result is the unsharded attention's, not an approximation.
+The backward runs the ordinary backward on the same extended sequence with
+zero dout for the halo rows (they contribute nothing), sends the halo rows'
+dk / dv back to rank r - 1, which adds them to its last W - 1 rows, and sums
+dsinks over the ranks.
+
+Full-context layers need every earlier shard's keys (a ring with a
+log-sum-exp merge); that is not built here.
+"""
+
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import ops
+
+
+def _rank_world(group):
+    """(rank, world size) in `group`; one rank when no process group exists."""
+    if not dist.is_available() or not dist.is_initialized():
+        return 0, 1
+    return dist.get_rank(group), dist.get_world_size(group)
+
+
+def _peer(group, rank: int) -> int:
+    """Global rank of `rank` within `group` (point-to-point calls take global ranks)."""
+    return rank if group is None else dist.get_global_rank(group, rank)
+
+
+def _exchange(send_next, recv_shape, dtype, device, group, rank, world):
+    """Send `send_next` to rank + 1 and receive a `recv_shape` tensor from rank - 1
+    (None on rank 0).  Receives are posted before sends, so no rank blocks."""
+    reqs = []
+    recv = None
+    if rank > 0:
+        recv = torch.empty(recv_shape, dtype=dtype, device=device)
+        reqs.append(dist.irecv(recv, src=_peer(group, rank - 1), group=group))
+    if rank + 1 < world:
+        reqs.append(dist.isend(send_next.contiguous(), dst=_peer(group, rank + 1), group=group))
+    for r in reqs:
+        r.wait()
+    return recv
+
+
+def _exchange_back(send_prev, recv_shape, dtype, device, group, rank, world):
+    """Send `send_prev` to rank - 1 and receive a `recv_shape` tensor from rank + 1
+    (None on the last rank)."""
+    reqs = []
+    recv = None
+    if rank + 1 < world:
+        recv = torch.empty(recv_shape, dtype=dtype, device=device)
+        reqs.append(dist.irecv(recv, src=_peer(group, rank + 1), group=group))
+    if rank > 0:
+        reqs.append(dist.isend(send_prev.contiguous(), dst=_peer(group, rank - 1), group=group))
+    for r in reqs:
+        r.wait()
+    return recv
+
+
+def halo_rows(window: int, s_loc: int, world: int) -> int:
+    """Rows of k / v a rank needs from its predecessor: window - 1 (none on one rank)."""
+    if window <= 0:
+        raise ValueError("context parallelism here covers the sliding-window layers (window > 0)")
+    halo = window - 1 if world > 1 else 0
+    if s_loc < halo:
+        raise ValueError(f"each shard needs at least window - 1 = {halo} tokens, got {s_loc}")
+    return halo
+
+
+def _positions(B: int, start: int, length: int, device) -> torch.Tensor:
+    pos = torch.arange(start, start + length, dtype=torch.int32, device=device)
+    return pos.unsqueeze(0).expand(B, length).contiguous()
+
+
+def kv_tail(k, v, halo: int):
+    """The last `halo` rows of this shard's k and v, heads concatenated: what
+    the next rank receives."""
+    s_loc = k.shape[1]
+    return torch.cat([k[:, s_loc - halo:], v[:, s_loc - halo:]], dim=2)
+
+
+def local_fwd(q, k, v, sinks, window: int, rope, rank: int, halo_kv=None, softmax_scale=None, attn_fwd=None):
+    """Rank `rank`'s rows given `halo_kv` (the previous rank's :func:`kv_tail`,
+    None on rank 0): the prefill over [halo | shard] at global positions,
+    the halo's query rows zero and dropped.  No communication."""
+    attn_fwd = attn_fwd or (lambda *a, **kw: ops.gptoss_attn_fwd(*a, return_lse=True, **kw))
+    B, s_loc, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if halo_kv is None:
+        pos = _positions(B, rank * s_loc, s_loc, q.device)
+        return attn_fwd(q, k, v, sinks, window=window, rope=rope, positions=pos, softmax_scale=softmax_scale)
+    halo = halo_kv.shape[1]
+    q_ext = torch.cat([torch.zeros((B, halo, Hq, D), dtype=q.dtype, device=q.device), q], dim=1)
+    k_ext = torch.cat([halo_kv[:, :, :Hkv], k], dim=1)
+    v_ext = torch.cat([halo_kv[:, :, Hkv:], v], dim=1)
+    pos = _positions(B, rank * s_loc - halo, halo + s_loc, q.device)
+    out, lse = attn_fwd(q_ext, k_ext, v_ext, sinks, window=window, rope=rope, positions=pos,
+                        softmax_scale=softmax_scale)
+    return out[:, halo:].contiguous(), lse[:, :, halo:].contiguous()
+
+
+def local_bwd(q, k, v, sinks, out, dout, lse, window: int, rope, rank: int, halo_kv=None, softmax_scale=None,
+              attn_bwd=None):
+    """Rank `rank`'s gradients given `halo_kv`: ``(dq, dk, dv, dsinks, dkv_halo)``
+    with dk / dv of its own rows (before the next rank's halo gradients are
+    added), its share of dsinks, and the halo rows' dk / dv (heads
+    concatenated, None on rank 0) that belong to the previous rank.  No
+    communication."""
+    attn_bwd = attn_bwd or ops.gptoss_attn_bwd
+    B, s_loc, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if halo_kv is None:
+        pos = _positions(B, rank * s_loc, s_loc, q.device)
+        dq, dk, dv, dsinks = attn_bwd(q, k, v, sinks, out, dout, lse, window=window, rope=rope, positions=pos,
+                                      softmax_scale=softmax_scale)
+        return dq, dk, dv, dsinks, None
+    halo = halo_kv.shape[1]
+    zq = torch.zeros((B, halo, Hq, D), dtype=q.dtype, device=q.device)
+    q_ext = torch.cat([zq, q], dim=1)
+    k_ext = torch.cat([halo_kv[:, :, :Hkv], k], dim=1)
+    v_ext = torch.cat([halo_kv[:, :, Hkv:], v], dim=1)
+    out_ext = torch.cat([zq, out], dim=1)
+    dout_ext = torch.cat([zq, dout], dim=1)  # the halo rows are not this rank's: no gradient flows in
+    # lse = +inf gives the halo rows zero weights (and zero sink share)
+    lse_ext = torch.cat([torch.full((B, Hq, halo), float("inf"), dtype=lse.dtype, device=lse.device), lse], dim=2)
+    pos = _positions(B, rank * s_loc - halo, halo + s_loc, q.device)
+    dq_e, dk_e, dv_e, dsinks = attn_bwd(q_ext, k_ext, v_ext, sinks, out_ext, dout_ext, lse_ext, window=window,
+                                        rope=rope, positions=pos, softmax_scale=softmax_scale)
+    return (dq_e[:, halo:].contiguous(), dk_e[:, halo:].contiguous(), dv_e[:, halo:].contiguous(), dsinks,
+            torch.cat([dk_e[:, :halo], dv_e[:, :halo]], dim=2))
+
+
+def add_halo_grads(dk, dv, back):
+    """Add the next rank's halo gradients `back` (heads concatenated) to the
+    last rows of dk / dv, summed in fp32 at least and rounded once."""
+    Hkv, halo, s_loc = dk.shape[2], back.shape[1], dk.shape[1]
+    tail = slice(s_loc - halo, s_loc)
+    acc = torch.promote_types(dk.dtype, torch.float32)
+    dk[:, tail] = (dk[:, tail].to(acc) + back[:, :, :Hkv].to(acc)).to(dk.dtype)
+    dv[:, tail] = (dv[:, tail].to(acc) + back[:, :, Hkv:].to(acc)).to(dv.dtype)
+
+
+def sliding_window_fwd(q, k, v, sinks, window: int, rope, group=None, softmax_scale: float | None = None,
+                       attn_fwd=None):
+    """This rank's rows of the sliding-window attention of the whole sequence.
+
+    q ``[B, S_loc, Hq, D]``, k / v ``[B, S_loc, Hkv, D]``: this rank's shard.
+    Returns ``(out [B, S_loc, Hq, D], lse [B, Hq, S_loc])``.  ``attn_fwd``
+    (keyword-compatible with :func:`ops.gptoss_attn_fwd`, returning
+    ``(out, lse)``) defaults to the CUDA prefill."""
+    rank, world = _rank_world(group)
+    B, s_loc, _, D = q.shape
+    Hkv = k.shape[2]
+    halo = halo_rows(window, s_loc, world)
+    got = None
+    if halo:
+        got = _exchange(kv_tail(k, v, halo), (B, halo, 2 * Hkv, D), k.dtype, k.device, group, rank, world)
+    return local_fwd(q, k, v, sinks, window, rope, rank, got, softmax_scale, attn_fwd)
+
+
+def sliding_window_bwd(q, k, v, sinks, out, dout, lse, window: int, rope, group=None,
+                       softmax_scale: float | None = None, attn_bwd=None):
+    """Gradients of this rank's shard for ``L = sum over all ranks of sum(dout * out)``.
+
+    q, k, v, sinks, window, rope as given to :func:`sliding_window_fwd`; out,
+    lse from it; dout this rank's ``[B, S_loc, Hq, D]``.  Returns ``(dq, dk,
+    dv, dsinks)`` for this rank's tokens, dsinks summed over the group.
+    ``attn_bwd`` (keyword-compatible with :func:`ops.gptoss_attn_bwd`)
+    defaults to the CUDA backward."""
+    rank, world = _rank_world(group)
+    B, s_loc, _, D = q.shape
+    Hkv = k.shape[2]
+    halo = halo_rows(window, s_loc, world)
+    got = None
+    if halo:
+        got = _exchange(kv_tail(k, v, halo), (B, halo, 2 * Hkv, D), k.dtype, k.device, group, rank, world)
+    dq, dk, dv, dsinks, dkv_halo = local_bwd(q, k, v, sinks, out, dout, lse, window, rope, rank, got,
+                                             softmax_scale, attn_bwd)
+    if halo:  # the halo rows' key / value gradients belong to the previous rank's last rows
+        back = _exchange_back(dkv_halo, (B, halo, 2 * Hkv, D), dk.dtype, dk.device, group, rank, world)
+        if back is not None:
+            add_halo_grads(dk, dv, back)
+    dsinks = dsinks.clone()
+    if world > 1:
+        dist.all_reduce(dsinks, op=dist.ReduceOp.SUM, group=group)
+    return dq, dk, dv, dsinks
