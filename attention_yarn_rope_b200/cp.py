@@ -54,8 +54,9 @@ def _exchange(send_next, recv_shape, dtype, device, group, rank, world):
     if rank > 0:
         recv = torch.empty(recv_shape, dtype=dtype, device=device)
         reqs.append(dist.irecv(recv, src=_peer(group, rank - 1), group=group))
-    if rank + 1 < world:
-        reqs.append(dist.isend(send_next.contiguous(), dst=_peer(group, rank + 1), group=group))
+    send = send_next.contiguous() if rank + 1 < world else None  # alive until the send completes
+    if send is not None:
+        reqs.append(dist.isend(send, dst=_peer(group, rank + 1), group=group))
     for r in reqs:
         r.wait()
     return recv
@@ -69,8 +70,9 @@ def _exchange_back(send_prev, recv_shape, dtype, device, group, rank, world):
     if rank + 1 < world:
         recv = torch.empty(recv_shape, dtype=dtype, device=device)
         reqs.append(dist.irecv(recv, src=_peer(group, rank + 1), group=group))
-    if rank > 0:
-        reqs.append(dist.isend(send_prev.contiguous(), dst=_peer(group, rank - 1), group=group))
+    send = send_prev.contiguous() if rank > 0 else None  # alive until the send completes
+    if send is not None:
+        reqs.append(dist.isend(send, dst=_peer(group, rank - 1), group=group))
     for r in reqs:
         r.wait()
     return recv

@@ -549,6 +549,15 @@ _KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C / C++ source without its comments (string literals kept): the hash
+    follows the code, not its documentation."""
+    import re
+
+    pat = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', re.S)
+    return pat.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", text)
+
+
 def kernel_src_hash(kernel):
     import hashlib
     import re
@@ -556,20 +565,23 @@ def kernel_src_hash(kernel):
     csrc = os.path.join(ROOT, "attention_yarn_rope_b200", "csrc")
     inc = os.path.join(ROOT, "include")
     root, launcher = _KERNEL_SOURCES[kernel]
+
+    def path_of(f):
+        return os.path.join(csrc, f) if os.path.exists(os.path.join(csrc, f)) else os.path.join(inc, f)
+
     seen, todo = [], [root]
     while todo:
         f = todo.pop()
         if f in seen:
             continue
         seen.append(f)
-        path = os.path.join(csrc, f) if os.path.exists(os.path.join(csrc, f)) else os.path.join(inc, f)
-        with open(path) as fh:
+        with open(path_of(f)) as fh:
             todo += re.findall(r'^#include "([^"]+)"', fh.read(), flags=re.M)
     h = hashlib.sha256()
     for f in sorted(seen) + [launcher]:
-        path = os.path.join(csrc, f) if os.path.exists(os.path.join(csrc, f)) else os.path.join(inc, f)
-        with open(path, "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+        with open(path_of(f)) as fh:
+            code = " ".join(_code_only(fh.read()).split())  # whitespace-insensitive too
+        h.update(f.encode() + b"\0" + code.encode())
     return h.hexdigest()[:12]
 
 

@@ -183,12 +183,16 @@ size_t gptoss_attn_bwd_workspace_size(int32_t total_tokens, int32_t Hq, int32_t 
  *   workspace  device memory of gptoss_attn_bwd_workspace_size(total_tokens,
  *          Hq, Hkv, D) bytes, 16-byte aligned, owned by the caller, contents
  *          need not be initialised.
- * Four kernels on `stream`: q / k rotation, D and dsinks, dk / dv (one CTA
- * per key tile and kv head), dq (one CTA per query tile and head).  The
- * rotated q / k enter the products as fp16 like the forward's; P is rounded
- * to bf16 and dS to fp16 for the products, accumulation is fp32.  dsinks is
- * summed with floating-point atomics (order not fixed); every other output
- * element has one writer. */
+ * Kernels on `stream`: q / k rotation; D and dsinks; dk / dv on the tcgen05
+ * tensor cores (one CTA per 128-key tile and kv head; sweeps longer than 64
+ * (head, 64-query tile) steps split into chunks that add into fp32
+ * accumulators, then one finishing kernel); dq (one CTA per query tile and
+ * head: tcgen05 for full context or windows of 1024+ keys, warp-level
+ * mma.sync for shorter windows).  The rotated q / k enter the products as
+ * fp16 like the forward's; P is rounded to bf16 and dS to fp16 for the
+ * products, accumulation is fp32.  dsinks and split dk / dv are summed with
+ * floating-point atomics (order not fixed); every other output element has
+ * one writer. */
 gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
                               const void* v, gptoss_strides sv, const void* out, gptoss_strides so,
                               const void* dout, gptoss_strides sdo, const float* lse, const float* sinks,

@@ -1,10 +1,9 @@
 """The benchmark's DRAM-traffic figures (profiles/traffic.txt) are reported
 only while the kernels they were captured on are unchanged: each line holds
 the hash of its kernel's sources (the include closure of the header that
-defines it plus its host launcher's text).  These CPU checks keep that
+defines it plus its host launcher, comments and whitespace removed).  These CPU checks keep that
 honest: the headline step's two kernels have a figure for the current
-sources, and the hash moves with any byte of the sources it covers and with
-nothing else."""
+sources, and the hash moves with the code it covers and with nothing else."""
 
 import os
 import shutil
@@ -32,6 +31,14 @@ def test_hash_covers_the_kernel_sources_only(tmp_path, monkeypatch):
     with open(tmp_path / "attention_yarn_rope_b200/csrc/attn_decode.cuh", "a") as f:
         f.write("\n// edited\n")
     assert bench.kernel_src_hash("attn_fwd_kernel") == h0
+    # comments and layout are documentation: the hash ignores them
     with open(tmp_path / "attention_yarn_rope_b200/csrc/fwd_softmax.cuh", "a") as f:
-        f.write("\n// edited\n")
+        f.write("\n// a comment\n/* another */\n\n")
+    assert bench.kernel_src_hash("attn_fwd_kernel") == h0
+    with open(tmp_path / "include/gptoss.h", "a") as f:
+        f.write("\n/* a documentation change */\n")
+    assert bench.kernel_src_hash("attn_fwd_kernel") == h0
+    # code is not
+    with open(tmp_path / "attention_yarn_rope_b200/csrc/fwd_softmax.cuh", "a") as f:
+        f.write("\nstatic const int edited = 1;\n")
     assert bench.kernel_src_hash("attn_fwd_kernel") != h0
