@@ -205,3 +205,119 @@ def sliding_window_bwd(q, k, v, sinks, out, dout, lse, window: int, rope, group=
     if world > 1:
         dist.all_reduce(dsinks, op=dist.ReduceOp.SUM, group=group)
     return dq, dk, dv, dsinks
+
+
+# ----------------------------------------------------------------------------
+# Packed (THD) inputs: rank r holds the contiguous tokens [r T_loc, (r + 1)
+# T_loc) of the packed stream, whose sequences may straddle the ranks.  The
+# extended stream [halo | shard] is re-packed with the global sequence
+# boundaries cut to it; positions restart at every sequence start, as in the
+# whole stream.  Halo tokens of a sequence that ends before the shard form
+# their own local sequence; their outputs are dropped like every halo row's.
+# ----------------------------------------------------------------------------
+def thd_local_layout(cu_seqlens, rank: int, t_loc: int, halo: int):
+    """Host-side layout of rank `rank`'s extended stream: ``(cu_local,
+    positions, start)`` -- the local sequence boundaries (int32, from 0), each
+    extended token's position inside its sequence (int32) and the global
+    index of the first extended token.  `cu_seqlens` is the global packing
+    (host integers)."""
+    cu = [int(x) for x in cu_seqlens]
+    start = rank * t_loc - (halo if rank > 0 else 0)
+    end = (rank + 1) * t_loc
+    if start < 0 or end > cu[-1]:
+        raise ValueError("the shards must tile the packed stream exactly")
+    bounds = [start] + [c for c in cu if start < c < end] + [end]
+    cu_local = [b - start for b in bounds]
+    pos = []
+    s = 0
+    for g in range(start, end):
+        while cu[s + 1] <= g:
+            s += 1
+        pos.append(g - cu[s])
+    return (torch.tensor(cu_local, dtype=torch.int32), torch.tensor(pos, dtype=torch.int32), start)
+
+
+def _thd_ext(x, halo_x, halo: int):
+    return x if halo_x is None else torch.cat([halo_x, x], dim=0)
+
+
+def local_fwd_thd(q, k, v, sinks, cu_seqlens, window: int, rope, rank: int, halo_kv=None, softmax_scale=None,
+                  attn_fwd=None):
+    """THD form of :func:`local_fwd`: q ``[T_loc, Hq, D]``, k / v ``[T_loc,
+    Hkv, D]``, `cu_seqlens` the global packing (host).  Returns ``(out
+    [T_loc, Hq, D], lse [Hq, T_loc])``.  No communication."""
+    attn_fwd = attn_fwd or (lambda *a, **kw: ops.gptoss_attn_fwd(*a, return_lse=True, **kw))
+    t_loc, Hq, D = q.shape
+    Hkv = k.shape[1]
+    halo = 0 if halo_kv is None else halo_kv.shape[0]
+    cu_l, pos, _ = thd_local_layout(cu_seqlens, rank, t_loc, halo)
+    q_ext = _thd_ext(q, torch.zeros((halo, Hq, D), dtype=q.dtype, device=q.device) if halo else None, halo)
+    k_ext = _thd_ext(k, halo_kv[:, :Hkv] if halo else None, halo)
+    v_ext = _thd_ext(v, halo_kv[:, Hkv:] if halo else None, halo)
+    max_len = int((cu_l[1:] - cu_l[:-1]).max())
+    out, lse = attn_fwd(q_ext, k_ext, v_ext, sinks, window=window, rope=rope, positions=pos.to(q.device),
+                        cu_seqlens=cu_l.to(q.device), max_seqlen=max_len, softmax_scale=softmax_scale)
+    return out[halo:].contiguous(), lse[:, halo:].contiguous()
+
+
+def local_bwd_thd(q, k, v, sinks, out, dout, lse, cu_seqlens, window: int, rope, rank: int, halo_kv=None,
+                  softmax_scale=None, attn_bwd=None):
+    """THD form of :func:`local_bwd`; returns ``(dq, dk, dv, dsinks,
+    dkv_halo)`` with dkv_halo ``[halo, 2 Hkv, D]`` (None on rank 0)."""
+    attn_bwd = attn_bwd or ops.gptoss_attn_bwd
+    t_loc, Hq, D = q.shape
+    Hkv = k.shape[1]
+    halo = 0 if halo_kv is None else halo_kv.shape[0]
+    cu_l, pos, _ = thd_local_layout(cu_seqlens, rank, t_loc, halo)
+    zq = torch.zeros((halo, Hq, D), dtype=q.dtype, device=q.device) if halo else None
+    q_ext = _thd_ext(q, zq, halo)
+    k_ext = _thd_ext(k, halo_kv[:, :Hkv] if halo else None, halo)
+    v_ext = _thd_ext(v, halo_kv[:, Hkv:] if halo else None, halo)
+    out_ext = _thd_ext(out, zq, halo)
+    dout_ext = _thd_ext(dout, zq, halo)  # no gradient flows into the halo rows
+    lse_ext = lse if not halo else torch.cat(
+        [torch.full((Hq, halo), float("inf"), dtype=lse.dtype, device=lse.device), lse], dim=1)
+    max_len = int((cu_l[1:] - cu_l[:-1]).max())
+    dq, dk, dv, dsinks = attn_bwd(q_ext, k_ext, v_ext, sinks, out_ext, dout_ext, lse_ext, window=window, rope=rope,
+                                  positions=pos.to(q.device), cu_seqlens=cu_l.to(q.device), max_seqlen=max_len,
+                                  softmax_scale=softmax_scale)
+    dkv_halo = torch.cat([dk[:halo], dv[:halo]], dim=1) if halo else None
+    return dq[halo:].contiguous(), dk[halo:].contiguous(), dv[halo:].contiguous(), dsinks, dkv_halo
+
+
+def sliding_window_fwd_thd(q, k, v, sinks, cu_seqlens, window: int, rope, group=None,
+                           softmax_scale: float | None = None, attn_fwd=None):
+    """:func:`sliding_window_fwd` for packed inputs: this rank's ``[T_loc, H,
+    D]`` tokens of a stream packed by `cu_seqlens` (global, host)."""
+    rank, world = _rank_world(group)
+    t_loc, _, D = q.shape
+    Hkv = k.shape[1]
+    halo = halo_rows(window, t_loc, world)
+    got = None
+    if halo:
+        tail = torch.cat([k[t_loc - halo:], v[t_loc - halo:]], dim=1)
+        got = _exchange(tail, (halo, 2 * Hkv, D), k.dtype, k.device, group, rank, world)
+    return local_fwd_thd(q, k, v, sinks, cu_seqlens, window, rope, rank, got, softmax_scale, attn_fwd)
+
+
+def sliding_window_bwd_thd(q, k, v, sinks, out, dout, lse, cu_seqlens, window: int, rope, group=None,
+                           softmax_scale: float | None = None, attn_bwd=None):
+    """:func:`sliding_window_bwd` for packed inputs."""
+    rank, world = _rank_world(group)
+    t_loc, _, D = q.shape
+    Hkv = k.shape[1]
+    halo = halo_rows(window, t_loc, world)
+    got = None
+    if halo:
+        tail = torch.cat([k[t_loc - halo:], v[t_loc - halo:]], dim=1)
+        got = _exchange(tail, (halo, 2 * Hkv, D), k.dtype, k.device, group, rank, world)
+    dq, dk, dv, dsinks, dkv_halo = local_bwd_thd(q, k, v, sinks, out, dout, lse, cu_seqlens, window, rope, rank,
+                                                 got, softmax_scale, attn_bwd)
+    if halo:
+        back = _exchange_back(dkv_halo, (halo, 2 * Hkv, D), dk.dtype, dk.device, group, rank, world)
+        if back is not None:
+            add_halo_grads(dk.unsqueeze(0), dv.unsqueeze(0), back.unsqueeze(0))
+    dsinks = dsinks.clone()
+    if world > 1:
+        dist.all_reduce(dsinks, op=dist.ReduceOp.SUM, group=group)
+    return dq, dk, dv, dsinks
