@@ -43,7 +43,7 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
         nvcc_path(),
         "-gencode", "arch=compute_100a,code=sm_100a",
         "-O3", "-lineinfo", "-std=c++17",
-        "--use_fast_math" if False else "-Xptxas=-O3",
+        "-Xptxas=-O3",
         "-Xcompiler", "-fPIC",
         "-shared", "-cudart", "static",
         "-I", os.path.join(ROOT, "include"),
