@@ -30,6 +30,12 @@ Contents
                definition by the chain rule, and the RoPE adjoint
                ``rope_transpose``.  The pages define the forward and describe
                training with it; they print no backward formula.
+``cp``         Attention of a query block over one key block at global
+               offsets (no sink) and the log-sum-exp merge of such blocks
+               with the sink folded once: the pieces of context parallelism
+               for full-context layers (``cp_size`` / ``cp_rank`` on the
+               ``gpt_oss.rope_utils`` page; the merge follows from the
+               definition in ``attention``).
 ``brute``      A second, independent formulation in scalar Python loops for
                tiny shapes (complex-multiply RoPE, softmax over the logits
                with the sink appended as one more column).
