@@ -53,3 +53,39 @@ def test_two_shards_sliding_window(cuda_device):
         got = np.concatenate([host(b[i]) for b in bwd], axis=1)
         assert_grad_parity(got, ref, f"cp {name}", E2E_MAX_REL, E2E_MEAN_REL)
     assert_dsinks(host(bwd[0][3]) + host(bwd[1][3]), rs, "cp")
+
+
+def test_two_shards_packed_stream(cuda_device):
+    # a packed stream of sequences 250, 210, 140 long split into two 300-token
+    # shards: the middle sequence straddles the boundary
+    from oracle.attention import attn_fwd_thd
+    from oracle.backward import attn_bwd_thd
+
+    rng = np.random.default_rng(157)
+    cu = [0, 250, 460, 600]
+    t_loc, Hq, Hkv, W = 300, 16, 2, 128
+    T = 2 * t_loc
+    q = bf16_round(rng.standard_normal((T, Hq, 64)))
+    k = bf16_round(rng.standard_normal((T, Hkv, 64)))
+    v = bf16_round(rng.standard_normal((T, Hkv, 64)))
+    dout = bf16_round(rng.standard_normal((T, Hq, 64)))
+    sinks = rng.standard_normal(Hq).astype(np.float32)
+    sh = [slice(0, t_loc), slice(t_loc, T)]
+    qd, kd, vd, dd = ([dev(a[s]) for s in sh] for a in (q, k, v, dout))
+    sd = f32(sinks)
+    halo_n = cp.halo_rows(W, t_loc, 2)
+    halo = [None, torch.cat([kd[0][t_loc - halo_n:], vd[0][t_loc - halo_n:]], dim=1)]
+    fwd = [cp.local_fwd_thd(qd[r], kd[r], vd[r], sd, cu, W, ROPE, r, halo[r]) for r in range(2)]
+    bwd = [cp.local_bwd_thd(qd[r], kd[r], vd[r], sd, fwd[r][0], dd[r], fwd[r][1], cu, W, ROPE, r, halo[r])
+           for r in range(2)]
+    cp.add_halo_grads(bwd[0][1].unsqueeze(0), bwd[0][2].unsqueeze(0), bwd[1][4].unsqueeze(0))
+    torch.cuda.synchronize()
+    assert ops.read_device_status() == 0
+    ref_o, ref_l = attn_fwd_thd(q, k, v, sinks, np.array(cu), 0.125, W, rope_tables=TABLES)
+    assert_parity(np.concatenate([host(f[0]) for f in fwd], axis=0), ref_o, "cp thd out")
+    assert_parity(np.concatenate([host(f[1]) for f in fwd], axis=1), ref_l, "cp thd lse")
+    rq, rk, rv, rs = attn_bwd_thd(q, k, v, sinks.astype(np.float64), np.array(cu), 0.125, W, dout, rope_tables=TABLES)
+    for i, (ref, name) in enumerate(((rq, "dq"), (rk, "dk"), (rv, "dv"))):
+        got = np.concatenate([host(b[i]) for b in bwd], axis=0)
+        assert_grad_parity(got, ref, f"cp thd {name}", E2E_MAX_REL, E2E_MEAN_REL)
+    assert_dsinks(host(bwd[0][3]) + host(bwd[1][3]), rs, "cp thd")
