@@ -18,7 +18,11 @@ Pins, each independent of the oracle's own code:
   logits with the sink appended as a column) agrees on tiny shapes, BSHD and
   packed THD, windows 1, 3 and longer than the sequence;
 * THD equals separate per-sequence calls; decode equals the last prefill row;
-  row-by-row sampling equals the full computation.
+  row-by-row sampling equals the full computation;
+* over 1100 rows (three of the oracle's 512-row blocks, windows 0 / 1 / 128 /
+  700) the output and log-sum-exp equal a whole-sequence restatement with
+  ``torch.softmax`` over the logits plus a sink column and
+  ``torch.logsumexp``, and with a -inf sink equal SDPA.
 """
 
 import math
@@ -210,3 +214,54 @@ def test_row_sampling_matches_full(window):
     for n, (t, h) in enumerate(rows_t):
         np.testing.assert_allclose(ro[n], out_t[t, h], rtol=1e-12, atol=1e-13)
         assert rl[n] == pytest.approx(lse_t[h, t], rel=1e-12)
+
+
+def _torch_sink_attention(q, k, v, sinks, scale, window):
+    """The definition restated with library routines over the whole sequence
+    at once: a full [L, L] logit matrix, the visibility mask built from
+    index grids, the sink as one more softmax column (``torch.softmax``) and
+    the log-sum-exp from ``torch.logsumexp``.  float64, CPU."""
+    L, Hq, _ = q.shape
+    G = Hq // k.shape[1]
+    qt = torch.from_numpy(q).permute(1, 0, 2)
+    kt = torch.from_numpy(k).permute(1, 0, 2).repeat_interleave(G, dim=0)
+    vt = torch.from_numpy(v).permute(1, 0, 2).repeat_interleave(G, dim=0)
+    logits = scale * qt @ kt.transpose(1, 2)
+    i = torch.arange(L)[:, None]
+    j = torch.arange(L)[None, :]
+    allowed = j <= i
+    if window > 0:
+        allowed = allowed & (i - j < window)
+    logits = logits.masked_fill(~allowed, float("-inf"))
+    col = torch.from_numpy(np.asarray(sinks, np.float64)).view(Hq, 1, 1).expand(Hq, L, 1)
+    full = torch.cat([logits, col], dim=-1)
+    w = torch.softmax(full, dim=-1)[..., :L]
+    return (w @ vt).permute(1, 0, 2).numpy(), torch.logsumexp(full, dim=-1).numpy()
+
+
+@pytest.mark.parametrize("window", [0, 1, 128, 700])
+def test_several_row_blocks_against_library_softmax(window):
+    # 1100 rows span three of the oracle's 512-row blocks; the band of the
+    # later blocks starts at r0 - window + 1, which this pins row by row
+    L, Hq, Hkv, D = 1100, 4, 2, 64
+    q, k, v = _rand((L, Hq, D), 70), _rand((L, Hkv, D), 71), _rand((L, Hkv, D), 72)
+    sinks = _rand(Hq, 73)
+    out, lse = sink_attention_sequence(q, k, v, sinks, 0.125, window)
+    ref_o, ref_l = _torch_sink_attention(q, k, v, sinks, 0.125, window)
+    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_l, rtol=1e-13, atol=0)
+    # and the row-by-row path on the rows around the block edges
+    pos = np.arange(L)
+    rows = [(0, h, i) for h in (0, 3) for i in (0, 511, 512, 513, 639, 640, 1023, 1024, 1099)]
+    ro, rl = attn_rows_bshd(q[None], k[None], v[None], sinks, 0.125, window, rows, positions=pos[None])
+    for n, (_, h, i) in enumerate(rows):
+        np.testing.assert_allclose(ro[n], out[i, h], rtol=0, atol=1e-12)
+        assert rl[n] == pytest.approx(lse[h, i], rel=1e-13)
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_several_row_blocks_minus_inf_sink_is_sdpa(window):
+    L, Hq, Hkv, D = 1100, 2, 1, 64
+    q, k, v = _rand((L, Hq, D), 74), _rand((L, Hkv, D), 75), _rand((L, Hkv, D), 76)
+    out, _ = sink_attention_sequence(q, k, v, np.full(Hq, -np.inf), 0.125, window)
+    np.testing.assert_allclose(out, _sdpa(q, k, v, 0.125, window), rtol=0, atol=1e-12)
