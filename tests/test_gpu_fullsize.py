@@ -1,14 +1,19 @@
 """GPU parity at the full workload sizes, in the launch configuration the
-benchmark times, checked on sampled outputs the oracle computes one by one:
+benchmark times.
 
-* sliding-window prefill B=4, S=4096, 64/8 heads, window 128, YaRN RoPE;
-* full-context prefill B=2, S=8192;
-* packed THD pair, 32768 tokens, full and window 128;
-* decode B=64 x 32768 and B=8 x 131072, full and window 128 (caches drawn
-  on the device, sampled sequences read back for the oracle).
+Every output element (and every lse) is compared with the float64 oracle for
 
-Sampled rows always include the tile edges (first / last row of a tile, the
-first and last token of a sequence) besides random ones.
+* sliding-window prefill B=4, S=4096, 64/8 heads, window 128, YaRN RoPE
+  (about ten seconds of oracle time on a few host cores);
+* the packed THD stream of 32768 tokens with window 128;
+* decode B=64 x 32768 and B=8 x 131072, full and window 128, every sequence
+  (caches drawn on the device and read back one sequence at a time).
+
+The two full-context prefills (B=2 x 8192 and the THD stream without a
+window: 1.1 and 1.4 TFLOP, hours of float64 host time) are checked on
+sampled rows that the oracle computes one by one; the samples always include
+the tile edges (first / last row of a tile, the first and last token of a
+sequence) besides random ones.
 """
 
 import numpy as np
@@ -28,9 +33,10 @@ from attention_yarn_rope_b200.workloads import (
     make_decode_device,
     make_prefill,
 )
-from oracle.attention import attn_decode, attn_rows_bshd, attn_rows_thd
+from oracle.attention import attn_decode, attn_fwd_bshd, attn_fwd_thd, attn_rows_bshd, attn_rows_thd
+from oracle.rope import rope
 from oracle.yarn import yarn_inv_freq_and_concentration
-from tests.gpu_util import assert_parity, dev, f32, host, i32
+from tests.gpu_util import assert_lse_parity, assert_parity, dev, f32, host, i32
 
 pytestmark = pytest.mark.gpu
 
@@ -48,8 +54,21 @@ def _rows_bshd(cfg, n, seed):
     return rows
 
 
-@pytest.mark.parametrize("cfg", [SLIDING, FULL], ids=lambda c: c.name)
-def test_prefill_full_size_sampled(cuda_device, cfg):
+def test_sliding_prefill_full_size_every_element(cuda_device):
+    cfg = SLIDING
+    x = make_prefill(cfg)
+    out, lse = ops.gptoss_attn_fwd(dev(x.q), dev(x.k), dev(x.v), f32(x.sinks), window=cfg.window,
+                                   rope=ops.RopeConfig.from_dict(cfg.rope), return_lse=True)
+    torch.cuda.synchronize()
+    o, l = host(out), host(lse)
+    del out, lse
+    ref_o, ref_l = attn_fwd_bshd(x.q, x.k, x.v, x.sinks, cfg.softmax_scale, cfg.window, rope_tables=_tables(cfg.rope))
+    assert_parity(o, ref_o, cfg.name + " out (every element)")
+    assert_lse_parity(l, ref_l, cfg.name + " lse (every element)")
+
+
+def test_full_prefill_full_size_sampled(cuda_device):
+    cfg = FULL
     x = make_prefill(cfg)
     out, lse = ops.gptoss_attn_fwd(dev(x.q), dev(x.k), dev(x.v), f32(x.sinks), window=cfg.window,
                                    rope=ops.RopeConfig.from_dict(cfg.rope), return_lse=True)
@@ -62,12 +81,11 @@ def test_prefill_full_size_sampled(cuda_device, cfg):
     got_o = np.stack([o[b, i, h] for (b, h, i) in rows])
     got_l = np.array([l[b, h, i] for (b, h, i) in rows])
     assert_parity(got_o, ref_o, cfg.name + " out")
-    assert_parity(got_l, ref_l, cfg.name + " lse")
+    assert_lse_parity(got_l, ref_l, cfg.name + " lse")
     assert np.all(np.isfinite(o))
 
 
-@pytest.mark.parametrize("cfg", [THD_FULL, THD_WINDOW], ids=lambda c: c.name)
-def test_thd_full_size_sampled(cuda_device, cfg):
+def _thd_call(cfg):
     x = make_prefill(cfg)
     cu = x.cu_seqlens
     lens = np.diff(cu)
@@ -75,27 +93,51 @@ def test_thd_full_size_sampled(cuda_device, cfg):
                                    cu_seqlens=i32(cu), max_seqlen=int(lens.max()),
                                    rope=ops.RopeConfig.from_dict(cfg.rope), return_lse=True)
     torch.cuda.synchronize()
+    return x, host(out), host(lse)
+
+
+def test_thd_window_full_size_every_element(cuda_device):
+    cfg = THD_WINDOW
+    x, o, l = _thd_call(cfg)
+    ref_o, ref_l = attn_fwd_thd(x.q, x.k, x.v, x.sinks, x.cu_seqlens, cfg.softmax_scale, cfg.window,
+                                rope_tables=_tables(cfg.rope))
+    assert_parity(o, ref_o, cfg.name + " out (every element)")
+    assert_lse_parity(l, ref_l, cfg.name + " lse (every element)")
+
+
+def test_thd_full_context_full_size_sampled(cuda_device):
+    cfg = THD_FULL
+    x, o, l = _thd_call(cfg)
+    cu = x.cu_seqlens
+    lens = np.diff(cu)
     rng = np.random.default_rng(6)
     T = int(cu[-1])
     rows = [(int(cu[s]), s % 64) for s in range(len(lens))] + [(int(cu[s + 1]) - 1, 7) for s in range(len(lens))]
     rows += [(int(rng.integers(T)), int(rng.integers(64))) for _ in range(40)]
     ref_o, ref_l = attn_rows_thd(x.q, x.k, x.v, x.sinks, cu, cfg.softmax_scale, cfg.window, rows,
                                  rope_tables=_tables(cfg.rope))
-    o = host(out)
-    l = host(lse)
     assert_parity(np.stack([o[t, h] for (t, h) in rows]), ref_o, cfg.name + " out")
-    assert_parity(np.array([l[h, t] for (t, h) in rows]), ref_l, cfg.name + " lse")
+    assert_lse_parity(np.array([l[h, t] for (t, h) in rows]), ref_l, cfg.name + " lse")
 
 
 @pytest.mark.parametrize("cfg", [DECODE_B64, DECODE_B64_W, DECODE_B8, DECODE_B8_W], ids=lambda c: c.name)
-def test_decode_full_size_sampled(cuda_device, cfg):
+def test_decode_full_size_every_sequence(cuda_device, cfg):
     q, kc, vc, sinks, seqlens = make_decode_device(cfg, cuda_device)
     out, lse = ops.gptoss_attn_decode(q, kc, vc, seqlens, sinks, window=cfg.window,
                                       rope=ops.RopeConfig.from_dict(cfg.rope), return_lse=True)
     torch.cuda.synchronize()
-    picks = sorted({0, cfg.B - 1, cfg.B // 2})
-    for b in picks:
-        ref_o, ref_l = attn_decode(host(q[b:b + 1]), host(kc[b:b + 1]), host(vc[b:b + 1]), [cfg.L], host(sinks),
-                                   0.125, cfg.window, rope_tables=_tables(cfg.rope))
-        assert_parity(host(out[b:b + 1]), ref_o, f"{cfg.name} b={b} out")
-        assert_parity(host(lse[b:b + 1]), ref_l, f"{cfg.name} b={b} lse")
+    tables = _tables(cfg.rope)
+    qh, sh = host(q), host(sinks)
+    lo = max(0, cfg.L - cfg.window) if cfg.window > 0 else 0
+    ref_o = np.zeros(qh.shape)
+    ref_l = np.zeros(qh.shape[:2])
+    # the query rotated by the oracle at its true position L - 1; the decode
+    # oracle then sees only the visible cache rows [lo, L), which travel to the
+    # host one sequence at a time
+    q_rot = rope(qh, np.full(cfg.B, cfg.L - 1), *tables)
+    for b in range(cfg.B):
+        ro, rl = attn_decode(q_rot[b:b + 1], host(kc[b:b + 1, lo:cfg.L]), host(vc[b:b + 1, lo:cfg.L]),
+                             [cfg.L - lo], sh, 0.125, cfg.window)
+        ref_o[b], ref_l[b] = ro[0], rl[0]
+    assert_parity(host(out), ref_o, f"{cfg.name} out (every sequence)")
+    assert_lse_parity(host(lse), ref_l, f"{cfg.name} lse (every sequence)")

@@ -13,7 +13,7 @@ from attention_yarn_rope_b200 import ops
 from attention_yarn_rope_b200.workloads import GPTOSS_ROPE, bf16_round
 from oracle.paged import attn_decode_paged, kv_append_paged
 from oracle.yarn import yarn_inv_freq_and_concentration
-from tests.gpu_util import assert_parity, dev, f32, host, i32
+from tests.gpu_util import assert_lse_parity, assert_parity, dev, f32, host, i32
 
 pytestmark = pytest.mark.gpu
 
@@ -44,7 +44,7 @@ def test_paged_decode_matches_oracle(cuda_device, block_size, window):
     torch.cuda.synchronize()
     ref, ref_lse = attn_decode_paged(q, kp, vp, table, block_size, lens, sinks, 0.125, window, TABLES)
     assert_parity(host(out), ref, f"paged out bs={block_size} w={window}")
-    assert_parity(host(lse), ref_lse, f"paged lse bs={block_size} w={window}")
+    assert_lse_parity(host(lse), ref_lse, f"paged lse bs={block_size} w={window}")
 
 
 def test_paged_equals_contiguous_bitwise(cuda_device):
@@ -178,7 +178,7 @@ def test_multi_token_decode_matches_oracle(cuda_device, window, q_len, Hq, Hkv):
     assert out.shape == (len(lens), q_len, Hq, 64) and lse.shape == (len(lens), q_len, Hq)
     ref, ref_lse = attn_decode_paged(q, kp, vp, table, bs, lens, sinks, 0.125, window, TABLES)
     assert_parity(host(out), ref, f"multi-token out q_len={q_len} G={Hq // Hkv} w={window}")
-    assert_parity(host(lse), ref_lse, f"multi-token lse q_len={q_len} G={Hq // Hkv} w={window}")
+    assert_lse_parity(host(lse), ref_lse, f"multi-token lse q_len={q_len} G={Hq // Hkv} w={window}")
 
 
 def test_multi_token_many_splits(cuda_device):

@@ -3,8 +3,8 @@
 Emulates the exact definition with only the roundings the prefill kernel
 makes -- rotated q / k rounded to fp16 for QK^T, unnormalised P rounded to
 bf16 for P V, the output rounded to bf16 -- and checks it against the float64
-oracle with the same bar the GPU tests use (every element within 1e-2 on the
-unit scale, mean-abs <= 1e-3).  It also shows why the QK^T operands are fp16:
+oracle with the same bar the GPU tests use (raw 1e-2 per element where
+|ref| <= 4, plus half a bf16 spacing above 4; mean-abs <= 1e-3).  It also shows why the QK^T operands are fp16:
 rounding them to bf16 instead breaks the bar at the YaRN concentration.
 """
 
@@ -14,6 +14,7 @@ from attention_yarn_rope_b200.workloads import bf16_round
 from oracle.attention import attn_fwd_bshd
 from oracle.rope import default_positions_bshd, rope
 from oracle.yarn import yarn_inv_freq_and_concentration
+from tests.gpu_util import out_bar
 
 TABS = yarn_inv_freq_and_concentration(64, 150000.0, 32.0, 4096, 1.0, 32.0)
 
@@ -52,8 +53,9 @@ def _case():
     return q, k, v, sinks
 
 
-def _scaled_max(got, ref):
-    return float((np.abs(got - ref) / np.maximum(1.0, np.abs(ref))).max())
+def _bar_used(got, ref):
+    """Largest share of the per-element bar that an element uses."""
+    return float((np.abs(got - ref) / out_bar(ref)).max())
 
 
 def test_kernel_number_formats_meet_the_bar():
@@ -61,7 +63,8 @@ def test_kernel_number_formats_meet_the_bar():
     for window in (0, 128):
         ref, _ = attn_fwd_bshd(q, k, v, sinks, 0.125, window, rope_tables=TABS)
         emu = _emulate(q, k, v, sinks, window, _f16)
-        assert _scaled_max(emu, ref) < 0.7e-2
+        assert _bar_used(emu, ref) < 0.9
+        assert np.abs(emu - ref)[np.abs(ref) <= 4].max() < 0.9e-2
         assert np.abs(emu - ref).mean() < 0.6e-3
 
 
