@@ -221,32 +221,64 @@ gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
-constexpr int kNoAllocMaxDevices = 64;
+constexpr int kScratchCacheSlots = 16;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
-// The array's name is a host-side stand-in in host code: its device address
-// comes from cudaGetSymbolAddress, once per device, with that device current.
-void* g_scratch_addr[kNoAllocMaxDevices];
-std::once_flag g_scratch_once[kNoAllocMaxDevices];
-cudaError_t g_scratch_err[kNoAllocMaxDevices];
+// In host code the array's name is a host-side stand-in, not a device
+// address.  The device address belongs to the CUDA context the library's
+// module is loaded into -- not to a device number: after cudaDeviceReset, or
+// with a non-primary driver context current, an address remembered per device
+// would be stale.  So the address is looked up with cudaGetSymbolAddress
+// (which allocates nothing) on the first call in each context, with that
+// context current, and remembered under the context's unique id (cuCtxGetId;
+// a process never reuses an id).  A full cache forgets its oldest entry; a
+// forgotten context just looks its address up again.
+struct ScratchSlot {
+  unsigned long long ctx_id;
+  void* addr;
+};
+std::mutex g_scratch_mu;
+ScratchSlot g_scratch_slots[kScratchCacheSlots];
+int g_scratch_used = 0, g_scratch_next = 0;
 
-void* scratch_address(int device, gptoss_status* st) {
-  if (device < 0 || device >= kNoAllocMaxDevices) {
-    *st = GPTOSS_ERR_UNSUPPORTED;
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
     return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+void* scratch_address(gptoss_status* st) {
+  static const PFN_cuCtxGetCurrent_v4000 get_current = driver_fn<PFN_cuCtxGetCurrent_v4000>("cuCtxGetCurrent");
+  static const PFN_cuCtxGetId_v12000 get_id = driver_fn<PFN_cuCtxGetId_v12000>("cuCtxGetId");
+  *st = GPTOSS_ERR_CUDA;
+  if (get_current == nullptr || get_id == nullptr) return nullptr;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return nullptr;
+  void* addr = nullptr;
+  if (ctx == nullptr) {
+    // no context current yet: the runtime binds the current device's primary
+    // context while it resolves the symbol
+    if (cudaGetSymbolAddress(&addr, g_decode_scratch) != cudaSuccess) return nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
   }
-  std::call_once(g_scratch_once[device], [device]() {
-    void* ptr = nullptr;
-    g_scratch_err[device] = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-    g_scratch_addr[device] = ptr;
-  });
-  if (g_scratch_err[device] != cudaSuccess || g_scratch_addr[device] == nullptr) {
-    *st = GPTOSS_ERR_CUDA;
-    return nullptr;
-  }
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  for (int i = 0; i < g_scratch_used; ++i)
+    if (g_scratch_slots[i].ctx_id == id) {
+      *st = GPTOSS_OK;
+      return g_scratch_slots[i].addr;
+    }
+  if (addr == nullptr && cudaGetSymbolAddress(&addr, g_decode_scratch) != cudaSuccess) return nullptr;
+  if (addr == nullptr) return nullptr;
+  const int slot = g_scratch_used < kScratchCacheSlots ? g_scratch_used++ : g_scratch_next++ % kScratchCacheSlots;
+  g_scratch_slots[slot] = ScratchSlot{id, addr};
   *st = GPTOSS_OK;
-  return g_scratch_addr[device];
+  return addr;
 }
 
 }  // namespace
@@ -262,10 +294,8 @@ extern "C" gptoss_status gptoss_attn_decode_noalloc(const void* q, const void* k
   const size_t need = gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D);
   if (need == 0) return D != kHeadDim ? GPTOSS_ERR_UNSUPPORTED : GPTOSS_ERR_INVALID_ARG;
   if (need > kNoAllocScratchBytes) return GPTOSS_ERR_UNSUPPORTED;  // partials exceed the fixed array
-  int device = 0;
-  if (cudaGetDevice(&device) != cudaSuccess) return GPTOSS_ERR_CUDA;
   gptoss_status st = GPTOSS_OK;
-  void* ws = scratch_address(device, &st);
+  void* ws = scratch_address(&st);
   if (ws == nullptr) return st;
   return gptoss_attn_decode(q, k_cache, v_cache, cache_seqlens, sinks, B, Lmax, Hq, Hkv, D, window, softmax_scale,
                             rope, out, lse, ws, kNoAllocScratchBytes, stream);

@@ -293,10 +293,13 @@ gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const
  *   whose gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D) exceeds
  *   16 MiB are rejected with GPTOSS_ERR_UNSUPPORTED (B=64 x 32768 needs
  *   8.7 MB, B=8 x 131072 needs 5.0 MB).
- *   The first call on a device looks the array's device address up
- *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.  Nothing in the array needs to start at zero:
- *   each call writes every partial it later reads.
+ *   The array's device address belongs to a CUDA context: the first call in
+ *   each context (the current one when the call is made) looks it up with
+ *   cudaGetSymbolAddress and remembers it under the context's unique id, so a
+ *   device reset or another driver context gets its own lookup, never a
+ *   stale address.  Make that first call before any stream capture.  Nothing
+ *   in the array needs to start at zero: each call writes every partial it
+ *   later reads.
  *   All calls share the one array, which keeps the last call's contents:
  *   calls whose executions overlap on the GPU (other streams, other host
  *   threads) race and must be serialised by the caller.
