@@ -158,9 +158,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
     if (t < cr.ntok) {
       const int64_t vb = static_cast<int64_t>(b) * p.q_len + cr.tok0 + t;
       const __nv_bfloat16* qr = p.q + (vb * p.Hq + g * G + row % G) * kHeadDim;
-      x = __bfloat162float(qr[j]);
-      y = __bfloat162float(qr[j + kPairs]);
-      if (p.tab.enabled) {
+      x = __bfloat162float(qr[rope_feature_a(j, p.tab.R)]);
+      y = __bfloat162float(qr[rope_feature_b(j, p.tab.R)]);
+      if (p.tab.enabled && j < p.tab.R) {
         const float2 cs = rope_cs(cr.n_first + t - 1, p.tab.inv_freq[j], p.tab.conc);
         const float xr = x * cs.x - y * cs.y;
         const float yr = y * cs.x + x * cs.y;
@@ -168,8 +168,8 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
         y = yr;
       }
     }
-    sm.q[row][j] = __float2bfloat16_rn(x);
-    sm.q[row][j + kPairs] = __float2bfloat16_rn(y);
+    sm.q[row][rope_feature_a(j, p.tab.R)] = __float2bfloat16_rn(x);
+    sm.q[row][rope_feature_b(j, p.tab.R)] = __float2bfloat16_rn(y);
   }
   __syncthreads();
 
@@ -484,17 +484,18 @@ __global__ void kv_append_paged_kernel(const __grid_constant__ AppendParams p) {
   const int64_t off = (static_cast<int64_t>(blk) * p.block_size + pos % p.block_size) * p.Hkv * kHeadDim +
                       static_cast<int64_t>(g) * kHeadDim;
   const int64_t src = ((static_cast<int64_t>(b) * p.q_len + tok) * p.Hkv + g) * kHeadDim;
-  float x = __bfloat162float(p.k_new[src + j]), y = __bfloat162float(p.k_new[src + j + kPairs]);
-  if (p.tab.enabled) {
+  const int fa = rope_feature_a(j, p.tab.R), fb = rope_feature_b(j, p.tab.R);
+  float x = __bfloat162float(p.k_new[src + fa]), y = __bfloat162float(p.k_new[src + fb]);
+  if (p.tab.enabled && j < p.tab.R) {
     const float2 cs = rope_cs(pos, p.tab.inv_freq[j], p.tab.conc);
     const float xr = x * cs.x - y * cs.y, yr = y * cs.x + x * cs.y;
     x = xr;
     y = yr;
   }
-  p.k_pool[off + j] = __float2bfloat16_rn(x);
-  p.k_pool[off + j + kPairs] = __float2bfloat16_rn(y);
-  p.v_pool[off + j] = p.v_new[src + j];
-  p.v_pool[off + j + kPairs] = p.v_new[src + j + kPairs];
+  p.k_pool[off + fa] = __float2bfloat16_rn(x);
+  p.k_pool[off + fb] = __float2bfloat16_rn(y);
+  p.v_pool[off + fa] = p.v_new[src + fa];
+  p.v_pool[off + fb] = p.v_new[src + fb];
 }
 
 }  // namespace gptoss

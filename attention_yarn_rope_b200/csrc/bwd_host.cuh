@@ -109,6 +109,7 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   } else {
     memset(&rp.tab, 0, sizeof(rp.tab));  // every inverse frequency 0: cos 1, sin 0
     rp.tab.conc = 1.f;
+    rp.tab.R = kPairs;
   }
   rp.cs_out = reinterpret_cast<float2*>(wsb + ws.cs);
   const int rgrid = (total_tokens + kRopeTokensPerCta - 1) / kRopeTokensPerCta;

@@ -51,7 +51,7 @@ gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cach
   if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
   if (Hq / Hkv > kDecMaxGroup) return GPTOSS_ERR_UNSUPPORTED;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
-  gptoss_status st = check_rope(rope, D);
+  gptoss_status st = check_rope(rope, D, /*allow_partial=*/true);
   if (st != GPTOSS_OK) return st;
   if (B == 0) return GPTOSS_OK;
   if (!q || !k_cache || !v_cache || !cache_seqlens || !sinks || !out || !workspace) return GPTOSS_ERR_INVALID_ARG;
@@ -181,7 +181,7 @@ gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const
   if (Hkv * kPairs > 1024) return GPTOSS_ERR_UNSUPPORTED;
   gptoss_status st = check_paged(max_blocks, block_size, num_blocks);
   if (st != GPTOSS_OK) return st;
-  st = check_rope(rope, D);
+  st = check_rope(rope, D, /*allow_partial=*/true);
   if (st != GPTOSS_OK) return st;
   if (B == 0) return GPTOSS_OK;
   if (!k_new || !v_new || !cache_seqlens || !block_table || !k_pool || !v_pool) return GPTOSS_ERR_INVALID_ARG;

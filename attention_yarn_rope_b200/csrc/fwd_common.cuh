@@ -13,11 +13,11 @@
 //                     tiles) rotated in place after TMA
 //   warps 4-7 / 8-11  softmax of head A / head B (thread = query row; warp w
 //                     reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31)
-//   warp 12           TMA producer (two Q tiles per unit into a double
-//                     buffer, K / V tiles into a 4-stage ring)
+//   warp 12           TMA producer of the K / V tiles (4-stage ring)
 //   warp 13           TMEM allocation; QK^T issue (fwd_mma_s_role)
 //   warp 14           P V issue (fwd_mma_pv_role)
-//   warp 15           idle (completes the register split)
+//   warp 15           TMA producer of the Q tiles (two per unit, 3-stage
+//                     ring: a unit's Q arrives while the two before it run)
 // setmaxnreg moves registers from the rope / producer / MMA warpgroups to the
 // two softmax warpgroups: launch 512 threads x 128 registers = 65536, split
 // 2 x 128 x 208 + 128 x 56 + 128 x 40 = 65536.  The host refuses to launch if
@@ -33,7 +33,8 @@
 namespace gptoss {
 
 constexpr int kFwdTile = 128;         // query rows and keys per tile
-constexpr int kFwdStages = 4;
+constexpr int kFwdStages = 4;         // K / V ring
+constexpr int kFwdQStages = 3;        // Q ring (units)
 constexpr int kFwdThreads = 512;
 constexpr int kFwdLaunchRegs = 128;   // 65536 / 512
 constexpr int kFwdTileBytes = kFwdTile * kHeadDim * 2;  // 16 KB
@@ -51,8 +52,8 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsRope + 128 * kRegsOther == kFw
 
 struct FwdParams {
   CUtensorMap tmap_q;  // dims (64, Hq, S or T, B or 1), box (64, 1, 128, 1)
-  CUtensorMap tmap_k;  // dims (64, Hkv, S or T, B or 1), box (64, 1, 128, 1)
-  CUtensorMap tmap_v;
+  CUtensorMap tmap_k;  // fp16 k of the workspace, dims (64, Hkv, S or T, B or 1), box (64, 1, 128, 1)
+  CUtensorMap tmap_v;  // fp16 v of the workspace, same layout
   const __nv_bfloat16* q;
   gptoss_strides sq;
   __nv_bfloat16* out;
@@ -62,7 +63,6 @@ struct FwdParams {
   const int32_t* positions;
   const int32_t* cu_seqlens;
   int B, S, T, Hq, Hkv, G, HP, window, n_qtiles, n_units;
-  int k_in_kernel;  // 1: K tiles are rotated in shared memory; 0: k arrives rotated (or RoPE is off)
   const float2* cs_tab;  // nullable: per-token (c cos, c sin) of the 32 pairs, [token][32]
   float scale_log2;
   uint64_t wait_ns;
@@ -70,11 +70,11 @@ struct FwdParams {
 };
 
 struct __align__(1024) FwdSmem {
-  uint8_t q[2][2][kFwdTileBytes];  // [buffer][head A/B], rotated, 128B-swizzled
+  uint8_t q[kFwdQStages][2][kFwdTileBytes];  // [stage][head A/B], rotated, 128B-swizzled
   uint8_t k[kFwdStages][kFwdTileBytes];
   uint8_t v[kFwdStages][kFwdTileBytes];
-  uint64_t q_loaded[2], q_full[2], q_empty[2];  // TMA landed / rotated / free again
-  uint64_t k_full[kFwdStages], k_ready[kFwdStages], k_empty[kFwdStages];
+  uint64_t q_loaded[kFwdQStages], q_full[kFwdQStages], q_empty[kFwdQStages];  // TMA landed / rotated / free
+  uint64_t k_full[kFwdStages], k_empty[kFwdStages];
   uint64_t v_full[kFwdStages], v_empty[kFwdStages];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];  // per head slot A/B
   uint64_t mma_final[2];  // the S and P V issuers' last products have completed

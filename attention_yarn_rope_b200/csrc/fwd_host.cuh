@@ -22,7 +22,7 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
   if (rope == nullptr) return GPTOSS_ERR_INVALID_ARG;
   if (B < 0 || S_or_T < 0 || Hq <= 0 || Hkv <= 0) return GPTOSS_ERR_INVALID_ARG;
   if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
-  gptoss_status st = check_rope(rope, D);
+  gptoss_status st = check_rope(rope, D, /*allow_partial=*/true);
   if (st != GPTOSS_OK) return st;
   const bool thd = cu_seqlens != nullptr;
   const int64_t ntok = thd ? S_or_T : static_cast<int64_t>(B) * S_or_T;
@@ -55,15 +55,25 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
   return check_launch();
 }
 
-// Workspace of gptoss_attn_fwd: rotated k (fp16, [token][Hkv][64]), then at a
-// 256-byte boundary each token's 32 (c cos, c sin) pairs ([token][32] float2).
-static size_t fwd_ws_k_bytes(int32_t total_tokens, int32_t Hkv) {
+// Workspace of gptoss_attn_fwd: k (rotated) and v as fp16, each dense
+// [token][Hkv][64] and rounded up to 256 bytes, then each token's 32
+// (c cos, c sin) pairs ([token][32] float2).
+static size_t fwd_ws_kv_bytes(int32_t total_tokens, int32_t Hkv) {
   return (static_cast<size_t>(total_tokens) * Hkv * kHeadDim * 2 + 255) & ~static_cast<size_t>(255);
 }
 
 size_t gptoss_attn_fwd_workspace_size(int32_t total_tokens, int32_t Hkv, int32_t D) {
   if (total_tokens < 0 || Hkv <= 0 || D != kHeadDim) return 0;
-  return fwd_ws_k_bytes(total_tokens, Hkv) + static_cast<size_t>(total_tokens) * kPairs * sizeof(float2);
+  return 2 * fwd_ws_kv_bytes(total_tokens, Hkv) + static_cast<size_t>(total_tokens) * kPairs * sizeof(float2);
+}
+
+// The identity rotation (every angle 0, concentration 1): the pre-pass and
+// the rope warps then only convert bf16 to fp16, exactly.
+static void identity_table(RopeTable* t) {
+  for (int j = 0; j < kPairs; ++j) t->inv_freq[j] = 0.0;
+  t->conc = 1.0f;
+  t->enabled = 1;
+  t->R = kPairs;
 }
 
 gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk, const void* v,
@@ -76,7 +86,7 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
   if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
-  gptoss_status st = check_rope(rope, D);
+  gptoss_status st = check_rope(rope, D, /*allow_partial=*/true);
   if (st != GPTOSS_OK) return st;
   const bool thd = cu_seqlens != nullptr;
   if (!thd && static_cast<int64_t>(B) * S != total_tokens) return GPTOSS_ERR_INVALID_ARG;
@@ -85,10 +95,10 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GPTOSS_ERR_INVALID_ARG;
   if (!strides_ok(sq, !thd) || !strides_ok(sk, !thd) || !strides_ok(sv, !thd) || !strides_ok(so, !thd))
     return GPTOSS_ERR_INVALID_ARG;
-  // with RoPE and a workspace, k is rotated once into it (fp16) instead of
-  // once per work unit inside the kernel
-  const bool k_pre = rope != nullptr && workspace != nullptr;
-  if (k_pre && (workspace_bytes < gptoss_attn_fwd_workspace_size(total_tokens, Hkv, D) || !aligned16(workspace)))
+  // k (rotated) and v are written once into the workspace as fp16, the
+  // operand format of both products
+  if (workspace == nullptr || !aligned16(workspace) ||
+      workspace_bytes < gptoss_attn_fwd_workspace_size(total_tokens, Hkv, D))
     return GPTOSS_ERR_INVALID_ARG;
   const int n_qtiles = (S + kFwdTile - 1) / kFwdTile;
   const int G = Hq / Hkv;
@@ -118,19 +128,16 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   st = make_tmap_4d(&p.tmap_q, q, kHeadDim, Hq, dimS, dimB, sq.head * 2, sq.tok * 2,
                          qb_stride == 0 ? 16 : qb_stride, kHeadDim, 1, kFwdTile, 1);
   if (st != GPTOSS_OK) return st;
-  const uint64_t kb_stride = thd ? dimS * sk.tok * 2 : static_cast<uint64_t>(sk.batch) * 2;
-  const uint64_t vb_stride = thd ? dimS * sv.tok * 2 : static_cast<uint64_t>(sv.batch) * 2;
-  if (k_pre) {  // dense fp16 [B, S, Hkv, D] / [T, Hkv, D] in the workspace
-    const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
-    st = make_tmap_4d(&p.tmap_k, workspace, kHeadDim, Hkv, dimS, dimB, kHeadDim * 2, tok_b,
-                      thd ? dimS * tok_b : static_cast<uint64_t>(S) * tok_b, kHeadDim, 1, kFwdTile, 1, true);
-  } else {
-    st = make_tmap_4d(&p.tmap_k, k, kHeadDim, Hkv, dimS, dimB, sk.head * 2, sk.tok * 2,
-                      kb_stride == 0 ? 16 : kb_stride, kHeadDim, 1, kFwdTile, 1);
-  }
+  // fp16 k and v: dense [B, S, Hkv, D] / [T, Hkv, D] in the workspace
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t kv_bytes = fwd_ws_kv_bytes(total_tokens, Hkv);
+  const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
+  const uint64_t seq_b = thd ? dimS * tok_b : static_cast<uint64_t>(S) * tok_b;
+  st = make_tmap_4d(&p.tmap_k, ws, kHeadDim, Hkv, dimS, dimB, kHeadDim * 2, tok_b, seq_b, kHeadDim, 1, kFwdTile, 1,
+                    true);
   if (st != GPTOSS_OK) return st;
-  st = make_tmap_4d(&p.tmap_v, v, kHeadDim, Hkv, dimS, dimB, sv.head * 2, sv.tok * 2,
-                         vb_stride == 0 ? 16 : vb_stride, kHeadDim, 1, kFwdTile, 1);
+  st = make_tmap_4d(&p.tmap_v, ws + kv_bytes, kHeadDim, Hkv, dimS, dimB, kHeadDim * 2, tok_b, seq_b, kHeadDim, 1,
+                    kFwdTile, 1, true);
   if (st != GPTOSS_OK) return st;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.sq = sq;
@@ -152,33 +159,35 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   p.n_units = static_cast<int>(n_units);
   p.scale_log2 = softmax_scale * kLog2e;
   p.wait_ns = wait_limit_ns();
+  // positions feed RoPE only: without RoPE the kernels take the identity table
   if (rope != nullptr) yarn_table(*rope, &p.tab);
-  else p.tab.enabled = 0;
-  p.k_in_kernel = rope != nullptr && !k_pre;
-  if (k_pre) {
-    RopeQkParams rp;
-    memset(&rp, 0, sizeof(rp));
-    rp.k = static_cast<const __nv_bfloat16*>(k);
-    rp.k_out = static_cast<__nv_bfloat16*>(workspace);  // fp16 bits (rope_qk_kernel<true>)
-    rp.sk = sk;
-    rp.sko.head = kHeadDim;
-    rp.sko.tok = static_cast<int64_t>(Hkv) * kHeadDim;
-    rp.sko.batch = thd ? 0 : static_cast<int64_t>(S) * Hkv * kHeadDim;
-    rp.tm.positions = positions;
-    rp.tm.cu_seqlens = cu_seqlens;
-    rp.tm.nseq = B;
-    rp.tm.S = thd ? 0 : S;
-    rp.tm.ntok = total_tokens;
-    rp.Hq = 0;
-    rp.Hkv = Hkv;
-    rp.tab = p.tab;
-    rp.cs_out = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + fwd_ws_k_bytes(total_tokens, Hkv));
-    p.cs_tab = rp.cs_out;
-    const int rgrid = (total_tokens + kRopeTokensPerCta - 1) / kRopeTokensPerCta;
-    rope_qk_kernel<true><<<rgrid, kRopeThreads, 0, as_stream(stream)>>>(rp);
-    st = check_launch();
-    if (st != GPTOSS_OK) return st;
-  }
+  else identity_table(&p.tab);
+  p.positions = rope != nullptr ? positions : nullptr;
+  RopeQkParams rp;
+  memset(&rp, 0, sizeof(rp));
+  rp.k = static_cast<const __nv_bfloat16*>(k);
+  rp.k_out = reinterpret_cast<__nv_bfloat16*>(ws);  // fp16 bits (rope_qk_kernel<true>)
+  rp.sk = sk;
+  rp.v = static_cast<const __nv_bfloat16*>(v);
+  rp.v_out = reinterpret_cast<__nv_bfloat16*>(ws + kv_bytes);
+  rp.sv = sv;
+  rp.sko.head = rp.svo.head = kHeadDim;
+  rp.sko.tok = rp.svo.tok = static_cast<int64_t>(Hkv) * kHeadDim;
+  rp.sko.batch = rp.svo.batch = thd ? 0 : static_cast<int64_t>(S) * Hkv * kHeadDim;
+  rp.tm.positions = p.positions;
+  rp.tm.cu_seqlens = cu_seqlens;
+  rp.tm.nseq = B;
+  rp.tm.S = thd ? 0 : S;
+  rp.tm.ntok = total_tokens;
+  rp.Hq = 0;
+  rp.Hkv = Hkv;
+  rp.tab = p.tab;
+  rp.cs_out = reinterpret_cast<float2*>(ws + 2 * kv_bytes);
+  p.cs_tab = rp.cs_out;
+  const int rgrid = (total_tokens + kRopeTokensPerCta - 1) / kRopeTokensPerCta;
+  rope_qk_kernel<true><<<rgrid, kRopeThreads, 0, as_stream(stream)>>>(rp);
+  st = check_launch();
+  if (st != GPTOSS_OK) return st;
   const size_t smem = sizeof(FwdSmem) + 1024;
   if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)

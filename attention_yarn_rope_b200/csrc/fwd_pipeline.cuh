@@ -13,26 +13,19 @@
 
 namespace gptoss {
 
-// =============================== TMA producer ===============================
-__device__ __forceinline__ void fwd_producer_role(const FwdParams& p, FwdSmem& sm) {
-  tma_prefetch_desc(&p.tmap_q);
+// =============================== TMA producers ===============================
+// K / V tiles of every unit, in unit order, into the 4-stage ring.
+__device__ __forceinline__ void fwd_producer_kv_role(const FwdParams& p, FwdSmem& sm) {
   tma_prefetch_desc(&p.tmap_k);
   tma_prefetch_desc(&p.tmap_v);
   const bool thd = p.cu_seqlens != nullptr;
-  uint32_t kv_it = 0, k_issued = 0, v_issued = 0, i = 0, q_issued = 0;
+  uint32_t kv_it = 0, k_issued = 0, v_issued = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
     Unit wu;
     if (!make_unit(p, u, wu)) continue;
     const int tok0 = thd ? wu.seq_start : 0;
     const int bc = thd ? 0 : wu.b;
-    // the unit's two raw Q tiles into the free half of the Q double buffer
-    const int qb = i & 1;
-    if (!mbar_wait(&sm.q_empty[qb], ((i >> 1) & 1) ^ 1, p.wait_ns)) break;
-    mbar_arrive_expect_tx(&sm.q_loaded[qb], 2 * kFwdTileBytes);
-    tma_load_4d(sm.q[qb][0], &p.tmap_q, &sm.q_loaded[qb], 0, wu.h0, tok0 + wu.q0, bc);
-    tma_load_4d(sm.q[qb][1], &p.tmap_q, &sm.q_loaded[qb], 0, wu.h1, tok0 + wu.q0, bc);
-    q_issued = ++i;
     for (int j = 0; j < wu.n_kt; ++j, ++kv_it) {
       const int s = kv_it % kFwdStages;
       const uint32_t ph = ((kv_it / kFwdStages) & 1) ^ 1;
@@ -48,12 +41,35 @@ __device__ __forceinline__ void fwd_producer_role(const FwdParams& p, FwdSmem& s
     }
   }
   // the copies of the last stages must land before the CTA exits
-  for (uint32_t it = q_issued > 2 ? q_issued - 2 : 0; it < q_issued; ++it)
-    mbar_wait(&sm.q_loaded[it & 1], (it >> 1) & 1, p.wait_ns);
   for (uint32_t it = k_issued > kFwdStages ? k_issued - kFwdStages : 0; it < k_issued; ++it)
     mbar_wait(&sm.k_full[it % kFwdStages], (it / kFwdStages) & 1, p.wait_ns);
   for (uint32_t it = v_issued > kFwdStages ? v_issued - kFwdStages : 0; it < v_issued; ++it)
     mbar_wait(&sm.v_full[it % kFwdStages], (it / kFwdStages) & 1, p.wait_ns);
+}
+
+// The two raw Q tiles of every unit into the 3-stage Q ring.  Its own warp,
+// so a Q load never queues behind a K / V stage that is still in use: with
+// two-tile units (128-key window) the Q of a unit must be requested two
+// units ahead to hide the HBM latency.
+__device__ __forceinline__ void fwd_producer_q_role(const FwdParams& p, FwdSmem& sm) {
+  tma_prefetch_desc(&p.tmap_q);
+  const bool thd = p.cu_seqlens != nullptr;
+  uint32_t i = 0;
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    Unit wu;
+    if (!make_unit(p, u, wu)) continue;
+    const int qs = i % kFwdQStages;
+    if (!mbar_wait(&sm.q_empty[qs], ((i / kFwdQStages) & 1) ^ 1, p.wait_ns)) break;
+    mbar_arrive_expect_tx(&sm.q_loaded[qs], 2 * kFwdTileBytes);
+    const int tok = (thd ? wu.seq_start : 0) + wu.q0;
+    const int bc = thd ? 0 : wu.b;
+    tma_load_4d(sm.q[qs][0], &p.tmap_q, &sm.q_loaded[qs], 0, wu.h0, tok, bc);
+    tma_load_4d(sm.q[qs][1], &p.tmap_q, &sm.q_loaded[qs], 0, wu.h1, tok, bc);
+    ++i;
+  }
+  // the copies of the last stages must land before the CTA exits
+  for (uint32_t it = i > kFwdQStages ? i - kFwdQStages : 0; it < i; ++it)
+    mbar_wait(&sm.q_loaded[it % kFwdQStages], (it / kFwdQStages) & 1, p.wait_ns);
 }
 
 // ================================ MMA issuers ================================
@@ -68,19 +84,18 @@ __device__ __forceinline__ void fwd_producer_role(const FwdParams& p, FwdSmem& s
 
 // S_X(t) = Q_X K(t)^T for both head slots, tile by tile.
 __device__ __forceinline__ void fwd_mma_s_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem) {
-  // fused RoPE leaves Q and K in shared memory as fp16; pre-rotated inputs stay bf16
-  const uint32_t idesc_s = p.tab.enabled ? idesc_f16_f32(128, 128) : idesc_bf16_f32(128, 128, false);
+  // Q (rotated or converted by the rope warps) and K (from the workspace) are fp16
+  constexpr uint32_t idesc_s = idesc_f16_f32(128, 128);
   uint32_t t = 0, kv_it = 0, i = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
     Unit wu;
     if (!make_unit(p, u, wu)) continue;
-    const int qb = i & 1;
-    if (!mbar_wait(&sm.q_full[qb], (i >> 1) & 1, p.wait_ns)) break;
+    const int qb = i % kFwdQStages;
+    if (!mbar_wait(&sm.q_full[qb], (i / kFwdQStages) & 1, p.wait_ns)) break;
     for (int j = 0; j < wu.n_kt; ++j, ++t, ++kv_it) {
       const int s = kv_it % kFwdStages;
-      uint64_t* k_in = p.k_in_kernel ? &sm.k_ready[s] : &sm.k_full[s];  // rotated in place, or as copied
-      if (!mbar_wait(k_in, (kv_it / kFwdStages) & 1, p.wait_ns)) { ok = false; break; }
+      if (!mbar_wait(&sm.k_full[s], (kv_it / kFwdStages) & 1, p.wait_ns)) { ok = false; break; }
       const uint64_t kdesc = sw128_desc(smem_u32(sm.k[s]));
 #pragma unroll 1
       for (int X = 0; X < 2; ++X) {
@@ -106,7 +121,7 @@ __device__ __forceinline__ void fwd_mma_s_role(const FwdParams& p, FwdSmem& sm, 
 // O_X += P_X(t) V(t) for both head slots (TS: P from TMEM, V N-major from
 // shared memory); the first tile of a unit starts O from zero.
 __device__ __forceinline__ void fwd_mma_pv_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem) {
-  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 64, true);
+  constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, true);  // fp16 P (TMEM) x fp16 V (workspace)
   uint32_t t = 0, kv_it = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -142,10 +157,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kFwdQStages; ++i) {
       mbar_init(&sm.q_loaded[i], 1);
       mbar_init(&sm.q_full[i], 128);
       mbar_init(&sm.q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.s_free[i], 128);
       mbar_init(&sm.p_full[i], 128);
@@ -153,7 +170,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     }
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.k_ready[s], 128);
       mbar_init(&sm.k_empty[s], 1);
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
@@ -181,9 +197,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     fwd_rope_role(p, sm);
   } else {
     reg_dealloc<kRegsOther>();
-    if (warp == 12 && lane == 0) fwd_producer_role(p, sm);
+    if (warp == 12 && lane == 0) fwd_producer_kv_role(p, sm);
     else if (warp == 13 && lane == 0) fwd_mma_s_role(p, sm, tmem);
     else if (warp == 14 && lane == 0) fwd_mma_pv_role(p, sm, tmem);
+    else if (warp == 15 && lane == 0) fwd_producer_q_role(p, sm);
   }
   tc_fence_before();
   __syncthreads();

@@ -5,29 +5,39 @@
 // QK^T overlaps the exponentials); classify each 32-key chunk for this warp
 // as hidden (skipped: its P is zero), partly visible (masked per element) or
 // fully visible; online softmax in log2 units with a running base m and sum
-// l; P in bf16 into TMEM, one half at a time.
+// l; P in fp16 into TMEM, one half at a time.
+//
+// P is fp16, not bf16: its 11-bit significand keeps the P V product's
+// rounding about eight times smaller, which the output needs -- a bf16
+// output of magnitude 2..4 already spends up to 7.8e-3 of the 1e-2 bar on its
+// own rounding.
 //
 // The base.  A row's first visible tile sets m to its maximum, so that tile's
-// largest P is exactly 1.  Later tiles reuse m as it stands and skip the row
-// maximum: any base gives the same O / l, and bf16 P and fp32 sums keep their
-// relative precision at any scale.  The only risk is range, so the tile's
-// sum is checked afterwards: above 2^64 (or not finite) the warp recomputes
-// tile against its true maximum (the scores are still in registers) and
-// rescales l and O.  In attention the
-// scores after the first tile rarely exceed it by 64 (log2 units), so the
-// redo path is cold; a row whose first tile is fully masked keeps m = -inf
-// and takes the maximum path again on the next one.
+// largest P is exactly 1 (and the row sum stays >= 1 from then on).  Later
+// tiles reuse m as it stands and skip the row maximum: any base gives the
+// same O / l, and fp16 P (down to its subnormals, far below 1 / l) and fp32
+// sums keep their precision at any scale the range allows.  The only risk
+// is range: fp16 ends at 65504, so the tile's sum is checked afterwards --
+// above 2^15 (or not finite) the warp recomputes the tile against its true
+// maximum (the scores are still in registers) and rescales l and O.  In
+// attention the scores after the first tile rarely exceed its maximum by 8
+// (log2 units) over a whole row, so the redo path is cold; a row whose first
+// tile is fully masked keeps m = -inf and takes the maximum path again on
+// the next one.
 //
 // Epilogue: the sink joins the max and the sum once -- M = max(m, sink),
 // l' = l 2^(m-M) + 2^(sink-M) (no term for sink = -inf) -- then
-// O 2^(m-M) / l' in bf16 and LSE = (M + log2 l') ln 2.
+// O 2^(m-M) / l' in bf16 and LSE = (M + log2 l') ln 2.  A unit's epilogue
+// runs inside the next unit's first tile (PendingRow below).
 #pragma once
 
 #include "fwd_common.cuh"
 
 namespace gptoss {
 
-constexpr float kMaxTileSum = 18446744073709551616.0f;  // 2^64
+// P enters P V as fp16 (largest finite value 65504): a tile whose row sum
+// stays at or below 2^15 has every element at or below 2^15.
+constexpr float kMaxTileSum = 32768.0f;  // 2^15
 
 // Row maximum of the raw scores over the chunks this warp can see (masked
 // elements already hold -inf); -inf when none is visible.
@@ -90,10 +100,50 @@ __device__ __forceinline__ void exp_half(const uint32_t (&sr)[4][32], const int 
         }
         rs0 += p0;
         rs1 += p1;
-        pk[cc * 16 + e] = pack_bf16(p0, p1);
+        pk[cc * 16 + e] = pack_f16(p0, p1);
       }
     }
   }
+}
+
+// A finished row awaiting its epilogue: the epilogue of a unit runs during
+// the next unit's first tile, right after that tile's wait for the previous
+// P V product -- which is this unit's last -- so the product's latency hides
+// behind the next unit's S read and first exponentials instead of stalling
+// the warp at the end of every unit.
+struct PendingRow {
+  float m, l, sink;
+  int64_t out_row;  // element offset of the output row (head included); -1: nothing to store
+  int64_t lse_idx;  // -1: no lse
+};
+
+// O / l with the sink folded once (M = max(m, sink), l' = l 2^(m - M) +
+// 2^(sink - M)), in bf16, and LSE = (M + log2 l') ln 2.  O must be complete.
+__device__ __forceinline__ void fwd_epilogue_row(const FwdParams& p, uint32_t o_addr, const PendingRow& pr) {
+  const float M = fmaxf(pr.m, pr.sink);
+  const float a = pr.m == -INFINITY ? 0.f : ex2_approx(pr.m - M);
+  const float l_fin = pr.l * a + (pr.sink == -INFINITY ? 0.f : ex2_approx(pr.sink - M));
+  const float inv = a / l_fin;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t ov[32];
+    tmem_ld32(o_addr + c * 32, ov);
+    tmem_wait_ld();
+    if (pr.out_row >= 0) {
+      __nv_bfloat16* dst = p.out + pr.out_row + c * 32;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        uint4 v;
+        const int e = c8 * 8;
+        v.x = pack_bf16(__uint_as_float(ov[e + 0]) * inv, __uint_as_float(ov[e + 1]) * inv);
+        v.y = pack_bf16(__uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+        v.z = pack_bf16(__uint_as_float(ov[e + 4]) * inv, __uint_as_float(ov[e + 5]) * inv);
+        v.w = pack_bf16(__uint_as_float(ov[e + 6]) * inv, __uint_as_float(ov[e + 7]) * inv);
+        *reinterpret_cast<uint4*>(dst + c8 * 8) = v;
+      }
+    }
+  }
+  if (pr.out_row >= 0 && pr.lse_idx >= 0) p.lse[pr.lse_idx] = (M + log2f(l_fin)) * kLn2;
 }
 
 __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem, int X) {
@@ -104,6 +154,8 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
   const bool thd = p.cu_seqlens != nullptr;
   const float sl = p.scale_log2;
   uint32_t t = 0;  // running tile count of this CTA
+  bool pending = false;
+  PendingRow pr;
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     Unit w;
     if (!make_unit(p, u, w)) continue;
@@ -154,6 +206,12 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
         }
         tmem_st32(lane_base + colP, pk);
       }
+      // the previous unit's rows: its last P V has completed (waited above),
+      // and this unit's first P V, which restarts O, waits for p_full below
+      if (j == 0 && pending) {
+        fwd_epilogue_row(p, lane_base + colO, pr);
+        pending = false;
+      }
       {
         uint32_t pk[32];
         exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
@@ -196,42 +254,28 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
       tc_fence_before();
       mbar_arrive(&sm.p_full[X]);
     }
-    // ---- epilogue: O / l, LSE ----
+    // this unit's epilogue waits for the next unit's first tile (or the end)
+    pr.m = m_run;
+    pr.l = l_run;
+    pr.sink = sink;
+    pr.out_row = -1;
+    pr.lse_idx = -1;
+    if (qi < w.L && !(X == 1 && w.dup)) {
+      pr.out_row = (thd ? static_cast<int64_t>(w.seq_start + qi) * p.so.tok
+                        : static_cast<int64_t>(w.b) * p.so.batch + static_cast<int64_t>(qi) * p.so.tok) +
+                   static_cast<int64_t>(h) * p.so.head;
+      if (p.lse != nullptr)
+        pr.lse_idx = thd ? static_cast<int64_t>(h) * p.T + w.seq_start + qi
+                         : (static_cast<int64_t>(w.b) * p.Hq + h) * p.S + qi;
+    }
+    pending = true;
+  }
+  if (pending) {  // the last unit: wait for its last P V product
     if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
     tc_fence_after();
-    uint32_t ov[2][32];
-    tmem_ld32(lane_base + colO, ov[0]);
-    tmem_ld32(lane_base + colO + 32, ov[1]);
-    tmem_wait_ld();
-    tc_fence_before();
-    if (qi < w.L && !(X == 1 && w.dup)) {
-      // fold the sink: M = max(m, sink), l = l 2^(m - M) + 2^(sink - M)
-      const float M = fmaxf(m_run, sink);
-      const float a = m_run == -INFINITY ? 0.f : ex2_approx(m_run - M);
-      const float l_fin = l_run * a + (sink == -INFINITY ? 0.f : ex2_approx(sink - M));
-      const float inv = a / l_fin;
-      const int64_t row = thd ? static_cast<int64_t>(w.seq_start + qi) * p.so.tok
-                              : static_cast<int64_t>(w.b) * p.so.batch + static_cast<int64_t>(qi) * p.so.tok;
-      __nv_bfloat16* dst = p.out + row + static_cast<int64_t>(h) * p.so.head;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint4 v;
-        const int c = c8 >> 2, e = (c8 & 3) * 8;
-        v.x = pack_bf16(__uint_as_float(ov[c][e + 0]) * inv, __uint_as_float(ov[c][e + 1]) * inv);
-        v.y = pack_bf16(__uint_as_float(ov[c][e + 2]) * inv, __uint_as_float(ov[c][e + 3]) * inv);
-        v.z = pack_bf16(__uint_as_float(ov[c][e + 4]) * inv, __uint_as_float(ov[c][e + 5]) * inv);
-        v.w = pack_bf16(__uint_as_float(ov[c][e + 6]) * inv, __uint_as_float(ov[c][e + 7]) * inv);
-        *reinterpret_cast<uint4*>(dst + c8 * 8) = v;
-      }
-      if (p.lse != nullptr) {
-        const float lse = (M + log2f(l_fin)) * kLn2;
-        if (thd)
-          p.lse[static_cast<int64_t>(h) * p.T + w.seq_start + qi] = lse;
-        else
-          p.lse[(static_cast<int64_t>(w.b) * p.Hq + h) * p.S + qi] = lse;
-      }
-    }
+    fwd_epilogue_row(p, lane_base + colO, pr);
   }
+  tc_fence_before();
 }
 
 }  // namespace gptoss

@@ -24,6 +24,7 @@ struct RopeTable {
   double inv_freq[kPairs];
   float conc;
   int enabled;  // 0: inputs already rotated, nothing to do
+  int R;        // rotary pairs, rotary_dim / 2: features [0, 2R) rotate in pairs (j, j + R), the rest pass through
 };
 
 // YaRN inverse frequencies and concentration (RotaryEmbedding on the NeMo
@@ -38,6 +39,7 @@ inline void yarn_table(const gptoss_rope_params& rp, RopeTable* t) {
   const int half = rdim / 2;
   const double two_pi = 6.283185307179586476925286766559;
   for (int j = 0; j < kPairs; ++j) t->inv_freq[j] = 0.0;
+  t->R = half;
   const double lnb = log(rp.base);
   if (rp.factor <= 1.0) {
     for (int j = 0; j < half; ++j) t->inv_freq[j] = exp(-2.0 * j / rdim * lnb);
@@ -64,13 +66,15 @@ inline gptoss_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? GPTOSS_OK : GPTOSS_ERR_CUDA;
 }
 
-// Validates rope params for this build (rotary_dim must equal head_dim 64).
-inline gptoss_status check_rope(const gptoss_rope_params* rp, int D) {
+// Validates rope params.  rotary_dim must be even and at most head_dim;
+// kernels that take partial rotary (allow_partial) need it a multiple of 16
+// (whole 16-byte chunks of pairs), the others need rotary_dim == head_dim.
+inline gptoss_status check_rope(const gptoss_rope_params* rp, int D, bool allow_partial = false) {
   if (rp == nullptr) return GPTOSS_OK;
   if (!(rp->base > 1.0) || !(rp->factor > 0.0) || rp->initial_context <= 0) return GPTOSS_ERR_INVALID_ARG;
   if (rp->factor > 1.0 && !(rp->ntk_alpha > 0.0 && rp->ntk_beta > rp->ntk_alpha)) return GPTOSS_ERR_INVALID_ARG;
-  if (rp->rotary_dim <= 0 || (rp->rotary_dim & 1)) return GPTOSS_ERR_INVALID_ARG;
-  if (rp->rotary_dim != D) return GPTOSS_ERR_UNSUPPORTED;
+  if (rp->rotary_dim <= 0 || (rp->rotary_dim & 1) || rp->rotary_dim > D) return GPTOSS_ERR_INVALID_ARG;
+  if (rp->rotary_dim != D && (!allow_partial || (rp->rotary_dim % 16) != 0)) return GPTOSS_ERR_UNSUPPORTED;
   return GPTOSS_OK;
 }
 

@@ -2,16 +2,20 @@
 //
 // Rule: NeMo AutoModel gpt_oss.rope_utils page, apply_rotary_emb_qk /
 // _apply_rotary_emb_qk: q and k rotated with the same tables, half-split
-// pairs (j, j+32), concentration applied, BSHD or packed THD with cu_seqlens.
+// pairs (j, j + R) with R = rotary_dim / 2, concentration applied, features
+// from rotary_dim on passed through unchanged (apply_rotary_emb, partial
+// rotary), BSHD or packed THD with cu_seqlens.
 //
 // Design (HBM-bound elementwise op): a CTA owns TB consecutive tokens.  Its
-// threads first build the (c cos, c sin) table of those tokens' 32 angles in
+// threads first build the (c cos, c sin) table of those tokens' R angles in
 // shared memory -- the angle p * inv_freq is formed and reduced modulo 2 pi
 // in double precision, then sincosf runs on the reduced angle -- and then
 // sweep every (token, head, 16-byte chunk) of q and k with 128-bit loads and
-// stores: chunk c of a head holds features [8c, 8c+8) and [32+8c, 40+8c),
-// i.e. 8 complete rotation pairs.  A warp covers 8 heads x 4 chunks of one
-// token, so its two loads fill whole 128-byte lines.
+// stores.  A rotation item takes chunk c (features [8c, 8c+8)) and its
+// partner chunk c + R/8 (features [R+8c, R+8c+8)): 8 complete pairs; a
+// pass-through item copies one chunk past 2R.  R = 32 (GPT-OSS) gives 4
+// rotation items per head: a warp covers 8 heads x 4 items of one token, so
+// its two loads fill whole 128-byte lines.
 #pragma once
 
 #include "host_util.cuh"
@@ -43,6 +47,12 @@ __device__ __forceinline__ void token_coords(const TokenMap& m, int t, int& seq,
   }
 }
 
+// The two features of rotation slot j (0 <= j < 32) with R rotary pairs:
+// slot j < R is the pair (j, j + R); slots j >= R cover the features past
+// the rotary ones, two each (2j, 2j + 1), which pass through unrotated.
+__host__ __device__ __forceinline__ int rope_feature_a(int j, int R) { return j < R ? j : 2 * j; }
+__host__ __device__ __forceinline__ int rope_feature_b(int j, int R) { return j < R ? j + R : 2 * j + 1; }
+
 // (c cos theta, c sin theta), theta = pos * f, reduced modulo 2 pi in double
 // (Cody-Waite with 2 pi split in two doubles), then sincosf on |r| <= pi.
 __device__ __forceinline__ float2 rope_cs(int pos, double f, float conc) {
@@ -59,7 +69,7 @@ __device__ __forceinline__ float2 rope_cs(int pos, double f, float conc) {
 }
 
 // Rotates the 8 pairs held by (lo, hi): lo = features [8c, 8c+8), hi = the
-// partners [32+8c, 40+8c); cs[e] = (c cos, c sin) of pair 8c+e.  The result
+// partners [R+8c, R+8c+8); cs[e] = (c cos, c sin) of pair 8c+e.  The result
 // is rounded to bf16, or to fp16 when kF16Out (the QK^T operand format of the
 // prefill kernel under fused RoPE).
 template <bool kF16Out>
@@ -84,22 +94,34 @@ struct RopeQkParams {
   __nv_bfloat16* q_out;
   __nv_bfloat16* k_out;
   gptoss_strides sq, sk, sqo, sko;
+  const __nv_bfloat16* v;  // nullable: v copied unrotated to v_out (in the output format)
+  __nv_bfloat16* v_out;
+  gptoss_strides sv, svo;
   TokenMap tm;
   int Hq, Hkv;
   RopeTable tab;
   float2* cs_out;  // nullable: each token's 32 (c cos, c sin) pairs, [token][32]
 };
 
+// Converts 8 bf16 values to fp16 (round to nearest even; exact for the
+// values fp16 represents).
+__device__ __forceinline__ void bf16x8_to_f16(uint4& x) {
+  uint32_t* w = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = pack_f16(bf16lo(w[i]), bf16hi(w[i]));
+}
+
 constexpr int kRopeTokensPerCta = 8;
 constexpr int kRopeThreads = 256;
 
-// q (Hq heads, may be 0) and k (Hkv heads) of TB tokens per CTA.  kF16Out:
-// fp16 results (k rotated once for the prefill kernel); otherwise bf16.
+// q (Hq heads, may be 0) and k (Hkv heads) of TB tokens per CTA, and v
+// (Hkv heads, unrotated) when p.v is set.  kF16Out: fp16 results (k rotated
+// and v converted once for the prefill kernel); otherwise bf16.
 template <bool kF16Out>
 __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_constant__ RopeQkParams p) {
   constexpr int TB = kRopeTokensPerCta;
   __shared__ float2 tab[TB][kPairs];
-  __shared__ int64_t tok_off[TB][4];  // element offsets of token rows: q, k, q_out, k_out
+  __shared__ int64_t tok_off[TB][6];  // element offsets of token rows: q, k, q_out, k_out, v, v_out
   const int t0 = blockIdx.x * TB;
   const int tid = threadIdx.x;
   if (tid < TB * kPairs) {
@@ -119,20 +141,41 @@ __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_cons
         tok_off[tt][1] = b * p.sk.batch + s * p.sk.tok;
         tok_off[tt][2] = b * p.sqo.batch + s * p.sqo.tok;
         tok_off[tt][3] = b * p.sko.batch + s * p.sko.tok;
+        tok_off[tt][4] = b * p.sv.batch + s * p.sv.tok;
+        tok_off[tt][5] = b * p.svo.batch + s * p.svo.tok;
       }
     }
   }
   __syncthreads();
-  const int H = p.Hq + p.Hkv;
-  const int items = TB * H * 4;
+  const int H = p.Hq + p.Hkv + (p.v != nullptr ? p.Hkv : 0);
+  const int n_rot = p.tab.R / 8;     // rotation items per head (chunk + partner)
+  const int per_head = 8 - n_rot;    // plus one pass-through item per chunk past 2R
+  const int items = TB * H * per_head;
   for (int it = tid; it < items; it += kRopeThreads) {
-    const int chunk = it & 3;
-    const int rest = it >> 2;
+    const int ci = it % per_head;
+    const int rest = it / per_head;
     const int hh = rest % H;
     const int tt = rest / H;
     if (t0 + tt >= p.tm.ntok) continue;
     const __nv_bfloat16* src;
     __nv_bfloat16* dst;
+    if (hh >= p.Hq + p.Hkv) {  // v: copied in the output format, not rotated
+      const int g = hh - p.Hq - p.Hkv;
+      src = p.v + tok_off[tt][4] + static_cast<int64_t>(g) * p.sv.head;
+      dst = p.v_out + tok_off[tt][5] + static_cast<int64_t>(g) * p.svo.head;
+      // the chunks this item would rotate or copy, copied (v is not rotated)
+      const int c0 = ci < n_rot ? ci : n_rot + ci;
+      const int c1 = ci < n_rot ? ci + n_rot : -1;
+      uint4 lo = *reinterpret_cast<const uint4*>(src + 8 * c0);
+      if (kF16Out) bf16x8_to_f16(lo);
+      *reinterpret_cast<uint4*>(dst + 8 * c0) = lo;
+      if (c1 >= 0) {
+        uint4 hi = *reinterpret_cast<const uint4*>(src + 8 * c1);
+        if (kF16Out) bf16x8_to_f16(hi);
+        *reinterpret_cast<uint4*>(dst + 8 * c1) = hi;
+      }
+      continue;
+    }
     if (hh < p.Hq) {
       src = p.q + tok_off[tt][0] + static_cast<int64_t>(hh) * p.sq.head;
       dst = p.q_out + tok_off[tt][2] + static_cast<int64_t>(hh) * p.sqo.head;
@@ -141,11 +184,18 @@ __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_cons
       src = p.k + tok_off[tt][1] + static_cast<int64_t>(g) * p.sk.head;
       dst = p.k_out + tok_off[tt][3] + static_cast<int64_t>(g) * p.sko.head;
     }
-    uint4 lo = *reinterpret_cast<const uint4*>(src + 8 * chunk);
-    uint4 hi = *reinterpret_cast<const uint4*>(src + 32 + 8 * chunk);
-    rotate8<kF16Out>(lo, hi, &tab[tt][8 * chunk]);
-    *reinterpret_cast<uint4*>(dst + 8 * chunk) = lo;
-    *reinterpret_cast<uint4*>(dst + 32 + 8 * chunk) = hi;
+    if (ci < n_rot) {
+      uint4 lo = *reinterpret_cast<const uint4*>(src + 8 * ci);
+      uint4 hi = *reinterpret_cast<const uint4*>(src + p.tab.R + 8 * ci);
+      rotate8<kF16Out>(lo, hi, &tab[tt][8 * ci]);
+      *reinterpret_cast<uint4*>(dst + 8 * ci) = lo;
+      *reinterpret_cast<uint4*>(dst + p.tab.R + 8 * ci) = hi;
+    } else {  // past the rotary features: passed through unchanged
+      const int c = n_rot + ci;
+      uint4 x = *reinterpret_cast<const uint4*>(src + 8 * c);
+      if (kF16Out) bf16x8_to_f16(x);
+      *reinterpret_cast<uint4*>(dst + 8 * c) = x;
+    }
   }
 }
 

@@ -91,14 +91,12 @@ def gptoss_attn_fwd_workspace_size(total_tokens: int, Hkv: int, D: int = 64) -> 
 
 def gptoss_attn_fwd(q, k, v, sinks, window: int = 0, softmax_scale: float | None = None,
                     rope: RopeConfig | None = None, positions=None, cu_seqlens=None, max_seqlen: int | None = None,
-                    out=None, return_lse: bool = False, lse=None, workspace=None, rotate_k_once: bool = True,
-                    stream=None):
+                    out=None, return_lse: bool = False, lse=None, workspace=None, stream=None):
     """Prefill sink attention.  BSHD when q is 4-D, packed THD when q is 3-D
     with ``cu_seqlens`` (then ``max_seqlen`` bounds the longest sequence).
-    With ``rope`` and ``rotate_k_once`` (default), k is rotated once into a
-    workspace (``workspace``, or a new device buffer of
-    ``gptoss_attn_fwd_workspace_size`` bytes); ``rotate_k_once=False`` rotates
-    k tiles inside the attention kernel instead.  Returns ``out`` or
+    k (rotated when ``rope`` is given) and v are written once into a
+    workspace as fp16 (``workspace``, or a new device buffer of
+    ``gptoss_attn_fwd_workspace_size`` bytes).  Returns ``out`` or
     ``(out, lse)``."""
     lib = _abi.load()
     thd = cu_seqlens is not None
@@ -123,15 +121,11 @@ def gptoss_attn_fwd(q, k, v, sinks, window: int = 0, softmax_scale: float | None
     _check_dev(q, k, v, sinks, out, lse, positions, cu_seqlens)
     scale = float(D) ** -0.5 if softmax_scale is None else float(softmax_scale)
     r = rope.to_c() if rope is not None else None
-    ws_bytes = 0
-    if rope is not None and rotate_k_once:
-        ws_bytes = int(lib.gptoss_attn_fwd_workspace_size(total, Hkv, D))
-        if workspace is None:
-            workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
-        _check_dev(workspace)
-        ws_bytes = workspace.numel() * workspace.element_size()
-    else:
-        workspace = None
+    if workspace is None:
+        need = int(lib.gptoss_attn_fwd_workspace_size(total, Hkv, D))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check_dev(workspace)
+    ws_bytes = workspace.numel() * workspace.element_size()
     st = lib.gptoss_attn_fwd(_ptr(q), _strides(q, thd), _ptr(k), _strides(k, thd), _ptr(v), _strides(v, thd),
                              _ptr(sinks), _ptr(positions), _ptr(cu_seqlens), B, S, total, Hq, Hkv, D, int(window),
                              scale, ctypes.byref(r) if r is not None else None, _ptr(out), _strides(out, thd),

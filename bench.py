@@ -614,29 +614,132 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg, budget_s=15.0):
-    """Times the oracle as it stands on (batch row, kv group) units of the
-    workload until about `budget_s` seconds of CPU work; TFLOP/s of the sample."""
-    from attention_yarn_rope_b200.workloads import make_prefill
+def _host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _tables_of(cfg):
     from oracle.yarn import yarn_inv_freq_and_concentration
 
-    x = make_prefill(cfg)
     r = cfg.rope
-    tables = yarn_inv_freq_and_concentration(cfg.D, r["base"], r["factor"], r["initial_context"], r["ntk_alpha"],
-                                             r["ntk_beta"])
-    units = [(b, g) for b in range(cfg.B) for g in range(cfg.Hkv)]
-    done_pairs, n = 0, 0
+    return yarn_inv_freq_and_concentration(cfg.D, r["base"], r["factor"], r["initial_context"], r["ntk_alpha"],
+                                           r["ntk_beta"])
+
+
+def _oracle_prefill_whole(cfg):
+    """The oracle's whole output for a prefill workload: seconds, visible pairs."""
+    import numpy as np
+
+    from attention_yarn_rope_b200.workloads import make_prefill
+    from oracle.attention import attn_fwd_bshd, attn_fwd_thd
+
+    x = make_prefill(cfg)
+    tables = _tables_of(cfg)
     t0 = time.perf_counter()
-    for b, g in units:
-        done_pairs += _oracle_unit(x, cfg, b, g, tables)
-        n += 1
+    if x.cu_seqlens is not None:
+        attn_fwd_thd(x.q, x.k, x.v, x.sinks, x.cu_seqlens, cfg.softmax_scale, cfg.window, rope_tables=tables)
+        pairs = visible_pairs(np.diff(x.cu_seqlens), cfg.window) * cfg.Hq
+    else:
+        attn_fwd_bshd(x.q, x.k, x.v, x.sinks, cfg.softmax_scale, cfg.window, rope_tables=tables)
+        pairs = visible_pairs([cfg.S] * cfg.B, cfg.window) * cfg.Hq
+    return time.perf_counter() - t0, pairs
+
+
+def _oracle_prefill_sample(cfg, budget_s):
+    """The oracle on (sequence, kv group) units of a prefill workload until
+    about ``budget_s`` seconds; returns seconds, pairs covered, pairs of the
+    whole workload and a description of the sample."""
+    import numpy as np
+
+    from attention_yarn_rope_b200.workloads import make_prefill
+    from oracle.attention import sink_attention_sequence
+    from oracle.rope import rope
+
+    x = make_prefill(cfg)
+    tables = _tables_of(cfg)
+    G = cfg.Hq // cfg.Hkv
+    if x.cu_seqlens is not None:
+        cu = x.cu_seqlens
+        seqs = [(int(cu[i]), int(cu[i + 1])) for i in range(len(cu) - 1)]
+        total = visible_pairs(np.diff(cu), cfg.window) * cfg.Hq
+        get = lambda s: (x.q[seqs[s][0]:seqs[s][1]], x.k[seqs[s][0]:seqs[s][1]], x.v[seqs[s][0]:seqs[s][1]])
+    else:
+        seqs = [(0, cfg.S)] * cfg.B
+        total = visible_pairs([cfg.S] * cfg.B, cfg.window) * cfg.Hq
+        get = lambda s: (x.q[s], x.k[s], x.v[s])
+    # shortest sequences first for a packed stream, so the sample spans several
+    order = sorted(range(len(seqs)), key=lambda s: seqs[s][1] - seqs[s][0])
+    pairs, n = 0, 0
+    t0 = time.perf_counter()
+    for s in order:
+        q, k, v = get(s)
+        L = q.shape[0]
+        pos = np.arange(L)
+        for g in range(cfg.Hkv):
+            qr = rope(q[:, g * G:(g + 1) * G], pos, *tables)
+            kr = rope(k[:, g:g + 1], pos, *tables)
+            sink_attention_sequence(qr, kr, v[:, g:g + 1], x.sinks[g * G:(g + 1) * G], cfg.softmax_scale,
+                                    cfg.window)
+            pairs += visible_pairs([L], cfg.window) * G
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    tf = 4 * cfg.D * done_pairs / dt / 1e12
-    return {"value": round(tf, 6), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{n} of {len(units)} (batch row, kv-group) units of {cfg.name} "
-                      f"({n * cfg.Hq // cfg.Hkv} query heads x {cfg.S} rows), float64 NumPy, {dt:.1f} s"}
+    return dt, pairs, total, f"{n} (sequence, kv-group) units"
+
+
+def _oracle_decode_sample(cfg, n_seq):
+    """The decode oracle on ``n_seq`` host-drawn sequences of the workload's
+    cache length; returns seconds and the visible K + V bytes they read."""
+    from attention_yarn_rope_b200.workloads import make_decode_host
+    from oracle.attention import attn_decode
+
+    x = make_decode_host(cfg, B=n_seq)
+    tables = _tables_of(cfg)
+    t0 = time.perf_counter()
+    attn_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.sinks, cfg.D ** -0.5, cfg.window, rope_tables=tables)
+    dt = time.perf_counter() - t0
+    vis = min(cfg.L, cfg.window) if cfg.window > 0 else cfg.L
+    return dt, n_seq * vis * cfg.Hkv * cfg.D * 2 * 2
+
+
+def cpu_baseline(cfg, budget_s=15.0, per_config=True):
+    """Times the oracle as it stands on the host cores: the whole output of
+    the sliding-window workload (the headline figure), and for every other
+    workload its whole output (windowed THD stream) or a bounded sample with
+    the whole-workload time extrapolated from it."""
+    from attention_yarn_rope_b200.workloads import (
+        DECODE_B8, DECODE_B8_W, DECODE_B64, DECODE_B64_W, FULL, THD_FULL, THD_WINDOW)
+
+    cores = _host_cores()
+    dt, pairs = _oracle_prefill_whole(cfg)
+    tf = 4 * cfg.D * pairs / dt / 1e12
+    res = {"value": round(tf, 6), "unit": UNIT, "cores": cores, "blas_threads": _blas_threads(), "kind": "oracle",
+           "sample": f"the whole output of {cfg.name} ({cfg.B} x {cfg.S} rows x {cfg.Hq} heads), float64 NumPy, "
+                     f"{dt:.1f} s on {cores} host cores"}
+    if not per_config:
+        return res
+    pc = {cfg.name: {"seconds": round(dt, 2), "tflops": round(tf, 6), "work": "whole output"}}
+    dt, pairs = _oracle_prefill_whole(THD_WINDOW)
+    pc[THD_WINDOW.name] = {"seconds": round(dt, 2), "tflops": round(4 * THD_WINDOW.D * pairs / dt / 1e12, 6),
+                           "work": "whole output"}
+    for c in (FULL, THD_FULL):
+        dt, pairs, total, what = _oracle_prefill_sample(c, budget_s / 2)
+        tf = 4 * c.D * pairs / dt / 1e12
+        pc[c.name] = {"seconds": round(dt, 2), "tflops": round(tf, 6), "work": f"sample: {what}",
+                      "est_whole_output_seconds": round(dt * total / pairs, 1)}
+    for c, n in ((DECODE_B64, 2), (DECODE_B64_W, 64), (DECODE_B8, 1), (DECODE_B8_W, 8)):
+        dt, nbytes = _oracle_decode_sample(c, n)
+        pc[c.name] = {"seconds": round(dt, 3), "gbs": round(nbytes / dt / 1e9, 4),
+                      "work": f"{n} of {c.B} sequences" + ("" if n == c.B else " (host-drawn, same shape)"),
+                      "est_whole_output_seconds": round(dt * c.B / n, 2)}
+    res["per_config"] = pc
+    return res
 
 
 def run_reference(args):

@@ -52,7 +52,7 @@ FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every case fails validati
 def _fwd(lib, **kw):
     a = dict(q=FAKE, sq=S_BSHD_Q, k=FAKE, sk=S_BSHD_K, v=FAKE, sv=S_BSHD_K, sinks=FAKE, pos=None, cu=None, B=1,
              S=4096, T=4096, Hq=64, Hkv=8, D=64, window=0, scale=0.125, rope=ctypes.byref(ROPE), out=FAKE,
-             so=S_BSHD_Q, lse=None, ws=None, ws_bytes=0)
+             so=S_BSHD_Q, lse=None, ws=FAKE, ws_bytes=1 << 40)
     a.update(kw)
     return lib.gptoss_attn_fwd(a["q"], a["sq"], a["k"], a["sk"], a["v"], a["sv"], a["sinks"], a["pos"], a["cu"],
                                a["B"], a["S"], a["T"], a["Hq"], a["Hkv"], a["D"], a["window"], a["scale"],
@@ -70,13 +70,18 @@ def test_attn_fwd_validation(lib):
     assert _fwd(lib, sinks=None) == _abi.GPTOSS_ERR_INVALID_ARG
     assert _fwd(lib, q=ctypes.c_void_p(0x10008)) == _abi.GPTOSS_ERR_INVALID_ARG  # not 16-byte aligned
     assert _fwd(lib, sq=_abi.Strides(0, 4097, 64)) == _abi.GPTOSS_ERR_INVALID_ARG  # stride not 16 B multiple
-    bad_rope = _abi.RopeParams(150000.0, 32.0, 4096, 32, 1.0, 32.0)
-    assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_UNSUPPORTED  # partial rotary
+    # partial rotary: any multiple of 16 up to head_dim; others are unsupported
+    bad_rope = _abi.RopeParams(150000.0, 32.0, 4096, 24, 1.0, 32.0)
+    assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_UNSUPPORTED
+    bad_rope = _abi.RopeParams(150000.0, 32.0, 4096, 80, 1.0, 32.0)
+    assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_INVALID_ARG  # beyond head_dim
     bad_rope = _abi.RopeParams(150000.0, 32.0, 4096, 64, 32.0, 1.0)
     assert _fwd(lib, rope=ctypes.byref(bad_rope)) == _abi.GPTOSS_ERR_INVALID_ARG  # alpha >= beta
-    # the rotated-k workspace: too small or misaligned
+    # the workspace (fp16 rotated k and v, per-token angle table): required,
+    # too small or misaligned is rejected
     need = lib.gptoss_attn_fwd_workspace_size(4096, 8, 64)
-    assert need == 4096 * 8 * 64 * 2 + 4096 * 32 * 8  # rotated k + per-token angle table
+    assert need == 2 * 4096 * 8 * 64 * 2 + 4096 * 32 * 8
+    assert _fwd(lib, ws=None, ws_bytes=0) == _abi.GPTOSS_ERR_INVALID_ARG
     assert _fwd(lib, ws=FAKE, ws_bytes=need - 16) == _abi.GPTOSS_ERR_INVALID_ARG
     assert _fwd(lib, ws=ctypes.c_void_p(0x10008), ws_bytes=need) == _abi.GPTOSS_ERR_INVALID_ARG
     # empty inputs are a successful no-op (nothing launched)

@@ -41,9 +41,9 @@ def test_tiny_workload(cuda_device):
     assert_lse_parity(host(lse), ref_lse, "tiny lse")
 
 
-# rope modes: k rotated once into the workspace, k tiles rotated inside the
-# kernel, or q and k rotated beforehand (no RoPE in the call)
-ROPE_MODES = ["k_once", "k_in_kernel", "prerotated"]
+# rope modes: RoPE fused into the call, or q and k rotated beforehand (no
+# RoPE in the call)
+ROPE_MODES = ["fused", "prerotated"]
 
 
 @pytest.mark.parametrize("window", [0, 1, 128, 200, 1000])
@@ -55,8 +55,7 @@ def test_bshd_multi_tile_ragged(cuda_device, window, mode):
     tabs = _tables(GPTOSS_ROPE)
     if mode != "prerotated":
         out, lse = ops.gptoss_attn_fwd(dev(q), dev(k), dev(v), f32(sinks), window=window,
-                                       rope=ops.RopeConfig.from_dict(GPTOSS_ROPE), return_lse=True,
-                                       rotate_k_once=mode == "k_once")
+                                       rope=ops.RopeConfig.from_dict(GPTOSS_ROPE), return_lse=True)
         torch.cuda.synchronize()
         ref, ref_lse = attn_fwd_bshd(q, k, v, sinks, 0.125, window, rope_tables=tabs)
     else:
@@ -84,8 +83,7 @@ def test_extreme_sinks(cuda_device, sink):
 
 
 @pytest.mark.parametrize("window", [0, 128])
-@pytest.mark.parametrize("k_once", [True, False])
-def test_thd_ragged_sequences(cuda_device, window, k_once):
+def test_thd_ragged_sequences(cuda_device, window):
     lens = [1, 129, 300, 77, 128, 256]
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     T, Hq, Hkv = int(cu[-1]), 16, 2
@@ -93,15 +91,14 @@ def test_thd_ragged_sequences(cuda_device, window, k_once):
     sinks = np.random.default_rng(24).standard_normal(Hq).astype(np.float32)
     out, lse = ops.gptoss_attn_fwd(dev(q), dev(k), dev(v), f32(sinks), window=window, cu_seqlens=i32(cu),
                                    max_seqlen=max(lens), rope=ops.RopeConfig.from_dict(GPTOSS_ROPE),
-                                   return_lse=True, rotate_k_once=k_once)
+                                   return_lse=True)
     torch.cuda.synchronize()
     ref, ref_lse = attn_fwd_thd(q, k, v, sinks, cu, 0.125, window, rope_tables=_tables(GPTOSS_ROPE))
     assert_parity(host(out), ref, "thd out")
     assert_lse_parity(host(lse), ref_lse, "thd lse")
 
 
-@pytest.mark.parametrize("k_once", [True, False])
-def test_explicit_positions_and_strided_io(cuda_device, k_once):
+def test_explicit_positions_and_strided_io(cuda_device):
     # q/k/v as views of one fused buffer; output into a strided view; positions offset by a prefix
     B, S, Hq, Hkv = 2, 200, 8, 2
     qkv = _rand((B, S, Hq + 2 * Hkv, 64), 31)
@@ -112,7 +109,7 @@ def test_explicit_positions_and_strided_io(cuda_device, k_once):
     big = torch.zeros((B, S, Hq + 8, 64), dtype=torch.bfloat16, device=cuda_device)
     out = big[:, :, 4:4 + Hq]
     ops.gptoss_attn_fwd(q, k, v, f32(sinks), window=128, rope=ops.RopeConfig.from_dict(GPTOSS_ROPE),
-                        positions=i32(pos), out=out, rotate_k_once=k_once)
+                        positions=i32(pos), out=out)
     torch.cuda.synchronize()
     ref, _ = attn_fwd_bshd(qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:], sinks, 0.125, 128,
                            rope_tables=_tables(GPTOSS_ROPE), positions=pos)
@@ -129,3 +126,37 @@ def test_gpt_oss_head_layout_two_tiles(cuda_device):
     torch.cuda.synchronize()
     ref, _ = attn_fwd_bshd(q, k, v, sinks, 0.125, 0, rope_tables=_tables(GPTOSS_ROPE))
     assert_parity(host(out), ref, "gpt-oss heads")
+
+
+@pytest.mark.parametrize("rotary_dim", [16, 32, 48])
+@pytest.mark.parametrize("window", [0, 128])
+def test_partial_rotary(cuda_device, rotary_dim, window):
+    # partial_rotary_factor = rotary_dim / 64: q and k rotate their first
+    # rotary_dim features in pairs (j, j + rotary_dim / 2); the rest pass through
+    B, S, Hq, Hkv = 2, 300, 16, 2
+    q, k, v = _rand((B, S, Hq, 64), 51), _rand((B, S, Hkv, 64), 52), _rand((B, S, Hkv, 64), 53)
+    sinks = np.random.default_rng(54).standard_normal(Hq).astype(np.float32)
+    cfg = ops.RopeConfig.from_dict(GPTOSS_ROPE, rotary_dim=rotary_dim)
+    out, lse = ops.gptoss_attn_fwd(dev(q), dev(k), dev(v), f32(sinks), window=window, rope=cfg, return_lse=True)
+    torch.cuda.synchronize()
+    tabs = yarn_inv_freq_and_concentration(64, 150000.0, 32.0, 4096, 1.0, 32.0,
+                                           partial_rotary_factor=rotary_dim / 64)
+    ref, ref_lse = attn_fwd_bshd(q, k, v, sinks, 0.125, window, rope_tables=tabs)
+    assert_parity(host(out), ref, f"partial rotary {rotary_dim} out w={window}")
+    assert_lse_parity(host(lse), ref_lse, f"partial rotary {rotary_dim} lse w={window}")
+
+
+def test_partial_rotary_thd_explicit_positions(cuda_device):
+    lens = [1, 200, 77]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T, Hq, Hkv = int(cu[-1]), 8, 2
+    q, k, v = _rand((T, Hq, 64), 55), _rand((T, Hkv, 64), 56), _rand((T, Hkv, 64), 57)
+    sinks = np.random.default_rng(58).standard_normal(Hq).astype(np.float32)
+    pos = np.random.default_rng(59).integers(0, 131072, T).astype(np.int32)
+    cfg = ops.RopeConfig.from_dict(GPTOSS_ROPE, rotary_dim=32)
+    out = ops.gptoss_attn_fwd(dev(q), dev(k), dev(v), f32(sinks), window=128, cu_seqlens=i32(cu),
+                              max_seqlen=max(lens), rope=cfg, positions=i32(pos))
+    torch.cuda.synchronize()
+    tabs = yarn_inv_freq_and_concentration(64, 150000.0, 32.0, 4096, 1.0, 32.0, partial_rotary_factor=0.5)
+    ref, _ = attn_fwd_thd(q, k, v, sinks, cu, 0.125, 128, rope_tables=tabs, positions=pos)
+    assert_parity(host(out), ref, "partial rotary thd out")

@@ -58,3 +58,21 @@ def test_decode_reuses_workspace_and_is_deterministic(cuda_device):
     assert torch.equal(o1, o2)
     ref, _ = attn_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.sinks, 0.125, 0, rope_tables=TABLES)
     assert_parity(host(o1), ref, "decode ws reuse")
+
+
+@pytest.mark.parametrize("rotary_dim", [16, 32])
+@pytest.mark.parametrize("window", [0, 128])
+def test_decode_partial_rotary(cuda_device, rotary_dim, window):
+    # partial_rotary_factor = rotary_dim / 64: the query rotates its first
+    # rotary_dim features only (the cache holds keys rotated the same way)
+    lens = [900, 1, 300]
+    x = make_decode_host(DECODE_B64, B=3, L=900, seqlens=lens, seed=104 + rotary_dim)
+    cfg = ops.RopeConfig.from_dict(GPTOSS_ROPE, rotary_dim=rotary_dim)
+    out, lse = ops.gptoss_attn_decode(dev(x.q), dev(x.k_cache), dev(x.v_cache), i32(x.seqlens), f32(x.sinks),
+                                      window=window, rope=cfg, return_lse=True)
+    torch.cuda.synchronize()
+    tabs = yarn_inv_freq_and_concentration(64, 150000.0, 32.0, 4096, 1.0, 32.0,
+                                           partial_rotary_factor=rotary_dim / 64)
+    ref, ref_lse = attn_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.sinks, 0.125, window, rope_tables=tabs)
+    assert_parity(host(out), ref, f"decode partial rotary {rotary_dim} out")
+    assert_lse_parity(host(lse), ref_lse, f"decode partial rotary {rotary_dim} lse")

@@ -231,3 +231,25 @@ def test_multi_token_of_one_equals_single_token(cuda_device):
     m = ops.gptoss_attn_decode_paged(dev(q[:, None]), dev(kp), dev(vp), i32(table), i32(lens), f32(sinks), rope=ROPE)
     torch.cuda.synchronize()
     assert torch.equal(m[:, 0], a)
+
+
+def test_partial_rotary_append_then_decode(cuda_device):
+    # rotary_dim 32: the appended key and the query rotate their first 32
+    # features; features 32..63 are copied as given
+    rng = np.random.default_rng(31)
+    lens = [300, 65]
+    bs = 64
+    q, kp, vp, table, sinks = _paged_case(lens, bs, seed=37)
+    k_new = bf16_round(rng.standard_normal((2, 2, 64)))
+    v_new = bf16_round(rng.standard_normal((2, 2, 64)))
+    cfg = ops.RopeConfig.from_dict(GPTOSS_ROPE, rotary_dim=32)
+    tabs = yarn_inv_freq_and_concentration(64, 150000.0, 32.0, 4096, 1.0, 32.0, partial_rotary_factor=0.5)
+    kd, vd = dev(kp), dev(vp)
+    ops.gptoss_kv_append_paged(dev(k_new), dev(v_new), i32(lens), i32(table), kd, vd, cfg)
+    out = ops.gptoss_attn_decode_paged(dev(q), kd, vd, i32(table), i32(lens), f32(sinks), rope=cfg)
+    torch.cuda.synchronize()
+    ref_k, ref_v = kv_append_paged(k_new, v_new, lens, table, bs, kp, vp, tabs)
+    np.testing.assert_allclose(host(kd), ref_k, rtol=2 ** -8, atol=1e-30)
+    np.testing.assert_array_equal(host(vd), ref_v)
+    ref, _ = attn_decode_paged(q, host(kd), host(vd), table, bs, lens, sinks, 0.125, 0, tabs)
+    assert_parity(host(out), ref, "partial rotary append then decode")

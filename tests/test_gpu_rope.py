@@ -80,3 +80,24 @@ def test_rope_strided_and_in_place(cuda_device):
     _check(host(qo), rope(qkv[:, :, :64], pos, inv, c))
     _check(host(t[:, :, 64:72]), rope(qkv[:, :, 64:72], pos, inv, c))
     np.testing.assert_array_equal(host(t[:, :, 72:]), qkv[:, :, 72:])  # v untouched
+
+
+@pytest.mark.parametrize("rotary_dim", [16, 32, 48])
+@pytest.mark.parametrize("rp", [PLAIN_ROPE, GPTOSS_ROPE], ids=["plain", "yarn"])
+def test_rope_partial_rotary(cuda_device, rp, rotary_dim):
+    # partial_rotary_factor = rotary_dim / 64: the first rotary_dim features
+    # rotate in pairs (j, j + rotary_dim / 2), the rest pass through untouched
+    rng = np.random.default_rng(rotary_dim)
+    B, S, Hq, Hkv = 2, 150, 8, 2
+    q = bf16_round(rng.standard_normal((B, S, Hq, 64)))
+    k = bf16_round(rng.standard_normal((B, S, Hkv, 64)))
+    qo, ko = ops.gptoss_rope_qk(dev(q), dev(k), ops.RopeConfig.from_dict(rp, rotary_dim=rotary_dim))
+    torch.cuda.synchronize()
+    inv, c = yarn_inv_freq_and_concentration(64, rp["base"], rp["factor"], rp["initial_context"], rp["ntk_alpha"],
+                                             rp["ntk_beta"], partial_rotary_factor=rotary_dim / 64)
+    assert len(inv) == rotary_dim // 2
+    pos = default_positions_bshd(B, S)
+    _check(host(qo), rope(q, pos, inv, c))
+    _check(host(ko), rope(k, pos, inv, c))
+    np.testing.assert_array_equal(host(qo)[..., rotary_dim:], q[..., rotary_dim:])
+    np.testing.assert_array_equal(host(ko)[..., rotary_dim:], k[..., rotary_dim:])
