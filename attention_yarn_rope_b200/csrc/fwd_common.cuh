@@ -20,7 +20,7 @@
 //                     ring: a unit's Q arrives while the two before it run)
 // setmaxnreg moves registers from the rope / producer / MMA warpgroups to the
 // two softmax warpgroups: launch 512 threads x 128 registers = 65536, split
-// 2 x 128 x 208 + 128 x 56 + 128 x 40 = 65536.  The host refuses to launch if
+// 2 x 128 x 208 + 128 x 48 + 128 x 48 = 65536.  The host refuses to launch if
 // the compiled kernel does not start at exactly 128 registers per thread.
 // TMEM columns (all 512): S_A [0,128) P_A [128,192) O_A [192,256),
 //                         S_B [256,384) P_B [384,448) O_B [448,512).
@@ -46,7 +46,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define GPTOSS_POLY_MASK 0x0000u
 #endif
 constexpr uint32_t kPolyMask = GPTOSS_POLY_MASK;
-constexpr uint32_t kRegsSoftmax = 208, kRegsRope = 56, kRegsOther = 40;
+constexpr uint32_t kRegsSoftmax = 208, kRegsRope = 48, kRegsOther = 48;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsRope + 128 * kRegsOther == kFwdThreads * kFwdLaunchRegs,
               "register split must add up to the launch allocation");
 
@@ -78,6 +78,7 @@ struct __align__(1024) FwdSmem {
   uint64_t v_full[kFwdStages], v_empty[kFwdStages];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];  // per head slot A/B
   uint64_t mma_final[2];  // the S and P V issuers' last products have completed
+  uint64_t turn[2][4];    // [head slot][warp]: this softmax warp may run its next exponentials
   uint32_t tmem_base;
 };
 

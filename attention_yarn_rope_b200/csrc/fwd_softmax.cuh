@@ -153,7 +153,9 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
   const uint32_t colS = X * 256, colP = X * 256 + 128, colO = X * 256 + 192;
   const bool thd = p.cu_seqlens != nullptr;
   const float sl = p.scale_log2;
-  uint32_t t = 0;  // running tile count of this CTA
+  uint32_t t = 0;        // running tile count of this CTA
+  uint32_t n_turns = 0;  // exponential turns this warp has taken
+  const int lane = threadIdx.x & 31;
   bool pending = false;
   PendingRow pr;
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
@@ -196,26 +198,34 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
       }
       float nb = m_run == -INFINITY ? 0.f : -m_run;
       float rs0 = 0.f, rs1 = 0.f;
+      // The exponentials of a tile are this warp's turn on its SMSP's MUFU
+      // unit, which it shares with the other head's warp of the same lane
+      // quarter: the two take turns tile by tile, so one reads S, stores P
+      // and waits on the pipeline while the other exponentiates.
+      // P(t) overwrites P(t-1): the previous P V product must have completed
+      // (waited here, while the other warp has its turn)
+      if (t > 0) {
+        if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
+        tc_fence_after();
+      }
+      if (X == 1 || n_turns > 0) {
+        if (!mbar_wait_warp(&sm.turn[X][wq], (X == 0 ? n_turns - 1 : n_turns) & 1, p.wait_ns)) return;
+      }
       {
         uint32_t pk[32];
         exp_half(sr, cls, 0, sl, nb, rs0, rs1, pk);
-        // P(t) overwrites P(t-1): the previous P V product must have completed
-        if (t > 0) {
-          if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
-          tc_fence_after();
-        }
         tmem_st32(lane_base + colP, pk);
+        exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
+        tmem_st32(lane_base + colP + 32, pk);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.turn[X ^ 1][wq]);
+      ++n_turns;
       // the previous unit's rows: its last P V has completed (waited above),
       // and this unit's first P V, which restarts O, waits for p_full below
       if (j == 0 && pending) {
         fwd_epilogue_row(p, lane_base + colO, pr);
         pending = false;
-      }
-      {
-        uint32_t pk[32];
-        exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
-        tmem_st32(lane_base + colP + 32, pk);
       }
       float rs = rs0 + rs1;
       if (__any_sync(0xffffffffu, !(rs <= kMaxTileSum))) {

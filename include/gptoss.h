@@ -77,7 +77,11 @@ typedef struct gptoss_rope_params {
   double base;             /* 150000 for GPT-OSS */
   double factor;           /* scaling_factor, 32 for GPT-OSS */
   int32_t initial_context; /* initial_context_length, 4096 */
-  int32_t rotary_dim;      /* int(head_dim * partial_rotary_factor); must equal D */
+  int32_t rotary_dim;      /* int(head_dim * partial_rotary_factor): features [0, rotary_dim)
+                              rotate in pairs (j, j + rotary_dim/2), the rest pass through
+                              unchanged; even, at most D.  gptoss_rope_qk, gptoss_attn_fwd, the
+                              decodes and the append take any multiple of 16 (partial rotary);
+                              gptoss_attn_bwd needs rotary_dim == D (else UNSUPPORTED) */
   double ntk_alpha;        /* 1 */
   double ntk_beta;         /* 32 */
 } gptoss_rope_params;
@@ -118,10 +122,11 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
  * sliding window, BSHD or packed THD.
  *   q [B,S,Hq,D] / [T,Hq,D], k and v [B,S,Hkv,D] / [T,Hkv,D], bf16, own
  *          strides.  rope != NULL: q and k are raw; q is rotated inside the
- *          kernel as its tiles are loaded, k likewise or once beforehand
- *          (see workspace); the rotated values enter the QK^T product as
- *          fp16, so c * |x| must stay below 65504;
- *          rope == NULL: q and k are already rotated (bf16 product).
+ *          attention kernel as its tiles are loaded, k once beforehand (see
+ *          workspace); rope == NULL: q and k are already rotated.  Both
+ *          products take fp16 operands (rotated q and k for QK^T; the
+ *          unnormalised probabilities and v for P V), so the rotated q and k
+ *          (c * |x|) and v must stay below 65504 in magnitude.
  *   sinks  fp32 [Hq], in the units of the scaled logits (may be -inf).
  *   positions / cu_seqlens as for gptoss_rope_qk (positions only used when
  *          rope != NULL).
@@ -132,16 +137,13 @@ gptoss_status gptoss_rope_qk(const void* q, gptoss_strides sq, const void* k, gp
  *   softmax_scale  head_dim^-0.5 for GPT-OSS.
  *   out    bf16, q's logical shape, strides so.
  *   lse    fp32, nullable: [B,Hq,S] (BSHD) or [Hq,T] (THD), natural log.
- *   workspace  nullable device memory of at least
+*   workspace  device memory of at least
  *          gptoss_attn_fwd_workspace_size(total_tokens, Hkv, D) bytes, 16-byte
- *          aligned, owned by the caller, contents need not be initialised;
- *          only used when rope != NULL.  Given one, a first kernel on the
- *          same stream rotates k once into it (fp16, dense) and stores every
- *          token's 32 RoPE angles (c cos, c sin), which the attention kernel
- *          reads for q; without one, every work unit rotates the k tiles it
- *          loads and forms the angles itself (same results, more work per
- *          key).  A workspace that is too small or misaligned is
- *          GPTOSS_ERR_INVALID_ARG. */
+ *          aligned, owned by the caller, contents need not be initialised.
+ *          A first kernel on the same stream writes into it k (rotated when
+ *          rope != NULL) and v as dense fp16, and every token's 32 RoPE
+ *          angles (c cos, c sin), which the attention kernel reads for q.
+ *          NULL, too small or misaligned is GPTOSS_ERR_INVALID_ARG. */
 gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
                               const void* v, gptoss_strides sv, const float* sinks,
                               const int32_t* positions, const int32_t* cu_seqlens, int32_t B,
@@ -150,9 +152,9 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
                               void* out, gptoss_strides so, float* lse, void* workspace,
                               size_t workspace_bytes, struct CUstream_st* stream);
 
-/* Workspace bytes for gptoss_attn_fwd: the rotated k (total_tokens x Hkv x D
- * fp16 values, rounded up to 256 bytes) and the angle table (total_tokens x
- * 32 fp32 pairs).  0 when a size is out of range. */
+/* Workspace bytes for gptoss_attn_fwd: k and v as fp16 (total_tokens x Hkv x
+ * D values each, each rounded up to 256 bytes) and the angle table
+ * (total_tokens x 32 fp32 pairs).  0 when a size is out of range. */
 size_t gptoss_attn_fwd_workspace_size(int32_t total_tokens, int32_t Hkv, int32_t D);
 
 /* Workspace bytes gptoss_attn_bwd needs: q and k rotated once (fp16), every
