@@ -32,6 +32,9 @@ EXPORTED = (
     "gptoss_rope_qk",
     "gptoss_attn_fwd",
     "gptoss_attn_fwd_workspace_size",
+    "gptoss_attn_fwd_block",
+    "gptoss_attn_fwd_block_workspace_size",
+    "gptoss_attn_merge",
     "gptoss_attn_decode_workspace_size",
     "gptoss_attn_decode",
     "gptoss_attn_decode_noalloc",
@@ -74,6 +77,11 @@ _SIGNATURES = {
                               _i32, _i32, _i32, _f32, ctypes.POINTER(RopeParams), _vp, Strides, _vp, _vp,
                               ctypes.c_size_t, _vp]),
     "gptoss_attn_fwd_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32]),
+    "gptoss_attn_fwd_block": (_st, [_vp, Strides, _vp, Strides, _vp, Strides, _i32, _i32, _i32, _i32, _i32, _i32,
+                                    _i32, _i32, _f32, ctypes.POINTER(RopeParams), _vp, _vp, _vp, ctypes.c_size_t,
+                                    _vp]),
+    "gptoss_attn_fwd_block_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
+    "gptoss_attn_merge": (_st, [_vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, Strides, _vp, _vp]),
     "gptoss_attn_decode_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
     "gptoss_attn_decode": (_st, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                  ctypes.POINTER(RopeParams), _vp, _vp, _vp, ctypes.c_size_t, _vp]),

@@ -22,8 +22,13 @@ zero dout for the halo rows (they contribute nothing), sends the halo rows'
 dk / dv back to rank r - 1, which adds them to its last W - 1 rows, and sums
 dsinks over the ranks.
 
-Full-context layers need every earlier shard's keys (a ring with a
-log-sum-exp merge); that is not built here.
+Full-context layers need every earlier shard's keys: :func:`full_context_fwd`
+passes the k / v shards around the ring of ranks (NCCL point-to-point, the
+next block's transfer overlapping the current block's attention); each rank
+runs the block form of the prefill (``gptoss_attn_fwd_block``: causal on the
+global token indices, no sink) of its query shard against every block at or
+before it, and merges the blocks with the sink folded in once
+(``gptoss_attn_merge``).  Forward only.
 """
 
 from __future__ import annotations
@@ -321,3 +326,43 @@ def sliding_window_bwd_thd(q, k, v, sinks, out, dout, lse, cu_seqlens, window: i
     if world > 1:
         dist.all_reduce(dsinks, op=dist.ReduceOp.SUM, group=group)
     return dq, dk, dv, dsinks
+
+
+def full_context_fwd(q, k, v, sinks, rope, group=None, softmax_scale: float | None = None, attn_block=None,
+                     merge=None):
+    """This rank's rows of the full-context attention of the whole sequence.
+
+    q ``[B, S_loc, Hq, D]``, k / v ``[B, S_loc, Hkv, D]``: this rank's shard
+    (tokens [rank S_loc, (rank + 1) S_loc) of every sequence), raw (RoPE at
+    the global positions inside the block prefill).  Returns ``(out [B, S_loc,
+    Hq, D], lse [B, Hq, S_loc])``.  Ring: at step s this rank holds the k / v
+    block of rank (rank - s) mod R; it forwards the block to rank + 1 while it
+    computes its queries against it, if that block lies at or before its shard
+    (a later rank's keys are all in the future of this shard's queries).
+    ``attn_block(q, k, v, q_start, k_start, rope=, softmax_scale=)`` returning
+    ``(out fp32, lse)`` and ``merge(outs [n, ...], lses [n, ...], sinks)``
+    returning ``(out, lse)`` default to the CUDA library."""
+    attn_block = attn_block or ops.gptoss_attn_fwd_block
+    merge = merge or (lambda outs, lses, snk: ops.gptoss_attn_merge(outs, lses, snk, lse=True))
+    rank, world = _rank_world(group)
+    s_loc = q.shape[1]
+    Hkv = k.shape[2]
+    held = torch.cat([k, v], dim=2).contiguous()  # the block held now: k and v heads concatenated
+    outs, lses = [], []
+    for step in range(world):
+        src = (rank - step) % world  # whose block is held
+        reqs, recv = [], None
+        if step + 1 < world:  # the ring moves on while this step computes
+            recv = torch.empty_like(held)
+            reqs.append(dist.irecv(recv, src=_peer(group, (rank - 1) % world), group=group))
+            reqs.append(dist.isend(held, dst=_peer(group, (rank + 1) % world), group=group))
+        if src <= rank:
+            o, l = attn_block(q, held[:, :, :Hkv], held[:, :, Hkv:], rank * s_loc, src * s_loc, rope=rope,
+                              softmax_scale=softmax_scale)
+            outs.append(o)
+            lses.append(l)
+        for r in reqs:
+            r.wait()
+        if recv is not None:
+            held = recv  # the sent block stays referenced by `reqs` until its send completed
+    return merge(torch.stack(outs), torch.stack(lses), sinks)

@@ -40,12 +40,6 @@ constexpr int kFwdLaunchRegs = 128;   // 65536 / 512
 constexpr int kFwdTileBytes = kFwdTile * kHeadDim * 2;  // 16 KB
 constexpr uint32_t kFwdTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Which of the 16 column pairs of every 32-key chunk take 2^x from the FMA-pipe
-// polynomial (bit e set) instead of the MUFU unit; balances the two pipes.
-#ifndef GPTOSS_POLY_MASK
-#define GPTOSS_POLY_MASK 0x0000u
-#endif
-constexpr uint32_t kPolyMask = GPTOSS_POLY_MASK;
 constexpr uint32_t kRegsSoftmax = 208, kRegsRope = 48, kRegsOther = 48;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsRope + 128 * kRegsOther == kFwdThreads * kFwdLaunchRegs,
               "register split must add up to the launch allocation");
@@ -59,10 +53,16 @@ struct FwdParams {
   __nv_bfloat16* out;
   gptoss_strides so;
   float* lse;
-  const float* sinks;
+  const float* sinks;         // nullable: no sink (the block form; the merge folds it in)
   const int32_t* positions;
   const int32_t* cu_seqlens;
   int B, S, T, Hq, Hkv, G, HP, window, n_qtiles, n_units;
+  // Block form (BSHD): the keys are another block of the sequence than the
+  // queries.  Query row i and key row j sit at global indices i + delta and
+  // j (delta = first query's global index - first key's, >= 0); Lk keys per
+  // batch row.  Self-attention: delta = 0, Lk = S.
+  int delta, Lk;
+  float* out_f32;             // nullable: fp32 output [B, S, Hq, 64] dense instead of bf16 out
   const float2* cs_tab;  // nullable: per-token (c cos, c sin) of the 32 pairs, [token][32]
   float scale_log2;
   uint64_t wait_ns;
@@ -78,13 +78,12 @@ struct __align__(1024) FwdSmem {
   uint64_t v_full[kFwdStages], v_empty[kFwdStages];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];  // per head slot A/B
   uint64_t mma_final[2];  // the S and P V issuers' last products have completed
-  uint64_t turn[2][4];    // [head slot][warp]: this softmax warp may run its next exponentials
   uint32_t tmem_base;
 };
 
 // One work unit: query tile q0 / 128 of heads (h0, h1) of sequence b.
 struct Unit {
-  int b, h0, h1, g, q0, L, seq_start, j_lo, n_kt;
+  int b, h0, h1, g, q0, L, Lk, seq_start, j_lo, n_kt;  // L query rows, Lk key rows
   bool dup;  // h1 repeats h0 (odd group size): computed, not stored
 };
 
@@ -104,11 +103,13 @@ __device__ __forceinline__ bool make_unit(const FwdParams& p, int u, Unit& w) {
   const bool thd = p.cu_seqlens != nullptr;
   w.seq_start = thd ? __ldg(p.cu_seqlens + w.b) : 0;
   w.L = thd ? __ldg(p.cu_seqlens + w.b + 1) - w.seq_start : p.S;
+  w.Lk = thd ? w.L : p.Lk;
   w.q0 = qt * kFwdTile;
   if (w.q0 >= w.L) return false;
+  // keys visible from the tile's rows: [q0 + delta - window + 1, q_last + delta]
   const int q_last = min(w.q0 + kFwdTile, w.L) - 1;
-  const int j_hi = q_last / kFwdTile;
-  w.j_lo = p.window > 0 ? max(0, w.q0 - p.window + 1) / kFwdTile : 0;
+  const int j_hi = min(q_last + p.delta, w.Lk - 1) / kFwdTile;
+  w.j_lo = p.window > 0 ? max(0, w.q0 + p.delta - p.window + 1) / kFwdTile : 0;
   w.n_kt = j_hi - w.j_lo + 1;
   return true;
 }

@@ -76,6 +76,144 @@ static void identity_table(RopeTable* t) {
   t->R = kPairs;
 }
 
+// One prefill call, validated: the self-attention entry point and the block
+// form both launch through here.
+struct PrefillCall {
+  const void *q, *k, *v;
+  gptoss_strides sq, sk, sv, so;
+  const float* sinks;            // nullable in the block form
+  const int32_t* positions;      // self-attention only
+  const int32_t* cu_seqlens;     // self-attention only
+  int32_t B, Sq, Sk, Tq, Tk;     // Sk / Tk: key rows per batch row / in all (self: equal to the query's)
+  int32_t Hq, Hkv, window, delta;
+  int32_t q_pos0, k_pos0;        // default positions of the first query / key row
+  float scale;
+  const gptoss_rope_params* rope;
+  void* out;                     // bf16, strides so
+  float* out_f32;                // block form: dense fp32 [B, Sq, Hq, 64]
+  float* lse;
+  void* workspace;
+  cudaStream_t stream;
+};
+
+static gptoss_status prefill_launch(const PrefillCall& c) {
+  const bool thd = c.cu_seqlens != nullptr;
+  const int n_qtiles = (c.Sq + kFwdTile - 1) / kFwdTile;
+  const int G = c.Hq / c.Hkv;
+  const int HP = (G + 1) / 2;  // head pairs per kv group
+  const int64_t n_units = static_cast<int64_t>(n_qtiles) * c.B * c.Hkv * HP;
+  if (n_units > INT32_MAX) return GPTOSS_ERR_UNSUPPORTED;
+  // The register split inside the kernel assumes exactly kFwdLaunchRegs
+  // registers per thread at launch; anything else could stall the split.
+  static int launch_regs = -1;
+  if (launch_regs < 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel) != cudaSuccess) return GPTOSS_ERR_CUDA;
+    launch_regs = fa.numRegs;
+  }
+  if (launch_regs != kFwdLaunchRegs) return GPTOSS_ERR_UNSUPPORTED;
+  int device = 0, n_sm = 0;
+  if (cudaGetDevice(&device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return GPTOSS_ERR_CUDA;
+  const int grid = static_cast<int>(n_units < n_sm ? n_units : n_sm);
+
+  FwdParams p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t dimQ = thd ? static_cast<uint64_t>(c.Tq) : static_cast<uint64_t>(c.Sq);
+  const uint64_t dimK = thd ? static_cast<uint64_t>(c.Tk) : static_cast<uint64_t>(c.Sk);
+  const uint64_t dimB = thd ? 1 : static_cast<uint64_t>(c.B);
+  const uint64_t qb_stride = thd ? dimQ * c.sq.tok * 2 : static_cast<uint64_t>(c.sq.batch) * 2;
+  gptoss_status st = make_tmap_4d(&p.tmap_q, c.q, kHeadDim, c.Hq, dimQ, dimB, c.sq.head * 2, c.sq.tok * 2,
+                                  qb_stride == 0 ? 16 : qb_stride, kHeadDim, 1, kFwdTile, 1);
+  if (st != GPTOSS_OK) return st;
+  // fp16 k and v: dense [B, Sk, Hkv, D] / [T, Hkv, D] in the workspace
+  uint8_t* ws = static_cast<uint8_t*>(c.workspace);
+  const size_t kv_bytes = fwd_ws_kv_bytes(c.Tk, c.Hkv);
+  const uint64_t tok_b = static_cast<uint64_t>(c.Hkv) * kHeadDim * 2;
+  const uint64_t seq_b = dimK * tok_b;
+  st = make_tmap_4d(&p.tmap_k, ws, kHeadDim, c.Hkv, dimK, dimB, kHeadDim * 2, tok_b, seq_b, kHeadDim, 1, kFwdTile, 1,
+                    true);
+  if (st != GPTOSS_OK) return st;
+  st = make_tmap_4d(&p.tmap_v, ws + kv_bytes, kHeadDim, c.Hkv, dimK, dimB, kHeadDim * 2, tok_b, seq_b, kHeadDim, 1,
+                    kFwdTile, 1, true);
+  if (st != GPTOSS_OK) return st;
+  p.q = static_cast<const __nv_bfloat16*>(c.q);
+  p.sq = c.sq;
+  p.out = static_cast<__nv_bfloat16*>(c.out);
+  p.so = c.so;
+  p.out_f32 = c.out_f32;
+  p.lse = c.lse;
+  p.sinks = c.sinks;
+  p.cu_seqlens = c.cu_seqlens;
+  p.B = c.B;
+  p.S = c.Sq;
+  p.T = c.Tq;
+  p.Hq = c.Hq;
+  p.Hkv = c.Hkv;
+  p.G = G;
+  p.HP = HP;
+  p.window = c.window;
+  p.delta = c.delta;
+  p.Lk = c.Sk;
+  p.n_qtiles = n_qtiles;
+  p.n_units = static_cast<int>(n_units);
+  p.scale_log2 = c.scale * kLog2e;
+  p.wait_ns = wait_limit_ns();
+  // positions feed RoPE only: without RoPE the kernels take the identity table
+  if (c.rope != nullptr) yarn_table(*c.rope, &p.tab);
+  else identity_table(&p.tab);
+  p.positions = c.rope != nullptr ? c.positions : nullptr;
+  // the first kernel: k rotated (at its positions) and v converted into the
+  // workspace as fp16, and the per-token angle table of the query tokens
+  const bool same_tokens = c.delta == 0 && c.Sk == c.Sq && c.q_pos0 == c.k_pos0;
+  float2* q_table = reinterpret_cast<float2*>(ws + 2 * kv_bytes);
+  RopeQkParams rp;
+  memset(&rp, 0, sizeof(rp));
+  rp.k = static_cast<const __nv_bfloat16*>(c.k);
+  rp.k_out = reinterpret_cast<__nv_bfloat16*>(ws);  // fp16 bits (rope_qk_kernel<true>)
+  rp.sk = c.sk;
+  rp.v = static_cast<const __nv_bfloat16*>(c.v);
+  rp.v_out = reinterpret_cast<__nv_bfloat16*>(ws + kv_bytes);
+  rp.sv = c.sv;
+  rp.sko.head = rp.svo.head = kHeadDim;
+  rp.sko.tok = rp.svo.tok = static_cast<int64_t>(c.Hkv) * kHeadDim;
+  rp.sko.batch = rp.svo.batch = thd ? 0 : static_cast<int64_t>(c.Sk) * c.Hkv * kHeadDim;
+  rp.tm.positions = p.positions;
+  rp.tm.cu_seqlens = c.cu_seqlens;
+  rp.tm.nseq = c.B;
+  rp.tm.S = thd ? 0 : c.Sk;
+  rp.tm.ntok = c.Tk;
+  rp.tm.pos_offset = c.k_pos0;
+  rp.Hq = 0;
+  rp.Hkv = c.Hkv;
+  rp.tab = p.tab;
+  rp.cs_out = same_tokens ? q_table : nullptr;
+  rope_qk_kernel<true><<<(c.Tk + kRopeTokensPerCta - 1) / kRopeTokensPerCta, kRopeThreads, 0, c.stream>>>(rp);
+  st = check_launch();
+  if (st != GPTOSS_OK) return st;
+  if (!same_tokens) {  // the block form: the query tokens' angle table on its own
+    RopeQkParams tp;
+    memset(&tp, 0, sizeof(tp));
+    tp.tm.nseq = c.B;
+    tp.tm.S = c.Sq;
+    tp.tm.ntok = c.Tq;
+    tp.tm.pos_offset = c.q_pos0;
+    tp.tab = p.tab;
+    tp.cs_out = q_table;
+    rope_qk_kernel<true><<<(c.Tq + kRopeTokensPerCta - 1) / kRopeTokensPerCta, kRopeThreads, 0, c.stream>>>(tp);
+    st = check_launch();
+    if (st != GPTOSS_OK) return st;
+  }
+  p.cs_tab = q_table;
+  const size_t smem = sizeof(FwdSmem) + 1024;
+  if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return GPTOSS_ERR_CUDA;
+  attn_fwd_kernel<<<grid, kFwdThreads, smem, c.stream>>>(p);
+  return check_launch();
+}
+
 gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk, const void* v,
                               gptoss_strides sv, const float* sinks, const int32_t* positions,
                               const int32_t* cu_seqlens, int32_t B, int32_t S, int32_t total_tokens, int32_t Hq,
@@ -100,100 +238,90 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
   if (workspace == nullptr || !aligned16(workspace) ||
       workspace_bytes < gptoss_attn_fwd_workspace_size(total_tokens, Hkv, D))
     return GPTOSS_ERR_INVALID_ARG;
-  const int n_qtiles = (S + kFwdTile - 1) / kFwdTile;
-  const int G = Hq / Hkv;
-  const int HP = (G + 1) / 2;  // head pairs per kv group
-  const int64_t n_units = static_cast<int64_t>(n_qtiles) * B * Hkv * HP;
-  if (n_units > INT32_MAX) return GPTOSS_ERR_UNSUPPORTED;
-  // The register split inside the kernel assumes exactly kFwdLaunchRegs
-  // registers per thread at launch; anything else could stall the split.
-  static int launch_regs = -1;
-  if (launch_regs < 0) {
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel) != cudaSuccess) return GPTOSS_ERR_CUDA;
-    launch_regs = fa.numRegs;
-  }
-  if (launch_regs != kFwdLaunchRegs) return GPTOSS_ERR_UNSUPPORTED;
-  int device = 0, n_sm = 0;
-  if (cudaGetDevice(&device) != cudaSuccess ||
-      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
-    return GPTOSS_ERR_CUDA;
-  const int grid = static_cast<int>(n_units < n_sm ? n_units : n_sm);
+  PrefillCall c;
+  memset(&c, 0, sizeof(c));
+  c.q = q;
+  c.k = k;
+  c.v = v;
+  c.sq = sq;
+  c.sk = sk;
+  c.sv = sv;
+  c.so = so;
+  c.sinks = sinks;
+  c.positions = positions;
+  c.cu_seqlens = cu_seqlens;
+  c.B = B;
+  c.Sq = c.Sk = S;
+  c.Tq = c.Tk = total_tokens;
+  c.Hq = Hq;
+  c.Hkv = Hkv;
+  c.window = window;
+  c.scale = softmax_scale;
+  c.rope = rope;
+  c.out = out;
+  c.lse = lse;
+  c.workspace = workspace;
+  c.stream = as_stream(stream);
+  return prefill_launch(c);
+}
 
-  FwdParams p;
-  memset(&p, 0, sizeof(p));
-  const uint64_t dimS = thd ? static_cast<uint64_t>(total_tokens) : static_cast<uint64_t>(S);
-  const uint64_t dimB = thd ? 1 : static_cast<uint64_t>(B);
-  const uint64_t qb_stride = thd ? dimS * sq.tok * 2 : static_cast<uint64_t>(sq.batch) * 2;
-  st = make_tmap_4d(&p.tmap_q, q, kHeadDim, Hq, dimS, dimB, sq.head * 2, sq.tok * 2,
-                         qb_stride == 0 ? 16 : qb_stride, kHeadDim, 1, kFwdTile, 1);
+size_t gptoss_attn_fwd_block_workspace_size(int32_t B, int32_t Sq, int32_t Sk, int32_t Hkv, int32_t D) {
+  if (B < 0 || Sq < 0 || Sk < 0 || Hkv <= 0 || D != kHeadDim) return 0;
+  const int64_t tq = static_cast<int64_t>(B) * Sq, tk = static_cast<int64_t>(B) * Sk;
+  if (tq > INT32_MAX || tk > INT32_MAX) return 0;
+  return 2 * fwd_ws_kv_bytes(static_cast<int32_t>(tk), Hkv) + static_cast<size_t>(tq) * kPairs * sizeof(float2);
+}
+
+gptoss_status gptoss_attn_fwd_block(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
+                                    const void* v, gptoss_strides sv, int32_t B, int32_t Sq, int32_t Sk,
+                                    int32_t q_start, int32_t k_start, int32_t Hq, int32_t Hkv, int32_t D,
+                                    float softmax_scale, const gptoss_rope_params* rope, float* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, struct CUstream_st* stream) {
+  if (B < 0 || Sq < 0 || Sk < 0 || Hq <= 0 || Hkv <= 0 || q_start < 0 || k_start < 0) return GPTOSS_ERR_INVALID_ARG;
+  if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
+  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
+  // the key block must start at or before the query shard (causal: a block
+  // after it is invisible), so every query row sees at least one key
+  if (k_start > q_start) return GPTOSS_ERR_INVALID_ARG;
+  gptoss_status st = check_rope(rope, D, /*allow_partial=*/true);
   if (st != GPTOSS_OK) return st;
-  // fp16 k and v: dense [B, S, Hkv, D] / [T, Hkv, D] in the workspace
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const size_t kv_bytes = fwd_ws_kv_bytes(total_tokens, Hkv);
-  const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
-  const uint64_t seq_b = thd ? dimS * tok_b : static_cast<uint64_t>(S) * tok_b;
-  st = make_tmap_4d(&p.tmap_k, ws, kHeadDim, Hkv, dimS, dimB, kHeadDim * 2, tok_b, seq_b, kHeadDim, 1, kFwdTile, 1,
-                    true);
-  if (st != GPTOSS_OK) return st;
-  st = make_tmap_4d(&p.tmap_v, ws + kv_bytes, kHeadDim, Hkv, dimS, dimB, kHeadDim * 2, tok_b, seq_b, kHeadDim, 1,
-                    kFwdTile, 1, true);
-  if (st != GPTOSS_OK) return st;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.sq = sq;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.so = so;
-  p.lse = lse;
-  p.sinks = sinks;
-  p.positions = positions;
-  p.cu_seqlens = cu_seqlens;
-  p.B = B;
-  p.S = S;
-  p.T = total_tokens;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = G;
-  p.HP = HP;
-  p.window = window;
-  p.n_qtiles = n_qtiles;
-  p.n_units = static_cast<int>(n_units);
-  p.scale_log2 = softmax_scale * kLog2e;
-  p.wait_ns = wait_limit_ns();
-  // positions feed RoPE only: without RoPE the kernels take the identity table
-  if (rope != nullptr) yarn_table(*rope, &p.tab);
-  else identity_table(&p.tab);
-  p.positions = rope != nullptr ? positions : nullptr;
-  RopeQkParams rp;
-  memset(&rp, 0, sizeof(rp));
-  rp.k = static_cast<const __nv_bfloat16*>(k);
-  rp.k_out = reinterpret_cast<__nv_bfloat16*>(ws);  // fp16 bits (rope_qk_kernel<true>)
-  rp.sk = sk;
-  rp.v = static_cast<const __nv_bfloat16*>(v);
-  rp.v_out = reinterpret_cast<__nv_bfloat16*>(ws + kv_bytes);
-  rp.sv = sv;
-  rp.sko.head = rp.svo.head = kHeadDim;
-  rp.sko.tok = rp.svo.tok = static_cast<int64_t>(Hkv) * kHeadDim;
-  rp.sko.batch = rp.svo.batch = thd ? 0 : static_cast<int64_t>(S) * Hkv * kHeadDim;
-  rp.tm.positions = p.positions;
-  rp.tm.cu_seqlens = cu_seqlens;
-  rp.tm.nseq = B;
-  rp.tm.S = thd ? 0 : S;
-  rp.tm.ntok = total_tokens;
-  rp.Hq = 0;
-  rp.Hkv = Hkv;
-  rp.tab = p.tab;
-  rp.cs_out = reinterpret_cast<float2*>(ws + 2 * kv_bytes);
-  p.cs_tab = rp.cs_out;
-  const int rgrid = (total_tokens + kRopeTokensPerCta - 1) / kRopeTokensPerCta;
-  rope_qk_kernel<true><<<rgrid, kRopeThreads, 0, as_stream(stream)>>>(rp);
-  st = check_launch();
-  if (st != GPTOSS_OK) return st;
-  const size_t smem = sizeof(FwdSmem) + 1024;
-  if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
-    return GPTOSS_ERR_CUDA;
-  attn_fwd_kernel<<<grid, kFwdThreads, smem, as_stream(stream)>>>(p);
-  return check_launch();
+  if (B == 0 || Sq == 0) return GPTOSS_OK;
+  if (Sk == 0) return GPTOSS_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(q_start) + Sq > INT32_MAX || static_cast<int64_t>(q_start) - k_start > INT32_MAX)
+    return GPTOSS_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out || !lse) return GPTOSS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GPTOSS_ERR_INVALID_ARG;
+  if (!strides_ok(sq, true) || !strides_ok(sk, true) || !strides_ok(sv, true)) return GPTOSS_ERR_INVALID_ARG;
+  const size_t need = gptoss_attn_fwd_block_workspace_size(B, Sq, Sk, Hkv, D);
+  if (need == 0 || workspace == nullptr || !aligned16(workspace) || workspace_bytes < need)
+    return GPTOSS_ERR_INVALID_ARG;
+  PrefillCall c;
+  memset(&c, 0, sizeof(c));
+  c.q = q;
+  c.k = k;
+  c.v = v;
+  c.sq = sq;
+  c.sk = sk;
+  c.sv = sv;
+  c.B = B;
+  c.Sq = Sq;
+  c.Sk = Sk;
+  c.Tq = B * Sq;
+  c.Tk = B * Sk;
+  c.Hq = Hq;
+  c.Hkv = Hkv;
+  c.window = 0;
+  c.delta = q_start - k_start;
+  c.q_pos0 = q_start;
+  c.k_pos0 = k_start;
+  c.scale = softmax_scale;
+  c.rope = rope;
+  c.out_f32 = out;
+  c.lse = lse;
+  c.workspace = workspace;
+  c.stream = as_stream(stream);
+  return prefill_launch(c);
 }
 
 }  // extern "C"

@@ -176,10 +176,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
     }
     mbar_init(&sm.mma_final[0], 1);
     mbar_init(&sm.mma_final[1], 1);
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&sm.turn[0][i], 1);
-      mbar_init(&sm.turn[1][i], 1);
-    }
     fence_mbar_init();
   }
   if (warp == 13) {

@@ -55,15 +55,16 @@ __device__ __forceinline__ float tile_max(const uint32_t (&sr)[4][32], const int
 }
 
 // Reads this warp's 32 rows x 128 scores of S from TMEM and sets the hidden
-// elements of partly visible chunks to -inf (row qi sees keys
-// [qi - window + 1, min(qi, L - 1)]; k0 is the tile's first key).
-__device__ __forceinline__ void load_masked_s(uint32_t taddr, const int (&cls)[4], int qi, int k0, int L,
+// elements of partly visible chunks to -inf (row qi, at key index gi =
+// qi + delta, sees keys [gi - window + 1, min(gi, Lk - 1)]; k0 is the tile's
+// first key).
+__device__ __forceinline__ void load_masked_s(uint32_t taddr, const int (&cls)[4], int gi, int k0, int Lk,
                                               int window, uint32_t (&sr)[4][32]) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, sr[c]);
   tmem_wait_ld();
-  const int c_hi = min(qi, L - 1) - k0;  // visible columns of this row: [c_lo, c_hi]
-  const int c_lo = window > 0 ? qi - window + 1 - k0 : -1;
+  const int c_hi = min(gi, Lk - 1) - k0;  // visible columns of this row: [c_lo, c_hi]
+  const int c_lo = window > 0 ? gi - window + 1 - k0 : -1;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     if (cls[c] == 1) {  // warp-uniform branch
@@ -90,14 +91,7 @@ __device__ __forceinline__ void exp_half(const uint32_t (&sr)[4][32], const int 
       for (int e = 0; e < 16; ++e) {
         const float x0 = fmaf(__uint_as_float(sr[c][2 * e]), sl, nb);
         const float x1 = fmaf(__uint_as_float(sr[c][2 * e + 1]), sl, nb);
-        float p0, p1;
-        if ((kPolyMask >> e) & 1u) {
-          p0 = exp2_poly(x0);
-          p1 = exp2_poly(x1);
-        } else {
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
-        }
+        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
         rs0 += p0;
         rs1 += p1;
         pk[cc * 16 + e] = pack_f16(p0, p1);
@@ -116,6 +110,7 @@ struct PendingRow {
   int64_t out_row;  // element offset of the output row (head included); -1: nothing to store
   int64_t lse_idx;  // -1: no lse
 };
+// (out_row indexes p.out with its strides, or the dense fp32 p.out_f32.)
 
 // O / l with the sink folded once (M = max(m, sink), l' = l 2^(m - M) +
 // 2^(sink - M)), in bf16, and LSE = (M + log2 l') ln 2.  O must be complete.
@@ -129,7 +124,18 @@ __device__ __forceinline__ void fwd_epilogue_row(const FwdParams& p, uint32_t o_
     uint32_t ov[32];
     tmem_ld32(o_addr + c * 32, ov);
     tmem_wait_ld();
-    if (pr.out_row >= 0) {
+    if (pr.out_row >= 0 && p.out_f32 != nullptr) {
+      float* dst = p.out_f32 + pr.out_row + c * 32;
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        float4 v;
+        v.x = __uint_as_float(ov[4 * c4 + 0]) * inv;
+        v.y = __uint_as_float(ov[4 * c4 + 1]) * inv;
+        v.z = __uint_as_float(ov[4 * c4 + 2]) * inv;
+        v.w = __uint_as_float(ov[4 * c4 + 3]) * inv;
+        *reinterpret_cast<float4*>(dst + 4 * c4) = v;
+      }
+    } else if (pr.out_row >= 0) {
       __nv_bfloat16* dst = p.out + pr.out_row + c * 32;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8) {
@@ -153,9 +159,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
   const uint32_t colS = X * 256, colP = X * 256 + 128, colO = X * 256 + 192;
   const bool thd = p.cu_seqlens != nullptr;
   const float sl = p.scale_log2;
-  uint32_t t = 0;        // running tile count of this CTA
-  uint32_t n_turns = 0;  // exponential turns this warp has taken
-  const int lane = threadIdx.x & 31;
+  uint32_t t = 0;  // running tile count of this CTA
   bool pending = false;
   PendingRow pr;
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
@@ -163,8 +167,9 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
     if (!make_unit(p, u, w)) continue;
     const int h = X == 0 ? w.h0 : w.h1;
     const int qi = w.q0 + r;
-    const int qw_lo = w.q0 + wq * 32, qw_hi = qw_lo + 31;  // rows of this warp
-    const float sink = __ldg(p.sinks + h) * kLog2e;
+    // rows of this warp, as key indices (query row i sits at key index i + delta)
+    const int qw_lo = w.q0 + wq * 32 + p.delta, qw_hi = qw_lo + 31;
+    const float sink = p.sinks != nullptr ? __ldg(p.sinks + h) * kLog2e : -INFINITY;
     float m_run = -INFINITY;
     float l_run = 0.f;
     for (int j = 0; j < w.n_kt; ++j, ++t) {
@@ -176,12 +181,12 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int kl = k0 + 32 * c, kh = kl + 31;
-        const bool hidden = kl > min(qw_hi, w.L - 1) || (p.window > 0 && kh < qw_lo - p.window + 1);
-        const bool full = kh <= qw_lo && kh <= w.L - 1 && (p.window == 0 || kl >= qw_hi - p.window + 1);
+        const bool hidden = kl > min(qw_hi, w.Lk - 1) || (p.window > 0 && kh < qw_lo - p.window + 1);
+        const bool full = kh <= qw_lo && kh <= w.Lk - 1 && (p.window == 0 || kl >= qw_hi - p.window + 1);
         cls[c] = hidden ? 0 : (full ? 2 : 1);
       }
       uint32_t sr[4][32];
-      load_masked_s(lane_base + colS, cls, qi, k0, w.L, p.window, sr);
+      load_masked_s(lane_base + colS, cls, qi + p.delta, k0, w.Lk, p.window, sr);
       tc_fence_before();
       mbar_arrive(&sm.s_free[X]);
       float alpha = 1.f;
@@ -198,29 +203,18 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
       }
       float nb = m_run == -INFINITY ? 0.f : -m_run;
       float rs0 = 0.f, rs1 = 0.f;
-      // The exponentials of a tile are this warp's turn on its SMSP's MUFU
-      // unit, which it shares with the other head's warp of the same lane
-      // quarter: the two take turns tile by tile, so one reads S, stores P
-      // and waits on the pipeline while the other exponentiates.
-      // P(t) overwrites P(t-1): the previous P V product must have completed
-      // (waited here, while the other warp has its turn)
-      if (t > 0) {
-        if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
-        tc_fence_after();
-      }
-      if (X == 1 || n_turns > 0) {
-        if (!mbar_wait_warp(&sm.turn[X][wq], (X == 0 ? n_turns - 1 : n_turns) & 1, p.wait_ns)) return;
-      }
       {
         uint32_t pk[32];
         exp_half(sr, cls, 0, sl, nb, rs0, rs1, pk);
+        // P(t) overwrites P(t-1): the previous P V product must have completed
+        if (t > 0) {
+          if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
+          tc_fence_after();
+        }
         tmem_st32(lane_base + colP, pk);
         exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
         tmem_st32(lane_base + colP + 32, pk);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.turn[X ^ 1][wq]);
-      ++n_turns;
       // the previous unit's rows: its last P V has completed (waited above),
       // and this unit's first P V, which restarts O, waits for p_full below
       if (j == 0 && pending) {
@@ -271,9 +265,11 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
     pr.out_row = -1;
     pr.lse_idx = -1;
     if (qi < w.L && !(X == 1 && w.dup)) {
-      pr.out_row = (thd ? static_cast<int64_t>(w.seq_start + qi) * p.so.tok
-                        : static_cast<int64_t>(w.b) * p.so.batch + static_cast<int64_t>(qi) * p.so.tok) +
-                   static_cast<int64_t>(h) * p.so.head;
+      pr.out_row = p.out_f32 != nullptr
+                       ? ((static_cast<int64_t>(w.b) * p.S + qi) * p.Hq + h) * kHeadDim
+                       : (thd ? static_cast<int64_t>(w.seq_start + qi) * p.so.tok
+                              : static_cast<int64_t>(w.b) * p.so.batch + static_cast<int64_t>(qi) * p.so.tok) +
+                             static_cast<int64_t>(h) * p.so.head;
       if (p.lse != nullptr)
         pr.lse_idx = thd ? static_cast<int64_t>(h) * p.T + w.seq_start + qi
                          : (static_cast<int64_t>(w.b) * p.Hq + h) * p.S + qi;

@@ -74,8 +74,10 @@ gptoss_status gptoss_selftest_wait_timeout(uint32_t limit_us, int32_t* result_de
 
 }  // extern "C"
 
-// the RoPE and prefill entry points
+// the RoPE and prefill entry points (self-attention and the block form)
 #include "fwd_host.cuh"
+// the log-sum-exp merge of key-block results
+#include "attn_merge.cuh"
 // the decode entry points (split-KV decode, paged cache, append, no-alloc)
 #include "decode_host.cuh"
 // the backward entry points

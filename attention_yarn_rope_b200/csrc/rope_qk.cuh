@@ -29,6 +29,7 @@ struct TokenMap {
   int nseq;                   // THD: number of sequences; BSHD: B
   int S;                      // BSHD sequence length
   int ntok;                   // B*S or T
+  int pos_offset;             // default positions: index in the sequence + pos_offset
 };
 
 // Token t -> (batch row or sequence, index inside it).
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_cons
     if (t < p.tm.ntok) {
       int seq, idx;
       token_coords(p.tm, t, seq, idx);
-      const int pos = p.tm.positions ? __ldg(p.tm.positions + t) : idx;
+      const int pos = p.tm.positions ? __ldg(p.tm.positions + t) : idx + p.tm.pos_offset;
       tab[tt][j] = rope_cs(pos, p.tab.inv_freq[j], p.tab.conc);
       if (p.cs_out != nullptr) p.cs_out[static_cast<int64_t>(t) * kPairs + j] = tab[tt][j];
       if (j == 0) {

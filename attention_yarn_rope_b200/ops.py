@@ -134,6 +134,60 @@ def gptoss_attn_fwd(q, k, v, sinks, window: int = 0, softmax_scale: float | None
     return (out, lse) if (return_lse or lse is not None) else out
 
 
+def gptoss_attn_fwd_block_workspace_size(B: int, Sq: int, Sk: int, Hkv: int, D: int = 64) -> int:
+    return int(_abi.load().gptoss_attn_fwd_block_workspace_size(int(B), int(Sq), int(Sk), int(Hkv), int(D)))
+
+
+def gptoss_attn_fwd_block(q, k, v, q_start: int, k_start: int, softmax_scale: float | None = None,
+                          rope: RopeConfig | None = None, out=None, lse=None, workspace=None, stream=None):
+    """One key block of a query shard (context parallelism, full context):
+    queries ``q [B,Sq,Hq,D]`` at global indices q_start.., keys / values
+    ``[B,Sk,Hkv,D]`` at k_start.. (k_start <= q_start), causal on the global
+    indices, no sink.  Returns ``(out fp32 [B,Sq,Hq,D], lse fp32 [B,Hq,Sq])``."""
+    lib = _abi.load()
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    if not (out.is_contiguous() and lse.is_contiguous()):
+        raise ValueError("out and lse must be contiguous")
+    if workspace is None:
+        need = gptoss_attn_fwd_block_workspace_size(B, Sq, Sk, Hkv, D)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check_dev(q, k, v, out, lse, workspace)
+    scale = float(D) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    r = rope.to_c() if rope is not None else None
+    st = lib.gptoss_attn_fwd_block(_ptr(q), _strides(q, False), _ptr(k), _strides(k, False), _ptr(v),
+                                   _strides(v, False), B, Sq, Sk, int(q_start), int(k_start), Hq, Hkv, D, scale,
+                                   ctypes.byref(r) if r is not None else None, _ptr(out), _ptr(lse),
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _abi.check("gptoss_attn_fwd_block", st)
+    return out, lse
+
+
+def gptoss_attn_merge(outs, lses, sinks, out=None, lse=None, stream=None):
+    """Merge block results of the same query rows and fold the sink in once:
+    ``outs [n,B,S,Hq,D]`` fp32, ``lses [n,B,Hq,S]`` fp32, ``sinks [Hq]`` fp32
+    (or None).  Returns ``out`` bf16 ``[B,S,Hq,D]`` or ``(out, lse)`` when
+    ``lse`` is given or requested with ``lse=True``."""
+    lib = _abi.load()
+    n, B, S, Hq, D = outs.shape
+    if not (outs.is_contiguous() and lses.is_contiguous()):
+        raise ValueError("outs and lses must be contiguous")
+    if out is None:
+        out = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, device=outs.device)
+    want_lse = lse is not None
+    if lse is True:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=outs.device)
+    _check_dev(outs, lses, sinks, out, lse if want_lse else None)
+    st = lib.gptoss_attn_merge(_ptr(outs), _ptr(lses), n, _ptr(sinks), B, S, Hq, D, _ptr(out), _strides(out, False),
+                               _ptr(lse) if want_lse else None, _stream(stream))
+    _abi.check("gptoss_attn_merge", st)
+    return (out, lse) if want_lse else out
+
+
 def gptoss_attn_bwd_workspace_size(total_tokens: int, Hq: int, Hkv: int, D: int = 64) -> int:
     return int(_abi.load().gptoss_attn_bwd_workspace_size(total_tokens, Hq, Hkv, D))
 

@@ -157,6 +157,47 @@ gptoss_status gptoss_attn_fwd(const void* q, gptoss_strides sq, const void* k, g
  * (total_tokens x 32 fp32 pairs).  0 when a size is out of range. */
 size_t gptoss_attn_fwd_workspace_size(int32_t total_tokens, int32_t Hkv, int32_t D);
 
+/* gptoss_attn_fwd_block -- one key block of a query shard, for context
+ * parallelism of the full-context layers (apply_rotary_emb_qk's cp_size /
+ * cp_rank on the rope_utils page): the prefill over queries at global token
+ * indices [q_start, q_start + Sq) against the keys at [k_start, k_start + Sk)
+ * of the same sequences, causal on the global indices (key j visible from
+ * query i iff k_start + j <= q_start + i), with NO sink.  Each row's output is
+ * normalised over the block's visible keys and lse is their log-sum-exp;
+ * gptoss_attn_merge folds the blocks and the sink together.
+ *   q [B,Sq,Hq,D], k and v [B,Sk,Hkv,D], bf16, BSHD strides (raw: rope !=
+ *          NULL rotates them at their global positions q_start + i and
+ *          k_start + j; rope == NULL takes them as rotated).  Both products
+ *          take fp16 operands, as in gptoss_attn_fwd.
+ *   k_start <= q_start (a block after the shard is invisible; skip it), so
+ *          every query row sees at least one key of the block.
+ *   out    fp32, dense [B,Sq,Hq,D] (kept in fp32 for the merge).
+ *   lse    fp32, dense [B,Hq,Sq], natural log, no sink.
+ *   workspace  device memory of gptoss_attn_fwd_block_workspace_size(B, Sq,
+ *          Sk, Hkv, D) bytes, 16-byte aligned (fp16 k and v of the block,
+ *          the queries' angle table); contents need not be initialised.
+ *   k_start > q_start or a bad size, pointer or stride: INVALID_ARG. */
+gptoss_status gptoss_attn_fwd_block(const void* q, gptoss_strides sq, const void* k, gptoss_strides sk,
+                                    const void* v, gptoss_strides sv, int32_t B, int32_t Sq, int32_t Sk,
+                                    int32_t q_start, int32_t k_start, int32_t Hq, int32_t Hkv, int32_t D,
+                                    float softmax_scale, const gptoss_rope_params* rope, float* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Workspace bytes for gptoss_attn_fwd_block (0 when a size is out of range). */
+size_t gptoss_attn_fwd_block_workspace_size(int32_t B, int32_t Sq, int32_t Sk, int32_t Hkv, int32_t D);
+
+/* gptoss_attn_merge -- the sink attention over the union of n_blocks key
+ * blocks from their gptoss_attn_fwd_block results (same query rows):
+ *   Z = exp(sink_h) + sum_b exp(lse_b),  out = sum_b exp(lse_b) out_b / Z,
+ *   lse = log Z; the sink enters once, here (sinks NULL: no sink).
+ *   outs   fp32 [n_blocks][B][S][Hq][D] dense (16-byte aligned).
+ *   lses   fp32 [n_blocks][B][Hq][S]; a block a row sees no key of has -inf.
+ *   out    bf16 [B,S,Hq,D] with BSHD strides so (8-byte aligned); lse
+ *          nullable fp32 [B,Hq,S]. */
+gptoss_status gptoss_attn_merge(const float* outs, const float* lses, int32_t n_blocks, const float* sinks,
+                                int32_t B, int32_t S, int32_t Hq, int32_t D, void* out, gptoss_strides so,
+                                float* lse, struct CUstream_st* stream);
+
 /* Workspace bytes gptoss_attn_bwd needs: q and k rotated once (fp16), every
  * token's 32 RoPE angles, and <dout, out> per row and head (fp32).  0 when a
  * size is out of range. */
