@@ -11,6 +11,8 @@ import ctypes
 import os
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptoss_attn.so")
+# the same library built with in-kernel range checks (GPTOSS_DEBUG_CHECKS)
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptoss_attn_debug.so")
 
 GPTOSS_OK = 0
 GPTOSS_ERR_INVALID_ARG = 1
@@ -104,21 +106,30 @@ _SIGNATURES = {
 _lib = None
 
 
+def _open(path: str) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{os.path.basename(path)} not found at {path}; build it with "
+            "`python -m attention_yarn_rope_b200.build_lib` (there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
 def load() -> ctypes.CDLL:
     """Load the in-tree library once.  Raises if it has not been built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise RuntimeError(
-                f"libgptoss_attn.so not found at {LIB_PATH}; build it with "
-                "`python -m attention_yarn_rope_b200.build_lib` (there is no CPU fallback)")
-        lib = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in _SIGNATURES.items():
-            fn = getattr(lib, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = lib
+        _lib = _open(LIB_PATH)
     return _lib
+
+
+def load_debug() -> ctypes.CDLL:
+    """The range-checking build (``build_lib --debug-checks``), loaded on its own."""
+    return _open(DEBUG_LIB_PATH)
 
 
 class GptossError(RuntimeError):

@@ -89,6 +89,12 @@ __device__ __forceinline__ BwdSeq bwd_seq(const BwdParams& p, int b) {
     const int a = __ldg(p.cu_seqlens + b);
     s.tok0 = a;
     s.L = __ldg(p.cu_seqlens + b + 1) - a;
+    // cu_seqlens: nondecreasing, within the T tokens, no sequence longer than
+    // S; a bad entry makes the sequence empty (skipped)
+    if (!index_ok(a >= 0 && s.L >= 0 && a + s.L <= p.T && s.L <= p.S)) {
+      s.tok0 = 0;
+      s.L = 0;
+    }
   } else {
     s.tok0 = static_cast<int64_t>(b) * p.S;
     s.L = p.S;

@@ -120,6 +120,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int g = blockIdx.x, split = blockIdx.y;
   const DecodeRows cr = decode_rows(p, blockIdx.z);
+  // cache_seqlens[b]: the q_len new tokens fit in the cache, 1 <= len <= Lmax
+  // (a failed check leaves this CTA's rows and partials unwritten)
+  if (!index_ok(cr.n_first >= 1 && cr.n_first + p.q_len - 1 - cr.tok0 <= p.Lmax)) return;
   const int b = cr.b;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G;
@@ -424,6 +427,7 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_con
   const int g = blockIdx.x, vb = blockIdx.y;  // virtual sequence (cache row, query token)
   const int b = vb / p.q_len, tok = vb - b * p.q_len;
   const DecodeRows cr = decode_rows(p, b * p.n_slices + tok / p.tpc);
+  if (!index_ok(cr.n_first >= 1 && cr.n_first + p.q_len - 1 - cr.tok0 <= p.Lmax)) return;
   const int n_last = cr.n_first + cr.ntok - 1;
   const int nsp = min(p.nsplit, (n_last - cr.lo_first + p.chunk - 1) / p.chunk);
   const int G = p.G;
@@ -469,7 +473,6 @@ struct AppendParams {
   RopeTable tab;
 };
 
-constexpr int kStatusBadIndex = 1;  // == GPTOSS_ERR_INVALID_ARG
 
 __global__ void kv_append_paged_kernel(const __grid_constant__ AppendParams p) {
   const int b = blockIdx.x, tok = blockIdx.y;

@@ -103,6 +103,9 @@ __device__ __forceinline__ bool make_unit(const FwdParams& p, int u, Unit& w) {
   const bool thd = p.cu_seqlens != nullptr;
   w.seq_start = thd ? __ldg(p.cu_seqlens + w.b) : 0;
   w.L = thd ? __ldg(p.cu_seqlens + w.b + 1) - w.seq_start : p.S;
+  // cu_seqlens: nondecreasing, within the T tokens, no sequence longer than S
+  // (every role decodes the same unit, so all skip a bad one together)
+  if (thd && !index_ok(w.seq_start >= 0 && w.L >= 0 && w.seq_start + w.L <= p.T && w.L <= p.S)) return false;
   w.Lk = thd ? w.L : p.Lk;
   w.q0 = qt * kFwdTile;
   if (w.q0 >= w.L) return false;

@@ -264,7 +264,9 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
     pr.sink = sink;
     pr.out_row = -1;
     pr.lse_idx = -1;
-    if (qi < w.L && !(X == 1 && w.dup)) {
+    // the row's logical coordinates (token, head) lie inside the call's tensors
+    if (qi < w.L && !(X == 1 && w.dup) &&
+        index_ok(h < p.Hq && (thd ? w.seq_start + qi < p.T : (w.b < p.B && qi < p.S)))) {
       pr.out_row = p.out_f32 != nullptr
                        ? ((static_cast<int64_t>(w.b) * p.S + qi) * p.Hq + h) * kHeadDim
                        : (thd ? static_cast<int64_t>(w.seq_start + qi) * p.so.tok

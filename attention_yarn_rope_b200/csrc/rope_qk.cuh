@@ -45,6 +45,8 @@ __device__ __forceinline__ void token_coords(const TokenMap& m, int t, int& seq,
     }
     seq = lo;
     idx = t - __ldg(m.cu_seqlens + lo);
+    // cu_seqlens nondecreasing around t: cu[lo] <= t < cu[lo + 1]
+    if (!index_ok(idx >= 0 && (lo + 1 > m.nseq || t < __ldg(m.cu_seqlens + lo + 1)))) idx = 0;
   }
 }
 

@@ -27,6 +27,25 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ void record_timeout() { atomicExch(&g_device_status, kStatusTimeout); }
 
+// Range checks of computed indices (the GPTOSS_DEBUG_CHECKS build).  A check
+// that fails records GPTOSS_ERR_INVALID_ARG in the device status word and its
+// caller skips the access; it never traps.  Release builds trust the indices
+// and the checks compile away.
+#ifdef GPTOSS_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+constexpr int kStatusBadIndex = 1;  // == GPTOSS_ERR_INVALID_ARG
+
+__device__ __forceinline__ bool index_ok(bool ok) {
+  if (kDebugChecks && !ok) {
+    atomicExch(&g_device_status, kStatusBadIndex);
+    return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
