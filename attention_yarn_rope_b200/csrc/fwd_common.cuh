@@ -39,7 +39,9 @@ constexpr int kFwdThreads = 512;
 constexpr int kFwdLaunchRegs = 128;   // 65536 / 512
 constexpr int kFwdTileBytes = kFwdTile * kHeadDim * 2;  // 16 KB
 constexpr uint32_t kFwdTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// A row's base moves when a tile's maximum exceeds it by more than this (log2
+// units): P = 2^(s - base) then stays at or below 2^15, inside fp16's range.
+constexpr float kRescaleThreshold = 15.0f;
 constexpr uint32_t kRegsSoftmax = 208, kRegsRope = 48, kRegsOther = 48;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsRope + 128 * kRegsOther == kFwdThreads * kFwdLaunchRegs,
               "register split must add up to the launch allocation");

@@ -13,8 +13,9 @@
 // own rounding.
 //
 // The base.  A row's first visible tile sets m to its maximum, so that tile's
-// largest P is exactly 1 (and the row sum stays >= 1 from then on).  Later
-// tiles reuse m as it stands and skip the row maximum: any base gives the
+// largest P is exactly 1 (and the row sum stays >= 1 from then on); while the
+// row has seen fewer than 64 keys it also takes later tiles' maxima.  After
+// that, tiles reuse m as it stands and skip the row maximum: any base gives the
 // same O / l, and fp16 P (down to its subnormals, far below 1 / l) and fp32
 // sums keep their precision at any scale the range allows.  The only risk
 // is range: fp16 ends at 65504, so the tile's sum is checked afterwards --
@@ -69,9 +70,14 @@ __device__ __forceinline__ void load_masked_s(uint32_t taddr, const int (&cls)[4
   for (int c = 0; c < 4; ++c) {
     if (cls[c] == 1) {  // warp-uniform branch
       const int lo_c = c_lo - 32 * c, hi_c = c_hi - 32 * c;
+      // this row's visible columns of the chunk, [lo_c, hi_c], as a bit mask:
+      // one bit test and select per element (measured: 9 % faster on the
+      // sliding window than comparing each column with both bounds)
+      const uint32_t upto = hi_c >= 31 ? 0xffffffffu : (hi_c < 0 ? 0u : (2u << hi_c) - 1u);
+      const uint32_t from = lo_c <= 0 ? 0xffffffffu : (lo_c > 31 ? 0u : ~((1u << lo_c) - 1u));
+      const uint32_t vis = upto & from;
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (e > hi_c || e < lo_c) sr[c][e] = __float_as_uint(-INFINITY);
+      for (int e = 0; e < 32; ++e) sr[c][e] = (vis & (1u << e)) ? sr[c][e] : __float_as_uint(-INFINITY);
     }
   }
 }
@@ -172,6 +178,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
     const float sink = p.sinks != nullptr ? __ldg(p.sinks + h) * kLog2e : -INFINITY;
     float m_run = -INFINITY;
     float l_run = 0.f;
+    int n_seen = 0;  // visible keys this row's base has seen so far
     for (int j = 0; j < w.n_kt; ++j, ++t) {
       const int k0 = (w.j_lo + j) * kFwdTile;
       if (!mbar_wait_warp(&sm.s_full[X], t & 1, p.wait_ns)) return;
@@ -191,54 +198,62 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
       mbar_arrive(&sm.s_free[X]);
       float alpha = 1.f;
       bool rescale = false;
-      // a row without a base yet takes its maximum (the whole warp does, so the
-      // branch stays uniform; rows that have a base keep it unless it grows by 2^8)
-      if (__any_sync(0xffffffffu, m_run == -INFINITY)) {
-        const float m_cand = tile_max(sr, cls) * sl;
-        if (m_cand > m_run + kRescaleThreshold) {
-          alpha = ex2_approx(m_run - m_cand);  // 0 when m_run is -inf
-          m_run = m_cand;
-          rescale = true;
+      // A row whose base rests on few keys (none yet, or fewer than 64) takes
+      // this tile's maximum -- the whole warp does, so the branch stays
+      // uniform.  With the maximum known, every P of the tile is at most
+      // 2^(max - base), so the base moves (the lazy O rescale) only when that
+      // would leave the fp16 range, and the tile needs no range check after
+      // its exponentials.  In the sliding window every unit starts with rows
+      // that see a handful of keys in their first tile; moving their base at
+      // every larger maximum, or redoing tiles whose sum passes 2^15, cost a
+      // quarter of the kernel.  Once a row has seen 64 keys its base stands
+      // and later tiles skip the maximum.
+      const int gi = qi + p.delta;  // this row's visible keys in the tile: [v_lo, v_hi]
+      const int v_hi = min(min(gi, w.Lk - 1), k0 + kFwdTile - 1);
+      const int v_lo = max(k0, p.window > 0 ? gi - p.window + 1 : k0);
+      const bool young = n_seen < 64;
+      n_seen += max(0, v_hi - v_lo + 1);
+      // One copy of the maximum and of the exponentials, in a rolled loop of at
+      // most two passes: the hot loop must fit the instruction cache (with a
+      // second, unrolled copy for the cold redo the warps stalled on
+      // instruction fetch).  A pass that takes the maximum needs no range
+      // check; a pass that fails the check takes the maximum and runs again
+      // only if some row's base moved.
+      bool max_pass = __any_sync(0xffffffffu, young);
+      bool waited = t == 0;  // P(t) overwrites P(t-1): the previous P V must have completed
+      float rs = 0.f;
+      for (int pass = 0;; ++pass) {
+        if (max_pass) {
+          const float m_cand = tile_max(sr, cls) * sl;
+          const bool moved = m_cand > m_run + kRescaleThreshold;
+          if (moved) {
+            alpha *= ex2_approx(m_run - m_cand);  // 0 when m_run is -inf
+            m_run = m_cand;
+            rescale = true;
+          }
+          if (pass > 0 && !__any_sync(0xffffffffu, moved)) break;  // the first pass's P stand
         }
-      }
-      float nb = m_run == -INFINITY ? 0.f : -m_run;
-      float rs0 = 0.f, rs1 = 0.f;
-      {
+        const float nb = m_run == -INFINITY ? 0.f : -m_run;
+        float rs0 = 0.f, rs1 = 0.f;
         uint32_t pk[32];
         exp_half(sr, cls, 0, sl, nb, rs0, rs1, pk);
-        // P(t) overwrites P(t-1): the previous P V product must have completed
-        if (t > 0) {
+        if (!waited) {
           if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
           tc_fence_after();
+          waited = true;
         }
         tmem_st32(lane_base + colP, pk);
         exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
         tmem_st32(lane_base + colP + 32, pk);
+        rs = rs0 + rs1;
+        if (max_pass || !__any_sync(0xffffffffu, !(rs <= kMaxTileSum))) break;
+        max_pass = true;
       }
       // the previous unit's rows: its last P V has completed (waited above),
       // and this unit's first P V, which restarts O, waits for p_full below
       if (j == 0 && pending) {
         fwd_epilogue_row(p, lane_base + colO, pr);
         pending = false;
-      }
-      float rs = rs0 + rs1;
-      if (__any_sync(0xffffffffu, !(rs <= kMaxTileSum))) {
-        // cold: rebase on the tile maximum and redo both halves (P(t) is not
-        // consumed before p_full, so overwriting it is safe)
-        const float m_new = fmaxf(m_run, tile_max(sr, cls) * sl);
-        if (m_new > m_run) {
-          alpha *= ex2_approx(m_run - m_new);
-          m_run = m_new;
-          rescale = true;
-        }
-        nb = m_run == -INFINITY ? 0.f : -m_run;
-        rs0 = rs1 = 0.f;
-        uint32_t pk[32];
-        exp_half(sr, cls, 0, sl, nb, rs0, rs1, pk);
-        tmem_st32(lane_base + colP, pk);
-        exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
-        tmem_st32(lane_base + colP + 32, pk);
-        rs = rs0 + rs1;
       }
       // warp-collective TMEM access: the whole warp rescales O when any row
       // needs it (alpha is 1 for the rows that do not)
