@@ -105,13 +105,16 @@ static gptoss_status prefill_launch(const PrefillCall& c) {
   if (n_units > INT32_MAX) return GPTOSS_ERR_UNSUPPORTED;
   // The register split inside the kernel assumes exactly kFwdLaunchRegs
   // registers per thread at launch; anything else could stall the split.
-  static int launch_regs = -1;
-  if (launch_regs < 0) {
+  // two instantiations: with a sliding window, and causal only
+  const auto kernel = c.window > 0 ? attn_fwd_kernel<true> : attn_fwd_kernel<false>;
+  static int launch_regs[2] = {-1, -1};
+  int& regs = launch_regs[c.window > 0 ? 1 : 0];
+  if (regs < 0) {
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel) != cudaSuccess) return GPTOSS_ERR_CUDA;
-    launch_regs = fa.numRegs;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return GPTOSS_ERR_CUDA;
+    regs = fa.numRegs;
   }
-  if (launch_regs != kFwdLaunchRegs) return GPTOSS_ERR_UNSUPPORTED;
+  if (regs != kFwdLaunchRegs) return GPTOSS_ERR_UNSUPPORTED;
   int device = 0, n_sm = 0;
   if (cudaGetDevice(&device) != cudaSuccess ||
       cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
@@ -207,10 +210,10 @@ static gptoss_status prefill_launch(const PrefillCall& c) {
   }
   p.cs_tab = q_table;
   const size_t smem = sizeof(FwdSmem) + 1024;
-  if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return GPTOSS_ERR_CUDA;
-  attn_fwd_kernel<<<grid, kFwdThreads, smem, c.stream>>>(p);
+  kernel<<<grid, kFwdThreads, smem, c.stream>>>(p);
   return check_launch();
 }
 

@@ -151,6 +151,7 @@ __device__ __forceinline__ void fwd_mma_pv_role(const FwdParams& p, FwdSmem& sm,
 }
 
 // ================================== kernel ==================================
+template <bool kWindow>
 __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_constant__ FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   FwdSmem& sm = *reinterpret_cast<FwdSmem*>(
@@ -191,7 +192,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   // rotation finishes sooner there, next to two busy softmax warpgroups)
   if (wg == 1 || wg == 2) {
     reg_alloc<kRegsSoftmax>();
-    fwd_softmax_role(p, sm, tmem, wg - 1);
+    fwd_softmax_role<kWindow>(p, sm, tmem, wg - 1);
   } else if (wg == 0) {
     reg_dealloc<kRegsRope>();
     fwd_rope_role(p, sm);

@@ -41,12 +41,14 @@ struct RopeLane {
 // (row_cs != nullptr and per_row) row r's 32 (c cos, c sin) pairs are read at
 // row_cs[16 r .. 16 r + 15] as float4.  Rows at or past n_valid (beyond the
 // sequence) are only converted to fp16: their scores are masked, but their
-// bits must be fp16 numbers, not bf16 ones read as fp16.  (Measured: rotating
-// row by row in a 4-way unrolled loop beats loading all 32 words up front.)
+// bits must be fp16 numbers, not bf16 ones read as fp16.  (Measured: a rolled
+// loop, row by row, beats 4-way unrolling by 5 % on the sliding window -- the
+// softmax warps' code shares the instruction cache -- and beats loading all
+// 32 words up front.)
 __device__ __forceinline__ void rotate_q_pair(const RopeLane& rl, uint8_t* ta, uint8_t* tb, float2 c0, float2 c1,
                                               int n_valid, bool per_row, const float4* row_cs, int pb) {
   const float2 one = make_float2(1.f, 0.f);
-#pragma unroll 4
+#pragma unroll 1
   for (int kk = 0; kk < 16; ++kk) {
     const int r = rl.ro + 8 * kk;
     float2 a0 = one, a1 = one;

@@ -58,26 +58,33 @@ __device__ __forceinline__ float tile_max(const uint32_t (&sr)[4][32], const int
 // Reads this warp's 32 rows x 128 scores of S from TMEM and sets the hidden
 // elements of partly visible chunks to -inf (row qi, at key index gi =
 // qi + delta, sees keys [gi - window + 1, min(gi, Lk - 1)]; k0 is the tile's
-// first key).
+// first key).  kWindow = false: no window, only the causal bound.
+template <bool kWindow>
 __device__ __forceinline__ void load_masked_s(uint32_t taddr, const int (&cls)[4], int gi, int k0, int Lk,
                                               int window, uint32_t (&sr)[4][32]) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, sr[c]);
   tmem_wait_ld();
   const int c_hi = min(gi, Lk - 1) - k0;  // visible columns of this row: [c_lo, c_hi]
-  const int c_lo = window > 0 ? gi - window + 1 - k0 : -1;
+  const int c_lo = kWindow ? gi - window + 1 - k0 : -1;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
     if (cls[c] == 1) {  // warp-uniform branch
       const int lo_c = c_lo - 32 * c, hi_c = c_hi - 32 * c;
-      // this row's visible columns of the chunk, [lo_c, hi_c], as a bit mask:
-      // one bit test and select per element (measured: 9 % faster on the
-      // sliding window than comparing each column with both bounds)
-      const uint32_t upto = hi_c >= 31 ? 0xffffffffu : (hi_c < 0 ? 0u : (2u << hi_c) - 1u);
-      const uint32_t from = lo_c <= 0 ? 0xffffffffu : (lo_c > 31 ? 0u : ~((1u << lo_c) - 1u));
-      const uint32_t vis = upto & from;
+      if (kWindow) {
+        // this row's visible columns of the chunk, [lo_c, hi_c], as a bit
+        // mask: one bit test and select per element (measured: 9 % faster on
+        // the sliding window than comparing each column with both bounds)
+        const uint32_t upto = hi_c >= 31 ? 0xffffffffu : (hi_c < 0 ? 0u : (2u << hi_c) - 1u);
+        const uint32_t from = lo_c <= 0 ? 0xffffffffu : (lo_c > 31 ? 0u : ~((1u << lo_c) - 1u));
+        const uint32_t vis = upto & from;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) sr[c][e] = (vis & (1u << e)) ? sr[c][e] : __float_as_uint(-INFINITY);
+        for (int e = 0; e < 32; ++e) sr[c][e] = (vis & (1u << e)) ? sr[c][e] : __float_as_uint(-INFINITY);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (e > hi_c) sr[c][e] = __float_as_uint(-INFINITY);
+      }
     }
   }
 }
@@ -158,7 +165,11 @@ __device__ __forceinline__ void fwd_epilogue_row(const FwdParams& p, uint32_t o_
   if (pr.out_row >= 0 && pr.lse_idx >= 0) p.lse[pr.lse_idx] = (M + log2f(l_fin)) * kLn2;
 }
 
+// kWindow: the call has a sliding window (window > 0); false compiles the
+// causal-only masks (a smaller loop for the full-context layers).
+template <bool kWindow>
 __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem, int X) {
+  const int window = kWindow ? p.window : 0;
   const int wq = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quarter
   const int r = threadIdx.x & 127;        // query row of the tile
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
@@ -188,12 +199,12 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int kl = k0 + 32 * c, kh = kl + 31;
-        const bool hidden = kl > min(qw_hi, w.Lk - 1) || (p.window > 0 && kh < qw_lo - p.window + 1);
-        const bool full = kh <= qw_lo && kh <= w.Lk - 1 && (p.window == 0 || kl >= qw_hi - p.window + 1);
+        const bool hidden = kl > min(qw_hi, w.Lk - 1) || (window > 0 && kh < qw_lo - window + 1);
+        const bool full = kh <= qw_lo && kh <= w.Lk - 1 && (window == 0 || kl >= qw_hi - window + 1);
         cls[c] = hidden ? 0 : (full ? 2 : 1);
       }
       uint32_t sr[4][32];
-      load_masked_s(lane_base + colS, cls, qi + p.delta, k0, w.Lk, p.window, sr);
+      load_masked_s<kWindow>(lane_base + colS, cls, qi + p.delta, k0, w.Lk, window, sr);
       tc_fence_before();
       mbar_arrive(&sm.s_free[X]);
       float alpha = 1.f;
@@ -210,7 +221,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
       // and later tiles skip the maximum.
       const int gi = qi + p.delta;  // this row's visible keys in the tile: [v_lo, v_hi]
       const int v_hi = min(min(gi, w.Lk - 1), k0 + kFwdTile - 1);
-      const int v_lo = max(k0, p.window > 0 ? gi - p.window + 1 : k0);
+      const int v_lo = max(k0, window > 0 ? gi - window + 1 : k0);
       const bool young = n_seen < 64;
       n_seen += max(0, v_hi - v_lo + 1);
       // One copy of the maximum and of the exponentials, in a rolled loop of at
