@@ -33,7 +33,7 @@
 namespace gptoss {
 
 constexpr int kFwdTile = 128;         // query rows and keys per tile
-constexpr int kFwdStages = 4;         // K / V ring
+constexpr int kFwdStages = 3;         // K / V ring (measured: 3 stages beat 4 by 2-4 %)
 constexpr int kFwdQStages = 3;        // Q ring (units)
 constexpr int kFwdThreads = 512;
 constexpr int kFwdLaunchRegs = 128;   // 65536 / 512
