@@ -417,7 +417,9 @@ def run_ours(args, torch, dist, rank, world, device):
 
 
 def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, args, bwd_cfgs=()):
-    res = {}
+    # the denominators of every frac_of_* below: MEASURED_PEAKS.json when the
+    # file is present ("measured"), else the pool's earlier figures ("fallback")
+    res = {"peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"], "source": peaks["source"]}}
     reps = max(3, min(args.steps, 20))
     for cfg in prefill_cfgs:
         case = prefill_case(torch, ops, cfg, device)
@@ -427,9 +429,9 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
         ms = timed_steps(torch, case["step"], reps, stream) / reps
         tf = case["flops"] / (ms * 1e-3) / 1e12
         gbs = case["bytes"] / (ms * 1e-3) / 1e9
-        res[cfg.name] = {"ms": round(ms, 4), "tflops": round(tf, 2), "frac_of_measured_bf16": round(
+        res[cfg.name] = {"ms": round(ms, 4), "tflops": round(tf, 2), "frac_of_bf16_peak": round(
             tf / peaks["bf16_tflops"], 4), "frac_of_2250_spec": round(tf / 2250.0, 4), "gbs": round(gbs, 1),
-            "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "visible_pairs": case["pairs"],
+            "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4), "visible_pairs": case["pairs"],
             "flops": case["flops"], "bytes": case["bytes"], "launches_per_call": 2}
         del case
         torch.cuda.empty_cache()
@@ -443,7 +445,7 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
         ms = timed_steps(torch, case["step"], reps, stream) / reps
         tf = case["flops"] / (ms * 1e-3) / 1e12
         res["bwd_" + cfg.name] = {"ms": round(ms, 4), "tflops": round(tf, 2),
-                                  "frac_of_measured_bf16": round(tf / peaks["bf16_tflops"], 4),
+                                  "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4),
                                   "gbs_io": round(case["bytes"] / (ms * 1e-3) / 1e9, 1), "flops": case["flops"],
                                   "io_bytes": case["bytes"], "launches_per_call": "4 (5 with split sweeps)",
                                   "note": "dK / dV on tcgen05 (TMEM); dQ on tcgen05 for long sweeps, mma.sync for short ones"}
@@ -460,7 +462,7 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
                          flush=(lambda: flush_buf.fill_(1)) if small else None) / reps
         gbs = case["bytes"] / (ms * 1e-3) / 1e9
         res[cfg.name] = {"ms": round(ms, 4), "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
-                         "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": case["kv_bytes"],
+                         "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": case["kv_bytes"],
                          "l2": "flushed between calls" if small else "cache > L2",
                          "launches_per_call": 1 if cfg.window and cfg.window <= 256 else 2}
         if cfg.window and cfg.window * 100 < cfg.L:
@@ -496,7 +498,7 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
         gbs = case["bytes"] / (ms * 1e-3) / 1e9
         res[f"decode_paged_b{cfg.B}_l{cfg.L}_bs{bs}_full"] = {
             "ms": round(ms, 4), "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
-            "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": case["kv_bytes"],
+            "frac_of_hbm_peak": round(gbs / peaks["hbm_gbs"], 4), "kv_bytes": case["kv_bytes"],
             "block_size": bs, "table": f"random permutation of the {nblk} blocks", "launches_per_call": 2}
         # four new tokens per sequence (draft tokens checked in one call): the
         # four share each CTA's pass over the cache (32 query rows per kv head)
@@ -546,6 +548,7 @@ _KERNEL_SOURCES = {
     "attn_fwd_kernel": ("fwd_pipeline.cuh", "fwd_host.cuh"),
     "rope_qk_kernel<true>": ("rope_qk.cuh", "fwd_host.cuh"),
     "attn_decode_split_kernel": ("attn_decode.cuh", "decode_host.cuh"),
+    "attn_bwd_dkdv_tc_kernel": ("attn_bwd_tc.cuh", "bwd_host.cuh"),
 }
 
 
