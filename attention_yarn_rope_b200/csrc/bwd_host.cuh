@@ -104,6 +104,7 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   rp.tm.ntok = total_tokens;
   rp.Hq = Hq;
   rp.Hkv = Hkv;
+  rp.D = kHeadDim;
   if (rope != nullptr) {
     yarn_table(*rope, &rp.tab);
   } else {

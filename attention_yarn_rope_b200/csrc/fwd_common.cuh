@@ -91,6 +91,9 @@ struct Unit {
 
 // Unit u of the static list (heaviest query tiles first).  Returns false for
 // a tile past the end of its packed sequence; every role skips the same units.
+// kPair: a unit holds two heads of a group (p.HP = ceil(G / 2) pairs);
+// otherwise one (p.HP = G), h1 = h0 and nothing is duplicated.
+template <bool kPair = true>
 __device__ __forceinline__ bool make_unit(const FwdParams& p, int u, Unit& w) {
   const int per_tile = p.B * p.Hkv * p.HP;
   const int qt = p.n_qtiles - 1 - u / per_tile;
@@ -99,9 +102,14 @@ __device__ __forceinline__ bool make_unit(const FwdParams& p, int u, Unit& w) {
   rest /= p.HP;
   w.g = rest % p.Hkv;
   w.b = rest / p.Hkv;
-  w.h0 = w.g * p.G + 2 * hp;
-  w.dup = (2 * hp + 1) >= p.G;
-  w.h1 = w.dup ? w.h0 : w.h0 + 1;
+  if (kPair) {
+    w.h0 = w.g * p.G + 2 * hp;
+    w.dup = (2 * hp + 1) >= p.G;
+    w.h1 = w.dup ? w.h0 : w.h0 + 1;
+  } else {
+    w.h0 = w.h1 = w.g * p.G + hp;
+    w.dup = false;
+  }
   const bool thd = p.cu_seqlens != nullptr;
   w.seq_start = thd ? __ldg(p.cu_seqlens + w.b) : 0;
   w.L = thd ? __ldg(p.cu_seqlens + w.b + 1) - w.seq_start : p.S;

@@ -126,14 +126,16 @@ struct PendingRow {
 // (out_row indexes p.out with its strides, or the dense fp32 p.out_f32.)
 
 // O / l with the sink folded once (M = max(m, sink), l' = l 2^(m - M) +
-// 2^(sink - M)), in bf16, and LSE = (M + log2 l') ln 2.  O must be complete.
+// 2^(sink - M)), in bf16, and LSE = (M + log2 l') ln 2.  O (kD columns) must
+// be complete.
+template <int kD>
 __device__ __forceinline__ void fwd_epilogue_row(const FwdParams& p, uint32_t o_addr, const PendingRow& pr) {
   const float M = fmaxf(pr.m, pr.sink);
   const float a = pr.m == -INFINITY ? 0.f : ex2_approx(pr.m - M);
   const float l_fin = pr.l * a + (pr.sink == -INFINITY ? 0.f : ex2_approx(pr.sink - M));
   const float inv = a / l_fin;
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
+  for (int c = 0; c < kD / 32; ++c) {
     uint32_t ov[32];
     tmem_ld32(o_addr + c * 32, ov);
     tmem_wait_ld();
@@ -166,9 +168,12 @@ __device__ __forceinline__ void fwd_epilogue_row(const FwdParams& p, uint32_t o_
 }
 
 // kWindow: the call has a sliding window (window > 0); false compiles the
-// causal-only masks (a smaller loop for the full-context layers).
-template <bool kWindow>
-__device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem, int X) {
+// causal-only masks (a smaller loop for the full-context layers).  kD: head
+// size, the width of O (64: two head slots per CTA, O_X at X * 256 + 192;
+// 128: one slot, O at 192 .. 319).  Smem: the kernel's shared-memory layout
+// (its s_full / s_free / p_full / o_done barriers per head slot).
+template <bool kWindow, int kD = kHeadDim, typename Smem = FwdSmem>
+__device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, Smem& sm, uint32_t tmem, int X) {
   const int window = kWindow ? p.window : 0;
   const int wq = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quarter
   const int r = threadIdx.x & 127;        // query row of the tile
@@ -181,7 +186,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
   PendingRow pr;
   for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
     Unit w;
-    if (!make_unit(p, u, w)) continue;
+    if (!make_unit<kD == kHeadDim>(p, u, w)) continue;
     const int h = X == 0 ? w.h0 : w.h1;
     const int qi = w.q0 + r;
     // rows of this warp, as key indices (query row i sits at key index i + delta)
@@ -263,14 +268,14 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
       // the previous unit's rows: its last P V has completed (waited above),
       // and this unit's first P V, which restarts O, waits for p_full below
       if (j == 0 && pending) {
-        fwd_epilogue_row(p, lane_base + colO, pr);
+        fwd_epilogue_row<kD>(p, lane_base + colO, pr);
         pending = false;
       }
       // warp-collective TMEM access: the whole warp rescales O when any row
       // needs it (alpha is 1 for the rows that do not)
       if (__any_sync(0xffffffffu, rescale && j > 0)) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < kD / 32; ++c) {
           uint32_t ov[32];
           tmem_ld32(lane_base + colO + c * 32, ov);
           tmem_wait_ld();
@@ -294,7 +299,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
     if (qi < w.L && !(X == 1 && w.dup) &&
         index_ok(h < p.Hq && (thd ? w.seq_start + qi < p.T : (w.b < p.B && qi < p.S)))) {
       pr.out_row = p.out_f32 != nullptr
-                       ? ((static_cast<int64_t>(w.b) * p.S + qi) * p.Hq + h) * kHeadDim
+                       ? ((static_cast<int64_t>(w.b) * p.S + qi) * p.Hq + h) * kD
                        : (thd ? static_cast<int64_t>(w.seq_start + qi) * p.so.tok
                               : static_cast<int64_t>(w.b) * p.so.batch + static_cast<int64_t>(qi) * p.so.tok) +
                              static_cast<int64_t>(h) * p.so.head;
@@ -307,7 +312,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, FwdSmem& sm
   if (pending) {  // the last unit: wait for its last P V product
     if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
     tc_fence_after();
-    fwd_epilogue_row(p, lane_base + colO, pr);
+    fwd_epilogue_row<kD>(p, lane_base + colO, pr);
   }
   tc_fence_before();
 }

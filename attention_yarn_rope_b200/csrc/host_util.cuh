@@ -15,13 +15,16 @@ namespace gptoss {
 
 constexpr int kHeadDim = 64;
 constexpr int kPairs = kHeadDim / 2;
+// the larger head size some entry points also take (RoPE, prefill, decode)
+constexpr int kMaxHeadDim = 128;
+constexpr int kMaxPairs = kMaxHeadDim / 2;
 constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
 constexpr float kLn2 = 0.6931471805599453f;     // ln(2)
 
 // Per-launch rotary table: inverse frequencies in double plus the
-// concentration.  Passed to kernels by value (268 bytes).
+// concentration.  Passed to kernels by value (524 bytes).
 struct RopeTable {
-  double inv_freq[kPairs];
+  double inv_freq[kMaxPairs];
   float conc;
   int enabled;  // 0: inputs already rotated, nothing to do
   int R;        // rotary pairs, rotary_dim / 2: features [0, 2R) rotate in pairs (j, j + R), the rest pass through
@@ -38,7 +41,7 @@ inline void yarn_table(const gptoss_rope_params& rp, RopeTable* t) {
   const int rdim = rp.rotary_dim;
   const int half = rdim / 2;
   const double two_pi = 6.283185307179586476925286766559;
-  for (int j = 0; j < kPairs; ++j) t->inv_freq[j] = 0.0;
+  for (int j = 0; j < kMaxPairs; ++j) t->inv_freq[j] = 0.0;
   t->R = half;
   const double lnb = log(rp.base);
   if (rp.factor <= 1.0) {

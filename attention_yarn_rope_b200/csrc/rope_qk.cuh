@@ -15,7 +15,8 @@
 // partner chunk c + R/8 (features [R+8c, R+8c+8)): 8 complete pairs; a
 // pass-through item copies one chunk past 2R.  R = 32 (GPT-OSS) gives 4
 // rotation items per head: a warp covers 8 heads x 4 items of one token, so
-// its two loads fill whole 128-byte lines.
+// its two loads fill whole 128-byte lines.  Head size D is 64 or 128 (D / 8
+// chunks per head row, R <= D / 2).
 #pragma once
 
 #include "host_util.cuh"
@@ -102,8 +103,9 @@ struct RopeQkParams {
   gptoss_strides sv, svo;
   TokenMap tm;
   int Hq, Hkv;
+  int D;           // head size: 64 or 128
   RopeTable tab;
-  float2* cs_out;  // nullable: each token's 32 (c cos, c sin) pairs, [token][32]
+  float2* cs_out;  // nullable: each token's D / 2 (c cos, c sin) pairs, [token][D / 2]
 };
 
 // Converts 8 bf16 values to fp16 (round to nearest even; exact for the
@@ -123,19 +125,20 @@ constexpr int kRopeThreads = 256;
 template <bool kF16Out>
 __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_constant__ RopeQkParams p) {
   constexpr int TB = kRopeTokensPerCta;
-  __shared__ float2 tab[TB][kPairs];
+  __shared__ float2 tab[TB][kMaxPairs];
   __shared__ int64_t tok_off[TB][6];  // element offsets of token rows: q, k, q_out, k_out, v, v_out
   const int t0 = blockIdx.x * TB;
   const int tid = threadIdx.x;
-  if (tid < TB * kPairs) {
-    const int tt = tid / kPairs, j = tid % kPairs;
+  const int np = p.D / 2;  // table entries per token
+  for (int ti = tid; ti < TB * np; ti += kRopeThreads) {
+    const int tt = ti / np, j = ti % np;
     const int t = t0 + tt;
     if (t < p.tm.ntok) {
       int seq, idx;
       token_coords(p.tm, t, seq, idx);
       const int pos = p.tm.positions ? __ldg(p.tm.positions + t) : idx + p.tm.pos_offset;
       tab[tt][j] = rope_cs(pos, p.tab.inv_freq[j], p.tab.conc);
-      if (p.cs_out != nullptr) p.cs_out[static_cast<int64_t>(t) * kPairs + j] = tab[tt][j];
+      if (p.cs_out != nullptr) p.cs_out[static_cast<int64_t>(t) * np + j] = tab[tt][j];
       if (j == 0) {
         const bool thd = p.tm.cu_seqlens != nullptr;
         const int64_t b = thd ? 0 : seq;
@@ -152,7 +155,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_qk_kernel(const __grid_cons
   __syncthreads();
   const int H = p.Hq + p.Hkv + (p.v != nullptr ? p.Hkv : 0);
   const int n_rot = p.tab.R / 8;     // rotation items per head (chunk + partner)
-  const int per_head = 8 - n_rot;    // plus one pass-through item per chunk past 2R
+  const int per_head = p.D / 8 - n_rot;  // plus one pass-through item per chunk past 2R
   const int items = TB * H * per_head;
   for (int it = tid; it < items; it += kRopeThreads) {
     const int ci = it % per_head;
