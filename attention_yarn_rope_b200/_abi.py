@@ -37,6 +37,8 @@ EXPORTED = (
     "gptoss_attn_fwd_block",
     "gptoss_attn_fwd_block_workspace_size",
     "gptoss_attn_merge",
+    "gptoss_qkv_rope_workspace_size",
+    "gptoss_qkv_rope",
     "gptoss_attn_decode_workspace_size",
     "gptoss_attn_decode",
     "gptoss_attn_decode_noalloc",
@@ -84,6 +86,10 @@ _SIGNATURES = {
                                     _vp]),
     "gptoss_attn_fwd_block_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
     "gptoss_attn_merge": (_st, [_vp, _vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, Strides, _vp, _vp]),
+    "gptoss_qkv_rope_workspace_size": (ctypes.c_size_t, [_i32, _i32]),
+    "gptoss_qkv_rope": (_st, [_vp, ctypes.c_int64, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                              ctypes.POINTER(RopeParams), _vp, Strides, _vp, Strides, _vp, Strides, _vp,
+                              ctypes.c_size_t, _vp]),
     "gptoss_attn_decode_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, _i32]),
     "gptoss_attn_decode": (_st, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
                                  ctypes.POINTER(RopeParams), _vp, _vp, _vp, ctypes.c_size_t, _vp]),

@@ -78,6 +78,8 @@ gptoss_status gptoss_selftest_wait_timeout(uint32_t limit_us, int32_t* result_de
 #include "fwd_host.cuh"
 // the log-sum-exp merge of key-block results
 #include "attn_merge.cuh"
+// the q / k / v projections with RoPE in the GEMM epilogue
+#include "qkv_rope.cuh"
 // the decode entry points (split-KV decode, paged cache, append, no-alloc)
 #include "decode_host.cuh"
 // the backward entry points

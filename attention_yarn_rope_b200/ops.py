@@ -188,6 +188,50 @@ def gptoss_attn_merge(outs, lses, sinks, out=None, lse=None, stream=None):
     return (out, lse) if want_lse else out
 
 
+def gptoss_qkv_rope_workspace_size(total_tokens: int, D: int = 64) -> int:
+    return int(_abi.load().gptoss_qkv_rope_workspace_size(int(total_tokens), int(D)))
+
+
+def gptoss_qkv_rope(x, w_qkv, b_qkv, Hq: int, Hkv: int, rope: RopeConfig | None = None, positions=None,
+                    cu_seqlens=None, q_out=None, k_out=None, v_out=None, workspace=None, stream=None):
+    """q, k, v projections of ``x`` (``[B,S,hidden]`` BSHD or ``[T,hidden]``
+    with ``cu_seqlens``) through the stacked weights ``w_qkv [(Hq + 2 Hkv) D,
+    hidden]`` and bias ``b_qkv`` (or None), q and k rotated when ``rope`` is
+    given.  D = w_qkv.shape[0] // (Hq + 2 Hkv).  Returns ``(q, k, v)``."""
+    lib = _abi.load()
+    thd = cu_seqlens is not None
+    N, hidden = w_qkv.shape
+    D = N // (Hq + 2 * Hkv)
+    if thd:
+        T = x.shape[0]
+        B, S_or_T = cu_seqlens.numel() - 1, T
+        lead = (T,)
+    else:
+        B, S = x.shape[0], x.shape[1]
+        S_or_T, T = S, B * S
+        lead = (B, S)
+    if x.shape[-1] != hidden or x.stride(-1) != 1:
+        raise ValueError("x must be [..., hidden] with hidden contiguous")
+    x_row_stride = x.stride(-2)
+    if not thd and x.stride(0) != S * x_row_stride:
+        raise ValueError("BSHD x must have uniform token rows")
+    q_out = torch.empty(lead + (Hq, D), dtype=torch.bfloat16, device=x.device) if q_out is None else q_out
+    k_out = torch.empty(lead + (Hkv, D), dtype=torch.bfloat16, device=x.device) if k_out is None else k_out
+    v_out = torch.empty(lead + (Hkv, D), dtype=torch.bfloat16, device=x.device) if v_out is None else v_out
+    if workspace is None and rope is not None:
+        workspace = torch.empty(int(lib.gptoss_qkv_rope_workspace_size(T, D)), dtype=torch.uint8, device=x.device)
+    _check_dev(x, w_qkv, b_qkv, positions, cu_seqlens, q_out, k_out, v_out, workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    r = rope.to_c() if rope is not None else None
+    st = lib.gptoss_qkv_rope(_ptr(x), int(x_row_stride), _ptr(w_qkv), _ptr(b_qkv), _ptr(positions),
+                             _ptr(cu_seqlens), B, S_or_T, hidden, Hq, Hkv, D,
+                             ctypes.byref(r) if r is not None else None, _ptr(q_out), _strides(q_out, thd),
+                             _ptr(k_out), _strides(k_out, thd), _ptr(v_out), _strides(v_out, thd), _ptr(workspace),
+                             ws_bytes, _stream(stream))
+    _abi.check("gptoss_qkv_rope", st)
+    return q_out, k_out, v_out
+
+
 def gptoss_attn_bwd_workspace_size(total_tokens: int, Hq: int, Hkv: int, D: int = 64) -> int:
     return int(_abi.load().gptoss_attn_bwd_workspace_size(total_tokens, Hq, Hkv, D))
 

@@ -198,6 +198,39 @@ gptoss_status gptoss_attn_merge(const float* outs, const float* lses, int32_t n_
                                 int32_t B, int32_t S, int32_t Hq, int32_t D, void* out, gptoss_strides so,
                                 float* lse, struct CUstream_st* stream);
 
+/* Workspace bytes for gptoss_qkv_rope: every token's D/2 RoPE angles
+ * (fp32 (c cos, c sin) pairs), plus 16.  0 when a size is out of range. */
+size_t gptoss_qkv_rope_workspace_size(int32_t total_tokens, int32_t D);
+
+/* gptoss_qkv_rope -- the q, k, v projections of the attention input with
+ * RoPE fused into the GEMM epilogue.  GptOssAttention's q_proj, k_proj and
+ * v_proj are Linear layers with bias (blog page "gpt-oss-20b 模型结构":
+ * 2880 -> 4096 / 512 / 512; y = x W^T + b); q and k, viewed as
+ * [token, head, D], are then rotated by the YaRN RoPE of the NeMo AutoModel
+ * gpt_oss.rope_utils page (apply_rotary_emb_qk, half-split pairs).
+ *   x          bf16 [T, hidden] rows of x_row_stride elements (T = B*S for
+ *              BSHD, S_or_T packed tokens with cu_seqlens); hidden % 8 == 0.
+ *   w_qkv      bf16 [(Hq + 2 Hkv) D, hidden], row-major: the q_proj rows,
+ *              then k_proj's, then v_proj's (caller-owned, read only).
+ *   b_qkv      bf16 [(Hq + 2 Hkv) D] in the same order; NULL: no bias.
+ *   positions, cu_seqlens, B, S_or_T: as gptoss_rope_qk (token positions).
+ *   rope       NULL: no rotation; else rotary_dim == D (full rotary;
+ *              GPTOSS_ERR_UNSUPPORTED otherwise).
+ *   q_out [.., Hq, D], k_out / v_out [.., Hkv, D]: bf16 with strides (D
+ *              contiguous, 16-byte aligned rows), BSHD or THD like x.
+ *   workspace  device, >= gptoss_qkv_rope_workspace_size(T, D) bytes when
+ *              rope != NULL (the angle table); else unused.
+ * D is 64 or 128; Hq D and Hkv D must be multiples of 128
+ * (GPTOSS_ERR_UNSUPPORTED otherwise).  Products accumulate in fp32 on the
+ * tensor cores; bias and rotation in fp32; outputs rounded to bf16.  Two
+ * launches (angle table, GEMM), asynchronous on `stream`. */
+gptoss_status gptoss_qkv_rope(const void* x, int64_t x_row_stride, const void* w_qkv, const void* b_qkv,
+                              const int32_t* positions, const int32_t* cu_seqlens, int32_t B, int32_t S_or_T,
+                              int32_t hidden, int32_t Hq, int32_t Hkv, int32_t D, const gptoss_rope_params* rope,
+                              void* q_out, gptoss_strides sq, void* k_out, gptoss_strides sk, void* v_out,
+                              gptoss_strides sv, void* workspace, size_t workspace_bytes,
+                              struct CUstream_st* stream);
+
 /* Workspace bytes gptoss_attn_bwd needs: q and k rotated once (fp16), every
  * token's 32 RoPE angles, and <dout, out> per row and head (fp32).  0 when a
  * size is out of range. */

@@ -27,7 +27,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from oracle.rope import rope
+from .rope import rope
 
 
 def linear(x: np.ndarray, w: np.ndarray, b: np.ndarray | None) -> np.ndarray:
