@@ -10,15 +10,16 @@
 //
 // Design: one persistent GEMM over the stacked output features, tensor-core
 // bound (x W^T is a dense contraction: 2 x 2880 FLOP per output).  Tiles of
-// 128 tokens x 128 output features, K in steps of 64 (128 bytes of bf16, one
-// swizzle span).  Warp 0 streams the x and W tiles with TMA through a ring of
-// stages; warp 1 issues tcgen05.mma (M128 N128 K16, bf16 -> fp32 in tensor
-// memory) into one of two 128-column accumulators; warps 2-5 drain the other
-// accumulator meanwhile -- each thread one token row: the tile's 128 // D
-// heads, bias added, q and k heads rotated with the token's angles (a
-// per-token table written by the first kernel of the call), rounded to bf16
-// and stored.  A 128-feature tile never straddles q, k and v (Hq D and Hkv D
-// are multiples of 128).
+// 128 tokens x 256 output features (measured: 1.0 PFLOP/s with 128 x 128
+// tiles, whose operands cross L2 twice as often per FLOP), K in steps of 64
+// (128 bytes of bf16, one swizzle span).  Warp 0 streams the x and W tiles
+// with TMA through a ring of stages; warp 1 issues tcgen05.mma (M128 N256
+// K16, bf16 -> fp32 in tensor memory) into one of two 256-column
+// accumulators; warps 2-5 drain the other accumulator meanwhile -- each
+// thread one token row: the tile's 256 / D heads, each wholly inside q, k or
+// v, bias added, q and k heads rotated with the token's angles (a per-token
+// table written by the first kernel of the call), rounded to bf16 and
+// stored.
 #pragma once
 
 #include "host_util.cuh"
@@ -27,15 +28,16 @@
 
 namespace gptoss {
 
-constexpr int kPjBM = 128, kPjBN = 128, kPjBK = 64;
-constexpr int kPjStages = 6;
+constexpr int kPjBM = 128, kPjBN = 256, kPjBK = 64;
+constexpr int kPjStages = 4;
 constexpr int kPjThreads = 192;                  // producer, MMA issuer, 4 epilogue warps
-constexpr int kPjTileBytes = kPjBM * kPjBK * 2;  // 16 KB
-constexpr uint32_t kPjTmemCols = 256;            // two 128-column accumulators
+constexpr int kPjABytes = kPjBM * kPjBK * 2;     // 16 KB of x per stage
+constexpr int kPjBBytes = kPjBN * kPjBK * 2;     // 32 KB of W per stage
+constexpr uint32_t kPjTmemCols = 512;            // two 256-column accumulators
 
 struct ProjParams {
   CUtensorMap tmap_x;  // x: dims (hidden, T), box (64, 128)
-  CUtensorMap tmap_w;  // stacked W: dims (hidden, N), box (64, 128)
+  CUtensorMap tmap_w;  // stacked W: dims (hidden, N), box (64, 256)
   const __nv_bfloat16* bias;  // [N] nullable
   const float2* cs;           // [T][D / 2] (c cos, c sin), nullable: no rotation
   __nv_bfloat16 *q, *k, *v;
@@ -45,8 +47,8 @@ struct ProjParams {
 };
 
 struct __align__(1024) ProjSmem {
-  uint8_t a[kPjStages][kPjTileBytes];
-  uint8_t b[kPjStages][kPjTileBytes];
+  uint8_t a[kPjStages][kPjABytes];
+  uint8_t b[kPjStages][kPjBBytes];
   uint64_t full[kPjStages], empty[kPjStages];
   uint64_t acc_full[2], acc_empty[2];
   uint32_t tmem_base;
@@ -62,7 +64,7 @@ __device__ __forceinline__ void proj_producer(const ProjParams& p, ProjSmem& sm)
     for (int ks = 0; ks < p.n_ksteps; ++ks, ++it) {
       const int s = it % kPjStages;
       if (!mbar_wait(&sm.empty[s], ((it / kPjStages) & 1) ^ 1, p.wait_ns)) { ok = false; break; }
-      mbar_arrive_expect_tx(&sm.full[s], 2 * kPjTileBytes);
+      mbar_arrive_expect_tx(&sm.full[s], kPjABytes + kPjBBytes);
       tma_load_4d(sm.a[s], &p.tmap_x, &sm.full[s], ks * kPjBK, m0, 0, 0);
       tma_load_4d(sm.b[s], &p.tmap_w, &sm.full[s], ks * kPjBK, n0, 0, 0);
     }
@@ -121,7 +123,8 @@ __device__ __forceinline__ void proj_epilogue(const ProjParams& p, ProjSmem& sm,
         tmem_ld32(lane_base + buf * kPjBN + hh * kD + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&a[32 * c]));
       tmem_wait_ld();
       const int col = n0 + hh * kD;  // first output feature of this head
-      if (t < p.T) {                 // a row past the tokens (zero-filled x) stores nothing
+      // a row past the tokens (zero-filled x) or a head past N (zero-filled W) stores nothing
+      if (t < p.T && col < p.N) {
         float y[kD];
         if (p.bias != nullptr) {
           const uint4* bb = reinterpret_cast<const uint4*>(p.bias + col);
@@ -237,8 +240,8 @@ gptoss_status gptoss_qkv_rope(const void* x, int64_t x_row_stride, const void* w
   using namespace gptoss;
   if (B < 0 || S_or_T < 0 || hidden <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
   if (D != kHeadDim && D != kMaxHeadDim) return GPTOSS_ERR_UNSUPPORTED;
-  // whole 128-feature tiles per projection; whole 16-byte rows of x
-  if ((Hq * D) % kPjBN || (Hkv * D) % kPjBN || hidden % 8) return GPTOSS_ERR_UNSUPPORTED;
+  // whole 16-byte rows of x
+  if (hidden % 8) return GPTOSS_ERR_UNSUPPORTED;
   gptoss_status st = check_rope(rope, D, /*allow_partial=*/false);
   if (st != GPTOSS_OK) return st;
   const bool thd = cu_seqlens != nullptr;
@@ -277,7 +280,7 @@ gptoss_status gptoss_qkv_rope(const void* x, int64_t x_row_stride, const void* w
   p.Hq = Hq;
   p.Hkv = Hkv;
   const int n_mtiles = static_cast<int>((T + kPjBM - 1) / kPjBM);
-  p.n_ntiles = N / kPjBN;
+  p.n_ntiles = (N + kPjBN - 1) / kPjBN;
   p.n_tiles = n_mtiles * p.n_ntiles;
   p.n_ksteps = (hidden + kPjBK - 1) / kPjBK;
   p.wait_ns = wait_limit_ns();

@@ -220,8 +220,8 @@ size_t gptoss_qkv_rope_workspace_size(int32_t total_tokens, int32_t D);
  *              contiguous, 16-byte aligned rows), BSHD or THD like x.
  *   workspace  device, >= gptoss_qkv_rope_workspace_size(T, D) bytes when
  *              rope != NULL (the angle table); else unused.
- * D is 64 or 128; Hq D and Hkv D must be multiples of 128
- * (GPTOSS_ERR_UNSUPPORTED otherwise).  Products accumulate in fp32 on the
+ * D is 64 or 128 and hidden a multiple of 8 (GPTOSS_ERR_UNSUPPORTED
+ * otherwise).  Products accumulate in fp32 on the
  * tensor cores; bias and rotation in fp32; outputs rounded to bf16.  Two
  * launches (angle table, GEMM), asynchronous on `stream`. */
 gptoss_status gptoss_qkv_rope(const void* x, int64_t x_row_stride, const void* w_qkv, const void* b_qkv,
