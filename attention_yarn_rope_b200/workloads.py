@@ -73,6 +73,10 @@ DECODE_B8_W = DecodeConfig("decode_b8_l131072_w128", 8, 131072, 64, 8, 64, 128, 
 
 PREFILL_CONFIGS = [TINY, SLIDING, FULL, THD_FULL, THD_WINDOW]
 DECODE_CONFIGS = [DECODE_B64, DECODE_B64_W, DECODE_B8, DECODE_B8_W]
+# Variants beyond GPT-OSS's own shapes: head size 128 (32 / 8 heads, full
+# rotary), and the q / k / v projection of the sliding layer's tokens.
+FULL_D128 = PrefillConfig("full_d128_b2_s8192_hq32", 2, 8192, 32, 8, 128, 0, GPTOSS_ROPE, seed=6)
+PROJ_HIDDEN = 2880  # GPT-OSS hidden size: q_proj 2880 -> 4096, k_proj / v_proj 2880 -> 512
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -186,7 +186,7 @@ def prefill_case(torch, ops, cfg, device, seed_offset=0):
     x = make_prefill(cfg, seed=cfg.seed + seed_offset)
     q, k, v = (to_torch_bf16(a, device) for a in (x.q, x.k, x.v))
     sinks = torch.from_numpy(x.sinks).to(device)
-    rope = ops.RopeConfig.from_dict(cfg.rope)
+    rope = ops.RopeConfig.from_dict(cfg.rope, rotary_dim=cfg.D)
     out = torch.empty_like(q)
     # k is rotated once per call into this workspace (allocated once, outside the timing)
     ws = torch.empty(ops.gptoss_attn_fwd_workspace_size(x.k.shape[0] * x.k.shape[1] if x.k.ndim == 4 else x.k.shape[0],
@@ -210,6 +210,27 @@ def prefill_case(torch, ops, cfg, device, seed_offset=0):
     io_bytes = sum(t.numel() * t.element_size() for t in (q, k, v, out))
     return dict(x=x, q=q, k=k, v=v, sinks=sinks, out=out, cu=cu, step=step, flops=flops, bytes=io_bytes,
                 pairs=pairs, rope=rope, lens=lens, ws=ws)
+
+
+def proj_case(torch, ops, device, B=4, S=4096, Hq=64, Hkv=8, D=64, seed=7):
+    """gptoss_qkv_rope over B x S tokens of GPT-OSS's hidden size: Linear-like
+    weights (N(0, 1 / hidden)), biases N(0, 0.01), x N(0, 1), all bf16."""
+    from attention_yarn_rope_b200.workloads import GPTOSS_ROPE, PROJ_HIDDEN
+
+    gen = torch.Generator(device=device).manual_seed(seed)
+    N = (Hq + 2 * Hkv) * D
+    x = torch.randn((B, S, PROJ_HIDDEN), generator=gen, device=device).to(torch.bfloat16)
+    w = (torch.randn((N, PROJ_HIDDEN), generator=gen, device=device) / PROJ_HIDDEN ** 0.5).to(torch.bfloat16)
+    b = (torch.randn((N,), generator=gen, device=device) * 0.1).to(torch.bfloat16)
+    rope = ops.RopeConfig.from_dict(GPTOSS_ROPE, rotary_dim=D)
+    q = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, device=device)
+    k = torch.empty((B, S, Hkv, D), dtype=torch.bfloat16, device=device)
+    v = torch.empty_like(k)
+    ws = torch.empty(ops.gptoss_qkv_rope_workspace_size(B * S, D), dtype=torch.uint8, device=device)
+
+    def step():
+        ops.gptoss_qkv_rope(x, w, b, Hq, Hkv, rope=rope, q_out=q, k_out=k, v_out=v, workspace=ws)
+    return dict(step=step, flops=2 * B * S * PROJ_HIDDEN * N)
 
 
 def bwd_case(torch, ops, cfg, device):
@@ -289,7 +310,7 @@ def decode_graph_us(torch, ops, cfg, case, flush, calls=100, reps=5):
 def run_ours(args, torch, dist, rank, world, device):
     from attention_yarn_rope_b200 import ops
     from attention_yarn_rope_b200.workloads import (
-        DECODE_B8, DECODE_B8_W, DECODE_B64, DECODE_B64_W, FULL, SLIDING, THD_FULL, THD_WINDOW)
+        DECODE_B8, DECODE_B8_W, DECODE_B64, DECODE_B64_W, FULL, FULL_D128, SLIDING, THD_FULL, THD_WINDOW)
 
     peaks = load_peaks()
     stream = torch.cuda.current_stream()
@@ -408,7 +429,7 @@ def run_ours(args, torch, dist, rank, world, device):
 
     if world == 1 and not args.no_extras:
         line["per_config"] = per_config(torch, ops, device, stream, peaks,
-                                        [FULL, THD_FULL, THD_WINDOW],
+                                        [FULL, THD_FULL, THD_WINDOW, FULL_D128],
                                         [DECODE_B64, DECODE_B64_W, DECODE_B8, DECODE_B8_W], args,
                                         bwd_cfgs=[SLIDING, FULL])
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -435,6 +456,19 @@ def per_config(torch, ops, device, stream, peaks, prefill_cfgs, decode_cfgs, arg
             "flops": case["flops"], "bytes": case["bytes"], "launches_per_call": 2}
         del case
         torch.cuda.empty_cache()
+    # the q / k / v projections with RoPE in the GEMM epilogue, for the
+    # sliding layer's 16384 tokens (x [4, 4096, 2880], GPT-OSS's 64 / 8 heads)
+    pj = proj_case(torch, ops, device)
+    for _ in range(3):
+        pj["step"]()
+    torch.cuda.synchronize()
+    ms = timed_steps(torch, pj["step"], reps, stream) / reps
+    tf = pj["flops"] / (ms * 1e-3) / 1e12
+    res["qkv_rope_b4_s4096_h2880"] = {"ms": round(ms, 4), "tflops": round(tf, 2),
+                                     "frac_of_bf16_peak": round(tf / peaks["bf16_tflops"], 4), "flops": pj["flops"],
+                                     "launches_per_call": 2, "note": "x W^T + b on tcgen05, RoPE of q and k in the epilogue"}
+    del pj
+    torch.cuda.empty_cache()
     # backward (training): dq, dk, dv, dsinks of the forward's output; 5
     # products per visible pair and head (S and dP recomputed, dV, dK, dQ)
     for cfg in bwd_cfgs:
