@@ -35,12 +35,20 @@
 namespace gptoss {
 
 constexpr int kDecTileKeys = 64;       // keys per pipeline stage
-constexpr int kDecStages = 6;
 constexpr int kDecConsumerWarps = 4;   // 16 keys of a stage each
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
-constexpr int kDecTileBytes = kDecTileKeys * kHeadDim * 2;  // 8 KB
 constexpr int kDecMaxGroup = 16;  // query heads per kv head
 constexpr int kDecMaxRows = 32;   // query rows of a CTA: two 16-row M fragments
+
+// Per head size kD (64 or 128): a stage holds one 64-key tile of K and one of
+// V, each kD / 64 halves of 64 features (a 128B-swizzled 64-row TMA box,
+// 8 KB); 96 KB of stages either way.
+template <int kD>
+struct DecCfg {
+  static constexpr int kTileBytes = kDecTileKeys * kD * 2;
+  static constexpr int kHalfBytes = kDecTileKeys * 64 * 2;
+  static constexpr int kStages = kD == 64 ? 6 : 3;
+};
 
 struct DecodeParams {
   CUtensorMap tmap_k;  // dims (64, Hkv, Lmax, B), box (64, 1, 64, 1)
@@ -83,14 +91,15 @@ __host__ __device__ inline int decode_chunk(int B, int Lmax, int Hkv) {
   return static_cast<int>(c);
 }
 
+template <int kD>
 struct __align__(1024) DecodeSmem {
-  uint8_t k[kDecStages][kDecTileBytes];
-  uint8_t v[kDecStages][kDecTileBytes];
-  __nv_bfloat16 q[kDecMaxRows][kHeadDim + 8];  // rotated query rows, padded
+  uint8_t k[DecCfg<kD>::kStages][DecCfg<kD>::kTileBytes];
+  uint8_t v[DecCfg<kD>::kStages][DecCfg<kD>::kTileBytes];  // directly after k (the merge uses both)
+  __nv_bfloat16 q[kDecMaxRows][kD + 8];  // rotated query rows, padded
   float wm[kDecConsumerWarps][kDecMaxRows];
   float wl[kDecConsumerWarps][kDecMaxRows];
-  uint64_t full[kDecStages];
-  uint64_t empty[kDecStages];
+  uint64_t full[DecCfg<kD>::kStages];
+  uint64_t empty[DecCfg<kD>::kStages];
 };
 
 // The query tokens one CTA serves and the keys they see.  CTA z = (b, slice)
@@ -112,11 +121,15 @@ __device__ __forceinline__ DecodeRows decode_rows(const DecodeParams& p, int z) 
   return r;
 }
 
-// RM = 16-row M fragments of query rows (1: up to 16 rows, 2: up to 32).
-template <int RM>
+// RM = 16-row M fragments of query rows (1: up to 16 rows, 2: up to 32);
+// kD = head size (64 or 128).
+template <int RM, int kD>
 __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int kStages = DecCfg<kD>::kStages;
+  constexpr int kHalf = DecCfg<kD>::kHalfBytes;
+  constexpr int kPairsD = kD / 2;
   extern __shared__ uint8_t smem_raw[];
-  DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
+  DecodeSmem<kD>& sm = *reinterpret_cast<DecodeSmem<kD>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int g = blockIdx.x, split = blockIdx.y;
   const DecodeRows cr = decode_rows(p, blockIdx.z);
@@ -134,11 +147,11 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   const int k_tile0 = p.block_table != nullptr ? (k_begin & ~(kDecTileKeys - 1)) : k_begin;
   if (k_begin >= k_end) {  // this split is past the sequence: the merge skips it
     if (p.direct) {        // (only an empty cache reaches here): the sink alone, O = 0
-      for (int idx = threadIdx.x; idx < cr.ntok * G * kHeadDim; idx += kDecThreads) {
-        const int row = idx / kHeadDim, t = row / G, head = g * G + row % G;
+      for (int idx = threadIdx.x; idx < cr.ntok * G * kD; idx += kDecThreads) {
+        const int row = idx / kD, t = row / G, head = g * G + row % G;
         const int64_t vb = static_cast<int64_t>(b) * p.q_len + cr.tok0 + t;
-        p.out[(vb * p.Hq + head) * kHeadDim + idx % kHeadDim] = __float2bfloat16_rn(0.f);
-        if (p.lse != nullptr && idx % kHeadDim == 0) p.lse[vb * p.Hq + head] = __ldg(p.sinks + head);
+        p.out[(vb * p.Hq + head) * kD + idx % kD] = __float2bfloat16_rn(0.f);
+        if (p.lse != nullptr && idx % kD == 0) p.lse[vb * p.Hq + head] = __ldg(p.sinks + head);
       }
     }
     return;
@@ -146,7 +159,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   const int ntile = (k_end - k_tile0 + kDecTileKeys - 1) / kDecTileKeys;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDecStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kDecConsumerWarps);
     }
@@ -154,13 +167,13 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   }
   // rotated query rows of this CTA (zero rows past its tokens); token t's
   // query sits at position n_first + t - 1
-  for (int idx = threadIdx.x; idx < 16 * RM * kPairs; idx += kDecThreads) {
-    const int row = idx / kPairs, j = idx % kPairs;
+  for (int idx = threadIdx.x; idx < 16 * RM * kPairsD; idx += kDecThreads) {
+    const int row = idx / kPairsD, j = idx % kPairsD;
     const int t = row / G;
     float x = 0.f, y = 0.f;
     if (t < cr.ntok) {
       const int64_t vb = static_cast<int64_t>(b) * p.q_len + cr.tok0 + t;
-      const __nv_bfloat16* qr = p.q + (vb * p.Hq + g * G + row % G) * kHeadDim;
+      const __nv_bfloat16* qr = p.q + (vb * p.Hq + g * G + row % G) * kD;
       x = __bfloat162float(qr[rope_feature_a(j, p.tab.R)]);
       y = __bfloat162float(qr[rope_feature_b(j, p.tab.R)]);
       if (p.tab.enabled && j < p.tab.R) {
@@ -182,9 +195,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       tma_prefetch_desc(&p.tmap_k);
       tma_prefetch_desc(&p.tmap_v);
       for (int it = 0; it < ntile; ++it) {
-        const int s = it % kDecStages;
-        if (!mbar_wait(&sm.empty[s], ((it / kDecStages) & 1) ^ 1, p.wait_ns)) break;
-        mbar_arrive_expect_tx(&sm.full[s], 2 * kDecTileBytes);
+        const int s = it % kStages;
+        if (!mbar_wait(&sm.empty[s], ((it / kStages) & 1) ^ 1, p.wait_ns)) break;
+        mbar_arrive_expect_tx(&sm.full[s], 2 * DecCfg<kD>::kTileBytes);
         const int key0 = k_tile0 + it * kDecTileKeys;
         int row = key0, bat = b;
         if (p.block_table != nullptr) {
@@ -196,13 +209,16 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
                                                   : p.num_blocks * p.block_size;
           bat = 0;
         }
-        tma_load_4d(sm.k[s], &p.tmap_k, &sm.full[s], 0, g, row, bat);
-        tma_load_4d(sm.v[s], &p.tmap_v, &sm.full[s], 0, g, row, bat);
+#pragma unroll
+        for (int hf = 0; hf < kD / 64; ++hf) {
+          tma_load_4d(sm.k[s] + hf * kHalf, &p.tmap_k, &sm.full[s], 64 * hf, g, row, bat);
+          tma_load_4d(sm.v[s] + hf * kHalf, &p.tmap_v, &sm.full[s], 64 * hf, g, row, bat);
+        }
       }
       // drain: every issued stage must land before the CTA may exit
-      const int first = ntile > kDecStages ? ntile - kDecStages : 0;
+      const int first = ntile > kStages ? ntile - kStages : 0;
       for (int it = first; it < ntile; ++it)
-        mbar_wait(&sm.full[it % kDecStages], (it / kDecStages) & 1, p.wait_ns);
+        mbar_wait(&sm.full[it % kStages], (it / kStages) & 1, p.wait_ns);
     }
     return;
   }
@@ -210,14 +226,14 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   // ---------------- consumer warps ----------------
   const int gr = lane >> 2, tq = lane & 3;  // fragment row / column-pair index
   // query A fragments of M fragment mi: rows 16 mi + gr and 16 mi + gr + 8
-  uint32_t qa[RM][4][4];
+  uint32_t qa[RM][kD / 16][4];
   // each of this thread's rows (mi, half) sees keys [klo, khi): its token's
   // range cut to this split; rows past the CTA's tokens see none
   int klo[RM][2], khi[RM][2];
 #pragma unroll
   for (int mi = 0; mi < RM; ++mi) {
 #pragma unroll
-    for (int kt = 0; kt < 4; ++kt) {
+    for (int kt = 0; kt < kD / 16; ++kt) {
       const int c0 = kt * 16 + 2 * tq;
       qa[mi][kt][0] = *reinterpret_cast<const uint32_t*>(&sm.q[16 * mi + gr][c0]);
       qa[mi][kt][1] = *reinterpret_cast<const uint32_t*>(&sm.q[16 * mi + gr + 8][c0]);
@@ -233,19 +249,19 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       khi[mi][hf] = t < cr.ntok ? min(k_end, n_t) : k_begin;
     }
   }
-  float o[RM][8][4];
+  float o[RM][kD / 8][4];
   float m[RM][2], l[RM][2];  // running max (log2 units) and this thread's share of the sums
 #pragma unroll
   for (int mi = 0; mi < RM; ++mi) {
 #pragma unroll
-    for (int dt = 0; dt < 8; ++dt) o[mi][dt][0] = o[mi][dt][1] = o[mi][dt][2] = o[mi][dt][3] = 0.f;
+    for (int dt = 0; dt < kD / 8; ++dt) o[mi][dt][0] = o[mi][dt][1] = o[mi][dt][2] = o[mi][dt][3] = 0.f;
     m[mi][0] = m[mi][1] = -INFINITY;
     l[mi][0] = l[mi][1] = 0.f;
   }
 
   for (int it = 0; it < ntile; ++it) {
-    const int s = it % kDecStages;
-    if (!mbar_wait(&sm.full[s], (it / kDecStages) & 1, p.wait_ns)) break;
+    const int s = it % kStages;
+    if (!mbar_wait(&sm.full[s], (it / kStages) & 1, p.wait_ns)) break;
     const uint32_t kb = smem_u32(sm.k[s]);
     const uint32_t vb = smem_u32(sm.v[s]);
     const int r0 = warp * 16;  // first key row of this warp in the tile
@@ -257,9 +273,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       for (int mi = 0; mi < RM; ++mi) sc[mi][nb][0] = sc[mi][nb][1] = sc[mi][nb][2] = sc[mi][nb][3] = 0.f;
       const int row = r0 + nb * 8 + (lane & 7);
 #pragma unroll
-      for (int kp = 0; kp < 2; ++kp) {
+      for (int kp = 0; kp < kD / 32; ++kp) {  // 32 features per step; half kp / 2 of the row
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(sw128_addr(kb, row, kp * 4 + (lane >> 3)), b0, b1, b2, b3);
+        ldsm_x4(sw128_addr(kb + (kp >> 1) * kHalf, row, (kp & 1) * 4 + (lane >> 3)), b0, b1, b2, b3);
 #pragma unroll
         for (int mi = 0; mi < RM; ++mi) {
           mma_bf16_16816(sc[mi][nb], qa[mi][2 * kp], b0, b1);
@@ -303,7 +319,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       l[mi][0] = l[mi][0] * a0 + (pr[mi][0][0] + pr[mi][0][1] + pr[mi][1][0] + pr[mi][1][1]);
       l[mi][1] = l[mi][1] * a1 + (pr[mi][0][2] + pr[mi][0][3] + pr[mi][1][2] + pr[mi][1][3]);
 #pragma unroll
-      for (int dt = 0; dt < 8; ++dt) {
+      for (int dt = 0; dt < kD / 8; ++dt) {
         o[mi][dt][0] *= a0;
         o[mi][dt][1] *= a0;
         o[mi][dt][2] *= a1;
@@ -315,10 +331,10 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
     // anything, so the warp zeroes its own V rows there before P V.
     const bool tail = key_base + 15 >= k_end;
     if (tail) {
-      for (int idx = lane; idx < 16 * 8; idx += 32) {  // 16 rows x 8 chunks of 16 bytes
-        const int rr = idx >> 3, ch = idx & 7;
+      for (int idx = lane; idx < 16 * 8 * (kD / 64); idx += 32) {  // halves x 16 rows x 8 chunks of 16 bytes
+        const int hf = idx >> 7, rr = (idx >> 3) & 15, ch = idx & 7;
         if (key_base + rr >= k_end)
-          *reinterpret_cast<uint4*>(sm.v[s] + (r0 + rr) * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(sm.v[s] + hf * kHalf + (r0 + rr) * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
       __syncwarp();
     }
@@ -333,10 +349,10 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
     }
     // O += P V over 8 feature blocks of 8; each V fragment serves every M fragment
 #pragma unroll
-    for (int dp = 0; dp < 4; ++dp) {
+    for (int dp = 0; dp < kD / 16; ++dp) {  // 16 features per step; half dp / 4 of the row
       uint32_t v0, v1, v2, v3;
       const int row = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-      ldsm_x4_t(sw128_addr(vb, row, 2 * dp + (lane >> 4)), v0, v1, v2, v3);
+      ldsm_x4_t(sw128_addr(vb + (dp >> 2) * kHalf, row, 2 * (dp & 3) + (lane >> 4)), v0, v1, v2, v3);
 #pragma unroll
       for (int mi = 0; mi < RM; ++mi) {
         mma_bf16_16816(o[mi][2 * dp], pa[mi], v0, v1);
@@ -349,10 +365,10 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   }
 
   // ---------------- merge the four warps ----------------
-  // The per-warp accumulators reuse the K stages once every warp is done
-  // (4 warps x 32 rows x 64 floats = 32 KB of the 48 KB).
+  // The per-warp accumulators reuse the K and V stages once every warp is
+  // done (4 warps x 32 rows x kD floats: at most 64 KB of the 96 KB).
   named_barrier_sync(1, kDecConsumerWarps * 32);
-  float(*wo)[kDecMaxRows][kHeadDim] = reinterpret_cast<float(*)[kDecMaxRows][kHeadDim]>(&sm.k[0][0]);
+  float(*wo)[kDecMaxRows][kD] = reinterpret_cast<float(*)[kDecMaxRows][kD]>(&sm.k[0][0]);
 #pragma unroll
   for (int mi = 0; mi < RM; ++mi) {
 #pragma unroll
@@ -366,7 +382,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       }
     }
 #pragma unroll
-    for (int dt = 0; dt < 8; ++dt) {
+    for (int dt = 0; dt < kD / 8; ++dt) {
       wo[warp][16 * mi + gr][dt * 8 + 2 * tq] = o[mi][dt][0];
       wo[warp][16 * mi + gr][dt * 8 + 2 * tq + 1] = o[mi][dt][1];
       wo[warp][16 * mi + gr + 8][dt * 8 + 2 * tq] = o[mi][dt][2];
@@ -375,8 +391,8 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
   }
   named_barrier_sync(1, kDecConsumerWarps * 32);
   const int tid = threadIdx.x;  // 128 consumer threads: (row, 4 features)
-  for (int idx = tid; idx < 16 * RM * 16; idx += kDecConsumerWarps * 32) {
-    const int row = idx >> 4, d4 = (idx & 15) * 4;
+  for (int idx = tid; idx < 16 * RM * (kD / 4); idx += kDecConsumerWarps * 32) {
+    const int row = idx / (kD / 4), d4 = (idx % (kD / 4)) * 4;
     const int t = row / G, h = row - t * G;
     if (t >= cr.ntok) continue;
     const int64_t vbq = static_cast<int64_t>(b) * p.q_len + cr.tok0 + t;  // virtual sequence of the row
@@ -407,12 +423,12 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
       uint2 r;
       r.x = pack_bf16(acc.x * inv, acc.y * inv);
       r.y = pack_bf16(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(p.out + (vbq * p.Hq + head) * kHeadDim + d4) = r;
+      *reinterpret_cast<uint2*>(p.out + (vbq * p.Hq + head) * kD + d4) = r;
       if (p.lse != nullptr && d4 == 0) p.lse[vbq * p.Hq + head] = (Mt + log2f(Lt)) * kLn2;
       continue;
     }
     const int64_t slot = ((vbq * p.Hkv + g) * p.nsplit + split) * G + h;
-    *reinterpret_cast<float4*>(p.ws_o + slot * kHeadDim + d4) = acc;
+    *reinterpret_cast<float4*>(p.ws_o + slot * kD + d4) = acc;
     if (d4 == 0) {
       p.ws_ml[slot * 2] = M;
       p.ws_ml[slot * 2 + 1] = L;
@@ -423,6 +439,7 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __
 // Merge the splits of one (virtual sequence, g): fold exp(sink) once,
 // normalise, write bf16.  The splits are those of the sequence's CTA group:
 // chunks of the union of its tokens' key ranges.
+template <int kD>
 __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_constant__ DecodeParams p) {
   const int g = blockIdx.x, vb = blockIdx.y;  // virtual sequence (cache row, query token)
   const int b = vb / p.q_len, tok = vb - b * p.q_len;
@@ -431,8 +448,8 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_con
   const int n_last = cr.n_first + cr.ntok - 1;
   const int nsp = min(p.nsplit, (n_last - cr.lo_first + p.chunk - 1) / p.chunk);
   const int G = p.G;
-  for (int idx = threadIdx.x; idx < G * 32; idx += 256) {
-    const int h = idx >> 5, d2 = (idx & 31) * 2;
+  for (int idx = threadIdx.x; idx < G * (kD / 2); idx += 256) {
+    const int h = idx / (kD / 2), d2 = (idx % (kD / 2)) * 2;
     const int head = g * G + h;
     const float sink = __ldg(p.sinks + head) * kLog2e;
     const int64_t base = (static_cast<int64_t>(vb) * p.Hkv + g) * p.nsplit;
@@ -445,7 +462,7 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_con
       const int64_t slot = (base + s) * G + h;
       const float sc = ex2_approx(p.ws_ml[slot * 2] - Ms);
       L += p.ws_ml[slot * 2 + 1] * sc;
-      const float2 ov = *reinterpret_cast<const float2*>(p.ws_o + slot * kHeadDim + d2);
+      const float2 ov = *reinterpret_cast<const float2*>(p.ws_o + slot * kD + d2);
       ox += ov.x * sc;
       oy += ov.y * sc;
     }
@@ -453,7 +470,7 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_con
     __nv_bfloat162 r;
     r.x = __float2bfloat16_rn(ox * inv);
     r.y = __float2bfloat16_rn(oy * inv);
-    *reinterpret_cast<__nv_bfloat162*>(p.out + (static_cast<int64_t>(vb) * p.Hq + head) * kHeadDim + d2) = r;
+    *reinterpret_cast<__nv_bfloat162*>(p.out + (static_cast<int64_t>(vb) * p.Hq + head) * kD + d2) = r;
     if (p.lse != nullptr && d2 == 0) p.lse[static_cast<int64_t>(vb) * p.Hq + head] = (M + log2f(L)) * kLn2;
   }
 }
@@ -463,20 +480,20 @@ __global__ void __launch_bounds__(256) attn_decode_merge_kernel(const __grid_con
 // (the cache holds post-RoPE keys, bf16), the values as given.  Block (b, i):
 // new token i of sequence b; thread (g, j): pair j of kv head g.
 struct AppendParams {
-  const __nv_bfloat16* k_new;  // [B, q_len, Hkv, 64]
+  const __nv_bfloat16* k_new;  // [B, q_len, Hkv, D]
   const __nv_bfloat16* v_new;
   const int32_t* seqlens;      // [B]
   const int32_t* block_table;  // [B, max_blocks]
-  __nv_bfloat16* k_pool;       // [num_blocks * block_size, Hkv, 64]
+  __nv_bfloat16* k_pool;       // [num_blocks * block_size, Hkv, D]
   __nv_bfloat16* v_pool;
-  int B, q_len, Hkv, max_blocks, block_size, num_blocks;
+  int B, q_len, Hkv, D, max_blocks, block_size, num_blocks;
   RopeTable tab;
 };
 
 
 __global__ void kv_append_paged_kernel(const __grid_constant__ AppendParams p) {
   const int b = blockIdx.x, tok = blockIdx.y;
-  const int g = threadIdx.x / kPairs, j = threadIdx.x % kPairs;
+  const int g = threadIdx.x / (p.D / 2), j = threadIdx.x % (p.D / 2);
   const int pos = __ldg(p.seqlens + b) - p.q_len + tok;
   const int jb = pos >= 0 ? pos / p.block_size : -1;
   const int blk = (jb >= 0 && jb < p.max_blocks) ? __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks + jb) : -1;
@@ -484,9 +501,9 @@ __global__ void kv_append_paged_kernel(const __grid_constant__ AppendParams p) {
     if (threadIdx.x == 0) atomicExch(&g_device_status, kStatusBadIndex);
     return;
   }
-  const int64_t off = (static_cast<int64_t>(blk) * p.block_size + pos % p.block_size) * p.Hkv * kHeadDim +
-                      static_cast<int64_t>(g) * kHeadDim;
-  const int64_t src = ((static_cast<int64_t>(b) * p.q_len + tok) * p.Hkv + g) * kHeadDim;
+  const int64_t off = (static_cast<int64_t>(blk) * p.block_size + pos % p.block_size) * p.Hkv * p.D +
+                      static_cast<int64_t>(g) * p.D;
+  const int64_t src = ((static_cast<int64_t>(b) * p.q_len + tok) * p.Hkv + g) * p.D;
   const int fa = rope_feature_a(j, p.tab.R), fb = rope_feature_b(j, p.tab.R);
   float x = __bfloat162float(p.k_new[src + fa]), y = __bfloat162float(p.k_new[src + fb]);
   if (p.tab.enabled && j < p.tab.R) {

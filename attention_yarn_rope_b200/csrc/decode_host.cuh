@@ -18,24 +18,24 @@ using namespace gptoss;
 extern "C" {
 
 size_t gptoss_attn_decode_workspace_size(int32_t B, int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D) {
-  if (B <= 0 || Lmax <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D != kHeadDim) return 0;
+  if (B <= 0 || Lmax <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || (D != kHeadDim && D != kMaxHeadDim)) return 0;
   const int chunk = decode_chunk(B, Lmax, Hkv);
   const int64_t nsplit = (Lmax + chunk - 1) / chunk;
   const int64_t slots = static_cast<int64_t>(B) * Hkv * nsplit * (Hq / Hkv);
-  return static_cast<size_t>(slots * (kHeadDim + 2) * sizeof(float));
+  return static_cast<size_t>(slots * (D + 2) * sizeof(float));
 }
 
 }  // extern "C"
 
 namespace {
 
-// A paged cache: pools [num_blocks * block_size, Hkv, 64] and the block table.
+// A paged cache: pools [num_blocks * block_size, Hkv, D] and the block table.
 struct PagedLayout {
   const int32_t* table;
   int32_t max_blocks, block_size, num_blocks;
 };
 
-// Decode over a contiguous cache [B, Lmax, Hkv, 64] (paged == nullptr) or a
+// Decode over a contiguous cache [B, Lmax, Hkv, D] (paged == nullptr) or a
 // paged one (Lmax = max_blocks * block_size, the caches are the pools).
 gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_seqlens,
                           const float* sinks, int32_t B, int32_t Lmax, int32_t Hq, int32_t Hkv, int32_t D,
@@ -48,7 +48,7 @@ gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cach
   if (BQ > 65535) return GPTOSS_ERR_UNSUPPORTED;  // grid z / y limit
   if (B < 0 || Lmax <= 0 || Hq <= 0 || Hkv <= 0 || window < 0) return GPTOSS_ERR_INVALID_ARG;
   if (Hq % Hkv) return GPTOSS_ERR_INVALID_ARG;
-  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (D != kHeadDim && D != kMaxHeadDim) return GPTOSS_ERR_UNSUPPORTED;
   if (Hq / Hkv > kDecMaxGroup) return GPTOSS_ERR_UNSUPPORTED;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
   gptoss_status st = check_rope(rope, D, /*allow_partial=*/true);
@@ -61,20 +61,19 @@ gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cach
   if (need == 0 || workspace_bytes < need) return GPTOSS_ERR_INVALID_ARG;
   const int64_t rows = paged ? static_cast<int64_t>(paged->num_blocks) * paged->block_size
                              : static_cast<int64_t>(B) * Lmax;
-  if (rows * Hkv * kHeadDim > (int64_t(1) << 40)) return GPTOSS_ERR_UNSUPPORTED;
+  if (rows * Hkv * D > (int64_t(1) << 40)) return GPTOSS_ERR_UNSUPPORTED;
 
   DecodeParams p;
   memset(&p, 0, sizeof(p));
-  const uint64_t tok_b = static_cast<uint64_t>(Hkv) * kHeadDim * 2;
+  const uint64_t tok_b = static_cast<uint64_t>(Hkv) * D * 2;
   // contiguous: (d, head, slot, sequence); paged: (d, head, pool row, 1)
   const uint64_t d2 = paged ? static_cast<uint64_t>(rows) : static_cast<uint64_t>(Lmax);
   const uint64_t d3 = paged ? 1 : static_cast<uint64_t>(B);
   const uint64_t bat_b = paged ? tok_b * d2 : tok_b * Lmax;
-  st = make_tmap_4d(&p.tmap_k, k_cache, kHeadDim, Hkv, d2, d3, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
-                    kDecTileKeys, 1);
+  // boxes of 64 features (a D = 128 row is two)
+  st = make_tmap_4d(&p.tmap_k, k_cache, D, Hkv, d2, d3, D * 2, tok_b, bat_b, kHeadDim, 1, kDecTileKeys, 1);
   if (st != GPTOSS_OK) return st;
-  st = make_tmap_4d(&p.tmap_v, v_cache, kHeadDim, Hkv, d2, d3, kHeadDim * 2, tok_b, bat_b, kHeadDim, 1,
-                    kDecTileKeys, 1);
+  st = make_tmap_4d(&p.tmap_v, v_cache, D, Hkv, d2, d3, D * 2, tok_b, bat_b, kHeadDim, 1, kDecTileKeys, 1);
   if (st != GPTOSS_OK) return st;
   const int G = Hq / Hkv;
   // tokens per CTA: as many as fill one 16-row M fragment, or two when q_len
@@ -96,7 +95,7 @@ gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cach
   p.seqlens = cache_seqlens;
   p.sinks = sinks;
   p.ws_o = static_cast<float*>(workspace);
-  p.ws_ml = p.ws_o + BQ * Hkv * nsplit_max * G * kHeadDim;
+  p.ws_ml = p.ws_o + BQ * Hkv * nsplit_max * G * D;
   p.B = B;
   p.q_len = q_len;
   p.tpc = tpc;
@@ -119,8 +118,10 @@ gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cach
   p.wait_ns = wait_limit_ns();
   if (rope != nullptr) yarn_table(*rope, &p.tab);
   else p.tab.enabled = 0;
-  const size_t smem = sizeof(DecodeSmem) + 1024;
-  auto kernel = rm == 1 ? attn_decode_split_kernel<1> : attn_decode_split_kernel<2>;
+  const bool d128 = D == kMaxHeadDim;
+  const size_t smem = (d128 ? sizeof(DecodeSmem<kMaxHeadDim>) : sizeof(DecodeSmem<kHeadDim>)) + 1024;
+  auto kernel = d128 ? (rm == 1 ? attn_decode_split_kernel<1, kMaxHeadDim> : attn_decode_split_kernel<2, kMaxHeadDim>)
+                     : (rm == 1 ? attn_decode_split_kernel<1, kHeadDim> : attn_decode_split_kernel<2, kHeadDim>);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return GPTOSS_ERR_CUDA;
@@ -129,7 +130,8 @@ gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cach
   kernel<<<grid, kDecThreads, smem, s>>>(p);
   if (check_launch() != GPTOSS_OK) return GPTOSS_ERR_CUDA;
   if (p.direct) return GPTOSS_OK;
-  attn_decode_merge_kernel<<<dim3(Hkv, static_cast<unsigned>(BQ)), 256, 0, s>>>(p);
+  if (d128) attn_decode_merge_kernel<kMaxHeadDim><<<dim3(Hkv, static_cast<unsigned>(BQ)), 256, 0, s>>>(p);
+  else attn_decode_merge_kernel<kHeadDim><<<dim3(Hkv, static_cast<unsigned>(BQ)), 256, 0, s>>>(p);
   return check_launch();
 }
 
@@ -177,8 +179,8 @@ gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const
                                      struct CUstream_st* stream) {
   if (B < 0 || q_len <= 0 || Hkv <= 0) return GPTOSS_ERR_INVALID_ARG;
   if (q_len > 65535) return GPTOSS_ERR_UNSUPPORTED;
-  if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
-  if (Hkv * kPairs > 1024) return GPTOSS_ERR_UNSUPPORTED;
+  if (D != kHeadDim && D != kMaxHeadDim) return GPTOSS_ERR_UNSUPPORTED;
+  if (Hkv * (D / 2) > 1024) return GPTOSS_ERR_UNSUPPORTED;
   gptoss_status st = check_paged(max_blocks, block_size, num_blocks);
   if (st != GPTOSS_OK) return st;
   st = check_rope(rope, D, /*allow_partial=*/true);
@@ -196,12 +198,13 @@ gptoss_status gptoss_kv_append_paged(const void* k_new, const void* v_new, const
   p.B = B;
   p.q_len = q_len;
   p.Hkv = Hkv;
+  p.D = D;
   p.max_blocks = max_blocks;
   p.block_size = block_size;
   p.num_blocks = num_blocks;
   if (rope != nullptr) yarn_table(*rope, &p.tab);
   else p.tab.enabled = 0;
-  kv_append_paged_kernel<<<dim3(B, q_len), Hkv * kPairs, 0, as_stream(stream)>>>(p);
+  kv_append_paged_kernel<<<dim3(B, q_len), Hkv * (D / 2), 0, as_stream(stream)>>>(p);
   return check_launch();
 }
 
@@ -292,7 +295,7 @@ extern "C" gptoss_status gptoss_attn_decode_noalloc(const void* q, const void* k
   if (B == 0) return gptoss_attn_decode(q, k_cache, v_cache, cache_seqlens, sinks, B, Lmax, Hq, Hkv, D, window,
                                         softmax_scale, rope, out, lse, nullptr, 0, stream);
   const size_t need = gptoss_attn_decode_workspace_size(B, Lmax, Hq, Hkv, D);
-  if (need == 0) return D != kHeadDim ? GPTOSS_ERR_UNSUPPORTED : GPTOSS_ERR_INVALID_ARG;
+  if (need == 0) return D != kHeadDim && D != kMaxHeadDim ? GPTOSS_ERR_UNSUPPORTED : GPTOSS_ERR_INVALID_ARG;
   if (need > kNoAllocScratchBytes) return GPTOSS_ERR_UNSUPPORTED;  // partials exceed the fixed array
   gptoss_status st = GPTOSS_OK;
   void* ws = scratch_address(&st);

@@ -2,8 +2,10 @@
 size) against the float64 oracle: gptoss_rope_qk with full and partial
 rotary, and the prefill (gptoss_attn_fwd) with RoPE fused or inputs
 pre-rotated, full and sliding windows, BSHD with a ragged last tile, packed
-THD, explicit positions and extreme sinks.  Every element of out and lse is
-compared against the same bar as at D = 64."""
+THD, explicit positions and extreme sinks; decode over a contiguous cache
+(full and 128 windows, full and partial rotary) and over a paged cache after
+appending 1 or 3 new tokens.  Every element of out and lse is compared
+against the same bar as at D = 64."""
 
 import numpy as np
 import pytest
@@ -109,3 +111,56 @@ def test_prefill_d128_rejects_partial_rotary(cuda_device):
     k = torch.zeros((1, 128, 1, D), dtype=torch.bfloat16, device=cuda_device)
     with pytest.raises(RuntimeError, match="UNSUPPORTED"):
         ops.gptoss_attn_fwd(q, k, k, torch.zeros(2, device=cuda_device), rope=_rope_cfg(64))
+
+
+# ---------------------------------------------------------------- decode, D = 128
+def _decode_case(lens, Hq=8, Hkv=2, seed=41):
+    rng = np.random.default_rng(seed)
+    B, L = len(lens), max(lens)
+    q = bf16_round(rng.standard_normal((B, Hq, D)))
+    kc = bf16_round(rng.standard_normal((B, L, Hkv, D)))
+    vc = bf16_round(rng.standard_normal((B, L, Hkv, D)))
+    sinks = rng.standard_normal(Hq).astype(np.float32)
+    return q, kc, vc, np.array(lens, np.int32), sinks
+
+
+@pytest.mark.parametrize("window", [0, 128])
+@pytest.mark.parametrize("rotary_dim", [128, 64])
+def test_decode_d128(cuda_device, window, rotary_dim):
+    from oracle.attention import attn_decode
+    q, kc, vc, lens, sinks = _decode_case([3000, 1, 517, 129, 2049])
+    out, lse = ops.gptoss_attn_decode(dev(q), dev(kc), dev(vc), i32(lens), f32(sinks), window=window,
+                                      rope=_rope_cfg(rotary_dim), return_lse=True)
+    torch.cuda.synchronize()
+    ref, ref_lse = attn_decode(q, kc, vc, lens, sinks, SCALE, window, rope_tables=_tables(rotary_dim))
+    assert_parity(host(out), ref, f"D=128 decode w={window} r={rotary_dim}")
+    assert_lse_parity(host(lse), ref_lse, f"D=128 decode lse w={window} r={rotary_dim}")
+
+
+@pytest.mark.parametrize("q_len", [1, 3])
+def test_paged_append_then_decode_d128(cuda_device, q_len):
+    from oracle.paged import attn_decode_paged, kv_append_paged
+    rng = np.random.default_rng(43)
+    lens = [129, 2000, 5]
+    bs, Hq, Hkv = 64, 16, 2
+    B = len(lens)
+    max_blocks = -(-max(lens) // bs)
+    num_blocks = B * max_blocks + 3
+    table = rng.permutation(num_blocks)[:B * max_blocks].reshape(B, max_blocks).astype(np.int32)
+    kp = bf16_round(rng.standard_normal((num_blocks, bs, Hkv, D)))
+    vp = bf16_round(rng.standard_normal((num_blocks, bs, Hkv, D)))
+    q = bf16_round(rng.standard_normal((B, q_len, Hq, D)))
+    sinks = rng.standard_normal(Hq).astype(np.float32)
+    k_new = bf16_round(rng.standard_normal((B, q_len, Hkv, D)))
+    v_new = bf16_round(rng.standard_normal((B, q_len, Hkv, D)))
+    kd, vd = dev(kp), dev(vp)
+    ops.gptoss_kv_append_paged(dev(k_new), dev(v_new), i32(lens), i32(table), kd, vd, _rope_cfg())
+    out, lse = ops.gptoss_attn_decode_paged(dev(q), kd, vd, i32(table), i32(lens), f32(sinks), window=128,
+                                            rope=_rope_cfg(), return_lse=True)
+    torch.cuda.synchronize()
+    ref_k, ref_v = kv_append_paged(k_new, v_new, lens, table, bs, kp, vp, _tables())
+    np.testing.assert_allclose(host(kd), ref_k, rtol=2 ** -8, atol=1e-30)
+    np.testing.assert_array_equal(host(vd), ref_v)
+    ref, ref_lse = attn_decode_paged(q, host(kd), host(vd), table, bs, lens, sinks, SCALE, 128, _tables())
+    assert_parity(host(out), ref, f"D=128 paged q_len={q_len}")
+    assert_lse_parity(host(lse), ref_lse, f"D=128 paged lse q_len={q_len}")
