@@ -60,7 +60,8 @@ def _fwd(lib, **kw):
 
 
 def test_attn_fwd_validation(lib):
-    assert _fwd(lib, D=128) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert _fwd(lib, D=96) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert _fwd(lib, D=128) == _abi.GPTOSS_ERR_UNSUPPORTED          # D = 128 takes full rotary only (rope has 64)
     assert _fwd(lib, Hkv=7) == _abi.GPTOSS_ERR_INVALID_ARG          # Hq % Hkv != 0
     assert _fwd(lib, window=-1) == _abi.GPTOSS_ERR_INVALID_ARG
     assert _fwd(lib, scale=0.0) == _abi.GPTOSS_ERR_INVALID_ARG
@@ -139,7 +140,8 @@ def test_rope_qk_validation(lib):
 def test_decode_validation_and_workspace(lib):
     ws = lib.gptoss_attn_decode_workspace_size(64, 32768, 64, 8, 64)
     assert ws > 0 and ws % 16 == 0
-    assert lib.gptoss_attn_decode_workspace_size(64, 32768, 64, 8, 128) == 0
+    assert lib.gptoss_attn_decode_workspace_size(64, 32768, 64, 8, 128) > ws  # D = 128: twice the partials
+    assert lib.gptoss_attn_decode_workspace_size(64, 32768, 64, 8, 96) == 0
     assert lib.gptoss_attn_decode_workspace_size(1, 32768, 64, 7, 64) == 0
 
     def call(**kw):
@@ -192,7 +194,8 @@ def test_paged_validation(lib):
 
     assert app(bs=100) == _abi.GPTOSS_ERR_UNSUPPORTED
     assert app(Hkv=33) == _abi.GPTOSS_ERR_UNSUPPORTED  # one thread per (head, pair): 33 x 32 > 1024
-    assert app(D=128) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert app(D=96) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert app(Hkv=17, D=128) == _abi.GPTOSS_ERR_UNSUPPORTED  # 17 x 64 threads > 1024
     assert app(kp=None) == _abi.GPTOSS_ERR_INVALID_ARG
     assert app(q_len=0) == _abi.GPTOSS_ERR_INVALID_ARG
     assert app(q_len=70000) == _abi.GPTOSS_ERR_UNSUPPORTED
@@ -224,3 +227,31 @@ def test_oracle_is_independent_of_the_cuda_path():
                 if line.startswith(("import ", "from ")):
                     mod = line.split()[1]
                     assert mod.split(".")[0] in {"numpy", "math", "cmath", "__future__", ""} or mod.startswith("."), (f, line)
+
+
+def test_qkv_rope_validation(lib):
+    S_Q = _abi.Strides(4096 * 64 * 64, 64 * 64, 64)
+    S_K = _abi.Strides(4096 * 8 * 64, 8 * 64, 64)
+    need = lib.gptoss_qkv_rope_workspace_size(4096, 64)
+    assert need >= 4096 * 32 * 8
+    assert lib.gptoss_qkv_rope_workspace_size(4096, 96) == 0
+    rp64 = _abi.RopeParams(150000.0, 32.0, 4096, 64, 1.0, 32.0)
+    rp32 = _abi.RopeParams(150000.0, 32.0, 4096, 32, 1.0, 32.0)
+
+    def call(**kw):
+        a = dict(x=FAKE, xs=2880, w=FAKE, b=FAKE, B=1, S=4096, hid=2880, Hq=64, Hkv=8, D=64,
+                 rope=ctypes.byref(rp64), q=FAKE, k=FAKE, v=FAKE, ws=FAKE, wsb=need)
+        a.update(kw)
+        return lib.gptoss_qkv_rope(a["x"], a["xs"], a["w"], a["b"], None, None, a["B"], a["S"], a["hid"], a["Hq"],
+                                   a["Hkv"], a["D"], a["rope"], a["q"], S_Q, a["k"], S_K, a["v"], S_K, a["ws"],
+                                   a["wsb"], None)
+
+    assert call(D=96) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert call(hid=2884, xs=2884) == _abi.GPTOSS_ERR_UNSUPPORTED       # rows of x not whole 16-byte units
+    assert call(rope=ctypes.byref(rp32)) == _abi.GPTOSS_ERR_UNSUPPORTED  # partial rotary is not fused here
+    assert call(Hkv=7) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(xs=2000) == _abi.GPTOSS_ERR_INVALID_ARG                  # row stride below hidden
+    assert call(w=None) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(ws=None) == _abi.GPTOSS_ERR_INVALID_ARG                  # RoPE needs the angle table
+    assert call(wsb=need - 16) == _abi.GPTOSS_ERR_INVALID_ARG
+    assert call(S=0) == _abi.GPTOSS_OK
