@@ -583,6 +583,8 @@ _KERNEL_SOURCES = {
     "rope_qk_kernel<true>": ("rope_qk.cuh", "fwd_host.cuh"),
     "attn_decode_split_kernel": ("attn_decode.cuh", "decode_host.cuh"),
     "attn_bwd_dkdv_tc_kernel": ("attn_bwd_tc.cuh", "bwd_host.cuh"),
+    "attn_fwd128_kernel": ("fwd128.cuh", "fwd_host.cuh"),
+    "qkv_rope_kernel": ("qkv_rope.cuh", "qkv_rope.cuh"),  # launched from its own header
 }
 
 
@@ -823,11 +825,20 @@ def profile_case(args):
     from attention_yarn_rope_b200 import ops
     from attention_yarn_rope_b200 import workloads as wl
 
-    cfgs = {c.name: c for c in wl.PREFILL_CONFIGS + wl.DECODE_CONFIGS}
+    device = "cuda:0"
+    if args.profile_case == "qkv_rope_b4_s4096_h2880":  # the fused projection (a GEMM, not a PrefillConfig)
+        B = args.profile_batch if args.profile_batch is not None else 4
+        case = proj_case(torch, ops, device, B=B)
+        for _ in range(args.warmup + args.steps):
+            case["step"]()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": args.profile_case, "B": B, "launches": args.warmup + args.steps,
+                          "flops_per_launch": case["flops"]}))
+        return 0
+    cfgs = {c.name: c for c in wl.PREFILL_CONFIGS + wl.DECODE_CONFIGS + [wl.FULL_D128]}
     cfg = cfgs[args.profile_case]
     if args.profile_batch is not None:
         cfg = dataclasses.replace(cfg, B=args.profile_batch)
-    device = "cuda:0"
     if isinstance(cfg, wl.DecodeConfig):
         case = decode_case(torch, ops, cfg, device)
     elif args.profile_bwd:
@@ -854,7 +865,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile-case", default=None,
                     help="only launch this workload's kernel warmup+steps times (for ncu), e.g. "
-                         "sliding_b4_s4096_w128, full_b2_s8192, decode_b64_l32768_full; no timing")
+                         "sliding_b4_s4096_w128, full_b2_s8192, decode_b64_l32768_full, "
+                         "full_d128_b2_s8192_hq32, qkv_rope_b4_s4096_h2880; no timing")
     ap.add_argument("--profile-batch", type=int, default=None, help="smaller batch for --profile-case")
     ap.add_argument("--profile-bwd", action="store_true",
                     help="with --profile-case of a prefill workload: launch its backward instead")
