@@ -39,7 +39,7 @@ def test_bounded_wait_gives_up_and_context_survives(cuda_device):
 
 
 def test_host_validation_raises(cuda_device):
-    q = torch.zeros((1, 16, 8, 128), dtype=torch.bfloat16, device=cuda_device)  # head_dim 128
+    q = torch.zeros((1, 16, 8, 96), dtype=torch.bfloat16, device=cuda_device)  # head_dim 96 (64 and 128 only)
     with pytest.raises(_abi.GptossError) as e:
         ops.gptoss_attn_fwd(q, q[:, :, :1], q[:, :, :1], torch.zeros(8, device=cuda_device))
     assert e.value.status == _abi.GPTOSS_ERR_UNSUPPORTED
