@@ -13,7 +13,8 @@
 // tensor maps as the D = 64 kernel.
 //   S  = Q K^T   (SS, M128 N128, 2 halves x 4 x K16, one accumulator)
 //   O += P V     (TS, M128 N64 per feature half, 8 x K16 each)
-// Tensor memory: S [0, 128), P [128, 192), O [192, 320).
+// Tensor memory: three S buffers [0, 384) (P over the first half of its S,
+// product t in buffer t mod 3), O [384, 512).
 // Warps: 0-3 rope (Q rotated in place: pair (j, j + 64) is word m of the
 // two halves at the same swizzled position), 4-7 softmax (fwd_softmax.cuh,
 // head slot 0), 8 K / V producer, 9 QK^T issuer and tensor-memory owner,
@@ -40,7 +41,9 @@ struct __align__(1024) Fwd128Smem {
   uint64_t q_loaded[kF128QStages], q_full[kF128QStages], q_empty[kF128QStages];
   uint64_t k_full[kF128Stages], k_empty[kF128Stages];
   uint64_t v_full[kF128Stages], v_empty[kF128Stages];
-  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];  // slot 0 only (the softmax role indexes a slot)
+  uint64_t s_full[2][kSBufs], p_full[kSBufs], s_empty[kSBufs];  // as in FwdSmem (slot 0 of s_full only)
+  uint64_t o_done[2];                                         // slot 0 only (the softmax role indexes a slot)
+  uint64_t s_free[2];                                         // unused (three-buffer layout)
   uint64_t mma_final[2];
   uint32_t tmem_base;
 };
@@ -187,7 +190,9 @@ __device__ __forceinline__ void fwd128_mma_s_role(const FwdParams& p, Fwd128Smem
     for (int j = 0; j < wu.n_kt; ++j, ++t, ++kv_it) {
       const int s = kv_it % kF128Stages;
       if (!mbar_wait(&sm.k_full[s], (kv_it / kF128Stages) & 1, p.wait_ns)) { ok = false; break; }
-      if (t > 0 && !mbar_wait(&sm.s_free[0], (t - 1) & 1, p.wait_ns)) { ok = false; break; }
+      // product t into S buffer t mod 3, once product t - 3's P V has read its P
+      const uint32_t b = t % kSBufs;
+      if (t >= kSBufs && !mbar_wait(&sm.s_empty[b], ((t / kSBufs) - 1) & 1, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
@@ -195,10 +200,10 @@ __device__ __forceinline__ void fwd128_mma_s_role(const FwdParams& p, Fwd128Smem
         const uint64_t kdesc = sw128_desc(smem_u32(sm.k[s][hf]));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem, qdesc + static_cast<uint64_t>(kk * 2), kdesc + static_cast<uint64_t>(kk * 2), idesc_s,
-                 (hf | kk) > 0 ? 1u : 0u);
+          mma_ss(tmem + b * 128, qdesc + static_cast<uint64_t>(kk * 2), kdesc + static_cast<uint64_t>(kk * 2),
+                 idesc_s, (hf | kk) > 0 ? 1u : 0u);
       }
-      mma_commit(&sm.s_full[0]);
+      mma_commit(&sm.s_full[0][b]);
       mma_commit(&sm.k_empty[s]);
       if (j == wu.n_kt - 1) mma_commit(&sm.q_empty[qb]);
     }
@@ -212,7 +217,7 @@ __device__ __forceinline__ void fwd128_mma_s_role(const FwdParams& p, Fwd128Smem
 // V read N-major); the first tile of a unit starts O from zero.
 __device__ __forceinline__ void fwd128_mma_pv_role(const FwdParams& p, Fwd128Smem& sm, uint32_t tmem) {
   constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, true);
-  constexpr uint32_t colP = 128, colO = 192;
+  constexpr uint32_t colO = kColO;  // O: columns 384 .. 511
   uint32_t t = 0, kv_it = 0;
   bool ok = true;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -221,7 +226,8 @@ __device__ __forceinline__ void fwd128_mma_pv_role(const FwdParams& p, Fwd128Sme
     for (int j = 0; j < wu.n_kt; ++j, ++t, ++kv_it) {
       const int s = kv_it % kF128Stages;
       if (!mbar_wait(&sm.v_full[s], (kv_it / kF128Stages) & 1, p.wait_ns)) { ok = false; break; }
-      if (!mbar_wait(&sm.p_full[0], t & 1, p.wait_ns)) { ok = false; break; }
+      const uint32_t b = t % kSBufs, colP = b * 128;  // P sits over the S it came from
+      if (!mbar_wait(&sm.p_full[b], (t / kSBufs) & 1, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
@@ -232,6 +238,7 @@ __device__ __forceinline__ void fwd128_mma_pv_role(const FwdParams& p, Fwd128Sme
                  (j == 0 && kk == 0) ? 0u : 1u);
       }
       mma_commit(&sm.o_done[0]);
+      mma_commit(&sm.s_empty[b]);  // the buffer may take product t + 3
       mma_commit(&sm.v_empty[s]);
     }
   }
@@ -251,12 +258,13 @@ __global__ void __launch_bounds__(kF128Threads, 1) attn_fwd128_kernel(const __gr
       mbar_init(&sm.q_full[i], 128);
       mbar_init(&sm.q_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 128);
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(&sm.s_full[0][i], 1);
+      mbar_init(&sm.s_full[1][i], 1);
       mbar_init(&sm.p_full[i], 128);
-      mbar_init(&sm.o_done[i], 1);
+      mbar_init(&sm.s_empty[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.o_done[i], 1);
     for (int s = 0; s < kF128Stages; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);

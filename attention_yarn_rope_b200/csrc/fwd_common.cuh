@@ -39,6 +39,19 @@ constexpr int kFwdThreads = 512;
 constexpr int kFwdLaunchRegs = 128;   // 65536 / 512
 constexpr int kFwdTileBytes = kFwdTile * kHeadDim * 2;  // 16 KB
 constexpr uint32_t kFwdTmemCols = 512;
+// Tensor memory, two layouts.  Three S buffers (the causal-only kernel at
+// D = 64, and D = 128): three 128-column S buffers at 128 b (P, fp16, is
+// written over the first 64 columns of the S it came from), then O from
+// column 384 (64 columns per head slot at D = 64, 128 at D = 128); score
+// products k = 0, 1, 2, .. (tile t of head slot X is k = t * slots + X) take
+// buffer k mod 3, whose previous product's P V must have completed first.
+// Per slot (the sliding-window kernel at D = 64): S_X at 256 X, P_X at
+// 256 X + 128, O_X at 256 X + 192; the next S of a slot is issued as soon
+// as its softmax has read the current one.  (Measured: the three-buffer
+// layout takes full causal from 1.86 to 1.57 ms but the sliding window from
+// 202 to 225 us, whose two-tile units then wait for a P V before each S.)
+constexpr int kSBufs = 3;
+constexpr uint32_t kColO = 384;
 // A row's base moves when a tile's maximum exceeds it by more than this (log2
 // units): P = 2^(s - base) then stays at or below 2^15, inside fp16's range.
 constexpr float kRescaleThreshold = 15.0f;
@@ -78,7 +91,22 @@ struct __align__(1024) FwdSmem {
   uint64_t q_loaded[kFwdQStages], q_full[kFwdQStages], q_empty[kFwdQStages];  // TMA landed / rotated / free
   uint64_t k_full[kFwdStages], k_empty[kFwdStages];
   uint64_t v_full[kFwdStages], v_empty[kFwdStages];
-  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];  // per head slot A/B
+  // Parity waits tell only adjacent phases apart, so every barrier is laid
+  // out so that its waiter has seen the previous phase complete and the next
+  // one cannot start before the waiter acts:
+  //   s_full[X][b]: slot X's product landed in S buffer b (a slot uses each
+  //     buffer once every three tiles, tile t being its use t / 3; per buffer
+  //     alone, a slot could poll before the other slot's earlier product in
+  //     that buffer had landed and take the old phase for its own);
+  //   p_full[b]: the product's P is in buffer b (the P V issuer takes products
+  //     in order; per slot, a slot's softmax could finish two tiles before
+  //     the issuer looks);
+  //   s_empty[b]: the P V that read buffer b's P completed.
+  uint64_t s_full[2][kSBufs], p_full[kSBufs], s_empty[kSBufs];
+  uint64_t o_done[2];  // per head slot A/B
+  // per-slot layout: s_full[X][0] and p_full[X] serve slot X, and s_free[X]
+  // tells the QK^T issuer that slot X's softmax has read its S
+  uint64_t s_free[2];
   uint64_t mma_final[2];  // the S and P V issuers' last products have completed
   uint32_t tmem_base;
 };

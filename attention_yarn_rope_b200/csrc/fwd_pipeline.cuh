@@ -82,7 +82,9 @@ __device__ __forceinline__ void fwd_producer_q_role(const FwdParams& p, FwdSmem&
 // tcgen05.commit tracks the issuing thread's own products, so each thread
 // signals its own consumers.
 
-// S_X(t) = Q_X K(t)^T for both head slots, tile by tile.
+// S_X(t) = Q_X K(t)^T for both head slots, tile by tile.  kTri: the
+// three-buffer layout, else per slot (fwd_common.cuh).
+template <bool kTri>
 __device__ __forceinline__ void fwd_mma_s_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem) {
   // Q (rotated or converted by the rope warps) and K (from the workspace) are fp16
   constexpr uint32_t idesc_s = idesc_f16_f32(128, 128);
@@ -99,14 +101,24 @@ __device__ __forceinline__ void fwd_mma_s_role(const FwdParams& p, FwdSmem& sm, 
       const uint64_t kdesc = sw128_desc(smem_u32(sm.k[s]));
 #pragma unroll 1
       for (int X = 0; X < 2; ++X) {
-        if (t > 0 && !mbar_wait(&sm.s_free[X], (t - 1) & 1, p.wait_ns)) { ok = false; break; }
+        uint32_t b, colS;
+        if (kTri) {  // product k = 2t + X into S buffer k mod 3, once product k - 3's P V has read its P
+          const uint32_t k = 2 * t + X;
+          b = k % kSBufs;
+          colS = b * 128;
+          if (k >= kSBufs && !mbar_wait(&sm.s_empty[b], ((k / kSBufs) - 1) & 1, p.wait_ns)) { ok = false; break; }
+        } else {  // slot X's own S, once its softmax has read the previous one
+          b = 0;
+          colS = X * 256;
+          if (t > 0 && !mbar_wait(&sm.s_free[X], (t - 1) & 1, p.wait_ns)) { ok = false; break; }
+        }
         tc_fence_after();
         const uint64_t qdesc = sw128_desc(smem_u32(sm.q[qb][X]));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + X * 256, qdesc + static_cast<uint64_t>(kk * 2), kdesc + static_cast<uint64_t>(kk * 2),
+          mma_ss(tmem + colS, qdesc + static_cast<uint64_t>(kk * 2), kdesc + static_cast<uint64_t>(kk * 2),
                  idesc_s, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.s_full[X]);
+        mma_commit(&sm.s_full[X][b]);
       }
       if (!ok) break;
       mma_commit(&sm.k_empty[s]);
@@ -120,6 +132,7 @@ __device__ __forceinline__ void fwd_mma_s_role(const FwdParams& p, FwdSmem& sm, 
 
 // O_X += P_X(t) V(t) for both head slots (TS: P from TMEM, V N-major from
 // shared memory); the first tile of a unit starts O from zero.
+template <bool kTri>
 __device__ __forceinline__ void fwd_mma_pv_role(const FwdParams& p, FwdSmem& sm, uint32_t tmem) {
   constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, true);  // fp16 P (TMEM) x fp16 V (workspace)
   uint32_t t = 0, kv_it = 0;
@@ -133,14 +146,17 @@ __device__ __forceinline__ void fwd_mma_pv_role(const FwdParams& p, FwdSmem& sm,
       const uint64_t vdesc = sw128_desc(smem_u32(sm.v[s]));
 #pragma unroll 1
       for (int X = 0; X < 2; ++X) {
-        if (!mbar_wait(&sm.p_full[X], t & 1, p.wait_ns)) { ok = false; break; }
+        const uint32_t k = 2 * t + X;
+        const uint32_t b = kTri ? k % kSBufs : X;  // three-buffer: P sits over the S it came from
+        if (!mbar_wait(&sm.p_full[b], (kTri ? k / kSBufs : t) & 1, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t colP = X * 256 + 128, colO = X * 256 + 192;
+        const uint32_t colP = kTri ? b * 128 : X * 256 + 128, colO = kTri ? kColO + X * 64 : X * 256 + 192;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + colO, tmem + colP + kk * 8, vdesc + static_cast<uint64_t>(kk * 128), idesc_o,
                  (j == 0 && kk == 0) ? 0u : 1u);
         mma_commit(&sm.o_done[X]);
+        if (kTri) mma_commit(&sm.s_empty[b]);  // the buffer may take product 2t + X + 3
       }
       if (!ok) break;
       mma_commit(&sm.v_empty[s]);
@@ -163,11 +179,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
       mbar_init(&sm.q_full[i], 128);
       mbar_init(&sm.q_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 128);
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(&sm.s_full[0][i], 1);
+      mbar_init(&sm.s_full[1][i], 1);
       mbar_init(&sm.p_full[i], 128);
+      mbar_init(&sm.s_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.o_done[i], 1);
+      mbar_init(&sm.s_free[i], 128);
     }
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
@@ -199,8 +219,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) attn_fwd_kernel(const __grid_c
   } else {
     reg_dealloc<kRegsOther>();
     if (warp == 12 && lane == 0) fwd_producer_kv_role(p, sm);
-    else if (warp == 13 && lane == 0) fwd_mma_s_role(p, sm, tmem);
-    else if (warp == 14 && lane == 0) fwd_mma_pv_role(p, sm, tmem);
+    else if (warp == 13 && lane == 0) fwd_mma_s_role<!kWindow>(p, sm, tmem);
+    else if (warp == 14 && lane == 0) fwd_mma_pv_role<!kWindow>(p, sm, tmem);
     else if (warp == 15 && lane == 0) fwd_producer_q_role(p, sm);
   }
   tc_fence_before();

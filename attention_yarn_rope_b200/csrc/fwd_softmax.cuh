@@ -169,16 +169,20 @@ __device__ __forceinline__ void fwd_epilogue_row(const FwdParams& p, uint32_t o_
 
 // kWindow: the call has a sliding window (window > 0); false compiles the
 // causal-only masks (a smaller loop for the full-context layers).  kD: head
-// size, the width of O (64: two head slots per CTA, O_X at X * 256 + 192;
-// 128: one slot, O at 192 .. 319).  Smem: the kernel's shared-memory layout
-// (its s_full / s_free / p_full / o_done barriers per head slot).
+// size, the width of O (64: two head slots per CTA, O_X at 384 + 64 X; 128:
+// one slot, O at 384 .. 511).  Smem: the kernel's shared-memory layout (its
+// s_full per slot and S buffer, p_full per S buffer, o_done per slot).
 template <bool kWindow, int kD = kHeadDim, typename Smem = FwdSmem>
 __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, Smem& sm, uint32_t tmem, int X) {
   const int window = kWindow ? p.window : 0;
   const int wq = (threadIdx.x >> 5) & 3;  // warp within the warpgroup = TMEM lane quarter
   const int r = threadIdx.x & 127;        // query row of the tile
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  const uint32_t colS = X * 256, colP = X * 256 + 128, colO = X * 256 + 192;
+  constexpr uint32_t kSlots = kD == kHeadDim ? 2 : 1;  // head slots per CTA
+  // the tensor-memory layout (fwd_common.cuh): three S buffers, or per slot
+  // for the sliding-window kernel at D = 64
+  constexpr bool kTri = !(kWindow && kD == kHeadDim);
+  const uint32_t colO = kTri ? kColO + (kD == kHeadDim ? X * 64 : 0) : X * 256 + 192;
   const bool thd = p.cu_seqlens != nullptr;
   const float sl = p.scale_log2;
   uint32_t t = 0;  // running tile count of this CTA
@@ -197,7 +201,13 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, Smem& sm, u
     int n_seen = 0;  // visible keys this row's base has seen so far
     for (int j = 0; j < w.n_kt; ++j, ++t) {
       const int k0 = (w.j_lo + j) * kFwdTile;
-      if (!mbar_wait_warp(&sm.s_full[X], t & 1, p.wait_ns)) return;
+      // three-buffer layout: score product t * slots + X sits in S buffer
+      // (t * slots + X) mod 3 and P goes over it; this is the slot's use t / 3
+      // of that buffer (each slot takes every buffer once in three tiles).
+      // Per-slot layout: S_X, then P_X beside it; b = X indexes p_full.
+      const uint32_t b = kTri ? (t * kSlots + X) % kSBufs : X;
+      const uint32_t colS = kTri ? b * 128 : X * 256, colP = kTri ? colS : colS + 128;
+      if (!mbar_wait_warp(&sm.s_full[X][kTri ? b : 0], (kTri ? t / kSBufs : t) & 1, p.wait_ns)) return;
       tc_fence_after();
       // chunk classes for this warp: 0 hidden, 1 partly visible, 2 visible
       int cls[4];
@@ -210,8 +220,10 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, Smem& sm, u
       }
       uint32_t sr[4][32];
       load_masked_s<kWindow>(lane_base + colS, cls, qi + p.delta, k0, w.Lk, window, sr);
-      tc_fence_before();
-      mbar_arrive(&sm.s_free[X]);
+      if (!kTri) {  // per slot: the next S may go into S_X now
+        tc_fence_before();
+        mbar_arrive(&sm.s_free[X]);
+      }
       float alpha = 1.f;
       bool rescale = false;
       // A row whose base rests on few keys (none yet, or fewer than 64) takes
@@ -236,7 +248,9 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, Smem& sm, u
       // check; a pass that fails the check takes the maximum and runs again
       // only if some row's base moved.
       bool max_pass = __any_sync(0xffffffffu, young);
-      bool waited = t == 0;  // P(t) overwrites P(t-1): the previous P V must have completed
+      // per slot: P(t) overwrites P(t-1), so the previous P V must have
+      // completed before the first store
+      bool waited = kTri || t == 0;
       float rs = 0.f;
       for (int pass = 0;; ++pass) {
         if (max_pass) {
@@ -258,6 +272,9 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, Smem& sm, u
           tc_fence_after();
           waited = true;
         }
+        // three-buffer layout: over the S columns this thread has already
+        // read (its own lane); the buffer's previous P was consumed before
+        // this S was computed
         tmem_st32(lane_base + colP, pk);
         exp_half(sr, cls, 1, sl, nb, rs0, rs1, pk);
         tmem_st32(lane_base + colP + 32, pk);
@@ -265,8 +282,17 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, Smem& sm, u
         if (max_pass || !__any_sync(0xffffffffu, !(rs <= kMaxTileSum))) break;
         max_pass = true;
       }
-      // the previous unit's rows: its last P V has completed (waited above),
-      // and this unit's first P V, which restarts O, waits for p_full below
+      // The previous tile's P V, waited for once per tile after this tile's P
+      // is stored (by then it has usually completed): every poll of o_done
+      // then follows the one of the phase before, so the parity test cannot
+      // mistake a phase two ahead for a completed one, and O holds every
+      // product up to this tile's.
+      if (kTri && t > 0) {
+        if (!mbar_wait_warp(&sm.o_done[X], (t - 1) & 1, p.wait_ns)) return;
+        tc_fence_after();
+      }
+      // the previous unit's rows (its last P V has completed); this unit's
+      // first P V, which restarts O, waits for p_full below
       if (j == 0 && pending) {
         fwd_epilogue_row<kD>(p, lane_base + colO, pr);
         pending = false;
@@ -287,7 +313,7 @@ __device__ __forceinline__ void fwd_softmax_role(const FwdParams& p, Smem& sm, u
       l_run = l_run * alpha + rs;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[X]);
+      mbar_arrive(&sm.p_full[b]);
     }
     // this unit's epilogue waits for the next unit's first tile (or the end)
     pr.m = m_run;
