@@ -7,19 +7,19 @@
 // every query row i that sees the key of P_ij dout_i, and dK' = scale * sum
 // dS_ij q'_i, dS_ij = P_ij (dP_ij - D_i), P_ij = exp(s_ij - lse_i).
 //
-// CTA = (128-key tile, kv head, sequence[, chunk of its sweep]), 10 warps:
-//   warps 0-7  softmax: warp w reads TMEM lanes 32 (w % 4) .. + 31 (key rows)
-//              and query columns 32 (w / 4) .. + 31 of the step; per step each
-//              thread reads its half row of S^T and dP^T from tensor memory,
-//              forms P^T (bf16) and dS^T (fp16) for those 32 queries and stores
+// CTA = (128-key tile, kv head, sequence[, chunk of its sweep]), 18 warps:
+//   warps 0-15 softmax: warp w reads TMEM lanes 32 (w % 4) .. + 31 (key rows)
+//              and query columns 16 (w / 4) .. + 15 of the step; per step each
+//              thread reads its quarter row of S^T and dP^T from tensor memory,
+//              forms P^T (bf16) and dS^T (fp16) for those 16 queries and stores
 //              them back to tensor memory for the gradient products; at the
 //              end warps 0-3 read and write dV, warps 4-7 dK (scale and c R^T),
 //              or add them into fp32 accumulators when sweeps are split;
-//   warp 8     producer: K and V tiles once (TMA), then per step the step's
+//   warp 16    producer: K and V tiles once (TMA), then per step the step's
 //              rotated q tile (fp16) and dout tile (bf16) by TMA and its 64
 //              lse and 64 D values by cp.async, kBwdTcStages ahead, all
 //              completing on the stage's qd_full barrier;
-//   warp 9     MMA issuer (one thread) and tensor-memory owner.
+//   warp 17    MMA issuer (one thread) and tensor-memory owner.
 // Per step (query head h, 64-query tile), all M = 128, N = 64, K = 4 x 16:
 //   S^T  = K Q^T            (SS, fp16, both K-major)
 //   dP^T = V dout^T         (SS, bf16, both K-major)
@@ -41,7 +41,13 @@ namespace gptoss {
 constexpr int kBwdTcKeys = 128;      // keys per CTA (the M side)
 constexpr int kBwdTcQ = 64;          // queries per step (the N side)
 constexpr int kBwdTcStages = 4;      // q / dout buffers: loads run 3 steps ahead of their use
-constexpr int kBwdTcSoftmax = 256;   // 8 softmax warps
+// 16 softmax warps: four per sub-partition, each thread 16 columns of a step
+// (measured: 8 warps of 32 columns left the per-step chain -- TMEM loads,
+// exponentials, stores -- unhidden, ~3300 cycles a step against ~500 of
+// tensor work)
+constexpr int kBwdTcSoftmax = 512;
+constexpr int kBwdTcSoftWarps = kBwdTcSoftmax / 32;
+constexpr int kBwdTcCols = 16;  // columns of a 64-column step per softmax thread
 constexpr int kBwdTcThreads = kBwdTcSoftmax + 64;  // + producer warp, MMA warp
 constexpr int kBwdTcChunkIt = 64;    // steps of one CTA when sweeps are split
 constexpr uint32_t kBwdTcTmemCols = 512;
@@ -59,6 +65,24 @@ struct __align__(1024) BwdTcSmem {
   uint64_t mma_done;
   uint32_t tmem_base;
 };
+
+// 32 lanes x 16 consecutive 32-bit columns (thread i reads lane base + i).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// 32 lanes x 8 consecutive 32-bit columns (thread i writes lane base + i).
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 
 // 32 lanes x 16 consecutive 32-bit columns (thread i writes lane base + i).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -212,9 +236,9 @@ __device__ __forceinline__ void bwd_tc_mma(const BwdParams& p, BwdTcSmem& sm, co
 template <bool kSplit>
 __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm, const BwdTcWork& w, int g,
                                                uint32_t tmem) {
-  const int tid = threadIdx.x;         // 0 .. 255
+  const int tid = threadIdx.x;         // 0 .. 511
   const int wq = (tid >> 5) & 3;       // TMEM lane quarter
-  const int ch = tid >> 7;             // query-column half of the step
+  const int ch = tid >> 7;             // query-column quarter of the step
   const int r = wq * 32 + (tid & 31);  // key row of the tile = TMEM lane
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   const int L = w.sq.L, W = p.window;
@@ -224,7 +248,7 @@ __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm
   const int n = w.it1 - w.it0;
   for (int t = 0; t < n; ++t) {
     const int it = w.it0 + t;
-    const int i0 = (w.qt0 + it % w.n_qt) * kBwdTcQ + ch * 32;  // this thread's first query column
+    const int i0 = (w.qt0 + it % w.n_qt) * kBwdTcQ + ch * kBwdTcCols;  // this thread's first query column
     const uint32_t X = t & 1;
     const int stg = t % kBwdTcStages;
     // the step's lse / D landed with its tiles (cp.async on qd_full); they
@@ -234,20 +258,21 @@ __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm
     if (!mbar_wait_warp(&sm.s_full[X], (t >> 1) & 1, p.wait_ns)) return;
     tc_fence_after();
     const uint32_t set = lane_base + X * kColSet;
-    uint32_t sv[32], dv[32];
-    tmem_ld32(set + ch * 32, sv);
-    tmem_ld32(set + kColDP + ch * 32, dv);
+    uint32_t sv[kBwdTcCols], dv[kBwdTcCols];
+    tmem_ld16(set + ch * kBwdTcCols, sv);
+    tmem_ld16(set + kColDP + ch * kBwdTcCols, dv);
     tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(&sm.s_free[X]);  // S^T / dP^T of set X may be overwritten
-    const float* lse = &sm.lsd[stg][ch * 32];
-    const float* dsum = &sm.lsd[stg][kBwdTcQ + ch * 32];
-    // every pair of this warp's 32 keys x 32 queries visible: no mask
+    const float* lse = &sm.lsd[stg][ch * kBwdTcCols];
+    const float* dsum = &sm.lsd[stg][kBwdTcQ + ch * kBwdTcCols];
+    // every pair of this warp's 32 keys x 16 queries visible: no mask
     const int jw = w.k0 + wq * 32;
-    const bool all_vis = jw + 31 <= i0 && i0 + 31 < L && jw + 31 < L && (W == 0 || i0 + 31 - jw < W);
-    uint32_t pk[16], dk[16];
+    const bool all_vis = jw + 31 <= i0 && i0 + kBwdTcCols - 1 < L && jw + 31 < L &&
+                         (W == 0 || i0 + kBwdTcCols - 1 - jw < W);
+    uint32_t pk[kBwdTcCols / 2], dk[kBwdTcCols / 2];
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) {
+    for (int e = 0; e < kBwdTcCols; e += 4) {
       const float4 l4 = *reinterpret_cast<const float4*>(lse + e);
       const float4 d4 = *reinterpret_cast<const float4*>(dsum + e);
       const float lv[4] = {l4.x * kLog2e, l4.y * kLog2e, l4.z * kLog2e, l4.w * kLog2e};
@@ -266,13 +291,14 @@ __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm
     }
     // P^T / dS^T of set X were last read by step t-2's gradient products,
     // which completed before step t's S^T (s_full covers all earlier products)
-    tmem_st16(set + kColP + ch * 16, pk);
-    tmem_st16(set + kColDS + ch * 16, dk);
+    tmem_st8(set + kColP + ch * (kBwdTcCols / 2), pk);
+    tmem_st8(set + kColDS + ch * (kBwdTcCols / 2), dk);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&sm.p_full[X]);
   }
   // ---- epilogue: warps 0-3 write dV, warps 4-7 dK, one key row per thread ----
+  if (ch >= 2) return;  // warp-uniform: warps 8-15 have no epilogue
   if (!mbar_wait_warp(&sm.mma_done, 0, p.wait_ns)) return;
   tc_fence_after();
   const int which = ch;  // 0: dV, 1: dK
@@ -348,7 +374,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dkdv_tc_kernel(cons
     mbar_init(&sm.mma_done, 1);
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kBwdTcSoftWarps + 1) {
     tmem_alloc(&sm.tmem_base, kBwdTcTmemCols);
     tmem_relinquish();
   }
@@ -356,21 +382,21 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dkdv_tc_kernel(cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp < 8) bwd_tc_softmax<kSplit>(p, sm, w, g, tmem);
-  else if (warp == 8) bwd_tc_producer(p, sm, w, g);
-  else if (warp == 9 && lane == 0) bwd_tc_mma(p, sm, w, tmem);
+  if (warp < kBwdTcSoftWarps) bwd_tc_softmax<kSplit>(p, sm, w, g, tmem);
+  else if (warp == kBwdTcSoftWarps) bwd_tc_producer(p, sm, w, g);
+  else if (warp == kBwdTcSoftWarps + 1 && lane == 0) bwd_tc_mma(p, sm, w, tmem);
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kBwdTcSoftWarps + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kBwdTcTmemCols);
   }
 }
 
 // ============================================================================
-// dQ on the tensor cores.  CTA = (128-query tile, head, sequence), 10 warps:
-// 8 softmax warps (TMEM lanes 32 (w % 4) .. = query rows, key columns
-// 32 (w / 4) .. of the step), a TMA producer (Q and dout tiles once, then each
+// dQ on the tensor cores.  CTA = (128-query tile, head, sequence), 18 warps:
+// 16 softmax warps (TMEM lanes 32 (w % 4) .. = query rows, key columns
+// 16 (w / 4) .. of the step), a TMA producer (Q and dout tiles once, then each
 // step's 64-key K and V tiles, 4 stages ahead), an MMA issuer.  Per step:
 //   S  = Q K^T, dP = dout V^T   (SS, K-major; M = 128 queries, N = 64 keys)
 //   dS = P (dP - D) -> tensor memory (fp16), P = exp(S scale - lse)
@@ -488,9 +514,9 @@ __device__ __forceinline__ void bwd_tcq_mma(const BwdParams& p, BwdTcQSmem& sm, 
 
 __device__ __forceinline__ void bwd_tcq_softmax(const BwdParams& p, BwdTcQSmem& sm, const BwdTcQWork& w,
                                                 uint32_t tmem) {
-  const int tid = threadIdx.x;         // 0 .. 255
+  const int tid = threadIdx.x;         // 0 .. 511
   const int wq = (tid >> 5) & 3;       // TMEM lane quarter
-  const int ch = tid >> 7;             // key-column half of the step
+  const int ch = tid >> 7;             // key-column quarter of the step
   const int r = wq * 32 + (tid & 31);  // query row of the tile = TMEM lane
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   const int L = w.sq.L, W = p.window;
@@ -506,21 +532,21 @@ __device__ __forceinline__ void bwd_tcq_softmax(const BwdParams& p, BwdTcQSmem& 
   const int iw = w.q0 + wq * 32;  // this warp's first query row
   for (int t = 0; t < w.n; ++t) {
     const uint32_t X = t & 1;
-    const int j0 = (w.kt0 + t) * kBwdTcQ + ch * 32;  // this thread's first key column
+    const int j0 = (w.kt0 + t) * kBwdTcQ + ch * kBwdTcCols;  // this thread's first key column
     if (!mbar_wait_warp(&sm.s_full[X], (t >> 1) & 1, p.wait_ns)) return;
     tc_fence_after();
     const uint32_t set = lane_base + X * kColSet;
-    uint32_t sv[32], dv[32];
-    tmem_ld32(set + ch * 32, sv);
-    tmem_ld32(set + kColDP + ch * 32, dv);
+    uint32_t sv[kBwdTcCols], dv[kBwdTcCols];
+    tmem_ld16(set + ch * kBwdTcCols, sv);
+    tmem_ld16(set + kColDP + ch * kBwdTcCols, dv);
     tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(&sm.s_free[X]);  // S / dP of set X may be overwritten
-    // every pair of this warp's 32 queries x 32 keys visible: no mask
-    const bool all_vis = j0 + 31 <= iw && iw + 31 < L && (W == 0 || iw + 31 - j0 < W);
-    uint32_t dk[16];
+    // every pair of this warp's 32 queries x 16 keys visible: no mask
+    const bool all_vis = j0 + kBwdTcCols - 1 <= iw && iw + 31 < L && (W == 0 || iw + 31 - j0 < W);
+    uint32_t dk[kBwdTcCols / 2];
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
+    for (int e = 0; e < kBwdTcCols; e += 2) {
       float ds[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
@@ -532,15 +558,15 @@ __device__ __forceinline__ void bwd_tcq_softmax(const BwdParams& p, BwdTcQSmem& 
     }
     // dS of set X was last read by step t-2's dQ product, which completed
     // before step t's S (s_full covers all earlier products)
-    tmem_st16(set + kColP + ch * 16, dk);
+    tmem_st8(set + kColP + ch * (kBwdTcCols / 2), dk);
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(&sm.p_full[X]);
   }
   // ---- epilogue: warps 0-3 write this query row of dq (scale, c R^T) ----
+  if (ch != 0) return;  // warp-uniform
   if (!mbar_wait_warp(&sm.mma_done, 0, p.wait_ns)) return;
   tc_fence_after();
-  if (ch != 0) return;  // warp-uniform
   uint32_t a[32], bb[32];
   tmem_ld32(lane_base + kColDQ, a);        // features [0, 32)
   tmem_ld32(lane_base + kColDQ + 32, bb);  // features [32, 64)
@@ -591,7 +617,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dq_tc_kernel(const 
     mbar_init(&sm.mma_done, 1);
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == kBwdTcSoftWarps + 1) {
     tmem_alloc(&sm.tmem_base, kBwdTcTmemCols);
     tmem_relinquish();
   }
@@ -599,12 +625,12 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dq_tc_kernel(const 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp < 8) bwd_tcq_softmax(p, sm, w, tmem);
-  else if (warp == 8 && lane == 0) bwd_tcq_producer(p, sm, w);
-  else if (warp == 9 && lane == 0) bwd_tcq_mma(p, sm, w, tmem);
+  if (warp < kBwdTcSoftWarps) bwd_tcq_softmax(p, sm, w, tmem);
+  else if (warp == kBwdTcSoftWarps && lane == 0) bwd_tcq_producer(p, sm, w);
+  else if (warp == kBwdTcSoftWarps + 1 && lane == 0) bwd_tcq_mma(p, sm, w, tmem);
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kBwdTcSoftWarps + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kBwdTcTmemCols);
   }
