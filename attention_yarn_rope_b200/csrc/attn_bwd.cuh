@@ -59,6 +59,7 @@ struct BwdParams {
   gptoss_strides sv, so, sdo;  // elements; BSHD uses batch, THD ignores it
   const float* lse;            // the forward's: BSHD [B, Hq, S], THD [Hq, T]
   float* dsum;                 // D, same layout as lse
+  float* lse2;                 // lse log2(e), same layout (the tcgen05 dK / dV kernel's copy)
   const float2* cs;            // [T][32] (c cos, c sin) of every token's pairs
   const float* sinks;          // [Hq]
   float* dsinks;               // [Hq], accumulated (zeroed before the launches)
@@ -147,7 +148,9 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const __grid_c
     for (int c = 0; c < 8; ++c) acc += dot8_bf16(__ldg(o + c), __ldg(d + c));
     const int64_t ri = bwd_row_index(p, b, h, i, sq.tok0);
     p.dsum[ri] = acc;
-    const float share = ex2_approx((__ldg(p.sinks + h) - __ldg(p.lse + ri)) * kLog2e);
+    const float lse = __ldg(p.lse + ri);
+    p.lse2[ri] = lse * kLog2e;
+    const float share = ex2_approx((__ldg(p.sinks + h) - lse) * kLog2e);
     atomicAdd(&part[h], -share * acc);
   }
   __syncthreads();

@@ -58,7 +58,7 @@ struct __align__(1024) BwdTcSmem {
   uint8_t v[kBwdTcKeys * 128];                 // V tile (bf16)
   uint8_t q[kBwdTcStages][kBwdTcQ * 128];      // rotated q tiles (fp16)
   uint8_t dout[kBwdTcStages][kBwdTcQ * 128];   // dout tiles (bf16)
-  float lsd[kBwdTcStages][2 * kBwdTcQ];        // per stage: lse [0, 64) and D [64, 128) of its queries
+  float lsd[kBwdTcStages][2 * kBwdTcQ];        // per stage: lse log2(e) [0, 64) and D [64, 128) of its queries
   uint64_t kv_full;
   uint64_t qd_full[kBwdTcStages], qd_empty[kBwdTcStages];
   uint64_t s_full[2], s_free[2], p_full[2];
@@ -103,6 +103,40 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
 
 // fp16 A and B with B read N-major (the q tile in dK += dS^T Q).
 __host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) { return idesc_f16_f32(M, N) | (1u << 16); }
+
+// Bits [max(lo, 0), min(hi, 15)] of a 16-bit mask (empty when lo > hi).
+__device__ __forceinline__ uint32_t col_mask16(int lo, int hi) {
+  const uint32_t upto = hi >= 15 ? 0xffffu : (hi < 0 ? 0u : (2u << hi) - 1u);
+  const uint32_t from = lo <= 0 ? 0xffffu : (lo > 15 ? 0u : (0xffffu << lo) & 0xffffu);
+  return upto & from;
+}
+
+// P^T (bf16) and dS^T = P^T (dP^T - D) (fp16) for 16 query columns of one key
+// row: P = 2^(s scale log2(e) - lse log2(e)), zero where bit c of `vis` is
+// clear (kMasked).  lse2 / dsum: the columns' lse in log2 units and D.
+template <bool kMasked>
+__device__ __forceinline__ void bwd_p_ds(const uint32_t (&sv)[16], const uint32_t (&dv)[16], const float4 (&l4s)[4],
+                                         const float4 (&d4s)[4], float sl, uint32_t vis, uint32_t (&pk)[8],
+                                         uint32_t (&dk)[8]) {
+#pragma unroll
+  for (int e = 0; e < 16; e += 4) {
+    const float4 l4 = l4s[e / 4];
+    const float4 d4 = d4s[e / 4];
+    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+    const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+    float pv[4], ds[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      pv[u] = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl, -lv[u]));
+      if (kMasked) pv[u] = (vis >> (e + u)) & 1u ? pv[u] : 0.f;
+      ds[u] = pv[u] * (__uint_as_float(dv[e + u]) - dd[u]);
+    }
+    pk[e / 2] = pack_bf16(pv[0], pv[1]);
+    pk[e / 2 + 1] = pack_bf16(pv[2], pv[3]);
+    dk[e / 2] = pack_f16(ds[0], ds[1]);
+    dk[e / 2 + 1] = pack_f16(ds[2], ds[3]);
+  }
+}
 
 // The CTA's sweep: steps [it0, it1) over (query head of the group, query
 // tile), query tiles [qt0, qt0 + n_qt) of the sequence.
@@ -165,14 +199,15 @@ __device__ __forceinline__ void bwd_tc_producer(const BwdParams& p, BwdTcSmem& s
       tma_load_4d(sm.q[s], &p.tmap_q, &sm.qd_full[s], 0, h, row0 + i0, bc);
       tma_load_4d(sm.dout[s], &p.tmap_do, &sm.qd_full[s], 0, h, row0 + i0, bc);
     }
-    // slots 4 lane .. 4 lane + 3: lse of queries [0, 64), D of [64, 128); a
-    // query past the sequence copies the last row's (finite, masked anyway)
+    // slots 4 lane .. 4 lane + 3: lse log2(e) of queries [0, 64) (scaled once
+    // by the preprocess kernel), D of [64, 128); a query past the sequence
+    // copies the last row's (finite, masked anyway)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int slot = 4 * lane + u;
       const int i = min(i0 + (slot & (kBwdTcQ - 1)), L - 1);
       const int64_t ri = bwd_row_index(p, w.b, h, i, w.sq.tok0);
-      cp_async4(smem_u32(&sm.lsd[s][slot]), (slot < kBwdTcQ ? p.lse : p.dsum) + ri);
+      cp_async4(smem_u32(&sm.lsd[s][slot]), (slot < kBwdTcQ ? p.lse2 : p.dsum) + ri);
     }
     cp_async_mbar_arrive_noinc(&sm.qd_full[s]);
   }
@@ -255,6 +290,13 @@ __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm
     // stay until this step's gradient products free the stage (qd_empty),
     // which follows this thread's p_full arrival below
     if (!mbar_wait_warp(&sm.qd_full[stg], (t / kBwdTcStages) & 1, p.wait_ns)) return;
+    // the step's lse / D columns, read while S^T / dP^T are still in flight
+    float4 l4s[4], d4s[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      l4s[e] = *reinterpret_cast<const float4*>(&sm.lsd[stg][ch * kBwdTcCols + 4 * e]);
+      d4s[e] = *reinterpret_cast<const float4*>(&sm.lsd[stg][kBwdTcQ + ch * kBwdTcCols + 4 * e]);
+    }
     if (!mbar_wait_warp(&sm.s_full[X], (t >> 1) & 1, p.wait_ns)) return;
     tc_fence_after();
     const uint32_t set = lane_base + X * kColSet;
@@ -264,30 +306,16 @@ __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm
     tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(&sm.s_free[X]);  // S^T / dP^T of set X may be overwritten
-    const float* lse = &sm.lsd[stg][ch * kBwdTcCols];
-    const float* dsum = &sm.lsd[stg][kBwdTcQ + ch * kBwdTcCols];
     // every pair of this warp's 32 keys x 16 queries visible: no mask
     const int jw = w.k0 + wq * 32;
     const bool all_vis = jw + 31 <= i0 && i0 + kBwdTcCols - 1 < L && jw + 31 < L &&
                          (W == 0 || i0 + kBwdTcCols - 1 - jw < W);
     uint32_t pk[kBwdTcCols / 2], dk[kBwdTcCols / 2];
-#pragma unroll
-    for (int e = 0; e < kBwdTcCols; e += 4) {
-      const float4 l4 = *reinterpret_cast<const float4*>(lse + e);
-      const float4 d4 = *reinterpret_cast<const float4*>(dsum + e);
-      const float lv[4] = {l4.x * kLog2e, l4.y * kLog2e, l4.z * kLog2e, l4.w * kLog2e};
-      const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-      float pv[4], ds[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const bool vis = all_vis || (j_ok && bwd_visible(i0 + e + u, j, L, W));
-        pv[u] = vis ? ex2_approx(__uint_as_float(sv[e + u]) * sl - lv[u]) : 0.f;
-        ds[u] = pv[u] * (__uint_as_float(dv[e + u]) - dd[u]);
-      }
-      pk[e / 2] = pack_bf16(pv[0], pv[1]);
-      pk[e / 2 + 1] = pack_bf16(pv[2], pv[3]);
-      dk[e / 2] = pack_f16(ds[0], ds[1]);
-      dk[e / 2 + 1] = pack_f16(ds[2], ds[3]);
+    if (all_vis) {
+      bwd_p_ds<false>(sv, dv, l4s, d4s, sl, 0u, pk, dk);
+    } else {  // this key's visible queries i0 + c: c in [j - i0, min(L - 1, j + W - 1) - i0]
+      const int hi = (W > 0 ? min(L - 1, j + W - 1) : L - 1) - i0;
+      bwd_p_ds<true>(sv, dv, l4s, d4s, sl, j_ok ? col_mask16(j - i0, hi) : 0u, pk, dk);
     }
     // P^T / dS^T of set X were last read by step t-2's gradient products,
     // which completed before step t's S^T (s_full covers all earlier products)
@@ -544,14 +572,16 @@ __device__ __forceinline__ void bwd_tcq_softmax(const BwdParams& p, BwdTcQSmem& 
     mbar_arrive(&sm.s_free[X]);  // S / dP of set X may be overwritten
     // every pair of this warp's 32 queries x 16 keys visible: no mask
     const bool all_vis = j0 + kBwdTcCols - 1 <= iw && iw + 31 < L && (W == 0 || iw + 31 - j0 < W);
+    // else this query's visible keys j0 + c: c in [i - W + 1 - j0, i - j0]
+    const uint32_t vis = all_vis ? 0xffffu : (i_ok ? col_mask16(W > 0 ? i - W + 1 - j0 : 0, i - j0) : 0u);
     uint32_t dk[kBwdTcCols / 2];
 #pragma unroll
     for (int e = 0; e < kBwdTcCols; e += 2) {
       float ds[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const bool vis = all_vis || (i_ok && bwd_visible(i, j0 + e + u, L, W));
-        const float pv = vis ? ex2_approx(__uint_as_float(sv[e + u]) * sl - lse2) : 0.f;
+        float pv = ex2_approx(fmaf(__uint_as_float(sv[e + u]), sl, -lse2));
+        pv = (vis >> (e + u)) & 1u ? pv : 0.f;
         ds[u] = pv * (__uint_as_float(dv[e + u]) - dd);
       }
       dk[e / 2] = pack_f16(ds[0], ds[1]);

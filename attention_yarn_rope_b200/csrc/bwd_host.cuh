@@ -21,10 +21,11 @@ namespace {
 inline size_t bwd_round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace: rotated q (fp16) | rotated k (fp16) | per-token (c cos, c sin)
-// table | D = <dout, out> (fp32, lse layout) | dK and dV fp32 accumulators of
-// split sweeps (adjacent, zeroed with one memset), each 256-byte aligned.
+// table | D = <dout, out> (fp32, lse layout) | lse log2(e) (fp32, lse layout)
+// | dK and dV fp32 accumulators of split sweeps (adjacent, zeroed with one
+// memset), each 256-byte aligned.
 struct BwdWorkspace {
-  size_t q, k, cs, d, acc, acc_bytes, total;
+  size_t q, k, cs, d, l2, acc, acc_bytes, total;
 };
 
 inline BwdWorkspace bwd_workspace(int64_t T, int Hq, int Hkv) {
@@ -33,7 +34,8 @@ inline BwdWorkspace bwd_workspace(int64_t T, int Hq, int Hkv) {
   w.k = w.q + bwd_round256(static_cast<size_t>(T) * Hq * kHeadDim * 2);
   w.cs = w.k + bwd_round256(static_cast<size_t>(T) * Hkv * kHeadDim * 2);
   w.d = w.cs + bwd_round256(static_cast<size_t>(T) * kPairs * sizeof(float2));
-  w.acc = w.d + bwd_round256(static_cast<size_t>(T) * Hq * sizeof(float));
+  w.l2 = w.d + bwd_round256(static_cast<size_t>(T) * Hq * sizeof(float));
+  w.acc = w.l2 + bwd_round256(static_cast<size_t>(T) * Hq * sizeof(float));
   w.acc_bytes = 2 * static_cast<size_t>(T) * Hkv * kHeadDim * sizeof(float);
   w.total = w.acc + bwd_round256(w.acc_bytes);
   return w;
@@ -132,6 +134,7 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   p.sdo = sdo;
   p.lse = lse;
   p.dsum = reinterpret_cast<float*>(wsb + ws.d);
+  p.lse2 = reinterpret_cast<float*>(wsb + ws.l2);
   p.cs = rp.cs_out;
   p.sinks = sinks;
   p.dsinks = dsinks;

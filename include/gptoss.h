@@ -232,8 +232,9 @@ gptoss_status gptoss_qkv_rope(const void* x, int64_t x_row_stride, const void* w
                               struct CUstream_st* stream);
 
 /* Workspace bytes gptoss_attn_bwd needs: q and k rotated once (fp16), every
- * token's 32 RoPE angles, and <dout, out> per row and head (fp32).  0 when a
- * size is out of range. */
+ * token's 32 RoPE angles, <dout, out> and lse log2(e) per row and head (fp32),
+ * and fp32 dk / dv accumulators for split sweeps.  0 when a size is out of
+ * range. */
 size_t gptoss_attn_bwd_workspace_size(int32_t total_tokens, int32_t Hq, int32_t Hkv, int32_t D);
 
 /* gptoss_attn_bwd -- gradients of gptoss_attn_fwd for L = sum(dout * out):

@@ -92,9 +92,10 @@ def test_attn_fwd_validation(lib):
 
 def test_attn_bwd_validation(lib):
     need = lib.gptoss_attn_bwd_workspace_size(4096, 64, 8, 64)
-    # rotated q and k (fp16) + per-token angle table + <dout, out> per row and head
-    # + fp32 dK and dV accumulators of split sweeps
-    assert need == 4096 * 64 * 64 * 2 + 4096 * 8 * 64 * 2 + 4096 * 32 * 8 + 4096 * 64 * 4 + 2 * 4096 * 8 * 64 * 4
+    # rotated q and k (fp16) + per-token angle table + <dout, out> and lse log2(e)
+    # per row and head + fp32 dK and dV accumulators of split sweeps
+    assert need == (4096 * 64 * 64 * 2 + 4096 * 8 * 64 * 2 + 4096 * 32 * 8 + 2 * 4096 * 64 * 4
+                    + 2 * 4096 * 8 * 64 * 4)
     assert lib.gptoss_attn_bwd_workspace_size(4096, 64, 7, 64) == 0
     assert lib.gptoss_attn_bwd_workspace_size(4096, 64, 8, 128) == 0
 
