@@ -40,7 +40,7 @@ namespace gptoss {
 
 constexpr int kBwdTcKeys = 128;      // keys per CTA (the M side)
 constexpr int kBwdTcQ = 64;          // queries per step (the N side)
-constexpr int kBwdTcStages = 4;      // q / dout buffers: loads run 3 steps ahead of their use
+constexpr int kBwdTcStages = 6;      // q / dout buffers: loads run 5 steps ahead of their use (measured: 6 beat 4 by 0.5 %)
 // 16 softmax warps: four per sub-partition, each thread 16 columns of a step
 // (measured: 8 warps of 32 columns left the per-step chain -- TMEM loads,
 // exponentials, stores -- unhidden, ~3300 cycles a step against ~500 of
@@ -49,7 +49,11 @@ constexpr int kBwdTcSoftmax = 512;
 constexpr int kBwdTcSoftWarps = kBwdTcSoftmax / 32;
 constexpr int kBwdTcCols = 16;  // columns of a 64-column step per softmax thread
 constexpr int kBwdTcThreads = kBwdTcSoftmax + 64;  // + producer warp, MMA warp
-constexpr int kBwdTcChunkIt = 64;    // steps of one CTA when sweeps are split
+// steps of one CTA when sweeps are split (measured on full causal S = 8192,
+// whose longest sweep has 1024 steps: 64 -> 7.24 ms, 128 -> 7.05, 192 -> 6.99,
+// 256 -> 7.01, 512 -> 7.07; fewer chunks add fewer fp32 partials, more leave
+// the longest CTAs running alone)
+constexpr int kBwdTcChunkIt = 192;
 constexpr uint32_t kBwdTcTmemCols = 512;
 constexpr uint32_t kColSet = 192, kColDP = 64, kColP = 128, kColDS = 160, kColDV = 384, kColDK = 448;
 
@@ -425,7 +429,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dkdv_tc_kernel(cons
 // dQ on the tensor cores.  CTA = (128-query tile, head, sequence), 18 warps:
 // 16 softmax warps (TMEM lanes 32 (w % 4) .. = query rows, key columns
 // 16 (w / 4) .. of the step), a TMA producer (Q and dout tiles once, then each
-// step's 64-key K and V tiles, 4 stages ahead), an MMA issuer.  Per step:
+// step's 64-key K and V tiles, kBwdTcStages ahead), an MMA issuer.  Per step:
 //   S  = Q K^T, dP = dout V^T   (SS, K-major; M = 128 queries, N = 64 keys)
 //   dS = P (dP - D) -> tensor memory (fp16), P = exp(S scale - lse)
 //   dQ += dS K                  (TS: dS from tensor memory, K read N-major)

@@ -261,7 +261,7 @@ size_t gptoss_attn_bwd_workspace_size(int32_t total_tokens, int32_t Hq, int32_t 
  *          Hq, Hkv, D) bytes, 16-byte aligned, owned by the caller, contents
  *          need not be initialised.
  * Kernels on `stream`: q / k rotation; D and dsinks; dk / dv on the tcgen05
- * tensor cores (one CTA per 128-key tile and kv head; sweeps longer than 64
+ * tensor cores (one CTA per 128-key tile and kv head; sweeps longer than 192
  * (head, 64-query tile) steps split into chunks that add into fp32
  * accumulators, then one finishing kernel); dq (one CTA per query tile and
  * head: tcgen05 for full context or windows of 1024+ keys, warp-level
