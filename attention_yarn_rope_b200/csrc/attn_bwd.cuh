@@ -61,6 +61,7 @@ struct BwdParams {
   float* dsum;                 // D, same layout as lse
   float* lse2;                 // lse log2(e), same layout (the tcgen05 dK / dV kernel's copy)
   const float2* cs;            // [T][32] (c cos, c sin) of every token's pairs
+  int R;                       // rotary pairs: features (j, j + R), j < R, rotate; [2R, 64) pass through
   const float* sinks;          // [Hq]
   float* dsinks;               // [Hq], accumulated (zeroed before the launches)
   __nv_bfloat16* dq;           // dense [T, Hq, 64]
@@ -177,9 +178,21 @@ __device__ __forceinline__ void load_a_frag(uint32_t (&a)[4][4], const __nv_bflo
   }
 }
 
+// RoPE taken back (the adjoint c R(theta)^T of gpt_oss.rope_utils'
+// apply_rotary_emb, R rotary pairs (j, j + R)): pair j's (x, y) = (g_j,
+// g_{j+R}) -> (x cc + y cs, y cc - x cs) with (cc, cs) = the row's (c cos, c
+// sin) of pair j; features past 2R pass through unchanged (they carry no
+// concentration).
+__device__ __forceinline__ void rope_t_pair(float x, float y, float2 c, float& xr, float& yr) {
+  xr = x * c.x + y * c.y;
+  yr = y * c.x - x * c.y;
+}
+
 // Writes a 16 x 64 fp32 accumulator (C fragments, rows gr / gr + 8) as bf16
-// rows, optionally scaled and taken back through RoPE: for pair (d, d + 32),
-// (x, y) -> (x cc + y cs, y cc - x cs) with (cc, cs) = the row's (c cos, c sin).
+// rows, optionally scaled and taken back through RoPE with R rotary pairs
+// (rope_t_pair); a thread's features d = 8 nf + 2 tq + e and their partners
+// d + R (fragment nf + R / 8) sit in the same thread.
+template <int R>
 __device__ __forceinline__ void store_rows(const float (&acc)[8][4], __nv_bfloat16* row_lo, __nv_bfloat16* row_hi,
                                            const float2* cs_lo, const float2* cs_hi, bool lo_ok, bool hi_ok,
                                            float scale, bool rotate, int tq) {
@@ -197,25 +210,26 @@ __device__ __forceinline__ void store_rows(const float (&acc)[8][4], __nv_bfloat
             pack_bf16(acc[nf][e0] * scale, acc[nf][e0 + 1] * scale);
       continue;
     }
+    constexpr int kNp = R / 8;  // partner offset in fragments
 #pragma unroll
-    for (int nf = 0; nf < 4; ++nf) {
-      const int d = 8 * nf + 2 * tq;  // pairs d, d + 1 and their partners d + 32, d + 33
+    for (int nf = 0; nf < kNp; ++nf) {
+      const int d = 8 * nf + 2 * tq;  // pairs d, d + 1 and their partners d + R, d + R + 1
       float xr[2], yr[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float x = acc[nf][e0 + e] * scale, y = acc[nf + 4][e0 + e] * scale;
-        const float2 c = __ldg(cs + d + e);
-        xr[e] = x * c.x + y * c.y;
-        yr[e] = y * c.x - x * c.y;
-      }
+      for (int e = 0; e < 2; ++e)
+        rope_t_pair(acc[nf][e0 + e] * scale, acc[nf + kNp][e0 + e] * scale, __ldg(cs + d + e), xr[e], yr[e]);
       *reinterpret_cast<uint32_t*>(row + d) = pack_bf16(xr[0], xr[1]);
-      *reinterpret_cast<uint32_t*>(row + d + 32) = pack_bf16(yr[0], yr[1]);
+      *reinterpret_cast<uint32_t*>(row + d + R) = pack_bf16(yr[0], yr[1]);
     }
+#pragma unroll
+    for (int nf = 2 * kNp; nf < 8; ++nf)  // past the rotary features
+      *reinterpret_cast<uint32_t*>(row + 8 * nf + 2 * tq) =
+          pack_bf16(acc[nf][e0] * scale, acc[nf][e0 + 1] * scale);
   }
 }
 
 // Split sweeps: dk = c R^T (scale dK_acc) and dv = dV_acc as bf16.  Thread
-// (token, kv head, pair j) handles features j and j + 32.
+// (token, kv head, j) handles features j and j + 32.
 __global__ void __launch_bounds__(256) attn_bwd_dkdv_finish_kernel(const __grid_constant__ BwdParams p) {
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= static_cast<int64_t>(p.T) * p.Hkv * kPairs) return;
@@ -223,10 +237,21 @@ __global__ void __launch_bounds__(256) attn_bwd_dkdv_finish_kernel(const __grid_
   const int64_t tg = idx / kPairs;  // token * Hkv + kv head
   const int64_t t = tg / p.Hkv;
   const int64_t row = tg * kHeadDim;
-  const float x = p.dk_acc[row + j] * p.scale, y = p.dk_acc[row + j + kPairs] * p.scale;
-  const float2 c = __ldg(p.cs + t * kPairs + j);
-  p.dk[row + j] = __float2bfloat16_rn(x * c.x + y * c.y);
-  p.dk[row + j + kPairs] = __float2bfloat16_rn(y * c.x - x * c.y);
+  // features j and j + 32: the rotary pair (j, j + R) is handled by its
+  // first feature's thread, features past 2R pass through
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int f = j + u * kPairs;
+    if (f < p.R) {
+      float xr, yr;
+      rope_t_pair(p.dk_acc[row + f] * p.scale, p.dk_acc[row + f + p.R] * p.scale, __ldg(p.cs + t * kPairs + f), xr,
+                  yr);
+      p.dk[row + f] = __float2bfloat16_rn(xr);
+      p.dk[row + f + p.R] = __float2bfloat16_rn(yr);
+    } else if (f >= 2 * p.R) {
+      p.dk[row + f] = __float2bfloat16_rn(p.dk_acc[row + f] * p.scale);
+    }
+  }
   p.dv[row + j] = __float2bfloat16_rn(p.dv_acc[row + j]);
   p.dv[row + j + kPairs] = __float2bfloat16_rn(p.dv_acc[row + j + kPairs]);
 }
@@ -237,6 +262,10 @@ struct __align__(128) BwdQSmem {
 };
 
 // 3 CTAs per SM: at most 170 registers a thread.
+// R: the call's rotary pairs (p.R), a template parameter so each
+// instantiation holds one RoPE transpose (measured: a runtime switch among
+// four cost the sliding-window backward 2.7 %).
+template <int R>
 __global__ void __launch_bounds__(kBwdThreads, 3) attn_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   __shared__ BwdQSmem sm;
   const int qt = p.n_tiles - 1 - static_cast<int>(blockIdx.x);  // the longest sweeps start first
@@ -351,8 +380,10 @@ __global__ void __launch_bounds__(kBwdThreads, 3) attn_bwd_dq_kernel(const __gri
     __syncthreads();  // the buffer is refilled two iterations on
   }
   const int64_t tl = sq.tok0 + il, th = sq.tok0 + ih;
-  store_rows(dq, p.dq + (tl * p.Hq + h) * kHeadDim, p.dq + (th * p.Hq + h) * kHeadDim, p.cs + tl * kPairs,
-             p.cs + th * kPairs, il_ok, ih_ok, p.scale, true, tq);
+  __nv_bfloat16* rl = p.dq + (tl * p.Hq + h) * kHeadDim;
+  __nv_bfloat16* rh = p.dq + (th * p.Hq + h) * kHeadDim;
+  const float2 *cl = p.cs + tl * kPairs, *ch = p.cs + th * kPairs;
+  store_rows<R>(dq, rl, rh, cl, ch, il_ok, ih_ok, p.scale, true, tq);
 }
 
 }  // namespace gptoss

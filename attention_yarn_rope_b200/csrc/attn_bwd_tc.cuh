@@ -105,6 +105,41 @@ __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// A row of dK or dQ in tensor memory (features [0, 32) in a, [32, 64) in
+// bb) scaled and taken back through RoPE with R rotary pairs (rope_t_pair),
+// as bf16 pairs: lo = features [0, 32), hi = [32, 64).
+template <int R>
+__device__ __forceinline__ void rope_t_row(const uint32_t (&a)[32], const uint32_t (&bb)[32], const float2* cs,
+                                           float scale, uint32_t (&lo)[16], uint32_t (&hi)[16]) {
+  auto g = [&](int f) { return __uint_as_float(f < 32 ? a[f] : bb[f - 32]) * scale; };
+  auto put = [&](int w, uint32_t v) {  // output word w: features 2w, 2w + 1
+    if (w < 16) lo[w] = v;
+    else hi[w - 16] = v;
+  };
+#pragma unroll
+  for (int j = 0; j < R; j += 2) {  // pairs j, j + 1 and their partners j + R, j + R + 1
+    float xr[2], yr[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) rope_t_pair(g(j + u), g(j + u + R), __ldg(cs + j + u), xr[u], yr[u]);
+    put(j / 2, pack_bf16(xr[0], xr[1]));
+    put((j + R) / 2, pack_bf16(yr[0], yr[1]));
+  }
+#pragma unroll
+  for (int f = 2 * R; f < 64; f += 2) put(f / 2, pack_bf16(g(f), g(f + 1)));  // past the rotary features
+}
+
+// rope_t_row for the call's rotary pairs (a multiple of 8: rotary_dim is a
+// multiple of 16).
+__device__ __forceinline__ void rope_t_row_r(int R, const uint32_t (&a)[32], const uint32_t (&bb)[32],
+                                             const float2* cs, float scale, uint32_t (&lo)[16], uint32_t (&hi)[16]) {
+  switch (R) {
+    case 8: rope_t_row<8>(a, bb, cs, scale, lo, hi); break;
+    case 16: rope_t_row<16>(a, bb, cs, scale, lo, hi); break;
+    case 24: rope_t_row<24>(a, bb, cs, scale, lo, hi); break;
+    default: rope_t_row<32>(a, bb, cs, scale, lo, hi); break;
+  }
+}
+
 // fp16 A and B with B read N-major (the q tile in dK += dS^T Q).
 __host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) { return idesc_f16_f32(M, N) | (1u << 16); }
 
@@ -360,21 +395,8 @@ __device__ __forceinline__ void bwd_tc_softmax(const BwdParams& p, BwdTcSmem& sm
       lo[e] = pack_bf16(__uint_as_float(a[2 * e]), __uint_as_float(a[2 * e + 1]));
       hi[e] = pack_bf16(__uint_as_float(bb[2 * e]), __uint_as_float(bb[2 * e + 1]));
     }
-  } else {  // pair (d, d + 32): (x, y) -> (x cc + y cs, y cc - x cs), after the scale
-    const float2* cs = p.cs + tok * kPairs;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      float xr[2], yr[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const float x = __uint_as_float(a[2 * e + u]) * p.scale, y = __uint_as_float(bb[2 * e + u]) * p.scale;
-        const float2 c = __ldg(cs + 2 * e + u);
-        xr[u] = x * c.x + y * c.y;
-        yr[u] = y * c.x - x * c.y;
-      }
-      lo[e] = pack_bf16(xr[0], xr[1]);
-      hi[e] = pack_bf16(yr[0], yr[1]);
-    }
+  } else {  // scale, then c R^T
+    rope_t_row_r(p.R, a, bb, p.cs + tok * kPairs, p.scale, lo, hi);
   }
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4) {
@@ -544,6 +566,7 @@ __device__ __forceinline__ void bwd_tcq_mma(const BwdParams& p, BwdTcQSmem& sm, 
   mbar_wait(&sm.mma_done, 0, p.wait_ns);
 }
 
+template <int R>
 __device__ __forceinline__ void bwd_tcq_softmax(const BwdParams& p, BwdTcQSmem& sm, const BwdTcQWork& w,
                                                 uint32_t tmem) {
   const int tid = threadIdx.x;         // 0 .. 511
@@ -608,21 +631,8 @@ __device__ __forceinline__ void bwd_tcq_softmax(const BwdParams& p, BwdTcQSmem& 
   if (!i_ok) return;
   const int64_t tok = w.sq.tok0 + i;
   __nv_bfloat16* dst = p.dq + (tok * p.Hq + w.h) * kHeadDim;
-  const float2* cs = p.cs + tok * kPairs;
   uint32_t lo[16], hi[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    float xr[2], yr[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const float x = __uint_as_float(a[2 * e + u]) * p.scale, y = __uint_as_float(bb[2 * e + u]) * p.scale;
-      const float2 c = __ldg(cs + 2 * e + u);
-      xr[u] = x * c.x + y * c.y;
-      yr[u] = y * c.x - x * c.y;
-    }
-    lo[e] = pack_bf16(xr[0], xr[1]);
-    hi[e] = pack_bf16(yr[0], yr[1]);
-  }
+  rope_t_row<R>(a, bb, p.cs + tok * kPairs, p.scale, lo, hi);
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4) {
     reinterpret_cast<uint4*>(dst)[q4] = make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
@@ -630,6 +640,9 @@ __device__ __forceinline__ void bwd_tcq_softmax(const BwdParams& p, BwdTcQSmem& 
   }
 }
 
+// R: the call's rotary pairs (p.R), a template parameter as for
+// attn_bwd_dq_kernel (measured: a runtime switch cost full causal 0.7 %).
+template <int R>
 __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dq_tc_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   BwdTcQSmem& sm = *reinterpret_cast<BwdTcQSmem*>(
@@ -659,7 +672,7 @@ __global__ void __launch_bounds__(kBwdTcThreads, 1) attn_bwd_dq_tc_kernel(const 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp < kBwdTcSoftWarps) bwd_tcq_softmax(p, sm, w, tmem);
+  if (warp < kBwdTcSoftWarps) bwd_tcq_softmax<R>(p, sm, w, tmem);
   else if (warp == kBwdTcSoftWarps && lane == 0) bwd_tcq_producer(p, sm, w);
   else if (warp == kBwdTcSoftWarps + 1 && lane == 0) bwd_tcq_mma(p, sm, w, tmem);
   tc_fence_before();

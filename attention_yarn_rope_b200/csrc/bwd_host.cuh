@@ -62,7 +62,7 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   if (D != kHeadDim) return GPTOSS_ERR_UNSUPPORTED;
   if (Hq > kBwdMaxHeads || B > 65535) return GPTOSS_ERR_UNSUPPORTED;
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return GPTOSS_ERR_INVALID_ARG;
-  gptoss_status st = check_rope(rope, D);
+  gptoss_status st = check_rope(rope, D, /*allow_partial=*/true);
   if (st != GPTOSS_OK) return st;
   const bool thd = cu_seqlens != nullptr;
   if (!thd && static_cast<int64_t>(B) * S != total_tokens) return GPTOSS_ERR_INVALID_ARG;
@@ -136,6 +136,7 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   p.dsum = reinterpret_cast<float*>(wsb + ws.d);
   p.lse2 = reinterpret_cast<float*>(wsb + ws.l2);
   p.cs = rp.cs_out;
+  p.R = rp.tab.R;
   p.sinks = sinks;
   p.dsinks = dsinks;
   p.dq = static_cast<__nv_bfloat16*>(dq);
@@ -212,14 +213,24 @@ gptoss_status gptoss_attn_bwd(const void* q, gptoss_strides sq, const void* k, g
   // windows of 1024+ keys: 16+ key tiles per query tile).  Short sweeps (a
   // 128-key window: 4-5 tiles) run faster on the mma.sync kernel, three
   // CTAs to an SM (measured, B=4 S=4096 W=128: 1.27 against 1.66 ms).
+  // both dQ kernels are instantiated per rotary pair count (a multiple of 8
+  // up to 32: check_rope admits rotary_dim in multiples of 16)
   if (window == 0 || window >= 1024) {
+    void (*dq)(BwdParams) = p.R == 8    ? attn_bwd_dq_tc_kernel<8>
+                            : p.R == 16 ? attn_bwd_dq_tc_kernel<16>
+                            : p.R == 24 ? attn_bwd_dq_tc_kernel<24>
+                                        : attn_bwd_dq_tc_kernel<32>;
     const size_t q_smem = sizeof(BwdTcQSmem) + 1024;
-    if (cudaFuncSetAttribute(attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(q_smem)) != cudaSuccess)
+    if (cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(q_smem)) !=
+        cudaSuccess)
       return GPTOSS_ERR_CUDA;
-    attn_bwd_dq_tc_kernel<<<dim3((S + 127) / 128, Hq, B), kBwdTcThreads, q_smem, s>>>(p);
+    dq<<<dim3((S + 127) / 128, Hq, B), kBwdTcThreads, q_smem, s>>>(p);
   } else {
-    attn_bwd_dq_kernel<<<dim3(p.n_tiles, Hq, B), kBwdThreads, 0, s>>>(p);
+    void (*dq)(BwdParams) = p.R == 8    ? attn_bwd_dq_kernel<8>
+                            : p.R == 16 ? attn_bwd_dq_kernel<16>
+                            : p.R == 24 ? attn_bwd_dq_kernel<24>
+                                        : attn_bwd_dq_kernel<32>;
+    dq<<<dim3(p.n_tiles, Hq, B), kBwdThreads, 0, s>>>(p);
   }
   return check_launch();
 }

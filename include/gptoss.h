@@ -43,8 +43,9 @@
  *   - Device-side conditions (a bounded pipeline wait that gave up, a block
  *     index outside a paged pool) are recorded in a device status word read
  *     by gptoss_read_device_status.
- *   - bf16 tensors are IEEE bfloat16; head_dim D must be 64 and contiguous
- *     (element stride 1); rotary_dim must equal D.
+ *   - bf16 tensors are IEEE bfloat16; head_dim D is 64 (128 where an entry
+ *     says so) and contiguous (element stride 1); rotary_dim: see
+ *     gptoss_rope_params.
  *   - No C++ exception crosses this ABI.
  */
 #ifndef GPTOSS_H_
@@ -79,9 +80,11 @@ typedef struct gptoss_rope_params {
   int32_t initial_context; /* initial_context_length, 4096 */
   int32_t rotary_dim;      /* int(head_dim * partial_rotary_factor): features [0, rotary_dim)
                               rotate in pairs (j, j + rotary_dim/2), the rest pass through
-                              unchanged; even, at most D.  gptoss_rope_qk, gptoss_attn_fwd, the
-                              decodes and the append take any multiple of 16 (partial rotary);
-                              gptoss_attn_bwd needs rotary_dim == D (else UNSUPPORTED) */
+                              unchanged; even, at most D.  gptoss_rope_qk, the decodes, the
+                              append, gptoss_attn_bwd, gptoss_attn_fwd at D = 64 and its block
+                              form take any multiple of 16 (partial rotary); gptoss_attn_fwd at
+                              D = 128 and gptoss_qkv_rope need rotary_dim == D (else
+                              UNSUPPORTED) */
   double ntk_alpha;        /* 1 */
   double ntk_beta;         /* 32 */
 } gptoss_rope_params;

@@ -105,10 +105,14 @@ def test_attn_bwd_validation(lib):
         a.update(kw)
         return lib.gptoss_attn_bwd(a["q"], a["sq"], FAKE, S_BSHD_K, FAKE, S_BSHD_K, FAKE, S_BSHD_Q, a["dout"],
                                    S_BSHD_Q, a["lse"], FAKE, None, None, a["B"], a["S"], a["T"], a["Hq"], a["Hkv"],
-                                   a["D"], a["window"], a["scale"], ctypes.byref(ROPE), a["dq"], FAKE, FAKE,
-                                   a["dsinks"], a["ws"], a["wsb"], None)
+                                   a["D"], a["window"], a["scale"], ctypes.byref(a.get("rope", ROPE)), a["dq"], FAKE,
+                                   FAKE, a["dsinks"], a["ws"], a["wsb"], None)
 
     assert call(D=128) == _abi.GPTOSS_ERR_UNSUPPORTED
+    # partial rotary: a multiple of 16 features (whole 8-pair groups of the
+    # RoPE transpose); others are unsupported
+    assert call(rope=_abi.RopeParams(150000.0, 32.0, 4096, 40, 1.0, 32.0)) == _abi.GPTOSS_ERR_UNSUPPORTED
+    assert call(rope=_abi.RopeParams(150000.0, 32.0, 4096, 80, 1.0, 32.0)) == _abi.GPTOSS_ERR_INVALID_ARG
     assert call(Hq=2048, Hkv=8) == _abi.GPTOSS_ERR_UNSUPPORTED      # more heads than the sink reduction holds
     assert call(Hkv=7) == _abi.GPTOSS_ERR_INVALID_ARG
     assert call(window=-1) == _abi.GPTOSS_ERR_INVALID_ARG

@@ -198,13 +198,13 @@ def test_bwd_no_rows(cuda_device):
 
 
 # Split sweeps: with G = 8 query heads per kv head, a key tile whose sweep
-# covers more than 16 query tiles (more than 128 (head, tile) steps) is cut
-# into chunks whose partial dK / dV add up in fp32 -- 1100 rows give key tile
-# 0 eighteen query tiles (two chunks); window 1000 seventeen.
-@pytest.mark.parametrize("window", [0, 1000])
+# covers more than 24 query tiles (more than 192 (head, tile) steps) is cut
+# into chunks whose partial dK / dV add up in fp32 -- 1700 rows give key tile
+# 0 twenty-seven query tiles (two chunks); window 1500 twenty-six.
+@pytest.mark.parametrize("window", [0, 1500])
 def test_bwd_split_sweeps(cuda_device, window):
     rng = np.random.default_rng(137)
-    B, S, Hq, Hkv = 1, 1100, 16, 2
+    B, S, Hq, Hkv = 1, 1700, 16, 2
     q, k, v, dout, sinks = _inputs(rng, (B, S), (B, S), Hq, Hkv)
     out, lse = _oracle_fwd(q, k, v, sinks, window, TABLES)
     got = _bwd(q, k, v, sinks, dout, out, lse, window, ROPE)
@@ -214,18 +214,18 @@ def test_bwd_split_sweeps(cuda_device, window):
 
 def test_bwd_split_sweeps_thd(cuda_device):
     rng = np.random.default_rng(139)
-    cu = np.array([0, 5, 1105, 1200], np.int64)  # lengths 5, 1100, 95
+    cu = np.array([0, 5, 1705, 1800], np.int64)  # lengths 5, 1700, 95
     T, Hq, Hkv = int(cu[-1]), 16, 2
     q, k, v, dout, sinks = _inputs(rng, (T,), (T,), Hq, Hkv)
     out, lse = _oracle_fwd(q, k, v, sinks, 0, TABLES, cu=cu)
-    got = _bwd(q, k, v, sinks, dout, out, lse, 0, ROPE, cu_seqlens=i32(cu), max_seqlen=1100)
+    got = _bwd(q, k, v, sinks, dout, out, lse, 0, ROPE, cu_seqlens=i32(cu), max_seqlen=1700)
     ref = attn_bwd_thd(q, k, v, sinks.astype(np.float64), cu, SCALE, 0, dout, rope_tables=TABLES, out=out)
     _check_all(got, ref, "split sweeps thd")
 
 
 def test_bwd_full_size_full_causal_slice(cuda_device):
     # the full-causal workload (B=2, S=8192, 64 / 8 heads): key tile 0 sweeps
-    # 128 query tiles x 8 heads, cut into 8 chunks.  The GPU forward supplies
+    # 128 query tiles x 8 heads, cut into 6 chunks.  The GPU forward supplies
     # out / lse everywhere except the checked slice (batch row 1, kv group 2),
     # where the oracle's stored output and lse stand in; that slice's dq / dk /
     # dv depend on nothing else
@@ -248,6 +248,24 @@ def test_bwd_full_size_full_causal_slice(cuda_device):
     assert_grad_parity(host(dq[b:b + 1, :, heads]), rq, "full causal dq")
     assert_grad_parity(host(dk[b:b + 1, :, g:g + 1]), rk, "full causal dk")
     assert_grad_parity(host(dv[b:b + 1, :, g:g + 1]), rv, "full causal dv")
+
+
+# Partial rotary (rotary_dim < 64): features [0, rotary_dim) rotate in pairs
+# (j, j + rotary_dim / 2), the rest pass through without the concentration;
+# the RoPE transpose in every backward epilogue follows.  W = 128 takes the
+# mma.sync dQ kernel, W = 0 the tcgen05 one; 1700 rows split key tile 0's
+# sweep (the finishing kernel's transpose).
+@pytest.mark.parametrize("rotary_dim,window,S", [(32, 128, 300), (16, 0, 300), (48, 0, 1700), (48, 128, 300)])
+def test_bwd_partial_rotary(cuda_device, rotary_dim, window, S):
+    rng = np.random.default_rng(151)
+    B, Hq, Hkv = 1, 16, 2
+    q, k, v, dout, sinks = _inputs(rng, (B, S), (B, S), Hq, Hkv)
+    tables = yarn_inv_freq_and_concentration(rotary_dim, 150000.0, 32.0, 4096, 1.0, 32.0)
+    rope = ops.RopeConfig.from_dict(GPTOSS_ROPE, rotary_dim=rotary_dim)
+    out, lse = _oracle_fwd(q, k, v, sinks, window, tables)
+    got = _bwd(q, k, v, sinks, dout, out, lse, window, rope)
+    ref = attn_bwd_bshd(q, k, v, sinks.astype(np.float64), SCALE, window, dout, rope_tables=tables, out=out)
+    _check_all(got, ref, f"rotary_dim={rotary_dim} w={window} S={S}")
 
 
 @pytest.mark.parametrize("window", [0, 1, 128])

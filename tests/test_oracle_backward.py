@@ -20,6 +20,7 @@ from oracle.rope import default_positions_bshd, rope
 from oracle.yarn import yarn_inv_freq_and_concentration
 
 TABLES = yarn_inv_freq_and_concentration(64, 150000.0, 32.0, 4096, 1.0, 32.0)
+TABLES_PARTIAL = yarn_inv_freq_and_concentration(32, 150000.0, 32.0, 4096, 1.0, 32.0)  # rotary_dim 32
 SCALE = 0.125
 
 
@@ -37,7 +38,7 @@ def _loss_bshd(q, k, v, sinks, dout, window, tables, positions=None):
     return float((out * dout).sum())
 
 
-@pytest.mark.parametrize("window,tables", [(0, TABLES), (3, TABLES), (0, None), (2, None)])
+@pytest.mark.parametrize("window,tables", [(0, TABLES), (3, TABLES), (0, None), (2, None), (0, TABLES_PARTIAL)])
 def test_finite_differences_bshd(window, tables):
     rng = np.random.default_rng(3)
     q, k, v, sinks, dout = _case(rng, 2, 6, 4, 2)
@@ -162,6 +163,23 @@ def test_rope_transpose_is_the_adjoint():
     assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(lhs))
     # and c^2 R^T R = c^2 I: the transpose undoes the rotation up to c^2
     np.testing.assert_allclose(rope_transpose(rope(x, pos, inv, c), pos, inv, c), c * c * x, rtol=0, atol=1e-12)
+
+
+def test_rope_transpose_partial_rotary():
+    # rotary_dim 32: pairs (j, j + 16) for j < 16 rotate; features 32..63 pass
+    # through unchanged (no concentration) in both directions
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((5, 3, 64))
+    y = rng.standard_normal((5, 3, 64))
+    pos = rng.integers(0, 100000, 5)
+    inv, c = TABLES_PARTIAL
+    assert inv.shape == (16,)
+    lhs = float((rope(x, pos, inv, c) * y).sum())
+    rhs = float((x * rope_transpose(y, pos, inv, c)).sum())
+    assert abs(lhs - rhs) <= 1e-11 * max(1.0, abs(lhs))
+    np.testing.assert_array_equal(rope_transpose(y, pos, inv, c)[..., 32:], y[..., 32:])
+    np.testing.assert_allclose(rope_transpose(rope(x, pos, inv, c), pos, inv, c)[..., :32], c * c * x[..., :32],
+                               rtol=0, atol=1e-12)
 
 
 def test_value_gradient_row_sums():
