@@ -43,6 +43,8 @@ constexpr int kDecMaxRows = 32;   // query rows of a CTA: two 16-row M fragments
 // Per head size kD (64 or 128): a stage holds one 64-key tile of K and one of
 // V, each kD / 64 halves of 64 features (a 128B-swizzled 64-row TMA box,
 // 8 KB); 96 KB of stages either way.
+constexpr int kDecShortStages = 2;  // K / V ring of short key ranges (see DecodeSmem)
+
 template <int kD>
 struct DecCfg {
   static constexpr int kTileBytes = kDecTileKeys * kD * 2;
@@ -91,16 +93,21 @@ __host__ __device__ inline int decode_chunk(int B, int Lmax, int Hkv) {
   return static_cast<int>(c);
 }
 
-template <int kD>
+// kStages: the K / V ring; short key ranges (a 128-key window: at most three
+// tiles) take a smaller ring, so more CTAs fit on an SM.
+template <int kD, int kStages = DecCfg<kD>::kStages>
 struct __align__(1024) DecodeSmem {
-  uint8_t k[DecCfg<kD>::kStages][DecCfg<kD>::kTileBytes];
-  uint8_t v[DecCfg<kD>::kStages][DecCfg<kD>::kTileBytes];  // directly after k (the merge uses both)
+  uint8_t k[kStages][DecCfg<kD>::kTileBytes];
+  uint8_t v[kStages][DecCfg<kD>::kTileBytes];  // directly after k (the merge uses both)
   __nv_bfloat16 q[kDecMaxRows][kD + 8];  // rotated query rows, padded
   float wm[kDecConsumerWarps][kDecMaxRows];
   float wl[kDecConsumerWarps][kDecMaxRows];
-  uint64_t full[DecCfg<kD>::kStages];
-  uint64_t empty[DecCfg<kD>::kStages];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
 };
+// the four warps' partial outputs reuse the K and V stages at the end
+template <int kD, int kStages>
+constexpr bool dec_merge_fits = kDecConsumerWarps * kDecMaxRows * kD * 4 <= 2 * kStages * DecCfg<kD>::kTileBytes;
 
 // The query tokens one CTA serves and the keys they see.  CTA z = (b, slice)
 // takes new tokens tok0 .. tok0 + ntok - 1 of sequence b; its query rows are
@@ -123,13 +130,13 @@ __device__ __forceinline__ DecodeRows decode_rows(const DecodeParams& p, int z) 
 
 // RM = 16-row M fragments of query rows (1: up to 16 rows, 2: up to 32);
 // kD = head size (64 or 128).
-template <int RM, int kD>
+template <int RM, int kD, int kStages = DecCfg<kD>::kStages>
 __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const __grid_constant__ DecodeParams p) {
-  constexpr int kStages = DecCfg<kD>::kStages;
+  static_assert(dec_merge_fits<kD, kStages>, "the warps' partial outputs must fit in the K / V stages");
   constexpr int kHalf = DecCfg<kD>::kHalfBytes;
   constexpr int kPairsD = kD / 2;
   extern __shared__ uint8_t smem_raw[];
-  DecodeSmem<kD>& sm = *reinterpret_cast<DecodeSmem<kD>*>(
+  DecodeSmem<kD, kStages>& sm = *reinterpret_cast<DecodeSmem<kD, kStages>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int g = blockIdx.x, split = blockIdx.y;
   const DecodeRows cr = decode_rows(p, blockIdx.z);

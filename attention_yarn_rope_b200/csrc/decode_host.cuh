@@ -119,9 +119,24 @@ gptoss_status decode_impl(const void* q, const void* k_cache, const void* v_cach
   if (rope != nullptr) yarn_table(*rope, &p.tab);
   else p.tab.enabled = 0;
   const bool d128 = D == kMaxHeadDim;
-  const size_t smem = (d128 ? sizeof(DecodeSmem<kMaxHeadDim>) : sizeof(DecodeSmem<kHeadDim>)) + 1024;
-  auto kernel = d128 ? (rm == 1 ? attn_decode_split_kernel<1, kMaxHeadDim> : attn_decode_split_kernel<2, kMaxHeadDim>)
-                     : (rm == 1 ? attn_decode_split_kernel<1, kHeadDim> : attn_decode_split_kernel<2, kHeadDim>);
+  // one split of at most four 64-key tiles (a 128-key window) takes the short
+  // K / V ring: a smaller CTA, more of them resident on an SM, and the range
+  // needs no deeper prefetch
+  const bool short_ring = p.direct && span <= 4 * kDecTileKeys;
+  size_t smem;
+  void (*kernel)(DecodeParams);
+  if (d128) {
+    smem = short_ring ? sizeof(DecodeSmem<kMaxHeadDim, kDecShortStages>) : sizeof(DecodeSmem<kMaxHeadDim>);
+    kernel = short_ring ? (rm == 1 ? attn_decode_split_kernel<1, kMaxHeadDim, kDecShortStages>
+                                   : attn_decode_split_kernel<2, kMaxHeadDim, kDecShortStages>)
+                        : (rm == 1 ? attn_decode_split_kernel<1, kMaxHeadDim> : attn_decode_split_kernel<2, kMaxHeadDim>);
+  } else {
+    smem = short_ring ? sizeof(DecodeSmem<kHeadDim, kDecShortStages>) : sizeof(DecodeSmem<kHeadDim>);
+    kernel = short_ring ? (rm == 1 ? attn_decode_split_kernel<1, kHeadDim, kDecShortStages>
+                                   : attn_decode_split_kernel<2, kHeadDim, kDecShortStages>)
+                        : (rm == 1 ? attn_decode_split_kernel<1, kHeadDim> : attn_decode_split_kernel<2, kHeadDim>);
+  }
+  smem += 1024;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return GPTOSS_ERR_CUDA;
