@@ -12,7 +12,10 @@
 // [0, 64) and [64, 128)), each a 128B-swizzled 128 x 64 box of the same
 // tensor maps as the D = 64 kernel.
 //   S  = Q K^T   (SS, M128 N128, 2 halves x 4 x K16, one accumulator)
-//   O += P V     (TS, M128 N64 per feature half, 8 x K16 each)
+//   O += P V     (TS, M128 N128, 8 x K16: the two feature halves of V are
+//                 consecutive 128B-swizzle atoms along N, 16 KB apart;
+//                 measured 1.2 % faster on full causal and 4.4 % on the
+//                 128-key window than two N64 products per K step)
 // Tensor memory: three S buffers [0, 384) (P over the first half of its S,
 // product t in buffer t mod 3), O [384, 512).
 // Warps: 0-3 rope (Q rotated in place: pair (j, j + 64) is word m of the
@@ -213,10 +216,10 @@ __device__ __forceinline__ void fwd128_mma_s_role(const FwdParams& p, Fwd128Smem
   mbar_wait(&sm.mma_final[0], 0, p.wait_ns);
 }
 
-// O_half += P V_half for the two feature halves (TS: P from tensor memory,
-// V read N-major); the first tile of a unit starts O from zero.
+// O += P V (TS: P from tensor memory, V read N-major, both feature halves in
+// one N = 128 product); the first tile of a unit starts O from zero.
 __device__ __forceinline__ void fwd128_mma_pv_role(const FwdParams& p, Fwd128Smem& sm, uint32_t tmem) {
-  constexpr uint32_t idesc_o = idesc_f16_f32(128, 64, true);
+  constexpr uint32_t idesc_o = idesc_f16_f32(128, 128, true);
   constexpr uint32_t colO = kColO;  // O: columns 384 .. 511
   uint32_t t = 0, kv_it = 0;
   bool ok = true;
@@ -229,14 +232,14 @@ __device__ __forceinline__ void fwd128_mma_pv_role(const FwdParams& p, Fwd128Sme
       const uint32_t b = t % kSBufs, colP = b * 128;  // P sits over the S it came from
       if (!mbar_wait(&sm.p_full[b], (t / kSBufs) & 1, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
+      // one N = 128 product per K step: the second 64-feature half of V is
+      // the next 128B-swizzle atom along N, 16 KB on (leading byte offset)
+      const uint64_t vdesc = (sw128_desc(smem_u32(sm.v[s][0])) & ~(static_cast<uint64_t>(0x3FFF) << 16)) |
+                             (static_cast<uint64_t>(kFwdTileBytes >> 4) << 16);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const uint64_t vdesc = sw128_desc(smem_u32(sm.v[s][hf]));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + colO + 64 * hf, tmem + colP + kk * 8, vdesc + static_cast<uint64_t>(kk * 128), idesc_o,
-                 (j == 0 && kk == 0) ? 0u : 1u);
-      }
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts(tmem + colO, tmem + colP + kk * 8, vdesc + static_cast<uint64_t>(kk * 128), idesc_o,
+               (j == 0 && kk == 0) ? 0u : 1u);
       mma_commit(&sm.o_done[0]);
       mma_commit(&sm.s_empty[b]);  // the buffer may take product t + 3
       mma_commit(&sm.v_empty[s]);
